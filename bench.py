@@ -1,0 +1,383 @@
+"""Benchmark of the SubMConv3d hot path on B200: neighbour-map build + bf16 forward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload headline|dense|shell_bf16]
+
+One step = one pass of the whole hot path over one synthetic input: the
+neighbour-map build (hash-table init, insert, 27-probe query + tile masks) and
+the bf16 tcgen05 forward, for the headline workload (128^3 grid, 8 sphere
+shells, 329,839 voxels, 128 -> 128 channels).  Inputs are resident in HBM
+when the timed region starts; the L2 is flushed (256 MB write) before every
+timed step; each step is timed with CUDA events on the launching stream.
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own replica on
+its own features (weak scaling, no collective on the data path); the job time
+is the max over ranks and `value` counts the voxels of all ranks.
+
+--impl reference times the CPU oracle (oracle/, C++ std::map + fp64 loop) on
+the host cores, on bounded samples of the same workload, and prints the same
+line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SubMConv3d fwd voxels/s and TFLOP/s at 128^3/128ch bf16; % of B200 roofline"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Algorithmic bytes of the map build per voxel: int32 (b,z,y,x) in + int32 [27] out.
+MAP_BYTES_PER_VOXEL = 16 + 27 * 4
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def _workload(name):
+    import workloads as WL
+    return WL.make_workload(name)
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons in the background."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.device_index = device_index
+        self.lines = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.device_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import sparse_voxel_conv_b200 as S
+    from sparse_voxel_conv_b200 import _abi
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+
+    wl = _workload(args.workload)
+    import workloads as WL
+    cin, cout = wl.channels[0], wl.channels[1]
+    n = wl.n
+    coords_h = torch.from_numpy(wl.coords)
+    feats_h = torch.from_numpy(WL.to_bf16_values(WL.make_features(n, cin, 1 + 1000 * rank)))
+    w_h = torch.from_numpy(wl.weights()[0])
+    coords = coords_h.to(dev)
+    feats = feats_h.to(dev).to(torch.bfloat16)
+    weight = w_h.to(dev).to(torch.bfloat16)
+    out = torch.empty((n, cout), dtype=torch.bfloat16, device=dev)
+    nbr = torch.empty((n, 27), dtype=torch.int32, device=dev)
+    ws_bytes = _abi.subm3d_map_workspace_bytes(n, wl.grid_dim, wl.batch)
+    workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(ev_fwd=None):
+        h = S.build_map(coords, wl.grid_dim, wl.batch, check=False, nbr=nbr, workspace=workspace)
+        if ev_fwd is not None:
+            ev_fwd[0].record(stream)
+        S.forward(h, feats, weight, out=out)
+        if ev_fwd is not None:
+            ev_fwd[1].record(stream)
+        return h
+
+    # correctness gate before timing: the map must be valid
+    h0 = step()
+    assert S.map_status(h0) == 0, "map build reported a data error"
+    nnz_total = int((nbr >= 0).sum().item())
+    assert _abi.subm3d_device_status() == 0
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    evf = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
+    smi_index = visible[dev.index].strip() if len(visible) > dev.index and visible[0] else dev.index
+    sampler = ClockSampler(smi_index)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record(stream)
+        step(evf[i])
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    assert _abi.subm3d_device_status() == 0
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    fwd_ms = [a.elapsed_time(b) for a, b in evf]
+    map_ms = [s - f for s, f in zip(step_ms, fwd_ms)]
+    total_ms = float(sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    # e2e through the public API with host buffers: H2D of this step's inputs
+    # from pinned memory, map build, forward, D2H of the output, every step.
+    coords_p = coords_h.pin_memory()
+    feats_p = feats_h.to(torch.bfloat16).pin_memory()
+    w_p = w_h.to(torch.bfloat16).pin_memory()
+    out_p = torch.empty((n, cout), dtype=torch.bfloat16).pin_memory()
+    h2d = coords_p.numel() * 4 + feats_p.numel() * 2 + w_p.numel() * 2
+    d2h = out_p.numel() * 2
+
+    def e2e_step():
+        coords.copy_(coords_p, non_blocking=True)
+        feats.copy_(feats_p, non_blocking=True)
+        weight.copy_(w_p, non_blocking=True)
+        step()
+        out_p.copy_(out, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    if rank == 0:
+        peaks, peak_src = _peaks()
+        flops = 2.0 * nnz_total * cin * cout
+        fwd_avg_s = statistics.mean(fwd_ms) / 1e3
+        map_avg_s = statistics.mean(map_ms) / 1e3
+        achieved_tf = flops / fwd_avg_s / 1e12
+        peak_tf = float(peaks["bf16_tflops"])
+        map_gbs = n * MAP_BYTES_PER_VOXEL / map_avg_s / 1e9
+        voxels_total = n * world
+        line = {
+            "metric": METRIC,
+            "value": voxels_total / (total_ms / 1e3 / K),
+            "unit": "voxels/s",
+            "n_gpus": world,
+            "steps": K,
+            "warmup": args.warmup,
+            "ms_per_step": total_ms / K,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": {
+                "workload": wl.name, "n_voxels": n, "nnz_avg": nnz_total / n, "cin": cin,
+                "cout": cout, "grid_dim": wl.grid_dim, "batch": wl.batch,
+                "step": "map build (3 kernels) + bf16 forward (1 kernel)",
+                "l2": f"flushed before every timed step ({L2_FLUSH_BYTES >> 20} MB write)",
+                "parallelism": f"replicas x{world}, no collective on the data path",
+            },
+            "tflops_effective": flops * world / (total_ms / 1e3 / K) / 1e12,
+            "roofline": {
+                "kernel": "subm3d_fwd_bf16_sm100",
+                "bound": "tensor", "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
+                "frac": achieved_tf / peak_tf, "traffic": None,
+                "peak_source": f"{peak_src} bf16 dense burst",
+                "fwd_ms_avg": fwd_avg_s * 1e3,
+            },
+            "map_build": {
+                "bound": "hbm", "achieved": map_gbs, "peak": float(peaks["hbm_gbs"]),
+                "unit": "GB/s", "frac": map_gbs / float(peaks["hbm_gbs"]),
+                "bytes_per_voxel": MAP_BYTES_PER_VOXEL, "ms_avg": map_avg_s * 1e3,
+            },
+            "e2e": {"value": voxels_total / (e2e_ms / 1e3 / K), "unit": "voxels/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms / K},
+            "gpu_launches": 4 * K,
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl, args.cpu_rows)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _oracle_inputs(wl):
+    import workloads as WL
+    x = WL.to_bf16_values(WL.make_features(wl.n, wl.channels[0], 1)).astype(np.float64)
+    w = wl.weights()[0].astype(np.float64)
+    return x, w
+
+
+def _oracle_step(wl, x, w, rows):
+    """One bounded oracle pass: the whole map (std::map) + the forward of `rows`."""
+    from oracle import cpp as C
+    t0 = time.perf_counter()
+    nbr = C.build_map(wl.coords, wl.grid_dim, wl.batch)
+    t1 = time.perf_counter()
+    C.forward(nbr, x, w, rows=rows, round_to_bf16=True)
+    t2 = time.perf_counter()
+    return t1 - t0, t2 - t1
+
+
+def cpu_baseline(wl, n_rows):
+    """The oracle as it stands on the host cores: map build of the full set plus
+    the forward of a sample of rows; voxels/s = 1 / (map_s / N + fwd_s / rows)."""
+    from oracle import cpp as C
+    rows = np.linspace(0, wl.n - 1, min(n_rows, wl.n)).astype(np.int64)
+    x, w = _oracle_inputs(wl)
+    map_s, fwd_s = _oracle_step(wl, x, w, rows)
+    per_voxel = map_s / wl.n + fwd_s / rows.size
+    return {"value": 1.0 / per_voxel, "unit": "voxels/s", "cores": C.num_threads(),
+            "kind": "oracle",
+            "sample": f"map build of all {wl.n} voxels ({map_s:.2f} s) + fp64 forward of "
+                      f"{rows.size} evenly spaced rows ({fwd_s:.2f} s)"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from oracle import cpp as C
+    wl = _workload(args.workload)
+    # rows per step shrink with K so that the whole run stays within minutes
+    n_rows = max(256, min(args.cpu_rows, 2_000_000 // max(1, args.steps), wl.n))
+    rows = np.linspace(0, wl.n - 1, n_rows).astype(np.int64)
+    x, w = _oracle_inputs(wl)
+    for _ in range(min(args.warmup, 3)):
+        _oracle_step(wl, x, w, rows[:256])
+    per_voxel = []
+    t_start = time.perf_counter()
+    for _ in range(args.steps):
+        map_s, fwd_s = _oracle_step(wl, x, w, rows)
+        per_voxel.append(map_s / wl.n + fwd_s / rows.size)
+    wall = time.perf_counter() - t_start
+    sec_per_voxel = statistics.mean(per_voxel)
+    value = 1.0 / sec_per_voxel
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "voxels/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": sec_per_voxel * wl.n * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "n_voxels": wl.n, "cin": wl.channels[0],
+                   "cout": wl.channels[1], "parallelism": "host cores (OpenMP)"},
+        "cpu_baseline": {"value": value, "unit": "voxels/s", "cores": C.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"per step: map build of all {wl.n} voxels + fp64 forward "
+                                   f"of {rows.size} evenly spaced rows; ms_per_step extrapolates "
+                                   f"to the full set; wall {wall:.1f} s"},
+        "e2e": {"value": value, "unit": "voxels/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="headline", choices=["headline", "dense", "shell_bf16"])
+    ap.add_argument("--cpu-rows", type=int, default=40000)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

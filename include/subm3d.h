@@ -1,0 +1,175 @@
+/*
+ * subm3d.h -- C ABI of the B200 (sm_100a) submanifold 3x3x3 sparse convolution.
+ *
+ * The op (lato.2_mrp_mlx, commit 97dcdfb54a message and CLAUDE.md "Key facts"):
+ * every SparseConv3d of the sparse-voxel generators is a submanifold
+ * convolution, kernel 3x3x3, stride 1, whose output sites are exactly its input
+ * sites.  For a set of N voxels p_i = (b, z, y, x):
+ *
+ *     out[i] = sum_{k=0}^{26} W[:, k, :] . feats[nbr[i][k]]      (nbr != -1)
+ *
+ * where nbr[i][k] is the row of the voxel at p_i + d_k, the 27 offsets d_k are
+ * ordered kz-major, k = 9*(dz+1) + 3*(dy+1) + (dx+1), and W is spconv's KRSC
+ * weight [Cout, kz, ky, kx, Cin] (same notes).  This is correlation; `flip`
+ * selects the mirrored kernel W[:, 26-k, :] because the pages leave the
+ * orientation unverified (same commit message, "--flip-kernel"; notes,
+ * "Unresolved").  The map is built once per coordinate set and reused by
+ * every layer on that set, as spconv does with indice_key (same message).
+ *
+ * Conventions for every entry point:
+ *   - All buffers are caller-owned.  Pointers marked (device) must point to
+ *     memory of the current CUDA device; (host) to host memory.  The library
+ *     never allocates device memory; the map's scratch space is a caller
+ *     workspace sized by subm3d_map_workspace_bytes().
+ *   - `stream` is a cudaStream_t (0 = legacy default stream).  Work is
+ *     enqueued on it and the call returns without waiting, unless noted.
+ *   - Argument errors are detected on the host, before anything is enqueued,
+ *     and returned synchronously.  Data errors in the coordinates are detected
+ *     on the device and reported by subm3d_map_status().
+ *   - Every function is safe to call from several host threads on different
+ *     streams; calls that share a workspace must be ordered by the caller.
+ */
+#ifndef SUBM3D_H_
+#define SUBM3D_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Symbol visibility: the library is built with hidden visibility and exports
+ * exactly the functions declared here. */
+#if defined(__GNUC__)
+#define SUBM3D_API __attribute__((visibility("default")))
+#else
+#define SUBM3D_API
+#endif
+
+#define SUBM3D_ABI_VERSION 1
+/* Number of kernel offsets, 3x3x3. */
+#define SUBM3D_KVOL 27
+/* Rows covered by one word of the per-tile offset mask. */
+#define SUBM3D_TILE_ROWS 128
+
+typedef enum {
+  SUBM3D_OK = 0,
+  SUBM3D_E_INVALID = 1,     /* null pointer, negative size, too-small workspace, bad enum  */
+  SUBM3D_E_RANGE = 2,       /* a coordinate lies outside [0,batch) x [0,grid_dim)^3        */
+  SUBM3D_E_DUPLICATE = 3,   /* a coordinate occurs more than once                          */
+  SUBM3D_E_TABLE_FULL = 4,  /* the hash table ran out of slots (only with a forced size)   */
+  SUBM3D_E_UNSUPPORTED = 5, /* shape, alignment or device the kernels do not handle        */
+  SUBM3D_E_CUDA = 6,        /* a CUDA runtime call failed (launch, copy, synchronize)     */
+  SUBM3D_E_TIMEOUT = 7      /* a bounded device-side wait ran out; the result is invalid   */
+} subm3d_status;
+
+typedef enum { SUBM3D_F32 = 0, SUBM3D_BF16 = 1 } subm3d_dtype;
+typedef enum { SUBM3D_ACT_NONE = 0, SUBM3D_ACT_GELU = 1 } subm3d_act;
+
+/* Opaque handle of a built neighbour map (host memory; see subm3d_build_map). */
+typedef struct subm3d_map subm3d_map;
+
+/* ABI version of the loaded library (SUBM3D_ABI_VERSION at build time). */
+SUBM3D_API int32_t subm3d_abi_version(void);
+
+/* Static, human-readable name of a status code (never NULL). */
+SUBM3D_API const char* subm3d_status_string(int32_t status);
+
+/*
+ * Workspace bytes subm3d_build_map() needs for N voxels in a batch x
+ * grid_dim^3 volume: a status word, one 32-bit offset mask per 128-row tile,
+ * and an open-addressing hash table of at least 2N slots.  Host-only, no CUDA
+ * call.  Returns 0 for arguments subm3d_build_map() would reject
+ * (N < 0, grid_dim < 1 or > 65535, batch < 1 or > 65535).
+ */
+SUBM3D_API size_t subm3d_map_workspace_bytes(int64_t n, int32_t grid_dim, int32_t batch);
+
+/*
+ * Build the neighbour map of a coordinate set ("sorted-key indice map, 27
+ * lookups/voxel", lato.2_mrp_mlx commit 97dcdfb54a; here a GPU hash table).
+ *
+ *   coords     (device) int32 [N, 4] rows (b, z, y, x), 16-byte aligned, any row order.
+ *   n          N >= 0; N < 2^31 - 1.
+ *   grid_dim   cubic extent; valid coordinates are 0 <= z, y, x < grid_dim (<= 65535).
+ *   batch      valid batch indices are 0 <= b < batch (<= 65535).
+ *   nbr        (device) int32 [N, 27] output, 16-byte aligned: row of the voxel at
+ *              p_i + d_k or -1 when it is absent or outside the grid.  Voxels of
+ *              different batch indices are never neighbours.
+ *   workspace  (device) >= subm3d_map_workspace_bytes(n, grid_dim, batch) bytes,
+ *              256-byte aligned.  Its head holds the tile masks the forward reads,
+ *              so it must stay alive, unmodified, as long as the handle is used.
+ *   stream     stream the build is enqueued on.
+ *   out_map    (host) receives a new handle; release it with subm3d_map_destroy().
+ *
+ * The map is bit-identical to the plain definition for every valid input and
+ * does not depend on the hash layout.  Coordinates outside the volume or
+ * repeated are reported by subm3d_map_status(); until it returns SUBM3D_OK the
+ * contents of nbr are unspecified.  Enqueues 3 kernels; no allocation.
+ * Testing knob: the environment variable SUBM3D_TABLE_CAPACITY, when set,
+ * caps the hash table at that many slots so that SUBM3D_E_TABLE_FULL can be
+ * exercised; probe loops stop after `capacity` steps instead of spinning.
+ */
+SUBM3D_API subm3d_status subm3d_build_map(const int32_t* coords, int64_t n, int32_t grid_dim,
+                               int32_t batch, int32_t* nbr, void* workspace,
+                               size_t workspace_bytes, void* stream, subm3d_map** out_map);
+
+/*
+ * Synchronizes the map's stream and returns the device-detected status of the
+ * build: SUBM3D_OK, SUBM3D_E_RANGE, SUBM3D_E_DUPLICATE or SUBM3D_E_TABLE_FULL
+ * (first in that order of precedence), or SUBM3D_E_CUDA.  Blocking.
+ */
+SUBM3D_API subm3d_status subm3d_map_status(const subm3d_map* map);
+
+/* Accessors (host, no CUDA call).  The pointers are the caller's buffers. */
+SUBM3D_API const int32_t* subm3d_map_nbr(const subm3d_map* map);        /* (device) [N, 27]          */
+SUBM3D_API const uint32_t* subm3d_map_tile_mask(const subm3d_map* map); /* (device) [ceil(N/128)]    */
+SUBM3D_API int64_t subm3d_map_size(const subm3d_map* map);              /* N                         */
+
+/* Frees the host handle only; the caller's nbr and workspace are untouched. */
+SUBM3D_API void subm3d_map_destroy(subm3d_map* map);
+
+/*
+ * Forward of one SubMConv3d layer over a built map (implicit gather-GEMM: the
+ * rows nbr[i][k] of feats are gathered tile by tile into shared memory and
+ * contracted against the weight slices; no scatter, no atomics, no [N,27,Cin]
+ * buffer).  out[i] = act( sum_k Wf[:, k, :] . feats[nbr[i][k]] ), with
+ * Wf[:, k] = W[:, k] (flip = 0, correlation) or W[:, 26-k] (flip != 0).
+ *
+ *   nbr        (device) int32 [N, 27] as written by subm3d_build_map().
+ *   tile_mask  (device) uint32 [ceil(N/128)]: bit k of word t is set when some row
+ *              of rows [128t, 128t+128) has nbr[.][k] != -1 (subm3d_map_tile_mask()).
+ *              NULL means every offset of every tile is visited.
+ *   n          N >= 0.  N = 0 enqueues nothing.
+ *   feats      (device) [N, Cin] row-major.
+ *   weight     (device) KRSC [Cout, 3, 3, 3, Cin] row-major.
+ *   out        (device) [N, Cout] row-major; must not overlap feats (E_INVALID).
+ *              feats, weight, out and nbr are 16-byte aligned for bf16 (else
+ *              SUBM3D_E_UNSUPPORTED), 4-byte aligned for fp32 (else E_INVALID).
+ *   dtype      SUBM3D_BF16: bf16 feats/weight/out, fp32 accumulation on the tensor
+ *              cores, Cin and Cout multiples of 16 (else SUBM3D_E_UNSUPPORTED).
+ *              SUBM3D_F32: fp32 throughout on CUDA-core FMA, any Cin, Cout >= 1.
+ *   act        SUBM3D_ACT_NONE, or SUBM3D_ACT_GELU (exact erf form) on the fp32 sum.
+ *
+ * The forward never fails on data.  SUBM3D_E_UNSUPPORTED is also returned when
+ * the current device is not sm_100.  A bounded device-side wait that runs out
+ * is reported by the next subm3d_device_status().
+ */
+SUBM3D_API subm3d_status subm3d_forward(const int32_t* nbr, const uint32_t* tile_mask, int64_t n,
+                             const void* feats, const void* weight, void* out,
+                             int32_t cin, int32_t cout, subm3d_dtype dtype, int32_t flip,
+                             subm3d_act act, void* stream);
+
+/*
+ * Synchronizes `stream`, then reads and clears the library's device error word
+ * of the current device: SUBM3D_E_TIMEOUT if a forward kernel gave up a
+ * bounded wait since the last call, else SUBM3D_OK (or SUBM3D_E_CUDA).
+ * Blocking.
+ */
+SUBM3D_API subm3d_status subm3d_device_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SUBM3D_H_ */

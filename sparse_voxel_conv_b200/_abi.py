@@ -1,0 +1,174 @@
+"""ctypes binding of libsubm3d.so (include/subm3d.h): argument marshalling only.
+
+Each function has the C name and passes torch tensors' device pointers and
+the current CUDA stream straight through.  Nothing here computes any part of
+the convolution; if the shared library is missing the import fails loudly,
+there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libsubm3d.so")
+
+SUBM3D_OK = 0
+SUBM3D_E_INVALID = 1
+SUBM3D_E_RANGE = 2
+SUBM3D_E_DUPLICATE = 3
+SUBM3D_E_TABLE_FULL = 4
+SUBM3D_E_UNSUPPORTED = 5
+SUBM3D_E_CUDA = 6
+SUBM3D_E_TIMEOUT = 7
+
+SUBM3D_F32 = 0
+SUBM3D_BF16 = 1
+SUBM3D_ACT_NONE = 0
+SUBM3D_ACT_GELU = 1
+SUBM3D_KVOL = 27
+SUBM3D_TILE_ROWS = 128
+
+
+class Subm3dError(RuntimeError):
+    """A non-OK subm3d_status returned by the library."""
+
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {subm3d_status_string(status)} (status {status})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python -m sparse_voxel_conv_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    sig = {
+        "subm3d_abi_version": (i32, []),
+        "subm3d_status_string": (ctypes.c_char_p, [i32]),
+        "subm3d_map_workspace_bytes": (sz, [i64, i32, i32]),
+        "subm3d_build_map": (ctypes.c_int, [vp, i64, i32, i32, vp, vp, sz, vp,
+                                            ctypes.POINTER(vp)]),
+        "subm3d_map_status": (ctypes.c_int, [vp]),
+        "subm3d_map_nbr": (vp, [vp]),
+        "subm3d_map_tile_mask": (vp, [vp]),
+        "subm3d_map_size": (i64, [vp]),
+        "subm3d_map_destroy": (None, [vp]),
+        "subm3d_forward": (ctypes.c_int, [vp, vp, i64, vp, vp, vp, i32, i32, ctypes.c_int, i32,
+                                          ctypes.c_int, vp]),
+        "subm3d_device_status": (ctypes.c_int, [vp]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _check(status: int, where: str) -> None:
+    if status != SUBM3D_OK:
+        raise Subm3dError(status, where)
+
+
+def subm3d_abi_version() -> int:
+    return int(lib.subm3d_abi_version())
+
+
+def subm3d_status_string(status: int) -> str:
+    return lib.subm3d_status_string(int(status)).decode()
+
+
+def subm3d_map_workspace_bytes(n: int, grid_dim: int, batch: int) -> int:
+    return int(lib.subm3d_map_workspace_bytes(int(n), int(grid_dim), int(batch)))
+
+
+class MapHandle:
+    """Owns a subm3d_map* and keeps the tensors it points into alive."""
+
+    def __init__(self, ptr: int, n: int, grid_dim: int, batch: int, nbr, workspace):
+        self._ptr = ptr
+        self.n = int(n)
+        self.grid_dim = int(grid_dim)
+        self.batch = int(batch)
+        self.nbr = nbr
+        self.workspace = workspace
+
+    @property
+    def ptr(self) -> int:
+        return self._ptr
+
+    def close(self) -> None:
+        if self._ptr:
+            lib.subm3d_map_destroy(self._ptr)
+            self._ptr = 0
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def subm3d_build_map(coords, n: int, grid_dim: int, batch: int, nbr, workspace,
+                     workspace_bytes: int | None = None, stream=None) -> MapHandle:
+    """Enqueue the map build; raises Subm3dError on an argument error."""
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    out = ctypes.c_void_p()
+    st = lib.subm3d_build_map(_ptr(coords), int(n), int(grid_dim), int(batch), _ptr(nbr),
+                              _ptr(workspace), int(workspace_bytes), _stream(stream),
+                              ctypes.byref(out))
+    _check(st, "subm3d_build_map")
+    return MapHandle(out.value, n, grid_dim, batch, nbr, workspace)
+
+
+def subm3d_map_status(handle: MapHandle) -> int:
+    """Blocking: the device-detected status of the build (an int status code)."""
+    return int(lib.subm3d_map_status(handle.ptr))
+
+
+def subm3d_map_nbr(handle: MapHandle) -> int:
+    return int(lib.subm3d_map_nbr(handle.ptr) or 0)
+
+
+def subm3d_map_tile_mask(handle: MapHandle) -> int:
+    return int(lib.subm3d_map_tile_mask(handle.ptr) or 0)
+
+
+def subm3d_map_size(handle: MapHandle) -> int:
+    return int(lib.subm3d_map_size(handle.ptr))
+
+
+def subm3d_forward(nbr, tile_mask, n: int, feats, weight, out, cin: int, cout: int,
+                   dtype: int, flip: bool, act: int, stream=None) -> None:
+    """Enqueue one layer's forward; raises Subm3dError on an argument error."""
+    st = lib.subm3d_forward(_ptr(nbr), _ptr(tile_mask), int(n), _ptr(feats), _ptr(weight),
+                            _ptr(out), int(cin), int(cout), int(dtype), 1 if flip else 0,
+                            int(act), _stream(stream))
+    _check(st, "subm3d_forward")
+
+
+def subm3d_device_status(stream=None) -> int:
+    """Blocking: SUBM3D_E_TIMEOUT if a forward kernel gave up a bounded wait."""
+    return int(lib.subm3d_device_status(_stream(stream)))

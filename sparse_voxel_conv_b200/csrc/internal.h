@@ -1,0 +1,53 @@
+// Declarations shared by the C-ABI layer (subm3d_api.cu) and the kernel files.
+// Not installed; the public surface is include/subm3d.h.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace subm3d {
+
+// Bits of the map build's device status word.
+constexpr uint32_t kErrRange = 1u;
+constexpr uint32_t kErrDuplicate = 2u;
+constexpr uint32_t kErrTableFull = 4u;
+
+constexpr int kTileRows = 128;  // rows per tile-mask word
+constexpr int kKvol = 27;
+
+// Placement of the map build's pieces inside the caller's workspace.
+struct MapLayout {
+  bool compact = true;      // 32-bit keys in 8-byte (key, row) slots; else 64-bit keys + row array
+  uint64_t capacity = 0;    // hash slots, a power of two >= 4
+  size_t status_off = 0;    // uint32 status word
+  size_t mask_off = 0;      // uint32 [n_tiles]
+  size_t table_off = 0;     // compact: uint64 [capacity]; wide: uint64 keys [capacity]
+  size_t rows_off = 0;      // wide only: int32 rows [capacity]
+  size_t total = 0;         // bytes
+  int64_t n_tiles = 0;
+};
+
+// Returns false when the arguments are out of the supported range.
+// forced_capacity (a power of two, or 0) caps the hash table for testing.
+bool map_layout(int64_t n, int32_t grid_dim, int32_t batch, uint64_t forced_capacity,
+                MapLayout* out);
+
+// Enqueues the three map-build kernels on `stream`.  Returns the launch error.
+cudaError_t launch_map_build(const int32_t* coords, int64_t n, int32_t grid_dim, int32_t batch,
+                             int32_t* nbr, void* workspace, const MapLayout& lay,
+                             cudaStream_t stream);
+
+// fp32 forward on CUDA-core FMA.
+cudaError_t launch_forward_f32(const int32_t* nbr, const uint32_t* tile_mask, int64_t n,
+                               const float* feats, const float* weight, float* out, int32_t cin,
+                               int32_t cout, int32_t flip, int32_t act, cudaStream_t stream);
+
+// bf16 forward on tcgen05 tensor cores (fp32 accumulation in TMEM).
+// err_word is the library's device error word (set when a bounded wait runs out).
+cudaError_t launch_forward_bf16(const int32_t* nbr, const uint32_t* tile_mask, int64_t n,
+                                const void* feats, const void* weight, void* out, int32_t cin,
+                                int32_t cout, int32_t flip, int32_t act, int32_t* err_word,
+                                cudaStream_t stream);
+
+}  // namespace subm3d

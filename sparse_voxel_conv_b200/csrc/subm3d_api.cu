@@ -1,0 +1,212 @@
+// C ABI of the submanifold 3x3x3 sparse convolution (include/subm3d.h):
+// argument checks, workspace sizing, the map handle, and kernel dispatch.
+// No device memory is allocated here; every buffer belongs to the caller.
+#include <cuda_runtime.h>
+
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+#include "subm3d.h"
+
+// The library's device error word: set to 1 by a forward kernel whose bounded
+// wait ran out; read and cleared by subm3d_device_status().
+static __device__ int32_t g_subm3d_error_word;
+
+struct subm3d_map {
+  const int32_t* nbr;
+  const uint32_t* tile_mask;
+  const uint32_t* status_word;
+  int64_t n;
+  int32_t grid_dim;
+  int32_t batch;
+  cudaStream_t stream;
+};
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Testing knob: SUBM3D_TABLE_CAPACITY caps the hash table at that many slots
+// (rounded up to a power of two), so that a full table can be exercised.
+uint64_t forced_capacity() {
+  const char* s = std::getenv("SUBM3D_TABLE_CAPACITY");
+  if (!s || !*s) return 0;
+  return std::strtoull(s, nullptr, 10);
+}
+
+// 1 when the current device is sm_100 (B200 class), 0 when it is not, -1 on error.
+int device_is_sm100(int* device_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  static std::mutex mu;
+  static signed char cache[64];
+  static bool init = false;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!init) {
+    std::memset(cache, -1, sizeof(cache));
+    init = true;
+  }
+  if (device_out) *device_out = dev;
+  if (dev >= 0 && dev < 64 && cache[dev] >= 0) return cache[dev];
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return -1;
+  const int ok = (major == 10 && minor == 0) ? 1 : 0;
+  if (dev >= 0 && dev < 64) cache[dev] = static_cast<signed char>(ok);
+  return ok;
+}
+
+int32_t* device_error_word() {
+  static std::mutex mu;
+  static int32_t* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_subm3d_error_word) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<int32_t*>(p);
+  }
+  return addr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t subm3d_abi_version(void) { return SUBM3D_ABI_VERSION; }
+
+const char* subm3d_status_string(int32_t status) {
+  switch (status) {
+    case SUBM3D_OK: return "ok";
+    case SUBM3D_E_INVALID: return "invalid argument";
+    case SUBM3D_E_RANGE: return "coordinate out of range";
+    case SUBM3D_E_DUPLICATE: return "duplicate coordinate";
+    case SUBM3D_E_TABLE_FULL: return "hash table full";
+    case SUBM3D_E_UNSUPPORTED: return "unsupported shape, alignment or device";
+    case SUBM3D_E_CUDA: return "CUDA runtime error";
+    case SUBM3D_E_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+size_t subm3d_map_workspace_bytes(int64_t n, int32_t grid_dim, int32_t batch) {
+  subm3d::MapLayout lay;
+  if (!subm3d::map_layout(n, grid_dim, batch, 0, &lay)) return 0;
+  return lay.total;
+}
+
+subm3d_status subm3d_build_map(const int32_t* coords, int64_t n, int32_t grid_dim,
+                               int32_t batch, int32_t* nbr, void* workspace,
+                               size_t workspace_bytes, void* stream, subm3d_map** out_map) {
+  if (!out_map) return SUBM3D_E_INVALID;
+  *out_map = nullptr;
+  if (n < 0 || !workspace) return SUBM3D_E_INVALID;
+  if (n > 0 && (!coords || !nbr)) return SUBM3D_E_INVALID;
+  subm3d::MapLayout lay;
+  if (!subm3d::map_layout(n, grid_dim, batch, forced_capacity(), &lay))
+    return (grid_dim < 1 || batch < 1) ? SUBM3D_E_INVALID : SUBM3D_E_UNSUPPORTED;
+  subm3d::MapLayout full;
+  subm3d::map_layout(n, grid_dim, batch, 0, &full);
+  if (workspace_bytes < full.total) return SUBM3D_E_INVALID;
+  if (!aligned(coords, 16) || !aligned(nbr, 16) || !aligned(workspace, 256))
+    return SUBM3D_E_INVALID;
+  auto* h = new (std::nothrow) subm3d_map;
+  if (!h) return SUBM3D_E_INVALID;
+  auto* ws = static_cast<uint8_t*>(workspace);
+  h->nbr = nbr;
+  h->tile_mask = reinterpret_cast<const uint32_t*>(ws + lay.mask_off);
+  h->status_word = reinterpret_cast<const uint32_t*>(ws + lay.status_off);
+  h->n = n;
+  h->grid_dim = grid_dim;
+  h->batch = batch;
+  h->stream = static_cast<cudaStream_t>(stream);
+  if (subm3d::launch_map_build(coords, n, grid_dim, batch, nbr, workspace, lay,
+                               h->stream) != cudaSuccess) {
+    delete h;
+    return SUBM3D_E_CUDA;
+  }
+  *out_map = h;
+  return SUBM3D_OK;
+}
+
+subm3d_status subm3d_map_status(const subm3d_map* map) {
+  if (!map) return SUBM3D_E_INVALID;
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, map->status_word, sizeof(word), cudaMemcpyDeviceToHost,
+                      map->stream) != cudaSuccess ||
+      cudaStreamSynchronize(map->stream) != cudaSuccess)
+    return SUBM3D_E_CUDA;
+  if (word & subm3d::kErrRange) return SUBM3D_E_RANGE;
+  if (word & subm3d::kErrDuplicate) return SUBM3D_E_DUPLICATE;
+  if (word & subm3d::kErrTableFull) return SUBM3D_E_TABLE_FULL;
+  return SUBM3D_OK;
+}
+
+const int32_t* subm3d_map_nbr(const subm3d_map* map) { return map ? map->nbr : nullptr; }
+const uint32_t* subm3d_map_tile_mask(const subm3d_map* map) {
+  return map ? map->tile_mask : nullptr;
+}
+int64_t subm3d_map_size(const subm3d_map* map) { return map ? map->n : -1; }
+void subm3d_map_destroy(subm3d_map* map) { delete map; }
+
+subm3d_status subm3d_forward(const int32_t* nbr, const uint32_t* tile_mask, int64_t n,
+                             const void* feats, const void* weight, void* out, int32_t cin,
+                             int32_t cout, subm3d_dtype dtype, int32_t flip, subm3d_act act,
+                             void* stream) {
+  if (n < 0 || cin < 1 || cout < 1) return SUBM3D_E_INVALID;
+  if (dtype != SUBM3D_F32 && dtype != SUBM3D_BF16) return SUBM3D_E_INVALID;
+  if (act != SUBM3D_ACT_NONE && act != SUBM3D_ACT_GELU) return SUBM3D_E_INVALID;
+  if (n > 0 && (!nbr || !feats || !weight || !out)) return SUBM3D_E_INVALID;
+  if (n >= 0x7FFFFFFFll) return SUBM3D_E_UNSUPPORTED;
+  if (n == 0) return SUBM3D_OK;
+  const size_t esz = dtype == SUBM3D_BF16 ? 2 : 4;
+  const auto* fb = static_cast<const uint8_t*>(feats);
+  const auto* ob = static_cast<const uint8_t*>(out);
+  if (fb < ob + static_cast<size_t>(n) * cout * esz && ob < fb + static_cast<size_t>(n) * cin * esz)
+    return SUBM3D_E_INVALID;  // out overlaps feats
+  auto s = static_cast<cudaStream_t>(stream);
+  const int flip01 = flip ? 1 : 0;
+  const int act01 = act == SUBM3D_ACT_GELU ? 1 : 0;
+  if (dtype == SUBM3D_F32) {
+    if (!aligned(nbr, 4) || !aligned(feats, 4) || !aligned(weight, 4) || !aligned(out, 4) ||
+        (tile_mask && !aligned(tile_mask, 4)))
+      return SUBM3D_E_INVALID;
+    return subm3d::launch_forward_f32(nbr, tile_mask, n, static_cast<const float*>(feats),
+                                      static_cast<const float*>(weight), static_cast<float*>(out),
+                                      cin, cout, flip01, act01, s) == cudaSuccess
+               ? SUBM3D_OK
+               : SUBM3D_E_CUDA;
+  }
+  if (cin % 16 != 0 || cout % 16 != 0) return SUBM3D_E_UNSUPPORTED;
+  if (!aligned(nbr, 16) || !aligned(feats, 16) || !aligned(weight, 16) || !aligned(out, 16) ||
+      (tile_mask && !aligned(tile_mask, 4)))
+    return SUBM3D_E_UNSUPPORTED;
+  const int sm100 = device_is_sm100(nullptr);
+  if (sm100 < 0) return SUBM3D_E_CUDA;
+  if (sm100 == 0) return SUBM3D_E_UNSUPPORTED;
+  int32_t* err = device_error_word();
+  if (!err) return SUBM3D_E_CUDA;
+  const cudaError_t e = subm3d::launch_forward_bf16(nbr, tile_mask, n, feats, weight, out, cin,
+                                                    cout, flip01, act01, err, s);
+  if (e == cudaErrorNotSupported) return SUBM3D_E_UNSUPPORTED;
+  return e == cudaSuccess ? SUBM3D_OK : SUBM3D_E_CUDA;
+}
+
+subm3d_status subm3d_device_status(void* stream) {
+  int32_t* err = device_error_word();
+  if (!err) return SUBM3D_E_CUDA;
+  auto s = static_cast<cudaStream_t>(stream);
+  int32_t word = 0;
+  const int32_t zero = 0;
+  if (cudaMemcpyAsync(&word, err, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaMemcpyAsync(err, &zero, sizeof(zero), cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return SUBM3D_E_CUDA;
+  return word ? SUBM3D_E_TIMEOUT : SUBM3D_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,156 @@
+"""User-facing API: SparseTensor, SubMConv3d with an indice_key map cache.
+
+The sparse-voxel generators the pages port (LATO.2, Pixal3D, the TRELLIS.2
+family) hold a SparseTensor (coordinates + features) and run SparseConv3d
+layers that are all submanifold 3x3x3 convolutions; the neighbour map is
+cached per coordinate set "the way spconv uses indice_key" (lato.2_mrp_mlx,
+commit 97dcdfb54a message).  torch provides device memory and streams only:
+every step of the op runs in libsubm3d.so's kernels.
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import _abi
+from ._abi import Subm3dError
+
+__all__ = ["MapHandle", "build_map", "forward", "SparseTensor", "SubMConv3d", "Subm3dError"]
+
+MapHandle = _abi.MapHandle
+
+_DTYPES = {torch.float32: _abi.SUBM3D_F32, torch.bfloat16: _abi.SUBM3D_BF16}
+_ACTS = {None: _abi.SUBM3D_ACT_NONE, "none": _abi.SUBM3D_ACT_NONE, "gelu": _abi.SUBM3D_ACT_GELU}
+
+
+def _cuda_contig(t: torch.Tensor, name: str, dtype=None) -> torch.Tensor:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.contiguous()
+
+
+def build_map(coords: torch.Tensor, grid_dim: int, batch: int = 1, stream=None,
+              check: bool = True, nbr: torch.Tensor | None = None,
+              workspace: torch.Tensor | None = None) -> MapHandle:
+    """Neighbour map of a coordinate set: int32 [N, 27] plus per-tile offset masks.
+
+    coords: int32 [N, 4] (b, z, y, x) on the GPU.  With check=True the call
+    waits for the build and raises Subm3dError on out-of-range or duplicate
+    coordinates; with check=False it stays asynchronous (call .status later).
+    nbr / workspace may be passed in to reuse memory.
+    """
+    coords = _cuda_contig(coords, "coords", torch.int32)
+    if coords.dim() != 2 or coords.shape[1] != 4:
+        raise ValueError("coords must have shape [N, 4]")
+    n = coords.shape[0]
+    ws_bytes = _abi.subm3d_map_workspace_bytes(n, grid_dim, batch)
+    if ws_bytes == 0:
+        raise Subm3dError(_abi.SUBM3D_E_UNSUPPORTED, "subm3d_map_workspace_bytes")
+    dev = coords.device
+    if nbr is None:
+        nbr = torch.empty((n, 27), dtype=torch.int32, device=dev)
+    if workspace is None or workspace.numel() * workspace.element_size() < ws_bytes:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    h = _abi.subm3d_build_map(coords, n, grid_dim, batch, nbr, workspace, ws_bytes, stream)
+    h.coords = coords
+    if check:
+        st = _abi.subm3d_map_status(h)
+        if st != _abi.SUBM3D_OK:
+            raise Subm3dError(st, "subm3d_build_map")
+    return h
+
+
+def map_status(h: MapHandle) -> int:
+    return _abi.subm3d_map_status(h)
+
+
+def tile_mask_tensor(h: MapHandle) -> torch.Tensor:
+    """The map's per-128-row-tile offset masks as an int32 view of its workspace."""
+    off = _abi.subm3d_map_tile_mask(h) - h.workspace.data_ptr()
+    n_tiles = (h.n + _abi.SUBM3D_TILE_ROWS - 1) // _abi.SUBM3D_TILE_ROWS
+    return h.workspace[off:off + 4 * n_tiles].view(torch.int32)
+
+
+def forward(h: MapHandle, feats: torch.Tensor, weight: torch.Tensor, flip: bool = False,
+            act: str | None = None, out: torch.Tensor | None = None, stream=None,
+            use_tile_mask: bool = True) -> torch.Tensor:
+    """One SubMConv3d layer: out[i] = act(sum_k Wf[:,k,:] . feats[nbr[i,k]]).
+
+    feats: [N, Cin] float32 or bfloat16; weight: KRSC [Cout, 3, 3, 3, Cin] (or
+    [Cout, 27, Cin]) of the same dtype.  Returns [N, Cout] of that dtype.
+    """
+    if feats.dtype not in _DTYPES:
+        raise ValueError(f"unsupported feature dtype {feats.dtype}")
+    feats = _cuda_contig(feats, "feats")
+    weight = _cuda_contig(weight, "weight", feats.dtype)
+    n, cin = feats.shape
+    if n != h.n:
+        raise ValueError(f"feats has {n} rows but the map has {h.n}")
+    cout = weight.shape[0]
+    if weight.numel() != cout * 27 * cin:
+        raise ValueError("weight must be KRSC [Cout, 3, 3, 3, Cin]")
+    if out is None:
+        out = torch.empty((n, cout), dtype=feats.dtype, device=feats.device)
+    mask_ptr = _abi.subm3d_map_tile_mask(h) if use_tile_mask else None
+    _abi.subm3d_forward(h.nbr, mask_ptr, n, feats, weight, out, cin, cout, _DTYPES[feats.dtype],
+                        flip, _ACTS[act], stream)
+    return out
+
+
+class SparseTensor:
+    """Voxel coordinates int32 [N, 4] (b, z, y, x) + features [N, C] on one GPU,
+    with the cache of neighbour maps built on this coordinate set."""
+
+    def __init__(self, coords: torch.Tensor, feats: torch.Tensor, grid_dim: int,
+                 batch: int = 1, cache: dict | None = None):
+        if coords.shape[0] != feats.shape[0]:
+            raise ValueError("coords and feats must have the same number of rows")
+        self.coords = coords
+        self.feats = feats
+        self.grid_dim = int(grid_dim)
+        self.batch = int(batch)
+        self.cache = {} if cache is None else cache
+
+    def replace(self, feats: torch.Tensor) -> "SparseTensor":
+        """Same coordinate set (and map cache), new features."""
+        return SparseTensor(self.coords, feats, self.grid_dim, self.batch, self.cache)
+
+    def get_map(self, indice_key: str) -> MapHandle:
+        h = self.cache.get(indice_key)
+        if h is None:
+            h = build_map(self.coords, self.grid_dim, self.batch)
+            self.cache[indice_key] = h
+        elif h.n != self.coords.shape[0]:
+            raise Subm3dError(_abi.SUBM3D_E_INVALID, f"cached map {indice_key!r} size mismatch")
+        return h
+
+
+class SubMConv3d(torch.nn.Module):
+    """Submanifold 3x3x3 convolution, stride 1, output sites = input sites.
+
+    The weight is a KRSC parameter [Cout, 3, 3, 3, Cin].  Layers sharing an
+    indice_key reuse one neighbour map per SparseTensor coordinate set.
+    flip selects the mirrored kernel; act=None or "gelu" (exact erf form).
+    No bias: the pages' op has none.
+    """
+
+    def __init__(self, in_channels: int, out_channels: int, indice_key: str = "subm0",
+                 flip: bool = False, act: str | None = None, dtype=torch.bfloat16,
+                 device=None):
+        super().__init__()
+        self.in_channels = in_channels
+        self.out_channels = out_channels
+        self.indice_key = indice_key
+        self.flip = flip
+        self.act = act
+        w = torch.empty((out_channels, 3, 3, 3, in_channels), dtype=torch.float32)
+        w.normal_(0.0, 1.0 / math.sqrt(27.0 * in_channels))
+        self.weight = torch.nn.Parameter(w.to(dtype=dtype, device=device), requires_grad=False)
+
+    def forward(self, x: SparseTensor) -> SparseTensor:
+        h = x.get_map(self.indice_key)
+        y = forward(h, x.feats, self.weight, flip=self.flip, act=self.act)
+        return x.replace(y)

@@ -1,0 +1,93 @@
+"""The C ABI library loads, exports every symbol include/*.h declares, and
+rejects bad arguments on the host before touching the device.  CPU only:
+no call here reaches a CUDA kernel."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def abi():
+    from sparse_voxel_conv_b200 import build
+    build.build()
+    from sparse_voxel_conv_b200 import _abi
+    return _abi
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        txt = open(h).read()
+        txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+        names |= set(re.findall(r"SUBM3D_API\s+[\w\s\*]*?\b(subm3d_\w+)\s*\(", txt))
+    return names
+
+
+def test_exports_every_declared_symbol(abi):
+    names = _declared()
+    assert len(names) >= 11
+    lib = ctypes.CDLL(abi.LIB_PATH)
+    for name in sorted(names):
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+
+
+def test_version_and_strings(abi):
+    assert abi.subm3d_abi_version() == 1
+    for st in range(8):
+        assert abi.subm3d_status_string(st) not in ("", "unknown status")
+    assert abi.subm3d_status_string(99) == "unknown status"
+
+
+def test_workspace_bytes(abi):
+    f = abi.subm3d_map_workspace_bytes
+    assert f(-1, 16, 1) == 0 and f(10, 0, 1) == 0 and f(10, 16, 0) == 0
+    assert f(10, 70000, 1) == 0 and f(10, 16, 70000) == 0
+    # compact form: 8-byte slots, capacity = max(1024, pow2 >= 2N)
+    n = 329839
+    ws = f(n, 128, 1)
+    assert ws >= 256 + 4 * ((n + 127) // 128) + 8 * (1 << 20)
+    assert ws < 256 + 4 * ((n + 127) // 128) + 8 * (1 << 20) + 1024
+    # wide form (batch > 4) adds a 4-byte row array
+    assert f(n, 128, 5) >= ws + 4 * (1 << 20)
+    assert f(0, 16, 1) > 0
+
+
+def test_build_map_argument_errors(abi):
+    lib = abi.lib
+    out = ctypes.c_void_p()
+    ws = abi.subm3d_map_workspace_bytes(100, 16, 1)
+    A = 1 << 20  # a 256-byte aligned fake address; never dereferenced on these paths
+    E_INVALID, E_UNSUP = abi.SUBM3D_E_INVALID, abi.SUBM3D_E_UNSUPPORTED
+    assert lib.subm3d_build_map(A, 100, 16, 1, A, A, ws, None, None) == E_INVALID
+    assert lib.subm3d_build_map(None, 100, 16, 1, A, A, ws, None, ctypes.byref(out)) == E_INVALID
+    assert lib.subm3d_build_map(A, -1, 16, 1, A, A, ws, None, ctypes.byref(out)) == E_INVALID
+    assert lib.subm3d_build_map(A, 100, 16, 1, A, A, ws - 1, None, ctypes.byref(out)) == E_INVALID
+    assert lib.subm3d_build_map(A + 4, 100, 16, 1, A, A, ws, None, ctypes.byref(out)) == E_INVALID
+    assert lib.subm3d_build_map(A, 100, 16, 1, A, A + 16, ws, None, ctypes.byref(out)) == E_INVALID
+    assert lib.subm3d_build_map(A, 100, 0, 1, A, A, ws, None, ctypes.byref(out)) == E_INVALID
+    assert lib.subm3d_build_map(A, 100, 70000, 1, A, A, ws, None, ctypes.byref(out)) == E_UNSUP
+    assert out.value is None
+
+
+def test_forward_argument_errors(abi):
+    lib = abi.lib
+    A, B, W = 1 << 20, 1 << 24, 1 << 28   # disjoint fake addresses
+    E_INVALID, E_UNSUP, OK = abi.SUBM3D_E_INVALID, abi.SUBM3D_E_UNSUPPORTED, abi.SUBM3D_OK
+    f = lib.subm3d_forward
+    # n = 0 is a no-op
+    assert f(None, None, 0, None, None, None, 16, 16, 1, 0, 0, None) == OK
+    assert f(A, None, -1, A, W, B, 16, 16, 1, 0, 0, None) == E_INVALID
+    assert f(A, None, 10, A, W, B, 0, 16, 1, 0, 0, None) == E_INVALID
+    assert f(A, None, 10, None, W, B, 16, 16, 1, 0, 0, None) == E_INVALID
+    assert f(A, None, 10, A, W, B, 16, 16, 7, 0, 0, None) == E_INVALID     # bad dtype
+    assert f(A, None, 10, A, W, B, 16, 16, 1, 0, 9, None) == E_INVALID     # bad act
+    assert f(A, None, 10, A, W, A + 64, 16, 16, 1, 0, 0, None) == E_INVALID  # out overlaps feats
+    assert f(A, None, 10, A, W, B, 8, 16, 1, 0, 0, None) == E_UNSUP        # bf16 Cin % 16
+    assert f(A, None, 10, A, W, B, 16, 24, 1, 0, 0, None) == E_UNSUP       # bf16 Cout % 16
+    assert f(A, None, 10, A + 8, W, B, 16, 16, 1, 0, 0, None) == E_UNSUP   # bf16 alignment
+    assert f(A, None, 10, A + 2, W, B, 3, 5, 0, 0, 0, None) == E_INVALID   # f32 alignment

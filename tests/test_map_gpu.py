@@ -1,0 +1,116 @@
+"""Neighbour-map build on the GPU vs the CPU oracle: bit-exact on every
+workload, under raster and random row order, for both key forms, plus the
+per-tile offset masks and the device-detected data errors."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as WL
+from oracle import cpp as C
+from tests.helpers import masks_from_nbr
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def S():
+    import sparse_voxel_conv_b200 as S
+    return S
+
+
+def _gpu_map(S, coords, grid, batch):
+    h = S.build_map(torch.from_numpy(np.ascontiguousarray(coords)).cuda(), grid, batch)
+    return h, h.nbr.cpu().numpy(), S.tile_mask_tensor(h).cpu().numpy().astype(np.int64) & 0x7FFFFFF
+
+
+@pytest.mark.parametrize("name", ["tiny", "shell", "headline", "dense", "batched"])
+def test_map_bit_exact(S, name):
+    wl = WL.make_workload(name)
+    h, nbr, masks = _gpu_map(S, wl.coords, wl.grid_dim, wl.batch)
+    ref = C.build_map(wl.coords, wl.grid_dim, wl.batch)
+    assert nbr.shape == ref.shape
+    assert np.array_equal(nbr, ref)
+    assert np.array_equal(masks, masks_from_nbr(ref))
+
+
+@pytest.mark.parametrize("name,seed", [("shell", 1), ("headline", 2), ("batched", 3)])
+def test_map_bit_exact_random_row_order(S, name, seed):
+    wl = WL.make_workload(name)
+    c = wl.coords[WL.permute_rows(wl.n, seed)]
+    _, nbr, masks = _gpu_map(S, c, wl.grid_dim, wl.batch)
+    ref = C.build_map(c, wl.grid_dim, wl.batch)
+    assert np.array_equal(nbr, ref)
+    assert np.array_equal(masks, masks_from_nbr(ref))
+
+
+@pytest.mark.parametrize("grid,batch,shift", [(2048, 1, 1900), (64, 6, 0), (65535, 9, 65500)])
+def test_map_wide_keys(S, grid, batch, shift):
+    # batch > 4 or grid_dim > 1024 takes the 64-bit key form
+    rng = np.random.default_rng(grid + batch)
+    parts = []
+    for b in range(batch):
+        c = WL.tiny_coords(seed=b)
+        c[:, 0] = b
+        c[:, 1:] += shift
+        parts.append(c)
+    c = np.concatenate(parts)[WL.permute_rows(sum(len(p) for p in parts), 4)]
+    del rng
+    _, nbr, masks = _gpu_map(S, c, grid, batch)
+    ref = C.build_map(c, grid, batch)
+    assert np.array_equal(nbr, ref)
+    assert np.array_equal(masks, masks_from_nbr(ref))
+
+
+def test_map_edge_sizes(S):
+    for c in (np.zeros((0, 4), np.int32), np.array([[0, 3, 3, 3]], np.int32),
+              WL.dense_coords(5)[:129], WL.dense_coords(2)):
+        grid = 5
+        h, nbr, masks = _gpu_map(S, c, grid, 1)
+        ref = C.build_map(c, grid, 1)
+        assert np.array_equal(nbr, ref)
+        assert np.array_equal(masks, masks_from_nbr(ref))
+
+
+def test_map_grid_boundary_no_wrap(S):
+    # voxels on opposite faces of the grid are not neighbours (no wrap-around)
+    g = 8
+    c = np.array([[0, 0, 0, 0], [0, g - 1, 0, 0], [0, 0, g - 1, 0], [0, 0, 0, g - 1],
+                  [0, g - 1, g - 1, g - 1]], np.int32)
+    _, nbr, _ = _gpu_map(S, c, g, 1)
+    assert np.array_equal(nbr, C.build_map(c, g, 1))
+    assert ((nbr >= 0).sum(axis=1) == 1).all()
+
+
+@pytest.mark.parametrize("bad,status", [([0, 0, 0, 16], 2), ([0, -1, 3, 3], 2), ([1, 1, 1, 1], 2),
+                                        (None, 3)])
+def test_map_data_errors(S, bad, status):
+    base = WL.tiny_coords()
+    extra = base[700:701] if bad is None else np.array([bad], np.int32)  # None: a duplicate
+    c = np.concatenate([base, extra])
+    with pytest.raises(S.Subm3dError) as e:
+        S.build_map(torch.from_numpy(c).cuda(), 16, 1)
+    assert e.value.status == status
+
+
+def test_map_table_full_is_reported_not_spun(S, monkeypatch):
+    monkeypatch.setenv("SUBM3D_TABLE_CAPACITY", "64")
+    c = torch.from_numpy(WL.tiny_coords()).cuda()
+    with pytest.raises(S.Subm3dError) as e:
+        S.build_map(c, 16, 1)
+    assert e.value.status == 4
+    monkeypatch.delenv("SUBM3D_TABLE_CAPACITY")
+    h = S.build_map(c, 16, 1)
+    assert np.array_equal(h.nbr.cpu().numpy(), C.build_map(WL.tiny_coords(), 16, 1))
+
+
+def test_map_async_status_and_reuse(S):
+    # build twice into the same buffers; the second build fully overwrites the first
+    c1 = torch.from_numpy(WL.shell_coords()).cuda()
+    h1 = S.build_map(c1, 64, 1, check=False)
+    assert S.map_status(h1) == 0
+    c2 = torch.from_numpy(WL.tiny_coords()).cuda()
+    nbr = torch.empty((c2.shape[0], 27), dtype=torch.int32, device="cuda")
+    h2 = S.build_map(c2, 16, 1, nbr=nbr, workspace=h1.workspace)
+    assert np.array_equal(h2.nbr.cpu().numpy(), C.build_map(WL.tiny_coords(), 16, 1))

@@ -85,17 +85,18 @@ def dense_coords(grid: int = 128, batch: int = 1) -> np.ndarray:
 
 
 def batched_coords(batch: int = 4, grid: int = 256, min_voxels: int = 250_000,
-                   seed0: int = 100, half: float = 1.0) -> np.ndarray:
+                   seed0: int = 100, half: float = 1.0, r_lo: float = 16.0,
+                   r_hi: float = 48.0) -> np.ndarray:
     """Batch of independent shell sets in a 256^3 grid.  Element b draws from
-    rng(100+b) and adds shells r ~ U[16,48], centre ~ U[r+1, 254-r]^3,
+    rng(100+b) and adds shells r ~ U[16,48], centre ~ U[r+1, grid-2-r]^3,
     half-width 1, until it holds at least 250k voxels (1,135,307 in total)."""
     parts = []
     for b in range(batch):
         rng = np.random.default_rng(seed0 + b)
         occ = np.zeros((grid,) * 3, bool)
         while int(occ.sum()) < min_voxels:
-            r = rng.uniform(16, 48)
-            c = rng.uniform(r + 1, 254 - r, size=3)
+            r = rng.uniform(r_lo, r_hi)
+            c = rng.uniform(r + 1, grid - 2 - r, size=3)
             _add_shell(occ, r, c, half)
         parts.append(_raster(occ, b))
     return np.concatenate(parts)

@@ -6,31 +6,37 @@
 // CLAUDE.md "Key facts").  An implicit gather-GEMM: no scatter, no atomics,
 // no [N, 27, Cin] buffer.
 //
-// One CTA computes a 128-row x BN-column output tile (BN = Cout split into
-// blocks of at most 256 columns) as one fp32 accumulator in tensor memory,
-// summing over every (offset k, 64-channel chunk j) step the tile needs:
+// Persistent kernel, one CTA per SM.  A work unit is a 128-row output tile x
+// BN output columns (Cout split into blocks of at most 256 columns); its fp32
+// accumulator lives in tensor memory and sums over every step (offset k,
+// channel chunk j) the tile needs.  A chunk is 64, 32 or 16 channels (rows of
+// 128, 64 or 32 bytes in the matching shared-memory swizzle), the widest that
+// divides Cin.  Roles (14 warps):
 //
-//   warps 0-3  gather: for step (k, j) copy 128 B of row nbr[r][k] of x (chunk j)
-//              into the A stage with cp.async, 16-byte pieces placed at their
-//              128-byte-swizzle positions; zero-fill where nbr = -1.  Lanes
-//              0-7 of a warp cover one 128-byte row segment, so every request
-//              is a full, aligned 128-byte line.  They then run the epilogue.
-//   warp 4     TMEM allocation; lane 0 issues tcgen05.mma (M=128, N=BN, K=16)
-//              and commits each stage back to the producers.
-//   warp 5     lane 0 loads the weight slice Wf[n0:n0+BN, k, 64j:64j+64] with a
-//              3-D TMA tiled load (128-byte swizzle), completing on the stage's
-//              mbarrier.
-//   epilogue   tcgen05.ld 32 columns at a time, optional exact-erf GELU,
-//              round to bf16 (RNE), 16-byte stores.
+//   warps 4-11 (gather)  256 threads fetch the A operand: for step (k, j) the
+//       128 rows x[nbr[r][k]][chunk j] are loaded with 16-byte read-only loads
+//       into registers, 4 steps ahead, then stored into the stage at their
+//       swizzled positions (zeros where nbr = -1).  Eight lanes cover one
+//       row segment, so every request is a whole aligned row segment.  A
+//       plain register pipeline keeps ~64 KB of gathers in flight per SM,
+//       which measured far above cp.async or TMA gather4 for these scattered
+//       128-byte rows.
+//   warp 13 (TMA)        bulk-copies each unit's nbr rows [128 x 27] into one
+//       of two shared buffers ahead of use, and loads the weight slice
+//       Wf[n0:n0+BN, k, chunk j] of every step with a 3-D TMA tiled load.
+//   warp 12 (MMA)        TMEM allocation; lane 0 issues tcgen05.mma (M=128,
+//       N=BN, K=16) into one of two accumulators and commits each stage back
+//       to the producers.
+//   warps 0-3 (epilogue) drain the other accumulator: tcgen05.ld, optional
+//       exact-erf GELU, bf16 round-to-nearest-even, 16-byte stores.
 //
-// Offsets with no neighbour in the whole tile (bit clear in the tile's mask
+// Offsets with no neighbour anywhere in the tile (bit clear in the tile's mask
 // word) are skipped.  Every wait is bounded (ptx.cuh); a wait that runs out
-// sets the library's device error word, the CTA drains its copies, frees its
-// tensor memory and exits.
+// sets the library's device error word, the CTA lets its copies land, frees
+// its tensor memory and exits.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
-#include <cudaTypedefs.h>
 
 #include <mutex>
 
@@ -40,41 +46,92 @@
 namespace subm3d {
 namespace {
 
-constexpr int BM = 128;                      // output rows per tile (= TMEM lanes)
-constexpr int KC = 64;                       // channels per stage: one 128-byte row
-constexpr int A_STAGE_BYTES = BM * 128;      // 16 KB
-constexpr int NUM_THREADS = 192;
-constexpr int MMA_WARP = 4;
-constexpr int TMA_WARP = 5;
+constexpr int BM = 128;  // output rows per tile (= TMEM lanes)
+constexpr int NUM_EPI_WARPS = 4;
+constexpr int NUM_GATHER_WARPS = 8;
+constexpr int GATHER_WARP0 = 4;
+constexpr int MMA_WARP = 12;
+constexpr int TMA_WARP = 13;
+constexpr int NUM_THREADS = 14 * 32;
+constexpr int GATHER_THREADS = NUM_GATHER_WARPS * 32;
+constexpr int kDepth = 4;  // gather steps in flight per thread
 constexpr int kSmemLimit = 227 * 1024;
+constexpr int kNbrTileBytes = BM * kKvol * 4;  // 13824
+constexpr uint32_t kCentreBit = 1u << 13;
 
 struct FwdArgs {
   const int32_t* nbr;
   const uint32_t* tile_mask;
-  int64_t n;
   const __nv_bfloat16* x;
+  int64_t n;
   __nv_bfloat16* out;
-  int32_t cin, cout, bn, n_kchunks, stages, flip, act;
+  int32_t cin, cout, bn, n_cblocks, n_kchunks, stages, flip, act;
+  int64_t n_tiles;
   uint32_t tmem_cols;
   int32_t* err_word;
 };
 
 struct SmemPlan {
-  int stages;
   size_t a_off, b_off, nbr_off, bar_off, bytes;
 };
 
-__host__ __device__ inline SmemPlan plan_smem(int bn, int stages) {
+__host__ __device__ inline SmemPlan plan_smem(int bn, int chunk, int stages) {
   SmemPlan p;
-  p.stages = stages;
+  const size_t a_bytes = static_cast<size_t>(BM) * chunk * 2;
+  const size_t b_bytes = static_cast<size_t>(bn) * chunk * 2;
   p.a_off = 0;
-  p.b_off = p.a_off + static_cast<size_t>(stages) * A_STAGE_BYTES;
-  p.nbr_off = p.b_off + static_cast<size_t>(stages) * bn * 128;
-  p.bar_off = p.nbr_off + BM * kKvol * 4;
-  // full[stages], empty[stages], acc, then tmem slot + abort word
-  p.bytes = p.bar_off + (2 * stages + 1) * 8 + 16 + 1024;  // + alignment slack
+  p.b_off = p.a_off + stages * a_bytes;
+  p.nbr_off = p.b_off + stages * b_bytes;
+  p.bar_off = p.nbr_off + 2 * kNbrTileBytes;
+  // full[S], empty[S], nbr_full[2], nbr_empty[2], acc_full[2], acc_empty[2], tmem slot, abort
+  p.bytes = p.bar_off + (2 * stages + 8) * 8 + 16 + 1024;  // + base alignment slack
   return p;
 }
+
+// The sequence of (unit, offset k, chunk j) steps a CTA runs; every role walks
+// the same sequence.  The centre offset is always included, so every unit has
+// at least one step.
+struct Steps {
+  int64_t u;      // current unit
+  int64_t n_units;
+  int local;      // index of the unit within this CTA (buffer / parity selector)
+  uint32_t rest;  // offsets of the unit still to come
+  int k, j;       // current offset and chunk
+  int it;         // global step counter
+  bool valid;
+
+  __device__ void load_unit(const FwdArgs& a) {
+    const int64_t tile = u / a.n_cblocks;
+    uint32_t m = (a.tile_mask ? __ldg(a.tile_mask + tile) : 0x7FFFFFFu) | kCentreBit;
+    k = __ffs(m) - 1;
+    rest = m & (m - 1);
+    j = 0;
+  }
+  __device__ void begin(const FwdArgs& a) {
+    n_units = a.n_tiles * a.n_cblocks;
+    u = blockIdx.x;
+    local = 0;
+    it = 0;
+    valid = u < n_units;
+    if (valid) load_unit(a);
+  }
+  // Advances one step; returns true when the step moved to a new unit (or ended).
+  __device__ bool next(const FwdArgs& a) {
+    ++it;
+    if (++j < a.n_kchunks) return false;
+    j = 0;
+    if (rest) {
+      k = __ffs(rest) - 1;
+      rest &= rest - 1;
+      return false;
+    }
+    u += gridDim.x;
+    ++local;
+    valid = u < n_units;
+    if (valid) load_unit(a);
+    return true;
+  }
+};
 
 __device__ __forceinline__ float gelu_erf(float v) {
   return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f));
@@ -85,51 +142,47 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// Waits until at most `lag` of this thread's cp.async groups are pending.
-__device__ __forceinline__ void cp_async_wait_dyn(int lag) {
-  switch (lag) {
-    case 0: cp_async_wait<0>(); break;
-    case 1: cp_async_wait<1>(); break;
-    case 2: cp_async_wait<2>(); break;
-    case 3: cp_async_wait<3>(); break;
-    case 4: cp_async_wait<4>(); break;
-    case 5: cp_async_wait<5>(); break;
-    case 6: cp_async_wait<6>(); break;
-    default: cp_async_wait<7>(); break;
-  }
-}
-
+template <int CHUNK>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     subm3d_fwd_bf16_sm100(const __grid_constant__ CUtensorMap wmap, const FwdArgs a) {
+  constexpr int ROW_BYTES = CHUNK * 2;              // 128, 64 or 32
+  constexpr int PPR = CHUNK / 8;                    // 16-byte pieces per row segment
+  constexpr int ROWS_PER_PASS = GATHER_THREADS / PPR;
+  constexpr int PPT = BM / ROWS_PER_PASS;           // pieces per gather thread per step
+  constexpr uint32_t A_STAGE = BM * ROW_BYTES;
+
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  const SmemPlan plan = plan_smem(a.bn, a.stages);
   const int S = a.stages;
+  const SmemPlan plan = plan_smem(a.bn, CHUNK, S);
+  const uint32_t b_stage = static_cast<uint32_t>(a.bn) * ROW_BYTES;
   uint8_t* stage_a = base + plan.a_off;
   uint8_t* stage_b = base + plan.b_off;
   int32_t* nbr_s = reinterpret_cast<int32_t*>(base + plan.nbr_off);
   uint64_t* full = reinterpret_cast<uint64_t*>(base + plan.bar_off);
   uint64_t* empty = full + S;
-  uint64_t* accbar = empty + S;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accbar + 1);
+  uint64_t* nbr_full = empty + S;
+  uint64_t* nbr_empty = nbr_full + 2;
+  uint64_t* acc_full = nbr_empty + 2;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int64_t tile = blockIdx.x;
-  const int64_t row0 = tile * BM;
-  const int n0 = blockIdx.y * a.bn;
-  const uint32_t mask = a.tile_mask ? __ldg(a.tile_mask + tile) : 0x7FFFFFFu;
-  const int n_iters = __popc(mask) * a.n_kchunks;
-  const uint32_t b_stage_bytes = static_cast<uint32_t>(a.bn) * 128u;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 128 + 1);  // 128 gather threads + the TMA thread's expect_tx
-      mbar_init(&empty[s], 1);       // one tcgen05.commit
+      mbar_init(&full[s], NUM_GATHER_WARPS + 1);  // one arrive per gather warp + TMA expect_tx
+      mbar_init(&empty[s], 1);                    // one tcgen05.commit
     }
-    mbar_init(accbar, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&nbr_full[b], 1);
+      mbar_init(&nbr_empty[b], NUM_GATHER_WARPS);
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], NUM_EPI_WARPS * 32);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -138,76 +191,193 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tmem_relinquish();
   }
   if (warp == TMA_WARP && lane == 0) tma_prefetch_desc(&wmap);
-  for (int e = threadIdx.x; e < BM * kKvol; e += NUM_THREADS) {
-    const int64_t r = row0 + e / kKvol;
-    nbr_s[e] = (r < a.n) ? __ldg(a.nbr + row0 * kKvol + e) : -1;
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp < 4) {
+  if (warp >= GATHER_WARP0 && warp < GATHER_WARP0 + NUM_GATHER_WARPS) {
     // ---------------------------------------------------------- gather ----
-    const int lag = S - 1 < 7 ? S - 1 : 7;
-    const int sub = lane >> 3;    // which of 4 rows this lane serves per pass
-    const int piece = lane & 7;   // which 16-byte piece of the 128-byte segment
-    uint32_t m = mask;
-    int it = 0;
+    const int gt = threadIdx.x - GATHER_WARP0 * 32;
+    const int piece = gt % PPR;
+    const int rbase = gt / PPR;
+    Steps ld, st;
+    ld.begin(a);
+    st.begin(a);
+    int ready_local = -1;
     bool ok = true;
-    while (m && ok) {
-      const int k = __ffs(m) - 1;
-      m &= m - 1;
-      for (int j = 0; j < a.n_kchunks; ++j, ++it) {
-        const int s = it % S;
-        if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1, abort_flag)) {
+    uint4 v[kDepth][PPT];
+
+    // Issue the loads of step `ld` into vd; returns false on a timed-out wait.
+    auto issue = [&](uint4 (&vd)[PPT]) -> bool {
+      if (ld.local != ready_local) {
+        if (!__all_sync(0xFFFFFFFFu,
+                        mbar_wait(&nbr_full[ld.local & 1], (ld.local >> 1) & 1, abort_flag)))
+          return false;
+        ready_local = ld.local;
+      }
+      const int32_t* nb = nbr_s + (ld.local & 1) * (BM * kKvol);
+      const int col = ld.j * CHUNK + piece * 8;
+#pragma unroll
+      for (int q = 0; q < PPT; ++q) {
+        const int r = rbase + q * ROWS_PER_PASS;
+        const int32_t src = nb[r * kKvol + ld.k];
+        if (src >= 0) {
+          vd[q] = ldg_nc_16(a.x + static_cast<int64_t>(src) * a.cin + col);
+        } else {
+          vd[q] = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      const int old_local = ld.local;
+      if (ld.next(a)) {  // the unit's last loads are issued: release its nbr buffer
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&nbr_empty[old_local & 1]);
+      }
+      return true;
+    };
+
+#pragma unroll
+    for (int d = 0; d < kDepth; ++d)
+      if (ok && ld.valid) ok = issue(v[d]);
+    while (ok && st.valid) {
+#pragma unroll
+      for (int d = 0; d < kDepth; ++d) {
+        if (!ok || !st.valid) break;
+        const int s = st.it % S;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[s], ((st.it / S) & 1) ^ 1, abort_flag))) {
           ok = false;
           break;
         }
-        const uint32_t a_base = smem_u32(stage_a + static_cast<size_t>(s) * A_STAGE_BYTES);
-        const int ch = j * KC + piece * 8;  // first channel of this piece
-        const bool piece_live = ch < a.cin;
+        const uint32_t a_base = smem_u32(stage_a) + static_cast<uint32_t>(s) * A_STAGE;
 #pragma unroll
-        for (int rr = 0; rr < 8; ++rr) {
-          const int r = warp * 32 + rr * 4 + sub;
-          const int32_t src = nbr_s[r * kKvol + k];
-          const bool live = piece_live && src >= 0;
-          const __nv_bfloat16* gp = live ? a.x + static_cast<int64_t>(src) * a.cin + ch : a.x;
-          const uint32_t dst = a_base + r * 128 + ((piece ^ (r & 7)) << 4);
-          if (piece_live) cp_async_16(dst, gp, live ? 16u : 0u);
+        for (int q = 0; q < PPT; ++q) {
+          const int r = rbase + q * ROWS_PER_PASS;
+          const int phys = piece ^ ((r * ROW_BYTES >> 7) & (PPR - 1));
+          sts_16(a_base + r * ROW_BYTES + (phys << 4), v[d][q]);
         }
-        cp_async_commit();
-        if (it >= lag) {
-          cp_async_wait_dyn(lag);
-          fence_proxy_async_smem();
-          mbar_arrive(&full[(it - lag) % S]);
-        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full[s]);
+        st.next(a);
+        if (ld.valid) ok = issue(v[d]);
       }
     }
-    cp_async_wait_all();
-    fence_proxy_async_smem();
-    if (ok) {
-      for (int t = (it - lag > 0 ? it - lag : 0); t < it; ++t) mbar_arrive(&full[t % S]);
+  } else if (warp == TMA_WARP) {
+    // ------------------------------------------------------------- TMA ----
+    const int64_t n_units = a.n_tiles * a.n_cblocks;
+    // Stage the nbr rows of the unit with local index l into buffer l & 1.
+    auto load_nbr = [&](int64_t u, int l) -> bool {
+      const int buf = l & 1;
+      if (!__all_sync(0xFFFFFFFFu,
+                      mbar_wait(&nbr_empty[buf], ((l >> 1) & 1) ^ 1, abort_flag)))
+        return false;
+      const int64_t row0 = (u / a.n_cblocks) * BM;
+      int32_t* dst = nbr_s + buf * (BM * kKvol);
+      if (row0 + BM <= a.n) {
+        if (lane == 0) {
+          fence_proxy_async_smem();  // earlier generic reads of this buffer come first
+          mbar_arrive_expect_tx(&nbr_full[buf], kNbrTileBytes);
+          bulk_load(smem_u32(dst), a.nbr + row0 * kKvol, kNbrTileBytes, &nbr_full[buf]);
+        }
+      } else {
+        const int rows = static_cast<int>(a.n - row0);
+        for (int e = lane; e < BM * kKvol; e += 32)
+          dst[e] = (e / kKvol < rows) ? __ldg(a.nbr + row0 * kKvol + e) : -1;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&nbr_full[buf]);
+      }
+      return true;
+    };
+    bool ok = true;
+    if (blockIdx.x < n_units) ok = load_nbr(blockIdx.x, 0);
+    Steps st;
+    st.begin(a);
+    int unit_local = -1;
+    while (ok && st.valid) {
+      if (st.local != unit_local) {  // entering a unit: prefetch the next unit's nbr rows
+        unit_local = st.local;
+        const int64_t nu = st.u + gridDim.x;
+        if (nu < n_units && !load_nbr(nu, st.local + 1)) {
+          ok = false;
+          break;
+        }
+      }
+      const int s = st.it % S;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[s], ((st.it / S) & 1) ^ 1, abort_flag))) {
+        ok = false;
+        break;
+      }
+      if (lane == 0) {
+        const int kw = a.flip ? (kKvol - 1 - st.k) : st.k;
+        const int n0 = static_cast<int>(st.u % a.n_cblocks) * a.bn;
+        mbar_arrive_expect_tx(&full[s], b_stage);
+        tma_load_3d(smem_u32(stage_b) + static_cast<uint32_t>(s) * b_stage, &wmap, &full[s],
+                    st.j * CHUNK, kw, n0);
+      }
+      __syncwarp();
+      st.next(a);
     }
-
-    // -------------------------------------------------------- epilogue ----
-    // tcgen05.ld is warp-collective: take the epilogue only if the whole warp can.
-    bool go = ok && n_iters > 0 && mbar_wait(accbar, 0, abort_flag);
-    go = __all_sync(0xFFFFFFFFu, go);
-    if (go) {
+    if (!ok) __nanosleep(20000);  // let TMA copies already issued land before exit
+  } else if (warp == MMA_WARP) {
+    // -------------------------------------------------------------- MMA ----
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(BM, static_cast<uint32_t>(a.bn));
+      Steps st;
+      st.begin(a);
+      bool ok = true;
+      while (ok && st.valid) {
+        const int local = st.local;
+        const int acc = local & 1;
+        if (!mbar_wait(&acc_empty[acc], ((local >> 1) & 1) ^ 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * a.bn);
+        bool first = true;
+        bool unit_done = false;
+        while (!unit_done) {
+          const int s = st.it % S;
+          if (!mbar_wait(&full[s], (st.it / S) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(stage_a) + static_cast<uint32_t>(s) * A_STAGE;
+          const uint32_t b0 = smem_u32(stage_b) + static_cast<uint32_t>(s) * b_stage;
+#pragma unroll
+          for (int kk = 0; kk < CHUNK / 16; ++kk) {
+            umma_bf16(d, smem_desc_sw(a0 + kk * 32, ROW_BYTES), smem_desc_sw(b0 + kk * 32, ROW_BYTES),
+                      idesc, (first && kk == 0) ? 0u : 1u);
+          }
+          first = false;
+          umma_commit(&empty[s]);
+          unit_done = st.next(a);
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[acc]);
+      }
+      if (!ok) __nanosleep(20000);  // let MMAs already issued finish before TMEM is freed
+    }
+  } else {
+    // --------------------------------------------------------- epilogue ----
+    const int64_t n_units = a.n_tiles * a.n_cblocks;
+    int local = 0;
+    for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x, ++local) {
+      const int acc = local & 1;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&acc_full[acc], (local >> 1) & 1, abort_flag))) break;
       tc_fence_after();
-      const int r = warp * 32 + lane;
-      const int64_t row = row0 + r;
-      const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+      const int64_t tile = u / a.n_cblocks;
+      const int n0 = static_cast<int>(u % a.n_cblocks) * a.bn;
+      const int64_t row = tile * BM + warp * 32 + lane;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) +
+                             static_cast<uint32_t>(acc * a.bn);
       __nv_bfloat16* orow = a.out + row * a.cout + n0;
       for (int c0 = 0; c0 < a.bn; c0 += 32) {
         const int width = a.bn - c0 >= 32 ? 32 : 16;
         uint32_t v[32];
         if (width == 32) {
-          tmem_ld_32x32b_x32(lane_addr + c0, v);
+          tmem_ld_32x32b_x32(taddr + c0, v);
         } else {
           uint32_t h[16];
-          tmem_ld_32x32b_x16(lane_addr + c0, h);
+          tmem_ld_32x32b_x16(taddr + c0, h);
 #pragma unroll
           for (int q = 0; q < 16; ++q) v[q] = h[q];
         }
@@ -219,8 +389,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             float f[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              const float acc = __uint_as_float(v[q * 8 + e]);
-              f[e] = a.act ? gelu_erf(acc) : acc;
+              const float accv = __uint_as_float(v[q * 8 + e]);
+              f[e] = a.act ? gelu_erf(accv) : accv;
             }
             uint4 pk;
             pk.x = pack_bf16x2(f[0], f[1]);
@@ -231,68 +401,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
-    } else if (n_iters == 0 && row0 + warp * 32 + lane < a.n) {
-      // A tile with no neighbours at all cannot occur for a valid map (every
-      // voxel is its own centre neighbour); write act(0) = 0 for safety.
-      __nv_bfloat16* orow = a.out + (row0 + warp * 32 + lane) * a.cout + n0;
-      for (int c = 0; c < a.bn && n0 + c < a.cout; ++c) orow[c] = __float2bfloat16_rn(0.f);
-    }
-  } else if (warp == MMA_WARP) {
-    // ------------------------------------------------------------- MMA ----
-    if (lane == 0 && n_iters > 0) {
-      const uint32_t idesc = idesc_bf16_f32(BM, static_cast<uint32_t>(a.bn));
-      uint32_t m = mask;
-      int it = 0;
-      bool ok = true;
-      while (m && ok) {
-        m &= m - 1;
-        for (int j = 0; j < a.n_kchunks; ++j, ++it) {
-          const int s = it % S;
-          if (!mbar_wait(&full[s], (it / S) & 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const int ksteps = (a.cin - j * KC >= KC ? KC : a.cin - j * KC) / 16;
-          const uint32_t a0 = smem_u32(stage_a + static_cast<size_t>(s) * A_STAGE_BYTES);
-          const uint32_t b0 = smem_u32(stage_b + static_cast<size_t>(s) * b_stage_bytes);
-          for (int kk = 0; kk < ksteps; ++kk) {
-            umma_bf16(tmem_base, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32),
-                      idesc, (it | kk) != 0 ? 1u : 0u);
-          }
-          umma_commit(&empty[s]);
-        }
-      }
-      // Always commit the accumulator barrier, so that the tensor memory is
-      // only released after every issued MMA has completed.
-      umma_commit(accbar);
-      if (!ok) {
-        volatile int no_abort = 0;
-        mbar_wait(accbar, 0, &no_abort);
-      }
-    }
-  } else {
-    // ------------------------------------------------------------- TMA ----
-    if (lane == 0 && n_iters > 0) {
-      uint32_t m = mask;
-      int it = 0;
-      bool ok = true;
-      while (m && ok) {
-        const int k = __ffs(m) - 1;
-        m &= m - 1;
-        const int kw = a.flip ? (kKvol - 1 - k) : k;
-        for (int j = 0; j < a.n_kchunks; ++j, ++it) {
-          const int s = it % S;
-          if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&full[s], b_stage_bytes);
-          tma_load_3d(smem_u32(stage_b + static_cast<size_t>(s) * b_stage_bytes), &wmap, &full[s],
-                      j * KC, kw, n0);
-        }
-      }
-      if (!ok) __nanosleep(20000);  // let TMA loads already issued land before exit
+      tc_fence_before();
+      mbar_arrive(&acc_empty[acc]);
     }
   }
 
@@ -324,17 +434,28 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Per-device one-time setup: opt in to the large dynamic shared memory size.
-cudaError_t ensure_attrs(int device) {
+// Per-device one-time setup: large dynamic shared memory opt-in and SM count.
+cudaError_t device_setup(int device, int* num_sms) {
   static std::mutex mu;
-  static bool done[64] = {};
+  static int sms[64] = {};
   if (device < 0 || device >= 64) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(mu);
-  if (done[device]) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(subm3d_fwd_bf16_sm100,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
-  if (e == cudaSuccess) done[device] = true;
-  return e;
+  if (sms[device] == 0) {
+    const void* kernels[3] = {reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<64>),
+                              reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<32>),
+                              reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<16>)};
+    for (const void* k : kernels) {
+      const cudaError_t e =
+          cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+      if (e != cudaSuccess) return e;
+    }
+    int count = 0;
+    const cudaError_t e = cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, device);
+    if (e != cudaSuccess) return e;
+    sms[device] = count;
+  }
+  *num_sms = sms[device];
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -348,47 +469,60 @@ cudaError_t launch_forward_bf16(const int32_t* nbr, const uint32_t* tile_mask, i
   int device = 0;
   cudaError_t e = cudaGetDevice(&device);
   if (e != cudaSuccess) return e;
-  if ((e = ensure_attrs(device)) != cudaSuccess) return e;
+  int num_sms = 0;
+  if ((e = device_setup(device, &num_sms)) != cudaSuccess) return e;
 
-  // Split Cout into n_blocks column blocks of equal width (a multiple of 16, <= 256).
-  const int n_blocks = (cout + 255) / 256;
-  int bn = (cout + n_blocks - 1) / n_blocks;
+  // Cout in n_cblocks column blocks of equal width (a multiple of 16, <= 256).
+  const int n_cblocks = (cout + 255) / 256;
+  int bn = (cout + n_cblocks - 1) / n_cblocks;
   bn = (bn + 15) / 16 * 16;
   uint32_t tmem_cols = 32;
-  while (tmem_cols < static_cast<uint32_t>(bn)) tmem_cols <<= 1;
+  while (tmem_cols < static_cast<uint32_t>(2 * bn)) tmem_cols <<= 1;
+  const int chunk = cin % 64 == 0 ? 64 : (cin % 32 == 0 ? 32 : 16);
   int stages = 8;
-  while (stages > 2 && plan_smem(bn, stages).bytes > static_cast<size_t>(kSmemLimit)) --stages;
-  const SmemPlan plan = plan_smem(bn, stages);
+  while (stages > 2 && plan_smem(bn, chunk, stages).bytes > static_cast<size_t>(kSmemLimit))
+    --stages;
+  const SmemPlan plan = plan_smem(bn, chunk, stages);
 
-  CUtensorMap map;
+  CUtensorMap wmap;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(cin), 27, static_cast<cuuint64_t>(cout)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(cin) * 2,
                                  static_cast<cuuint64_t>(cin) * 27 * 2};
-  const cuuint32_t box[3] = {KC, 1, static_cast<cuuint32_t>(bn)};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(chunk), 1, static_cast<cuuint32_t>(bn)};
   const cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(weight), dims,
-                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  const CUtensorMapSwizzle swz =
+      chunk == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                  : (chunk == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+  if (encode(&wmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(weight), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
 
   FwdArgs a;
   a.nbr = nbr;
   a.tile_mask = tile_mask;
-  a.n = n;
   a.x = static_cast<const __nv_bfloat16*>(feats);
+  a.n = n;
   a.out = static_cast<__nv_bfloat16*>(out);
   a.cin = cin;
   a.cout = cout;
   a.bn = bn;
-  a.n_kchunks = (cin + KC - 1) / KC;
+  a.n_cblocks = n_cblocks;
+  a.n_kchunks = cin / chunk;
   a.stages = stages;
   a.flip = flip;
   a.act = act;
+  a.n_tiles = (n + BM - 1) / BM;
   a.tmem_cols = tmem_cols;
   a.err_word = err_word;
-  const dim3 grid(static_cast<unsigned>((n + BM - 1) / BM), static_cast<unsigned>(n_blocks));
-  subm3d_fwd_bf16_sm100<<<grid, NUM_THREADS, plan.bytes, stream>>>(map, a);
+  const int64_t units = a.n_tiles * n_cblocks;
+  const unsigned grid = static_cast<unsigned>(units < num_sms ? units : num_sms);
+  if (chunk == 64)
+    subm3d_fwd_bf16_sm100<64><<<grid, NUM_THREADS, plan.bytes, stream>>>(wmap, a);
+  else if (chunk == 32)
+    subm3d_fwd_bf16_sm100<32><<<grid, NUM_THREADS, plan.bytes, stream>>>(wmap, a);
+  else
+    subm3d_fwd_bf16_sm100<16><<<grid, NUM_THREADS, plan.bytes, stream>>>(wmap, a);
   return cudaGetLastError();
 }
 

@@ -160,6 +160,7 @@ __global__ void __launch_bounds__(kQueryThreads)
   const int local = threadIdx.x / kKvol;
   const int k = threadIdx.x - local * kKvol;
   const int64_t i = static_cast<int64_t>(blockIdx.x) * kQueryVoxels + local;
+  uint32_t bits = 0u;
   if (i < n) {
     int32_t found = -1;
     if (k == 13) {
@@ -200,8 +201,11 @@ __global__ void __launch_bounds__(kQueryThreads)
       }
     }
     nbr[static_cast<int64_t>(blockIdx.x) * kQueryThreads + threadIdx.x] = found;
-    if (found >= 0) atomicOr(&s_mask, 1u << k);
+    bits = found >= 0 ? (1u << k) : 0u;
   }
+  // one shared atomic per warp instead of one per thread
+  bits = __reduce_or_sync(0xFFFFFFFFu, bits);
+  if ((threadIdx.x & 31) == 0 && bits != 0u) atomicOr(&s_mask, bits);
   __syncthreads();
   if (threadIdx.x == 0 && s_mask != 0u) {
     atomicOr(tile_mask + (static_cast<int64_t>(blockIdx.x) * kQueryVoxels) / kTileRows, s_mask);

@@ -79,9 +79,11 @@ SUBM3D_API const char* subm3d_status_string(int32_t status);
 /*
  * Workspace bytes subm3d_build_map() needs for N voxels in a batch x
  * grid_dim^3 volume: a status word, one 32-bit offset mask per 128-row tile,
- * and an open-addressing hash table of at least 2N slots.  Host-only, no CUDA
- * call.  Returns 0 for arguments subm3d_build_map() would reject
- * (N < 0, grid_dim < 1 or > 65535, batch < 1 or > 65535).
+ * and the lookup table -- a direct-address table of batch * grid_dim^3 int32
+ * cells when that is at most 64 MB, else an open-addressing hash table of at
+ * least 2N slots (8 bytes each, 12 with batch > 4 or grid_dim > 1024).
+ * Host-only, no CUDA call.  Returns 0 for arguments subm3d_build_map() would
+ * reject (N < 0, grid_dim < 1 or > 65535, batch < 1 or > 65535).
  */
 SUBM3D_API size_t subm3d_map_workspace_bytes(int64_t n, int32_t grid_dim, int32_t batch);
 
@@ -106,9 +108,11 @@ SUBM3D_API size_t subm3d_map_workspace_bytes(int64_t n, int32_t grid_dim, int32_
  * does not depend on the hash layout.  Coordinates outside the volume or
  * repeated are reported by subm3d_map_status(); until it returns SUBM3D_OK the
  * contents of nbr are unspecified.  Enqueues 3 kernels; no allocation.
- * Testing knob: the environment variable SUBM3D_TABLE_CAPACITY, when set,
- * caps the hash table at that many slots so that SUBM3D_E_TABLE_FULL can be
- * exercised; probe loops stop after `capacity` steps instead of spinning.
+ * Testing knobs, read from the environment by this function and by
+ * subm3d_map_workspace_bytes() alike: SUBM3D_MAP_KIND=hash selects the hash
+ * table even where the direct table fits; SUBM3D_TABLE_CAPACITY=<slots> caps
+ * the hash table (and selects it) so that SUBM3D_E_TABLE_FULL can be
+ * exercised -- probe loops stop after `capacity` steps instead of spinning.
  */
 SUBM3D_API subm3d_status subm3d_build_map(const int32_t* coords, int64_t n, int32_t grid_dim,
                                int32_t batch, int32_t* nbr, void* workspace,

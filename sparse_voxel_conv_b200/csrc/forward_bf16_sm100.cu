@@ -6,34 +6,44 @@
 // CLAUDE.md "Key facts").  An implicit gather-GEMM: no scatter, no atomics,
 // no [N, 27, Cin] buffer.
 //
-// Persistent kernel, one CTA per SM.  A work unit is a 128-row output tile x
-// BN output columns (Cout split into blocks of at most 256 columns); its fp32
-// accumulator lives in tensor memory and sums over every step (offset k,
-// channel chunk j) the tile needs.  A chunk is 64, 32 or 16 channels (rows of
-// 128, 64 or 32 bytes in the matching shared-memory swizzle), the widest that
-// divides Cin.  Roles (14 warps):
+// Orientation of the contraction.  A tcgen05.mma with M = 128 costs the same
+// number of cycles for any N up to 256, so it reaches the tensor-core peak
+// only at N = 256.  The layer widths here are 64-128 channels, so the output
+// channels are the M side and a tile of 256 voxels is the N side:
 //
-//   warps 4-11 (gather)  256 threads fetch the A operand: for step (k, j) the
-//       128 rows x[nbr[r][k]][chunk j] are loaded with 16-byte read-only loads
-//       into registers, 4 steps ahead, then stored into the stage at their
+//     D[o, v] += sum_c Wf[o, k, c] * x[nbr[v][k], c]      (D in tensor memory)
+//
+// with A = the weight slice (128 output channels x a channel chunk, loaded by
+// TMA) and B = the gathered input rows (256 voxels x the chunk).  Both are
+// K-major in the 128/64/32-byte swizzle layout matching the chunk of 64/32/16
+// channels (the widest that divides Cin).
+//
+// Persistent kernel, one CTA per SM.  A work unit is a 256-voxel tile x a
+// block of 128 output channels; its fp32 accumulator (128 lanes x 256 columns)
+// sums over every step (offset k, chunk j) the tile needs.  Roles (14 warps):
+//
+//   warps 4-11 (gather)  256 threads fetch B: for step (k, j) the 256 rows
+//       x[nbr[v][k]][chunk j] are loaded with 16-byte read-only loads into
+//       registers, 2-4 steps ahead, then stored into the stage at their
 //       swizzled positions (zeros where nbr = -1).  Eight lanes cover one
-//       row segment, so every request is a whole aligned row segment.  A
-//       plain register pipeline keeps ~64 KB of gathers in flight per SM,
-//       which measured far above cp.async or TMA gather4 for these scattered
-//       128-byte rows.
-//   warp 13 (TMA)        bulk-copies each unit's nbr rows [128 x 27] into one
+//       128-byte row segment, so every request is a whole aligned segment.
+//       This plain register pipeline measured far above cp.async or TMA
+//       gather4 for these scattered rows.
+//   warp 13 (TMA)        bulk-copies each unit's nbr rows [256 x 27] into one
 //       of two shared buffers ahead of use, and loads the weight slice
-//       Wf[n0:n0+BN, k, chunk j] of every step with a 3-D TMA tiled load.
-//   warp 12 (MMA)        TMEM allocation; lane 0 issues tcgen05.mma (M=128,
-//       N=BN, K=16) into one of two accumulators and commits each stage back
-//       to the producers.
-//   warps 0-3 (epilogue) drain the other accumulator: tcgen05.ld, optional
-//       exact-erf GELU, bf16 round-to-nearest-even, 16-byte stores.
+//       Wf[o0:o0+128, k, chunk j] of every step with a 3-D TMA tiled load
+//       (rows past Cout read as zero).
+//   warp 12 (MMA)        TMEM allocation (512 columns: two accumulators); lane 0
+//       issues tcgen05.mma (M=128, N=256, K=16) and commits each stage back.
+//   warps 0-3 (epilogue) drain the other accumulator: warp w holds channels
+//       32w..32w+31; tcgen05.ld 32 voxels at a time, optional exact-erf GELU,
+//       bf16 round-to-nearest-even, a transpose through shared memory, and
+//       16-byte stores of whole 64-byte channel runs of each voxel's row.
 //
-// Offsets with no neighbour anywhere in the tile (bit clear in the tile's mask
-// word) are skipped.  Every wait is bounded (ptx.cuh); a wait that runs out
-// sets the library's device error word, the CTA lets its copies land, frees
-// its tensor memory and exits.
+// Offsets with no neighbour anywhere in the tile (bit clear in both 128-row
+// mask words) are skipped.  Every wait is bounded (ptx.cuh); a wait that runs
+// out sets the library's device error word, the CTA lets its copies land,
+// frees its tensor memory and exits.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -46,7 +56,8 @@
 namespace subm3d {
 namespace {
 
-constexpr int BM = 128;  // output rows per tile (= TMEM lanes)
+constexpr int TV = 256;  // voxels per tile (MMA N)
+constexpr int TO = 128;  // output channels per unit (MMA M, TMEM lanes)
 constexpr int NUM_EPI_WARPS = 4;
 constexpr int NUM_GATHER_WARPS = 8;
 constexpr int GATHER_WARP0 = 4;
@@ -54,35 +65,36 @@ constexpr int MMA_WARP = 12;
 constexpr int TMA_WARP = 13;
 constexpr int NUM_THREADS = 14 * 32;
 constexpr int GATHER_THREADS = NUM_GATHER_WARPS * 32;
-constexpr int kDepth = 4;  // gather steps in flight per thread
 constexpr int kSmemLimit = 227 * 1024;
-constexpr int kNbrTileBytes = BM * kKvol * 4;  // 13824
+constexpr int kNbrTileBytes = TV * kKvol * 4;             // 27648
+constexpr int kEpiStageBytes = NUM_EPI_WARPS * 32 * 64;  // 32 voxels x 32 channels bf16 per warp
+constexpr uint32_t kTmemCols = 2 * TV;
 constexpr uint32_t kCentreBit = 1u << 13;
 
 struct FwdArgs {
   const int32_t* nbr;
-  const uint32_t* tile_mask;
+  const uint32_t* tile_mask;  // one word per 128 rows
   const __nv_bfloat16* x;
   int64_t n;
   __nv_bfloat16* out;
-  int32_t cin, cout, bn, n_cblocks, n_kchunks, stages, flip, act;
+  int32_t cin, cout, n_oblocks, n_kchunks, stages, flip, act;
   int64_t n_tiles;
-  uint32_t tmem_cols;
   int32_t* err_word;
 };
 
 struct SmemPlan {
-  size_t a_off, b_off, nbr_off, bar_off, bytes;
+  size_t a_off, b_off, nbr_off, epi_off, bar_off, bytes;
 };
 
-__host__ __device__ inline SmemPlan plan_smem(int bn, int chunk, int stages) {
+__host__ __device__ inline SmemPlan plan_smem(int chunk, int stages) {
   SmemPlan p;
-  const size_t a_bytes = static_cast<size_t>(BM) * chunk * 2;
-  const size_t b_bytes = static_cast<size_t>(bn) * chunk * 2;
+  const size_t a_bytes = static_cast<size_t>(TO) * chunk * 2;
+  const size_t b_bytes = static_cast<size_t>(TV) * chunk * 2;
   p.a_off = 0;
   p.b_off = p.a_off + stages * a_bytes;
   p.nbr_off = p.b_off + stages * b_bytes;
-  p.bar_off = p.nbr_off + 2 * kNbrTileBytes;
+  p.epi_off = p.nbr_off + 2 * kNbrTileBytes;
+  p.bar_off = p.epi_off + kEpiStageBytes;
   // full[S], empty[S], nbr_full[2], nbr_empty[2], acc_full[2], acc_empty[2], tmem slot, abort
   p.bytes = p.bar_off + (2 * stages + 8) * 8 + 16 + 1024;  // + base alignment slack
   return p;
@@ -101,14 +113,20 @@ struct Steps {
   bool valid;
 
   __device__ void load_unit(const FwdArgs& a) {
-    const int64_t tile = u / a.n_cblocks;
-    uint32_t m = (a.tile_mask ? __ldg(a.tile_mask + tile) : 0x7FFFFFFu) | kCentreBit;
+    const int64_t tile = u / a.n_oblocks;
+    uint32_t m = 0x7FFFFFFu;
+    if (a.tile_mask) {
+      const int64_t w = 2 * tile;
+      const int64_t n_words = (a.n + kTileRows - 1) / kTileRows;
+      m = __ldg(a.tile_mask + w) | (w + 1 < n_words ? __ldg(a.tile_mask + w + 1) : 0u);
+    }
+    m |= kCentreBit;
     k = __ffs(m) - 1;
     rest = m & (m - 1);
     j = 0;
   }
   __device__ void begin(const FwdArgs& a) {
-    n_units = a.n_tiles * a.n_cblocks;
+    n_units = a.n_tiles * a.n_oblocks;
     u = blockIdx.x;
     local = 0;
     it = 0;
@@ -137,29 +155,27 @@ __device__ __forceinline__ float gelu_erf(float v) {
   return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f));
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-
 template <int CHUNK>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     subm3d_fwd_bf16_sm100(const __grid_constant__ CUtensorMap wmap, const FwdArgs a) {
-  constexpr int ROW_BYTES = CHUNK * 2;              // 128, 64 or 32
-  constexpr int PPR = CHUNK / 8;                    // 16-byte pieces per row segment
+  constexpr int ROW_BYTES = CHUNK * 2;  // 128, 64 or 32
+  constexpr int PPR = CHUNK / 8;        // 16-byte pieces per row segment
   constexpr int ROWS_PER_PASS = GATHER_THREADS / PPR;
-  constexpr int PPT = BM / ROWS_PER_PASS;           // pieces per gather thread per step
-  constexpr uint32_t A_STAGE = BM * ROW_BYTES;
+  constexpr int PPT = TV / ROWS_PER_PASS;  // pieces per gather thread per step
+  // gather steps in flight per thread: ~64 KB of loads in flight per SM
+  constexpr int kDepth = PPT >= 8 ? 2 : (PPT >= 4 ? 3 : 4);
+  constexpr uint32_t A_STAGE = TO * ROW_BYTES;
+  constexpr uint32_t B_STAGE = TV * ROW_BYTES;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const int S = a.stages;
-  const SmemPlan plan = plan_smem(a.bn, CHUNK, S);
-  const uint32_t b_stage = static_cast<uint32_t>(a.bn) * ROW_BYTES;
+  const SmemPlan plan = plan_smem(CHUNK, S);
   uint8_t* stage_a = base + plan.a_off;
   uint8_t* stage_b = base + plan.b_off;
   int32_t* nbr_s = reinterpret_cast<int32_t*>(base + plan.nbr_off);
+  uint8_t* epi_s = base + plan.epi_off;
   uint64_t* full = reinterpret_cast<uint64_t*>(base + plan.bar_off);
   uint64_t* empty = full + S;
   uint64_t* nbr_full = empty + S;
@@ -187,7 +203,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     fence_mbar_init();
   }
   if (warp == MMA_WARP) {
-    tmem_alloc(tmem_slot, a.tmem_cols);
+    tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
   if (warp == TMA_WARP && lane == 0) tma_prefetch_desc(&wmap);
@@ -216,17 +232,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           return false;
         ready_local = ld.local;
       }
-      const int32_t* nb = nbr_s + (ld.local & 1) * (BM * kKvol);
+      const int32_t* nb = nbr_s + (ld.local & 1) * (TV * kKvol);
       const int col = ld.j * CHUNK + piece * 8;
 #pragma unroll
       for (int q = 0; q < PPT; ++q) {
         const int r = rbase + q * ROWS_PER_PASS;
         const int32_t src = nb[r * kKvol + ld.k];
-        if (src >= 0) {
-          vd[q] = ldg_nc_16(a.x + static_cast<int64_t>(src) * a.cin + col);
-        } else {
-          vd[q] = make_uint4(0u, 0u, 0u, 0u);
-        }
+        vd[q] = src >= 0 ? ldg_nc_16(a.x + static_cast<int64_t>(src) * a.cin + col)
+                         : make_uint4(0u, 0u, 0u, 0u);
       }
       const int old_local = ld.local;
       if (ld.next(a)) {  // the unit's last loads are issued: release its nbr buffer
@@ -248,12 +261,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ok = false;
           break;
         }
-        const uint32_t a_base = smem_u32(stage_a) + static_cast<uint32_t>(s) * A_STAGE;
+        const uint32_t b_base = smem_u32(stage_b) + static_cast<uint32_t>(s) * B_STAGE;
 #pragma unroll
         for (int q = 0; q < PPT; ++q) {
           const int r = rbase + q * ROWS_PER_PASS;
           const int phys = piece ^ ((r * ROW_BYTES >> 7) & (PPR - 1));
-          sts_16(a_base + r * ROW_BYTES + (phys << 4), v[d][q]);
+          sts_16(b_base + r * ROW_BYTES + (phys << 4), v[d][q]);
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -264,16 +277,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp == TMA_WARP) {
     // ------------------------------------------------------------- TMA ----
-    const int64_t n_units = a.n_tiles * a.n_cblocks;
+    const int64_t n_units = a.n_tiles * a.n_oblocks;
     // Stage the nbr rows of the unit with local index l into buffer l & 1.
     auto load_nbr = [&](int64_t u, int l) -> bool {
       const int buf = l & 1;
       if (!__all_sync(0xFFFFFFFFu,
                       mbar_wait(&nbr_empty[buf], ((l >> 1) & 1) ^ 1, abort_flag)))
         return false;
-      const int64_t row0 = (u / a.n_cblocks) * BM;
-      int32_t* dst = nbr_s + buf * (BM * kKvol);
-      if (row0 + BM <= a.n) {
+      const int64_t row0 = (u / a.n_oblocks) * TV;
+      int32_t* dst = nbr_s + buf * (TV * kKvol);
+      if (row0 + TV <= a.n) {
         if (lane == 0) {
           fence_proxy_async_smem();  // earlier generic reads of this buffer come first
           mbar_arrive_expect_tx(&nbr_full[buf], kNbrTileBytes);
@@ -281,7 +294,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       } else {
         const int rows = static_cast<int>(a.n - row0);
-        for (int e = lane; e < BM * kKvol; e += 32)
+        for (int e = lane; e < TV * kKvol; e += 32)
           dst[e] = (e / kKvol < rows) ? __ldg(a.nbr + row0 * kKvol + e) : -1;
         __syncwarp();
         if (lane == 0) mbar_arrive(&nbr_full[buf]);
@@ -309,10 +322,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (lane == 0) {
         const int kw = a.flip ? (kKvol - 1 - st.k) : st.k;
-        const int n0 = static_cast<int>(st.u % a.n_cblocks) * a.bn;
-        mbar_arrive_expect_tx(&full[s], b_stage);
-        tma_load_3d(smem_u32(stage_b) + static_cast<uint32_t>(s) * b_stage, &wmap, &full[s],
-                    st.j * CHUNK, kw, n0);
+        const int o0 = static_cast<int>(st.u % a.n_oblocks) * TO;
+        mbar_arrive_expect_tx(&full[s], A_STAGE);
+        tma_load_3d(smem_u32(stage_a) + static_cast<uint32_t>(s) * A_STAGE, &wmap, &full[s],
+                    st.j * CHUNK, kw, o0);
       }
       __syncwarp();
       st.next(a);
@@ -321,7 +334,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == MMA_WARP) {
     // -------------------------------------------------------------- MMA ----
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(BM, static_cast<uint32_t>(a.bn));
+      const uint32_t idesc = idesc_bf16_f32(TO, TV);
       Steps st;
       st.begin(a);
       bool ok = true;
@@ -330,7 +343,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int acc = local & 1;
         if (!mbar_wait(&acc_empty[acc], ((local >> 1) & 1) ^ 1, abort_flag)) break;
         tc_fence_after();
-        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * a.bn);
+        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * TV);
         bool first = true;
         bool unit_done = false;
         while (!unit_done) {
@@ -341,11 +354,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           tc_fence_after();
           const uint32_t a0 = smem_u32(stage_a) + static_cast<uint32_t>(s) * A_STAGE;
-          const uint32_t b0 = smem_u32(stage_b) + static_cast<uint32_t>(s) * b_stage;
+          const uint32_t b0 = smem_u32(stage_b) + static_cast<uint32_t>(s) * B_STAGE;
 #pragma unroll
           for (int kk = 0; kk < CHUNK / 16; ++kk) {
-            umma_bf16(d, smem_desc_sw(a0 + kk * 32, ROW_BYTES), smem_desc_sw(b0 + kk * 32, ROW_BYTES),
-                      idesc, (first && kk == 0) ? 0u : 1u);
+            umma_bf16(d, smem_desc_sw(a0 + kk * 32, ROW_BYTES),
+                      smem_desc_sw(b0 + kk * 32, ROW_BYTES), idesc,
+                      (first && kk == 0) ? 0u : 1u);
           }
           first = false;
           umma_commit(&empty[s]);
@@ -358,48 +372,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // --------------------------------------------------------- epilogue ----
-    const int64_t n_units = a.n_tiles * a.n_cblocks;
+    const int64_t n_units = a.n_tiles * a.n_oblocks;
+    const uint32_t stage = smem_u32(epi_s) + static_cast<uint32_t>(warp) * (32 * 64);
     int local = 0;
     for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x, ++local) {
       const int acc = local & 1;
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&acc_full[acc], (local >> 1) & 1, abort_flag))) break;
       tc_fence_after();
-      const int64_t tile = u / a.n_cblocks;
-      const int n0 = static_cast<int>(u % a.n_cblocks) * a.bn;
-      const int64_t row = tile * BM + warp * 32 + lane;
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(warp * 32) << 16) +
-                             static_cast<uint32_t>(acc * a.bn);
-      __nv_bfloat16* orow = a.out + row * a.cout + n0;
-      for (int c0 = 0; c0 < a.bn; c0 += 32) {
-        const int width = a.bn - c0 >= 32 ? 32 : 16;
+      const int64_t row0 = (u / a.n_oblocks) * TV;
+      const int o_warp = static_cast<int>(u % a.n_oblocks) * TO + warp * 32;  // this warp's channels
+      const uint32_t taddr =
+          tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(acc * TV);
+      for (int c0 = 0; c0 < TV; c0 += 32) {
         uint32_t v[32];
-        if (width == 32) {
-          tmem_ld_32x32b_x32(taddr + c0, v);
-        } else {
-          uint32_t h[16];
-          tmem_ld_32x32b_x16(taddr + c0, h);
-#pragma unroll
-          for (int q = 0; q < 16; ++q) v[q] = h[q];
-        }
+        tmem_ld_32x32b_x32(taddr + c0, v);  // lane = channel o_warp + lane, 32 voxels
         tmem_ld_wait();
-        if (row < a.n) {
+        // transpose through shared memory: [voxel 0..31][channel 0..31] bf16
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            if (q * 8 >= width || n0 + c0 + q * 8 >= a.cout) continue;
-            float f[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float accv = __uint_as_float(v[q * 8 + e]);
-              f[e] = a.act ? gelu_erf(accv) : accv;
-            }
-            uint4 pk;
-            pk.x = pack_bf16x2(f[0], f[1]);
-            pk.y = pack_bf16x2(f[2], f[3]);
-            pk.z = pack_bf16x2(f[4], f[5]);
-            pk.w = pack_bf16x2(f[6], f[7]);
-            *reinterpret_cast<uint4*>(orow + c0 + q * 8) = pk;
-          }
+        for (int e = 0; e < 32; ++e) {
+          float f = __uint_as_float(v[e]);
+          if (a.act) f = gelu_erf(f);
+          const __nv_bfloat16 h = __float2bfloat16_rn(f);
+          sts_u16(stage + e * 64 + lane * 2, *reinterpret_cast<const uint16_t*>(&h));
         }
+        __syncwarp();
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const int vv = p * 8 + lane / 4;  // voxel within the 32
+          const int q = lane % 4;           // 8-channel group
+          const uint4 val = lds_16(stage + vv * 64 + q * 16);
+          const int64_t row = row0 + c0 + vv;
+          const int o = o_warp + q * 8;
+          if (row < a.n && o < a.cout)
+            *reinterpret_cast<uint4*>(a.out + row * a.cout + o) = val;
+        }
+        __syncwarp();
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
@@ -410,7 +417,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   if (warp == MMA_WARP) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, a.tmem_cols);
+    tmem_dealloc(tmem_base, kTmemCols);
   }
   if (threadIdx.x == 0 && *abort_flag) atomicExch(a.err_word, 1);
 }
@@ -472,23 +479,18 @@ cudaError_t launch_forward_bf16(const int32_t* nbr, const uint32_t* tile_mask, i
   int num_sms = 0;
   if ((e = device_setup(device, &num_sms)) != cudaSuccess) return e;
 
-  // Cout in n_cblocks column blocks of equal width (a multiple of 16, <= 256).
-  const int n_cblocks = (cout + 255) / 256;
-  int bn = (cout + n_cblocks - 1) / n_cblocks;
-  bn = (bn + 15) / 16 * 16;
-  uint32_t tmem_cols = 32;
-  while (tmem_cols < static_cast<uint32_t>(2 * bn)) tmem_cols <<= 1;
   const int chunk = cin % 64 == 0 ? 64 : (cin % 32 == 0 ? 32 : 16);
-  int stages = 8;
-  while (stages > 2 && plan_smem(bn, chunk, stages).bytes > static_cast<size_t>(kSmemLimit))
-    --stages;
-  const SmemPlan plan = plan_smem(bn, chunk, stages);
+  int stages = 12;
+  while (stages > 2 && plan_smem(chunk, stages).bytes > static_cast<size_t>(kSmemLimit)) --stages;
+  const SmemPlan plan = plan_smem(chunk, stages);
 
+  // Weight viewed as [Cout][27][Cin]; a box is 128 output channels x 1 offset x
+  // one channel chunk.  Output channels past Cout read as zero.
   CUtensorMap wmap;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(cin), 27, static_cast<cuuint64_t>(cout)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(cin) * 2,
                                  static_cast<cuuint64_t>(cin) * 27 * 2};
-  const cuuint32_t box[3] = {static_cast<cuuint32_t>(chunk), 1, static_cast<cuuint32_t>(bn)};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(chunk), 1, static_cast<cuuint32_t>(TO)};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUtensorMapSwizzle swz =
       chunk == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
@@ -506,16 +508,14 @@ cudaError_t launch_forward_bf16(const int32_t* nbr, const uint32_t* tile_mask, i
   a.out = static_cast<__nv_bfloat16*>(out);
   a.cin = cin;
   a.cout = cout;
-  a.bn = bn;
-  a.n_cblocks = n_cblocks;
+  a.n_oblocks = (cout + TO - 1) / TO;
   a.n_kchunks = cin / chunk;
   a.stages = stages;
   a.flip = flip;
   a.act = act;
-  a.n_tiles = (n + BM - 1) / BM;
-  a.tmem_cols = tmem_cols;
+  a.n_tiles = (n + TV - 1) / TV;
   a.err_word = err_word;
-  const int64_t units = a.n_tiles * n_cblocks;
+  const int64_t units = a.n_tiles * a.n_oblocks;
   const unsigned grid = static_cast<unsigned>(units < num_sms ? units : num_sms);
   if (chunk == 64)
     subm3d_fwd_bf16_sm100<64><<<grid, NUM_THREADS, plan.bytes, stream>>>(wmap, a);

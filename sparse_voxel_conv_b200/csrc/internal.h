@@ -16,21 +16,35 @@ constexpr uint32_t kErrTableFull = 4u;
 constexpr int kTileRows = 128;  // rows per tile-mask word
 constexpr int kKvol = 27;
 
+// The two lookup structures of the map build (see map_build.cu).
+enum class MapKind { kDirect, kHash };
+
+// Largest direct-address table (batch * grid_dim^3 int32 cells) the build uses.
+constexpr size_t kDirectTableMaxBytes = size_t(64) << 20;
+
+// Testing knobs: force the hash table, or cap its capacity (which implies it).
+struct MapOptions {
+  bool force_hash = false;
+  uint64_t forced_capacity = 0;  // a power of two, or 0
+};
+
 // Placement of the map build's pieces inside the caller's workspace.
 struct MapLayout {
-  bool compact = true;      // 32-bit keys in 8-byte (key, row) slots; else 64-bit keys + row array
+  MapKind kind = MapKind::kDirect;
+  bool compact = true;      // hash: 32-bit keys in 8-byte (key, row) slots; else 64-bit keys + rows
   uint64_t capacity = 0;    // hash slots, a power of two >= 4
+  uint64_t cells = 0;       // direct: batch * grid_dim^3
   size_t status_off = 0;    // uint32 status word
   size_t mask_off = 0;      // uint32 [n_tiles]
-  size_t table_off = 0;     // compact: uint64 [capacity]; wide: uint64 keys [capacity]
-  size_t rows_off = 0;      // wide only: int32 rows [capacity]
+  size_t table_off = 0;     // direct: int32 [cells]; hash: uint64 [capacity] (slots or keys)
+  size_t table_bytes = 0;   // bytes of the table (a multiple of 16)
+  size_t rows_off = 0;      // hash, wide keys only: int32 rows [capacity]
   size_t total = 0;         // bytes
   int64_t n_tiles = 0;
 };
 
 // Returns false when the arguments are out of the supported range.
-// forced_capacity (a power of two, or 0) caps the hash table for testing.
-bool map_layout(int64_t n, int32_t grid_dim, int32_t batch, uint64_t forced_capacity,
+bool map_layout(int64_t n, int32_t grid_dim, int32_t batch, const MapOptions& opt,
                 MapLayout* out);
 
 // Enqueues the three map-build kernels on `stream`.  Returns the launch error.

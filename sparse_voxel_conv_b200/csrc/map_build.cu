@@ -1,33 +1,30 @@
-// Neighbour-map build for the submanifold 3x3x3 convolution: a GPU hash table
-// over packed (b, z, y, x) keys, then 27 probes per voxel.
+// Neighbour-map build for the submanifold 3x3x3 convolution.
 //
 // The pages build a "sorted-key indice map (27 lookups/voxel vectorised)"
-// (lato.2_mrp_mlx, commit 97dcdfb54a message).  On the B200 the table is an
-// open-addressing hash table with linear probing that stays resident in L2
-// (8 MB at 330k voxels, 32 MB at 2.1M), built with 64-bit atomicCAS:
+// (lato.2_mrp_mlx, commit 97dcdfb54a message).  Here the lookup structure is
+// one of two GPU tables over packed (b, z, y, x) keys, chosen per call:
 //
-//   map_init    fills the table with EMPTY, zeroes the status word and the
-//               per-tile offset masks (one grid-stride pass);
-//   map_insert  one thread per voxel: 16-byte coordinate load, range check,
-//               key pack, CAS into the first free slot of its probe sequence;
-//               an equal key already present flags a duplicate;
-//   map_query   one thread per (voxel, offset) pair, so the [N,27] int32 map is
-//               written with fully coalesced stores; each thread probes one
-//               neighbour key.  A block covers 32 voxels and ORs the offsets it
-//               found into the mask word of its 128-row tile.
+//   direct  when batch * grid_dim^3 int32 cells fit in 64 MB (every 128^3
+//           volume): cell -> row, -1 when empty.  A collision-free perfect
+//           hash: insert is one plain store per voxel, a lookup is one load,
+//           and voxels adjacent in raster order look up adjacent cells, so the
+//           27 lookups of a warp coalesce.  A duplicate coordinate leaves one
+//           of its rows in the cell; the other row sees a foreign row at its
+//           own centre offset and raises the duplicate flag.
+//   hash    otherwise: open addressing with linear probing, capacity a power
+//           of two >= 2N.  With batch <= 4 and grid_dim <= 1024 a key is
+//           b:2|z:10|y:10|x:10 and a slot the 8-byte word (key << 32 | row),
+//           published by one 64-bit CAS; else a key is b:16|z:16|y:16|x:16 in
+//           a uint64 array with a separate int32 row array.  The home slot is
+//           4 * h(key >> 2) + (key & 3), h a 32-bit avalanche mix, so the
+//           x-neighbours of a voxel usually share a 32-byte sector.  Probe
+//           loops are bounded by the capacity; a full table raises a flag.
 //
-// Keys: with batch <= 4 and grid_dim <= 1024 a key is b:2|z:10|y:10|x:10 and a
-// slot is the 8-byte word (key << 32 | row), so one CAS publishes key and row
-// together and one load returns both.  Otherwise a key is b:16|z:16|y:16|x:16
-// in a uint64 array with a separate int32 row array (rows are read only after
-// the insert kernel has finished).
-//
-// Locality: the home slot of a key is 4 * h(key >> 2) + (key & 3), h a 32-bit
-// avalanche mix, so the x-neighbours (dx = -1, 0, +1) of a voxel usually sit in
-// the same 32-byte sector and the 27 probes of one voxel touch ~10 sectors.
-//
-// Every probe loop is bounded by the capacity; a full table sets kErrTableFull
-// instead of spinning.
+// Kernels: map_init (table <- empty, status <- 0), map_insert (one thread per
+// voxel: 16-byte coordinate load, range check, insert), map_query (one block
+// per 128-row tile, one thread per voxel: 27 lookups into shared memory, then
+// the [128, 27] block and the tile's offset mask are written with coalesced
+// stores; no atomics on the output).
 #include <cuda_runtime.h>
 
 #include "internal.h"
@@ -55,35 +52,19 @@ __device__ __forceinline__ uint32_t mix64to32(unsigned long long k) {
   return static_cast<uint32_t>(k);
 }
 
-struct CompactKeys {
-  using key_t = uint32_t;
-  __device__ static key_t pack(int b, int z, int y, int x) {
-    return (static_cast<uint32_t>(b) << 30) | (static_cast<uint32_t>(z) << 20) |
-           (static_cast<uint32_t>(y) << 10) | static_cast<uint32_t>(x);
-  }
-  __device__ static uint32_t home(key_t key, uint32_t capmask) {
-    return ((mix32(key >> 2) << 2) | (key & 3u)) & capmask;
-  }
-};
-
-struct WideKeys {
-  using key_t = unsigned long long;
-  __device__ static key_t pack(int b, int z, int y, int x) {
-    return (static_cast<unsigned long long>(b) << 48) |
-           (static_cast<unsigned long long>(z) << 32) |
-           (static_cast<unsigned long long>(y) << 16) | static_cast<unsigned long long>(x);
-  }
-  __device__ static uint32_t home(key_t key, uint32_t capmask) {
-    return ((mix64to32(key >> 2) << 2) | static_cast<uint32_t>(key & 3u)) & capmask;
-  }
-};
-
-__global__ void map_init(uint4* table, size_t table_words16, uint32_t* head, size_t head_words) {
-  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
-  const size_t t0 = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const uint4 ones = make_uint4(~0u, ~0u, ~0u, ~0u);
-  for (size_t t = t0; t < table_words16; t += stride) table[t] = ones;
-  for (size_t t = t0; t < head_words; t += stride) head[t] = 0u;
+__device__ __forceinline__ uint32_t pack32(int b, int z, int y, int x) {
+  return (static_cast<uint32_t>(b) << 30) | (static_cast<uint32_t>(z) << 20) |
+         (static_cast<uint32_t>(y) << 10) | static_cast<uint32_t>(x);
+}
+__device__ __forceinline__ unsigned long long pack64(int b, int z, int y, int x) {
+  return (static_cast<unsigned long long>(b) << 48) | (static_cast<unsigned long long>(z) << 32) |
+         (static_cast<unsigned long long>(y) << 16) | static_cast<unsigned long long>(x);
+}
+__device__ __forceinline__ uint32_t home32(uint32_t key, uint32_t capmask) {
+  return ((mix32(key >> 2) << 2) | (key & 3u)) & capmask;
+}
+__device__ __forceinline__ uint32_t home64(unsigned long long key, uint32_t capmask) {
+  return ((mix64to32(key >> 2) << 2) | static_cast<uint32_t>(key & 3u)) & capmask;
 }
 
 __device__ __forceinline__ bool in_volume(int4 c, int grid, int batch) {
@@ -91,6 +72,31 @@ __device__ __forceinline__ bool in_volume(int4 c, int grid, int batch) {
          static_cast<unsigned>(c.y) < static_cast<unsigned>(grid) &&
          static_cast<unsigned>(c.z) < static_cast<unsigned>(grid) &&
          static_cast<unsigned>(c.w) < static_cast<unsigned>(grid);
+}
+
+__device__ __forceinline__ int64_t cell_of(int b, int z, int y, int x, int grid) {
+  return ((static_cast<int64_t>(b) * grid + z) * grid + y) * grid + x;
+}
+
+// Fills `words16` 16-byte words of the table with all-ones and zeroes the status word.
+__global__ void map_init(uint4* table, size_t words16, uint32_t* status) {
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  const size_t t0 = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const uint4 ones = make_uint4(~0u, ~0u, ~0u, ~0u);
+  for (size_t t = t0; t < words16; t += stride) table[t] = ones;
+  if (t0 == 0) *status = 0u;
+}
+
+__global__ void map_insert_direct(const int4* __restrict__ coords, int64_t n, int grid, int batch,
+                                  int32_t* __restrict__ cells, uint32_t* status) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const int4 c = __ldg(coords + i);
+  if (!in_volume(c, grid, batch)) {
+    atomicOr(status, kErrRange);
+    return;
+  }
+  cells[cell_of(c.x, c.y, c.z, c.w, grid)] = static_cast<int32_t>(i);
 }
 
 __global__ void map_insert_compact(const int4* __restrict__ coords, int64_t n, int grid, int batch,
@@ -103,10 +109,10 @@ __global__ void map_insert_compact(const int4* __restrict__ coords, int64_t n, i
     atomicOr(status, kErrRange);
     return;
   }
-  const uint32_t key = CompactKeys::pack(c.x, c.y, c.z, c.w);
+  const uint32_t key = pack32(c.x, c.y, c.z, c.w);
   const unsigned long long entry =
       (static_cast<unsigned long long>(key) << 32) | static_cast<uint32_t>(i);
-  uint32_t slot = CompactKeys::home(key, capmask);
+  uint32_t slot = home32(key, capmask);
   for (uint64_t step = 0; step <= capmask; ++step) {
     const unsigned long long prev = atomicCAS(table + slot, kEmpty, entry);
     if (prev == kEmpty) return;
@@ -129,8 +135,8 @@ __global__ void map_insert_wide(const int4* __restrict__ coords, int64_t n, int 
     atomicOr(status, kErrRange);
     return;
   }
-  const unsigned long long key = WideKeys::pack(c.x, c.y, c.z, c.w);
-  uint32_t slot = WideKeys::home(key, capmask);
+  const unsigned long long key = pack64(c.x, c.y, c.z, c.w);
+  uint32_t slot = home64(key, capmask);
   for (uint64_t step = 0; step <= capmask; ++step) {
     const unsigned long long prev = atomicCAS(keys + slot, kEmpty, key);
     if (prev == kEmpty) {
@@ -146,69 +152,89 @@ __global__ void map_insert_wide(const int4* __restrict__ coords, int64_t n, int 
   atomicOr(status, kErrTableFull);
 }
 
-constexpr int kQueryVoxels = 32;                     // voxels per query block
-constexpr int kQueryThreads = kQueryVoxels * kKvol;  // 864
+enum class Kind { kDirect, kCompact, kWide };
 
-template <bool kCompact>
-__global__ void __launch_bounds__(kQueryThreads)
-    map_query(const int4* __restrict__ coords, int64_t n, int grid,
-              const unsigned long long* __restrict__ table, const int32_t* __restrict__ rows,
-              uint32_t capmask, int32_t* __restrict__ nbr, uint32_t* __restrict__ tile_mask) {
-  __shared__ uint32_t s_mask;
-  if (threadIdx.x == 0) s_mask = 0u;
-  __syncthreads();
-  const int local = threadIdx.x / kKvol;
-  const int k = threadIdx.x - local * kKvol;
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * kQueryVoxels + local;
+struct Tables {
+  const int32_t* cells;             // direct
+  const unsigned long long* table;  // compact slots or wide keys
+  const int32_t* rows;              // wide rows
+  uint32_t capmask;
+};
+
+template <Kind K>
+__device__ __forceinline__ int32_t lookup(const Tables& t, int b, int z, int y, int x, int grid) {
+  if constexpr (K == Kind::kDirect) {
+    return __ldg(t.cells + cell_of(b, z, y, x, grid));
+  } else if constexpr (K == Kind::kCompact) {
+    const uint32_t key = pack32(b, z, y, x);
+    uint32_t slot = home32(key, t.capmask);
+    for (uint64_t step = 0; step <= t.capmask; ++step) {
+      const unsigned long long e = __ldg(t.table + slot);
+      if (e == kEmpty) return -1;
+      if (static_cast<uint32_t>(e >> 32) == key)
+        return static_cast<int32_t>(static_cast<uint32_t>(e));
+      slot = (slot + 1) & t.capmask;
+    }
+    return -1;
+  } else {
+    const unsigned long long key = pack64(b, z, y, x);
+    uint32_t slot = home64(key, t.capmask);
+    for (uint64_t step = 0; step <= t.capmask; ++step) {
+      const unsigned long long e = __ldg(t.table + slot);
+      if (e == kEmpty) return -1;
+      if (e == key) return __ldg(t.rows + slot);
+      slot = (slot + 1) & t.capmask;
+    }
+    return -1;
+  }
+}
+
+template <Kind K>
+__global__ void __launch_bounds__(kTileRows)
+    map_query(const int4* __restrict__ coords, int64_t n, int grid, int batch, Tables t,
+              int32_t* __restrict__ nbr, uint32_t* __restrict__ tile_mask, uint32_t* status) {
+  __shared__ __align__(16) int32_t s_nbr[kTileRows * kKvol];
+  __shared__ uint32_t s_bits[kTileRows / 32];
+  const int r = threadIdx.x;
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kTileRows;
+  const int64_t i = row0 + r;
   uint32_t bits = 0u;
   if (i < n) {
-    int32_t found = -1;
-    if (k == 13) {
-      found = static_cast<int32_t>(i);  // the centre offset is the voxel itself
-    } else {
-      const int4 c = __ldg(coords + i);
-      const int z = c.y + (k / 9) - 1;
-      const int y = c.z + (k / 3) % 3 - 1;
-      const int x = c.w + k % 3 - 1;
-      if (static_cast<unsigned>(z) < static_cast<unsigned>(grid) &&
-          static_cast<unsigned>(y) < static_cast<unsigned>(grid) &&
-          static_cast<unsigned>(x) < static_cast<unsigned>(grid)) {
-        if constexpr (kCompact) {
-          const uint32_t key = CompactKeys::pack(c.x, z, y, x);
-          uint32_t slot = CompactKeys::home(key, capmask);
-          for (uint64_t step = 0; step <= capmask; ++step) {
-            const unsigned long long e = table[slot];
-            if (e == kEmpty) break;
-            if (static_cast<uint32_t>(e >> 32) == key) {
-              found = static_cast<int32_t>(static_cast<uint32_t>(e));
-              break;
-            }
-            slot = (slot + 1) & capmask;
-          }
-        } else {
-          const unsigned long long key = WideKeys::pack(c.x, z, y, x);
-          uint32_t slot = WideKeys::home(key, capmask);
-          for (uint64_t step = 0; step <= capmask; ++step) {
-            const unsigned long long e = table[slot];
-            if (e == kEmpty) break;
-            if (e == key) {
-              found = rows[slot];
-              break;
-            }
-            slot = (slot + 1) & capmask;
-          }
-        }
+    const int4 c = __ldg(coords + i);
+    if (in_volume(c, grid, batch)) {
+#pragma unroll
+      for (int k = 0; k < kKvol; ++k) {
+        const int z = c.y + k / 9 - 1;
+        const int y = c.z + (k / 3) % 3 - 1;
+        const int x = c.w + k % 3 - 1;
+        int32_t found = -1;
+        if (static_cast<unsigned>(z) < static_cast<unsigned>(grid) &&
+            static_cast<unsigned>(y) < static_cast<unsigned>(grid) &&
+            static_cast<unsigned>(x) < static_cast<unsigned>(grid))
+          found = lookup<K>(t, c.x, z, y, x, grid);
+        s_nbr[r * kKvol + k] = found;
+        bits |= (found >= 0 ? 1u : 0u) << k;
       }
+      if (K == Kind::kDirect && s_nbr[r * kKvol + 13] != static_cast<int32_t>(i))
+        atomicOr(status, kErrDuplicate);  // another row owns this voxel's cell
+    } else {
+#pragma unroll
+      for (int k = 0; k < kKvol; ++k) s_nbr[r * kKvol + k] = -1;
     }
-    nbr[static_cast<int64_t>(blockIdx.x) * kQueryThreads + threadIdx.x] = found;
-    bits = found >= 0 ? (1u << k) : 0u;
   }
-  // one shared atomic per warp instead of one per thread
   bits = __reduce_or_sync(0xFFFFFFFFu, bits);
-  if ((threadIdx.x & 31) == 0 && bits != 0u) atomicOr(&s_mask, bits);
+  if ((r & 31) == 0) s_bits[r >> 5] = bits;
   __syncthreads();
-  if (threadIdx.x == 0 && s_mask != 0u) {
-    atomicOr(tile_mask + (static_cast<int64_t>(blockIdx.x) * kQueryVoxels) / kTileRows, s_mask);
+  if (r == 0) tile_mask[blockIdx.x] = s_bits[0] | s_bits[1] | s_bits[2] | s_bits[3];
+  const int rows = static_cast<int>(n - row0 < kTileRows ? n - row0 : kTileRows);
+  int32_t* dst = nbr + row0 * kKvol;
+  if (rows == kTileRows) {
+    // 13824 bytes = 864 16-byte words; each tile's nbr block starts 16-byte aligned
+    const int4* src4 = reinterpret_cast<const int4*>(s_nbr);
+    int4* dst4 = reinterpret_cast<int4*>(dst);
+    for (int e = r; e < kTileRows * kKvol / 4; e += kTileRows) dst4[e] = src4[e];
+  } else {
+    for (int e = r; e < rows * kKvol; e += kTileRows) dst[e] = s_nbr[e];
   }
 }
 
@@ -216,26 +242,38 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 }  // namespace
 
-bool map_layout(int64_t n, int32_t grid_dim, int32_t batch, uint64_t forced_capacity,
+bool map_layout(int64_t n, int32_t grid_dim, int32_t batch, const MapOptions& opt,
                 MapLayout* out) {
   if (n < 0 || n >= 0x7FFFFFFFll || grid_dim < 1 || grid_dim > 65535 || batch < 1 ||
       batch > 65535)
     return false;
   MapLayout lay;
+  const double cells = static_cast<double>(batch) * grid_dim * grid_dim * grid_dim;
+  const bool direct_fits = cells * 4.0 <= static_cast<double>(kDirectTableMaxBytes);
+  lay.kind = (direct_fits && !opt.force_hash && opt.forced_capacity == 0) ? MapKind::kDirect
+                                                                         : MapKind::kHash;
   lay.compact = (batch <= 4 && grid_dim <= 1024);
   uint64_t cap = 1024;
   while (cap < 2ull * static_cast<uint64_t>(n)) cap <<= 1;
-  if (forced_capacity != 0 && forced_capacity < cap) {
+  if (opt.forced_capacity != 0 && opt.forced_capacity < cap) {
     cap = 4;
-    while (cap < forced_capacity) cap <<= 1;
+    while (cap < opt.forced_capacity) cap <<= 1;
   }
   lay.capacity = cap;
+  lay.cells = direct_fits ? static_cast<uint64_t>(cells) : 0;
   lay.n_tiles = (n + kTileRows - 1) / kTileRows;
   lay.status_off = 0;
   lay.mask_off = 256;
   lay.table_off = align_up(lay.mask_off + static_cast<size_t>(lay.n_tiles) * 4, 256);
-  lay.rows_off = align_up(lay.table_off + cap * 8, 256);
-  lay.total = lay.compact ? lay.rows_off : align_up(lay.rows_off + cap * 4, 256);
+  if (lay.kind == MapKind::kDirect) {
+    lay.table_bytes = align_up(lay.cells * 4, 256);
+    lay.rows_off = lay.table_off + lay.table_bytes;
+    lay.total = lay.rows_off;
+  } else {
+    lay.table_bytes = cap * 8;
+    lay.rows_off = align_up(lay.table_off + lay.table_bytes, 256);
+    lay.total = lay.compact ? lay.rows_off : align_up(lay.rows_off + cap * 4, 256);
+  }
   *out = lay;
   return true;
 }
@@ -246,33 +284,42 @@ cudaError_t launch_map_build(const int32_t* coords, int64_t n, int32_t grid_dim,
   auto* ws = static_cast<uint8_t*>(workspace);
   auto* status = reinterpret_cast<uint32_t*>(ws + lay.status_off);
   auto* mask = reinterpret_cast<uint32_t*>(ws + lay.mask_off);
-  auto* table = reinterpret_cast<unsigned long long*>(ws + lay.table_off);
-  auto* rows = reinterpret_cast<int32_t*>(ws + lay.rows_off);
-  const uint32_t capmask = static_cast<uint32_t>(lay.capacity - 1);
-  // head = status word (+ padding) and the mask words, all cleared to zero
-  const size_t head_words = (lay.table_off - lay.status_off) / 4;
-  const size_t table_words16 = lay.capacity * 8 / 16;
+  auto* table = ws + lay.table_off;
+  const size_t words16 = lay.table_bytes / 16;
   {
-    const size_t work = table_words16 > head_words ? table_words16 : head_words;
-    size_t blocks = (work + 255) / 256;
-    if (blocks > 148 * 16) blocks = 148 * 16;
+    size_t blocks = (words16 + 255) / 256;
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    if (blocks == 0) blocks = 1;
     map_init<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(reinterpret_cast<uint4*>(table),
-                                                               table_words16, status, head_words);
+                                                               words16, status);
   }
   if (n == 0) return cudaGetLastError();
   const auto* c4 = reinterpret_cast<const int4*>(coords);
   const unsigned ins_blocks = static_cast<unsigned>((n + 255) / 256);
-  const unsigned q_blocks = static_cast<unsigned>((n + kQueryVoxels - 1) / kQueryVoxels);
-  if (lay.compact) {
-    map_insert_compact<<<ins_blocks, 256, 0, stream>>>(c4, n, grid_dim, batch, table, capmask,
-                                                       status);
-    map_query<true><<<q_blocks, kQueryThreads, 0, stream>>>(c4, n, grid_dim, table, nullptr,
-                                                            capmask, nbr, mask);
+  const unsigned q_blocks = static_cast<unsigned>(lay.n_tiles);
+  Tables t{};
+  t.capmask = static_cast<uint32_t>(lay.capacity - 1);
+  if (lay.kind == MapKind::kDirect) {
+    t.cells = reinterpret_cast<const int32_t*>(table);
+    map_insert_direct<<<ins_blocks, 256, 0, stream>>>(c4, n, grid_dim, batch,
+                                                      reinterpret_cast<int32_t*>(table), status);
+    map_query<Kind::kDirect><<<q_blocks, kTileRows, 0, stream>>>(c4, n, grid_dim, batch, t, nbr,
+                                                                 mask, status);
+  } else if (lay.compact) {
+    t.table = reinterpret_cast<const unsigned long long*>(table);
+    map_insert_compact<<<ins_blocks, 256, 0, stream>>>(
+        c4, n, grid_dim, batch, reinterpret_cast<unsigned long long*>(table), t.capmask, status);
+    map_query<Kind::kCompact><<<q_blocks, kTileRows, 0, stream>>>(c4, n, grid_dim, batch, t, nbr,
+                                                                  mask, status);
   } else {
-    map_insert_wide<<<ins_blocks, 256, 0, stream>>>(c4, n, grid_dim, batch, table, rows, capmask,
-                                                    status);
-    map_query<false><<<q_blocks, kQueryThreads, 0, stream>>>(c4, n, grid_dim, table, rows,
-                                                             capmask, nbr, mask);
+    auto* rows = reinterpret_cast<int32_t*>(ws + lay.rows_off);
+    t.table = reinterpret_cast<const unsigned long long*>(table);
+    t.rows = rows;
+    map_insert_wide<<<ins_blocks, 256, 0, stream>>>(c4, n, grid_dim, batch,
+                                                    reinterpret_cast<unsigned long long*>(table),
+                                                    rows, t.capmask, status);
+    map_query<Kind::kWide><<<q_blocks, kTileRows, 0, stream>>>(c4, n, grid_dim, batch, t, nbr,
+                                                               mask, status);
   }
   return cudaGetLastError();
 }

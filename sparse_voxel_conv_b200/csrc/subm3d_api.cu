@@ -28,12 +28,18 @@ namespace {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-// Testing knob: SUBM3D_TABLE_CAPACITY caps the hash table at that many slots
-// (rounded up to a power of two), so that a full table can be exercised.
-uint64_t forced_capacity() {
-  const char* s = std::getenv("SUBM3D_TABLE_CAPACITY");
-  if (!s || !*s) return 0;
-  return std::strtoull(s, nullptr, 10);
+// Testing knobs read from the environment at every call:
+//   SUBM3D_TABLE_CAPACITY=<slots>  caps the hash table (and selects it), so that
+//                                  a full table can be exercised;
+//   SUBM3D_MAP_KIND=hash           uses the hash table even where the direct
+//                                  table would fit.
+subm3d::MapOptions options_from_env() {
+  subm3d::MapOptions o;
+  const char* cap = std::getenv("SUBM3D_TABLE_CAPACITY");
+  if (cap && *cap) o.forced_capacity = std::strtoull(cap, nullptr, 10);
+  const char* kind = std::getenv("SUBM3D_MAP_KIND");
+  if (kind && std::strcmp(kind, "hash") == 0) o.force_hash = true;
+  return o;
 }
 
 // 1 when the current device is sm_100 (B200 class), 0 when it is not, -1 on error.
@@ -95,7 +101,7 @@ const char* subm3d_status_string(int32_t status) {
 
 size_t subm3d_map_workspace_bytes(int64_t n, int32_t grid_dim, int32_t batch) {
   subm3d::MapLayout lay;
-  if (!subm3d::map_layout(n, grid_dim, batch, 0, &lay)) return 0;
+  if (!subm3d::map_layout(n, grid_dim, batch, options_from_env(), &lay)) return 0;
   return lay.total;
 }
 
@@ -107,11 +113,9 @@ subm3d_status subm3d_build_map(const int32_t* coords, int64_t n, int32_t grid_di
   if (n < 0 || !workspace) return SUBM3D_E_INVALID;
   if (n > 0 && (!coords || !nbr)) return SUBM3D_E_INVALID;
   subm3d::MapLayout lay;
-  if (!subm3d::map_layout(n, grid_dim, batch, forced_capacity(), &lay))
+  if (!subm3d::map_layout(n, grid_dim, batch, options_from_env(), &lay))
     return (grid_dim < 1 || batch < 1) ? SUBM3D_E_INVALID : SUBM3D_E_UNSUPPORTED;
-  subm3d::MapLayout full;
-  subm3d::map_layout(n, grid_dim, batch, 0, &full);
-  if (workspace_bytes < full.total) return SUBM3D_E_INVALID;
+  if (workspace_bytes < lay.total) return SUBM3D_E_INVALID;
   if (!aligned(coords, 16) || !aligned(nbr, 16) || !aligned(workspace, 256))
     return SUBM3D_E_INVALID;
   auto* h = new (std::nothrow) subm3d_map;

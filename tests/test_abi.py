@@ -43,17 +43,24 @@ def test_version_and_strings(abi):
     assert abi.subm3d_status_string(99) == "unknown status"
 
 
-def test_workspace_bytes(abi):
+def test_workspace_bytes(abi, monkeypatch):
+    monkeypatch.delenv("SUBM3D_MAP_KIND", raising=False)
+    monkeypatch.delenv("SUBM3D_TABLE_CAPACITY", raising=False)
     f = abi.subm3d_map_workspace_bytes
     assert f(-1, 16, 1) == 0 and f(10, 0, 1) == 0 and f(10, 16, 0) == 0
     assert f(10, 70000, 1) == 0 and f(10, 16, 70000) == 0
-    # compact form: 8-byte slots, capacity = max(1024, pow2 >= 2N)
     n = 329839
-    ws = f(n, 128, 1)
-    assert ws >= 256 + 4 * ((n + 127) // 128) + 8 * (1 << 20)
-    assert ws < 256 + 4 * ((n + 127) // 128) + 8 * (1 << 20) + 1024
-    # wide form (batch > 4) adds a 4-byte row array
-    assert f(n, 128, 5) >= ws + 4 * (1 << 20)
+    head = 256 + 4 * ((n + 127) // 128)
+    # direct table: one int32 per cell of a volume up to 64 MB
+    assert head + 4 * 128 ** 3 <= f(n, 128, 1) < head + 4 * 128 ** 3 + 1024
+    assert head + 4 * 256 ** 3 <= f(n, 256, 1) < head + 4 * 256 ** 3 + 1024
+    # larger volumes: hash table, 8-byte slots, capacity max(1024, pow2 >= 2N)
+    assert head + 8 * (1 << 20) <= f(n, 512, 1) < head + 8 * (1 << 20) + 1024
+    # wide keys (batch > 4 or grid > 1024) add a 4-byte row array
+    assert f(n, 2048, 1) >= head + 12 * (1 << 20)
+    monkeypatch.setenv("SUBM3D_MAP_KIND", "hash")
+    assert head + 8 * (1 << 20) <= f(n, 128, 1) < head + 8 * (1 << 20) + 1024
+    assert f(n, 128, 5) >= head + 12 * (1 << 20)
     assert f(0, 16, 1) > 0
 
 

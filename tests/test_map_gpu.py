@@ -20,13 +20,24 @@ def S():
     return S
 
 
+@pytest.fixture(params=["auto", "hash"])
+def kind(request, monkeypatch):
+    """auto: the direct table where the volume fits in 64 MB, else the hash
+    table; hash: the hash table everywhere (testing knob SUBM3D_MAP_KIND)."""
+    if request.param == "hash":
+        monkeypatch.setenv("SUBM3D_MAP_KIND", "hash")
+    else:
+        monkeypatch.delenv("SUBM3D_MAP_KIND", raising=False)
+    return request.param
+
+
 def _gpu_map(S, coords, grid, batch):
     h = S.build_map(torch.from_numpy(np.ascontiguousarray(coords)).cuda(), grid, batch)
     return h, h.nbr.cpu().numpy(), S.tile_mask_tensor(h).cpu().numpy().astype(np.int64) & 0x7FFFFFF
 
 
 @pytest.mark.parametrize("name", ["tiny", "shell", "headline", "dense", "batched"])
-def test_map_bit_exact(S, name):
+def test_map_bit_exact(S, kind, name):
     wl = WL.make_workload(name)
     h, nbr, masks = _gpu_map(S, wl.coords, wl.grid_dim, wl.batch)
     ref = C.build_map(wl.coords, wl.grid_dim, wl.batch)
@@ -36,7 +47,7 @@ def test_map_bit_exact(S, name):
 
 
 @pytest.mark.parametrize("name,seed", [("shell", 1), ("headline", 2), ("batched", 3)])
-def test_map_bit_exact_random_row_order(S, name, seed):
+def test_map_bit_exact_random_row_order(S, kind, name, seed):
     wl = WL.make_workload(name)
     c = wl.coords[WL.permute_rows(wl.n, seed)]
     _, nbr, masks = _gpu_map(S, c, wl.grid_dim, wl.batch)
@@ -46,7 +57,7 @@ def test_map_bit_exact_random_row_order(S, name, seed):
 
 
 @pytest.mark.parametrize("grid,batch,shift", [(2048, 1, 1900), (64, 6, 0), (65535, 9, 65500)])
-def test_map_wide_keys(S, grid, batch, shift):
+def test_map_wide_keys(S, kind, grid, batch, shift):
     # batch > 4 or grid_dim > 1024 takes the 64-bit key form
     rng = np.random.default_rng(grid + batch)
     parts = []
@@ -63,7 +74,7 @@ def test_map_wide_keys(S, grid, batch, shift):
     assert np.array_equal(masks, masks_from_nbr(ref))
 
 
-def test_map_edge_sizes(S):
+def test_map_edge_sizes(S, kind):
     for c in (np.zeros((0, 4), np.int32), np.array([[0, 3, 3, 3]], np.int32),
               WL.dense_coords(5)[:129], WL.dense_coords(2)):
         grid = 5
@@ -73,7 +84,7 @@ def test_map_edge_sizes(S):
         assert np.array_equal(masks, masks_from_nbr(ref))
 
 
-def test_map_grid_boundary_no_wrap(S):
+def test_map_grid_boundary_no_wrap(S, kind):
     # voxels on opposite faces of the grid are not neighbours (no wrap-around)
     g = 8
     c = np.array([[0, 0, 0, 0], [0, g - 1, 0, 0], [0, 0, g - 1, 0], [0, 0, 0, g - 1],
@@ -85,7 +96,7 @@ def test_map_grid_boundary_no_wrap(S):
 
 @pytest.mark.parametrize("bad,status", [([0, 0, 0, 16], 2), ([0, -1, 3, 3], 2), ([1, 1, 1, 1], 2),
                                         (None, 3)])
-def test_map_data_errors(S, bad, status):
+def test_map_data_errors(S, kind, bad, status):
     base = WL.tiny_coords()
     extra = base[700:701] if bad is None else np.array([bad], np.int32)  # None: a duplicate
     c = np.concatenate([base, extra])

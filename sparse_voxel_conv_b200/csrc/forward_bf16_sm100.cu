@@ -104,12 +104,13 @@ __host__ __device__ inline SmemPlan plan_smem(int chunk, int stages) {
 // the same sequence.  The centre offset is always included, so every unit has
 // at least one step.
 struct Steps {
-  int64_t u;      // current unit
+  int64_t u;       // current unit
   int64_t n_units;
-  int local;      // index of the unit within this CTA (buffer / parity selector)
-  uint32_t rest;  // offsets of the unit still to come
-  int k, j;       // current offset and chunk
-  int it;         // global step counter
+  int local;       // index of the unit within this CTA (buffer / parity selector)
+  uint32_t rest;   // offsets of the unit still to come
+  int k, j;        // current offset and chunk
+  int slot;        // stage slot of the current step (step counter mod stages)
+  uint32_t phase;  // parity of the slot's current use (step counter / stages, mod 2)
   bool valid;
 
   __device__ void load_unit(const FwdArgs& a) {
@@ -129,13 +130,17 @@ struct Steps {
     n_units = a.n_tiles * a.n_oblocks;
     u = blockIdx.x;
     local = 0;
-    it = 0;
+    slot = 0;
+    phase = 0;
     valid = u < n_units;
     if (valid) load_unit(a);
   }
   // Advances one step; returns true when the step moved to a new unit (or ended).
   __device__ bool next(const FwdArgs& a) {
-    ++it;
+    if (++slot == a.stages) {
+      slot = 0;
+      phase ^= 1u;
+    }
     if (++j < a.n_kchunks) return false;
     j = 0;
     if (rest) {
@@ -155,7 +160,7 @@ __device__ __forceinline__ float gelu_erf(float v) {
   return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f));
 }
 
-template <int CHUNK>
+template <int CHUNK, bool GELU>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     subm3d_fwd_bf16_sm100(const __grid_constant__ CUtensorMap wmap, const FwdArgs a) {
   constexpr int ROW_BYTES = CHUNK * 2;  // 128, 64 or 32
@@ -238,8 +243,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int q = 0; q < PPT; ++q) {
         const int r = rbase + q * ROWS_PER_PASS;
         const int32_t src = nb[r * kKvol + ld.k];
-        vd[q] = src >= 0 ? ldg_nc_16(a.x + static_cast<int64_t>(src) * a.cin + col)
-                         : make_uint4(0u, 0u, 0u, 0u);
+        vd[q] = ldg_nc_16_pred(a.x + static_cast<int64_t>(src < 0 ? 0 : src) * a.cin + col,
+                               src >= 0);
       }
       const int old_local = ld.local;
       if (ld.next(a)) {  // the unit's last loads are issued: release its nbr buffer
@@ -256,8 +261,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
       for (int d = 0; d < kDepth; ++d) {
         if (!ok || !st.valid) break;
-        const int s = st.it % S;
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[s], ((st.it / S) & 1) ^ 1, abort_flag))) {
+        const int s = st.slot;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[s], st.phase ^ 1u, abort_flag))) {
           ok = false;
           break;
         }
@@ -315,8 +320,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           break;
         }
       }
-      const int s = st.it % S;
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[s], ((st.it / S) & 1) ^ 1, abort_flag))) {
+      const int s = st.slot;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[s], st.phase ^ 1u, abort_flag))) {
         ok = false;
         break;
       }
@@ -347,8 +352,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         bool first = true;
         bool unit_done = false;
         while (!unit_done) {
-          const int s = st.it % S;
-          if (!mbar_wait(&full[s], (st.it / S) & 1, abort_flag)) {
+          const int s = st.slot;
+          if (!mbar_wait(&full[s], st.phase, abort_flag)) {
             ok = false;
             break;
           }
@@ -383,6 +388,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int o_warp = static_cast<int>(u % a.n_oblocks) * TO + warp * 32;  // this warp's channels
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(acc * TV);
+#pragma unroll 1
       for (int c0 = 0; c0 < TV; c0 += 32) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(taddr + c0, v);  // lane = channel o_warp + lane, 32 voxels
@@ -391,7 +397,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           float f = __uint_as_float(v[e]);
-          if (a.act) f = gelu_erf(f);
+          if constexpr (GELU) f = gelu_erf(f);
           const __nv_bfloat16 h = __float2bfloat16_rn(f);
           sts_u16(stage + e * 64 + lane * 2, *reinterpret_cast<const uint16_t*>(&h));
         }
@@ -448,9 +454,12 @@ cudaError_t device_setup(int device, int* num_sms) {
   if (device < 0 || device >= 64) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(mu);
   if (sms[device] == 0) {
-    const void* kernels[3] = {reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<64>),
-                              reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<32>),
-                              reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<16>)};
+    const void* kernels[6] = {reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<64, false>),
+                              reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<32, false>),
+                              reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<16, false>),
+                              reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<64, true>),
+                              reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<32, true>),
+                              reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<16, true>)};
     for (const void* k : kernels) {
       const cudaError_t e =
           cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
@@ -517,12 +526,15 @@ cudaError_t launch_forward_bf16(const int32_t* nbr, const uint32_t* tile_mask, i
   a.err_word = err_word;
   const int64_t units = a.n_tiles * a.n_oblocks;
   const unsigned grid = static_cast<unsigned>(units < num_sms ? units : num_sms);
+  auto launch = [&](auto kernel) {
+    kernel<<<grid, NUM_THREADS, plan.bytes, stream>>>(wmap, a);
+  };
   if (chunk == 64)
-    subm3d_fwd_bf16_sm100<64><<<grid, NUM_THREADS, plan.bytes, stream>>>(wmap, a);
+    act ? launch(subm3d_fwd_bf16_sm100<64, true>) : launch(subm3d_fwd_bf16_sm100<64, false>);
   else if (chunk == 32)
-    subm3d_fwd_bf16_sm100<32><<<grid, NUM_THREADS, plan.bytes, stream>>>(wmap, a);
+    act ? launch(subm3d_fwd_bf16_sm100<32, true>) : launch(subm3d_fwd_bf16_sm100<32, false>);
   else
-    subm3d_fwd_bf16_sm100<16><<<grid, NUM_THREADS, plan.bytes, stream>>>(wmap, a);
+    act ? launch(subm3d_fwd_bf16_sm100<16, true>) : launch(subm3d_fwd_bf16_sm100<16, false>);
   return cudaGetLastError();
 }
 

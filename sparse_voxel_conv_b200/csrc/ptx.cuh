@@ -55,11 +55,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase of `bar` with the given parity to complete.  Returns
-// false (and sets *abort) when the wait exceeds kWaitLimitNs, or returns false
-// at once when another role of the CTA has already set *abort.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Slow path of mbar_wait, kept out of line so that the many wait sites of a
+// warp-specialised kernel share one copy of the polling loop.
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort) {
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -73,12 +71,32 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Waits for the phase of `bar` with the given parity to complete.  Returns
+// false (and sets *abort) when the wait exceeds kWaitLimitNs, or returns false
+// at once when another role of the CTA has already set *abort.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort);
+}
+
 // 16-byte global load that bypasses L1 allocation (read-only data).
 __device__ __forceinline__ uint4 ldg_nc_16(const void* p) {
   uint4 v;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
+  return v;
+}
+
+// 16-byte read-only load when `pred` is nonzero, else zeros (no branch).
+__device__ __forceinline__ uint4 ldg_nc_16_pred(const void* p, uint32_t pred) {
+  uint4 v = make_uint4(0u, 0u, 0u, 0u);
+  asm volatile(
+      "{\n\t.reg .pred q;\n\t"
+      "setp.ne.b32 q, %5, 0;\n\t"
+      "@q ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];\n\t}"
+      : "+r"(v.x), "+r"(v.y), "+r"(v.z), "+r"(v.w)
+      : "l"(p), "r"(pred));
   return v;
 }
 

@@ -55,6 +55,28 @@ def _workload(name):
     return WL.make_workload(name)
 
 
+def feature_seed(rank: int) -> int:
+    """Seed of a replica's features: every rank convolves its own input."""
+    return 1 + 1000 * rank
+
+
+def max_over_ranks(value: float, device) -> float:
+    """The job's time is the slowest rank's: all-reduce MAX of a float (a
+    no-op without an initialised process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank: int, world: int, job_seconds: float) -> float:
+    """Weak-scaling throughput: the units every rank processed / the job time."""
+    return units_per_rank * world / job_seconds
+
+
 class ClockSampler:
     """Samples nvidia-smi clocks and throttle reasons in the background."""
 
@@ -139,7 +161,7 @@ def run_ours(args):
     cin, cout = wl.channels[0], wl.channels[1]
     n = wl.n
     coords_h = torch.from_numpy(wl.coords)
-    feats_h = torch.from_numpy(WL.to_bf16_values(WL.make_features(n, cin, 1 + 1000 * rank)))
+    feats_h = torch.from_numpy(WL.to_bf16_values(WL.make_features(n, cin, feature_seed(rank))))
     w_h = torch.from_numpy(wl.weights()[0])
     coords = coords_h.to(dev)
     feats = feats_h.to(dev).to(torch.bfloat16)
@@ -195,11 +217,7 @@ def run_ours(args):
     step_ms = [a.elapsed_time(b) for a, b in ev]
     fwd_ms = [a.elapsed_time(b) for a, b in evf]
     map_ms = [s - f for s, f in zip(step_ms, fwd_ms)]
-    total_ms = float(sum(step_ms))
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(float(sum(step_ms)), dev)
 
     # e2e through the public API with host buffers: H2D of this step's inputs
     # from pinned memory, map build, forward, D2H of the output, every step.
@@ -228,11 +246,7 @@ def run_ours(args):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
 
     if rank == 0:
         peaks, peak_src = _peaks()
@@ -245,7 +259,7 @@ def run_ours(args):
         voxels_total = n * world
         line = {
             "metric": METRIC,
-            "value": voxels_total / (total_ms / 1e3 / K),
+            "value": job_rate(n, world, total_ms / 1e3 / K),
             "unit": "voxels/s",
             "n_gpus": world,
             "steps": K,
@@ -276,7 +290,7 @@ def run_ours(args):
                 "unit": "GB/s", "frac": map_gbs / float(peaks["hbm_gbs"]),
                 "bytes_per_voxel": MAP_BYTES_PER_VOXEL, "ms_avg": map_avg_s * 1e3,
             },
-            "e2e": {"value": voxels_total / (e2e_ms / 1e3 / K), "unit": "voxels/s",
+            "e2e": {"value": job_rate(n, world, e2e_ms / 1e3 / K), "unit": "voxels/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms / K},
             "gpu_launches": 4 * K,

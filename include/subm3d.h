@@ -165,6 +165,46 @@ SUBM3D_API subm3d_status subm3d_forward(const int32_t* nbr, const uint32_t* tile
                              subm3d_act act, void* stream);
 
 /*
+ * Largest N subm3d_build_map_noalloc() accepts.  Its fixed scratch array holds a
+ * hash table for this many voxels: about 12 MB of device memory.
+ */
+#define SUBM3D_NOALLOC_MAX_VOXELS 524288
+
+/*
+ * Allocation-free map build.  The paper has no counterpart to this entry point;
+ * it exists for callers that cannot allocate device memory when they build a
+ * map -- a plugin inside a host framework that owns and accounts for every
+ * device allocation, or a serving loop that must never call cudaMalloc or
+ * cudaFree once running, since those calls synchronise the device and cost
+ * hundreds of microseconds.  It builds the same map as subm3d_build_map()
+ * (always with the hash table) but takes no workspace: its scratch (status word
+ * and hash table) is a fixed device array inside the library, about 12 MB,
+ * which exists on every GPU the process loads the library on, until exit.
+ * It calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ *   coords     (device) int32 [N, 4] (b, z, y, x), 16-byte aligned.
+ *   n          0 <= N <= SUBM3D_NOALLOC_MAX_VOXELS; a larger N returns
+ *              SUBM3D_E_UNSUPPORTED before anything is enqueued.
+ *   grid_dim, batch   as for subm3d_build_map().
+ *   nbr        (device) int32 [N, 27] output, 16-byte aligned.
+ *   tile_mask  (device) uint32 [ceil(N/128)] output, the per-tile offset masks
+ *              that subm3d_forward() takes.
+ *   stream     stream the work is enqueued on.
+ *
+ * Blocking: enqueues the build and a copy of the masks out of the scratch,
+ * synchronizes `stream`, and returns the build's status (SUBM3D_OK,
+ * SUBM3D_E_RANGE, SUBM3D_E_DUPLICATE, SUBM3D_E_TABLE_FULL) or an argument or
+ * CUDA error.  The first call on each device looks up the scratch array's
+ * device address (cudaGetSymbolAddress); make that first call before any
+ * stream capture.  Every call uses the same scratch array and starts by
+ * clearing it, so calls whose work overlaps on the GPU (unordered streams,
+ * several host threads) race and must be serialized by the caller.
+ */
+SUBM3D_API subm3d_status subm3d_build_map_noalloc(const int32_t* coords, int64_t n,
+                                                  int32_t grid_dim, int32_t batch, int32_t* nbr,
+                                                  uint32_t* tile_mask, void* stream);
+
+/*
  * Synchronizes `stream`, then reads and clears the library's device error word
  * of the current device: SUBM3D_E_TIMEOUT if a forward kernel gave up a
  * bounded wait since the last call, else SUBM3D_OK (or SUBM3D_E_CUDA).

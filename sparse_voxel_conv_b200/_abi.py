@@ -59,6 +59,7 @@ def _load() -> ctypes.CDLL:
         "subm3d_forward": (ctypes.c_int, [vp, vp, i64, vp, vp, vp, i32, i32, ctypes.c_int, i32,
                                           ctypes.c_int, vp]),
         "subm3d_device_status": (ctypes.c_int, [vp]),
+        "subm3d_build_map_noalloc": (ctypes.c_int, [vp, i64, i32, i32, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -172,3 +173,15 @@ def subm3d_forward(nbr, tile_mask, n: int, feats, weight, out, cin: int, cout: i
 def subm3d_device_status(stream=None) -> int:
     """Blocking: SUBM3D_E_TIMEOUT if a forward kernel gave up a bounded wait."""
     return int(lib.subm3d_device_status(_stream(stream)))
+
+
+SUBM3D_NOALLOC_MAX_VOXELS = 524288
+
+
+def subm3d_build_map_noalloc(coords, n: int, grid_dim: int, batch: int, nbr, tile_mask,
+                             stream=None) -> int:
+    """Allocation-free map build into caller-given nbr [N, 27] and tile_mask
+    [ceil(N/128)] buffers, using the library's fixed scratch array.  Blocking;
+    returns the status code (no exception), as the C function does."""
+    return int(lib.subm3d_build_map_noalloc(_ptr(coords), int(n), int(grid_dim), int(batch),
+                                            _ptr(nbr), _ptr(tile_mask), _stream(stream)))

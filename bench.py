@@ -50,6 +50,30 @@ def _peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def _profiled_traffic(workload: str):
+    """DRAM bytes per forward launch from the committed ncu summary, when the
+    forward kernel's source is unchanged since that capture (hash match) and
+    the capture was of this workload; else None."""
+    import hashlib
+    import re
+    if workload != "headline":
+        return None
+    prof = os.path.join(ROOT, "profiles", "fwd_bf16_headline.md")
+    csrc = os.path.join(ROOT, "sparse_voxel_conv_b200", "csrc")
+    try:
+        text = open(prof).read()
+        h = hashlib.sha256()
+        for f in ("forward_bf16_sm100.cu", "ptx.cuh"):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    except OSError:
+        return None
+    sha = re.search(r"source_sha256_16:\s*([0-9a-f]{16})", text)
+    traffic = re.search(r"traffic_bytes_per_launch:\s*(\d+)", text)
+    if not sha or not traffic or sha.group(1) != h.hexdigest()[:16]:
+        return None
+    return int(traffic.group(1))
+
+
 def _workload(name):
     import workloads as WL
     return WL.make_workload(name)
@@ -281,7 +305,8 @@ def run_ours(args):
             "roofline": {
                 "kernel": "subm3d_fwd_bf16_sm100",
                 "bound": "tensor", "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
-                "frac": achieved_tf / peak_tf, "traffic": None,
+                "frac": achieved_tf / peak_tf, "traffic": _profiled_traffic(args.workload),
+                "traffic_unit": "bytes per launch (ncu dram read+write)",
                 "peak_source": f"{peak_src} bf16 dense burst",
                 "fwd_ms_avg": fwd_avg_s * 1e3,
             },

@@ -23,12 +23,11 @@
 // sums over every step (offset k, chunk j) the tile needs.  Roles (14 warps):
 //
 //   warps 4-11 (gather)  256 threads fetch B: for step (k, j) the 256 rows
-//       x[nbr[v][k]][chunk j] are loaded with 16-byte read-only loads into
-//       registers, 2-4 steps ahead, then stored into the stage at their
-//       swizzled positions (zeros where nbr = -1).  Eight lanes cover one
-//       128-byte row segment, so every request is a whole aligned segment.
-//       This plain register pipeline measured far above cp.async or TMA
-//       gather4 for these scattered rows.
+//       x[nbr[v][k]][chunk j] are copied with 16-byte cp.async straight into
+//       their swizzled positions in the stage (zero-fill where nbr = -1); each
+//       thread's cp.async.mbarrier.arrive.noinc completes the stage barrier
+//       when its copies have landed.  Eight lanes cover one 128-byte row
+//       segment, so every request is a whole aligned segment.
 //   warp 13 (TMA)        bulk-copies each unit's nbr rows [256 x 27] into one
 //       of two shared buffers ahead of use, and loads the weight slice
 //       Wf[o0:o0+128, k, chunk j] of every step with a 3-D TMA tiled load
@@ -61,9 +60,9 @@ constexpr int TO = 128;  // output channels per unit (MMA M, TMEM lanes)
 constexpr int NUM_EPI_WARPS = 4;
 constexpr int NUM_GATHER_WARPS = 8;
 constexpr int GATHER_WARP0 = 4;
-constexpr int MMA_WARP = 12;
-constexpr int TMA_WARP = 13;
-constexpr int NUM_THREADS = 14 * 32;
+constexpr int MMA_WARP = GATHER_WARP0 + NUM_GATHER_WARPS;
+constexpr int TMA_WARP = MMA_WARP + 1;
+constexpr int NUM_THREADS = (TMA_WARP + 1) * 32;
 constexpr int GATHER_THREADS = NUM_GATHER_WARPS * 32;
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kNbrTileBytes = TV * kKvol * 4;             // 27648
@@ -107,7 +106,8 @@ struct Steps {
   int64_t u;       // current unit
   int64_t n_units;
   int local;       // index of the unit within this CTA (buffer / parity selector)
-  uint32_t rest;   // offsets of the unit still to come
+  uint32_t mask;   // offsets of the unit
+  uint32_t rest;   // offsets still to come in the current chunk
   int k, j;        // current offset and chunk
   int slot;        // stage slot of the current step (step counter mod stages)
   uint32_t phase;  // parity of the slot's current use (step counter / stages, mod 2)
@@ -122,6 +122,7 @@ struct Steps {
       m = __ldg(a.tile_mask + w) | (w + 1 < n_words ? __ldg(a.tile_mask + w + 1) : 0u);
     }
     m |= kCentreBit;
+    mask = m;
     k = __ffs(m) - 1;
     rest = m & (m - 1);
     j = 0;
@@ -141,13 +142,20 @@ struct Steps {
       slot = 0;
       phase ^= 1u;
     }
-    if (++j < a.n_kchunks) return false;
-    j = 0;
+    // chunk-major: all offsets of chunk j, then chunk j+1, so that the steps of
+    // x-adjacent offsets (which gather largely the same rows, shifted by one
+    // voxel) follow each other and can share cached rows
     if (rest) {
       k = __ffs(rest) - 1;
       rest &= rest - 1;
       return false;
     }
+    if (++j < a.n_kchunks) {
+      k = __ffs(mask) - 1;
+      rest = mask & (mask - 1);
+      return false;
+    }
+    j = 0;
     u += gridDim.x;
     ++local;
     valid = u < n_units;
@@ -167,8 +175,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   constexpr int PPR = CHUNK / 8;        // 16-byte pieces per row segment
   constexpr int ROWS_PER_PASS = GATHER_THREADS / PPR;
   constexpr int PPT = TV / ROWS_PER_PASS;  // pieces per gather thread per step
-  // gather steps in flight per thread: ~64 KB of loads in flight per SM
-  constexpr int kDepth = PPT >= 8 ? 2 : (PPT >= 4 ? 3 : 4);
   constexpr uint32_t A_STAGE = TO * ROW_BYTES;
   constexpr uint32_t B_STAGE = TV * ROW_BYTES;
 
@@ -195,7 +201,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], NUM_GATHER_WARPS + 1);  // one arrive per gather warp + TMA expect_tx
+      mbar_init(&full[s], GATHER_THREADS + 1);  // every gather thread's cp.async arrive + TMA
       mbar_init(&empty[s], 1);                    // one tcgen05.commit
     }
     for (int b = 0; b < 2; ++b) {
@@ -219,67 +225,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp >= GATHER_WARP0 && warp < GATHER_WARP0 + NUM_GATHER_WARPS) {
     // ---------------------------------------------------------- gather ----
+    // Per step: wait for the slot, read this thread's row indices, issue its
+    // 16-byte cp.async copies straight into the swizzled stage (zero-fill
+    // where nbr = -1), and let the hardware arrive on the stage's barrier when
+    // they have landed.  No register staging: the copies of up to `stages`
+    // steps are in flight at once.
     const int gt = threadIdx.x - GATHER_WARP0 * 32;
     const int piece = gt % PPR;
     const int rbase = gt / PPR;
-    Steps ld, st;
-    ld.begin(a);
+    uint32_t dst_off[PPT];  // swizzled byte offset of each piece in a stage
+#pragma unroll
+    for (int q = 0; q < PPT; ++q) {
+      const int r = rbase + q * ROWS_PER_PASS;
+      dst_off[q] = r * ROW_BYTES + ((piece ^ ((r * ROW_BYTES >> 7) & (PPR - 1))) << 4);
+    }
+    Steps st;
     st.begin(a);
     int ready_local = -1;
-    bool ok = true;
-    uint4 v[kDepth][PPT];
-
-    // Issue the loads of step `ld` into vd; returns false on a timed-out wait.
-    auto issue = [&](uint4 (&vd)[PPT]) -> bool {
-      if (ld.local != ready_local) {
+    while (st.valid) {
+      if (st.local != ready_local) {
         if (!__all_sync(0xFFFFFFFFu,
-                        mbar_wait(&nbr_full[ld.local & 1], (ld.local >> 1) & 1, abort_flag)))
-          return false;
-        ready_local = ld.local;
+                        mbar_wait(&nbr_full[st.local & 1], (st.local >> 1) & 1, abort_flag)))
+          break;
+        ready_local = st.local;
       }
-      const int32_t* nb = nbr_s + (ld.local & 1) * (TV * kKvol);
-      const int col = ld.j * CHUNK + piece * 8;
+      const int s = st.slot;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[s], st.phase ^ 1u, abort_flag))) break;
+      const int32_t* nb = nbr_s + (st.local & 1) * (TV * kKvol) + rbase * kKvol + st.k;
+      const __nv_bfloat16* xcol = a.x + st.j * CHUNK + piece * 8;
+      const uint32_t b_base = smem_u32(stage_b) + static_cast<uint32_t>(s) * B_STAGE;
 #pragma unroll
       for (int q = 0; q < PPT; ++q) {
-        const int r = rbase + q * ROWS_PER_PASS;
-        const int32_t src = nb[r * kKvol + ld.k];
-        vd[q] = ldg_nc_16_pred(a.x + static_cast<int64_t>(src < 0 ? 0 : src) * a.cin + col,
-                               src >= 0);
+        const int32_t src = nb[q * ROWS_PER_PASS * kKvol];
+        cp_async_16(b_base + dst_off[q],
+                    src >= 0 ? xcol + static_cast<int64_t>(src) * a.cin : a.x, src >= 0 ? 16u : 0u);
       }
-      const int old_local = ld.local;
-      if (ld.next(a)) {  // the unit's last loads are issued: release its nbr buffer
+      cp_async_mbar_arrive_noinc(&full[s]);
+      const int old_local = st.local;
+      if (st.next(a)) {  // the unit's last copies are issued: release its nbr buffer
         __syncwarp();
         if (lane == 0) mbar_arrive(&nbr_empty[old_local & 1]);
       }
-      return true;
-    };
-
-#pragma unroll
-    for (int d = 0; d < kDepth; ++d)
-      if (ok && ld.valid) ok = issue(v[d]);
-    while (ok && st.valid) {
-#pragma unroll
-      for (int d = 0; d < kDepth; ++d) {
-        if (!ok || !st.valid) break;
-        const int s = st.slot;
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[s], st.phase ^ 1u, abort_flag))) {
-          ok = false;
-          break;
-        }
-        const uint32_t b_base = smem_u32(stage_b) + static_cast<uint32_t>(s) * B_STAGE;
-#pragma unroll
-        for (int q = 0; q < PPT; ++q) {
-          const int r = rbase + q * ROWS_PER_PASS;
-          const int phys = piece ^ ((r * ROW_BYTES >> 7) & (PPR - 1));
-          sts_16(b_base + r * ROW_BYTES + (phys << 4), v[d][q]);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&full[s]);
-        st.next(a);
-        if (ld.valid) ok = issue(v[d]);
-      }
     }
+    cp_async_wait_all();
   } else if (warp == TMA_WARP) {
     // ------------------------------------------------------------- TMA ----
     const int64_t n_units = a.n_tiles * a.n_oblocks;

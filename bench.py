@@ -37,6 +37,10 @@ sys.path.insert(0, ROOT)
 METRIC = "SubMConv3d fwd voxels/s and TFLOP/s at 128^3/128ch bf16; % of B200 roofline"
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Kernels one map build launches: table init, insert, query, and the x-run
+# position layout (run count, run scan, placement, E index table).
+MAP_LAUNCHES = 7
+
 # Algorithmic bytes of the map build per voxel: int32 (b,z,y,x) in + int32 [27] out.
 MAP_BYTES_PER_VOXEL = 16 + 27 * 4
 
@@ -58,12 +62,12 @@ def _profiled_traffic(workload: str):
     import re
     if workload != "headline":
         return None
-    prof = os.path.join(ROOT, "profiles", "fwd_bf16_headline.md")
+    prof = os.path.join(ROOT, "profiles", "fwd_bf16_runs_headline.md")
     csrc = os.path.join(ROOT, "sparse_voxel_conv_b200", "csrc")
     try:
         text = open(prof).read()
         h = hashlib.sha256()
-        for f in ("forward_bf16_sm100.cu", "ptx.cuh"):
+        for f in ("forward_bf16_runs_sm100.cu", "ptx.cuh"):
             h.update(open(os.path.join(csrc, f), "rb").read())
     except OSError:
         return None
@@ -297,13 +301,13 @@ def run_ours(args):
             "config": {
                 "workload": wl.name, "n_voxels": n, "nnz_avg": nnz_total / n, "cin": cin,
                 "cout": cout, "grid_dim": wl.grid_dim, "batch": wl.batch,
-                "step": "map build (3 kernels) + bf16 forward (1 kernel)",
+                "step": f"map build ({MAP_LAUNCHES} kernels) + bf16 x-run forward (1 kernel)",
                 "l2": f"flushed before every timed step ({L2_FLUSH_BYTES >> 20} MB write)",
                 "parallelism": f"replicas x{world}, no collective on the data path",
             },
             "tflops_effective": flops * world / (total_ms / 1e3 / K) / 1e12,
             "roofline": {
-                "kernel": "subm3d_fwd_bf16_sm100",
+                "kernel": "subm3d_fwd_bf16_runs_sm100",
                 "bound": "tensor", "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
                 "frac": achieved_tf / peak_tf, "traffic": _profiled_traffic(args.workload),
                 "traffic_unit": "bytes per launch (ncu dram read+write)",
@@ -318,7 +322,7 @@ def run_ours(args):
             "e2e": {"value": job_rate(n, world, e2e_ms / 1e3 / K), "unit": "voxels/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms / K},
-            "gpu_launches": 4 * K,
+            "gpu_launches": (MAP_LAUNCHES + 1) * K,
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:

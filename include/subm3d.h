@@ -81,8 +81,11 @@ SUBM3D_API const char* subm3d_status_string(int32_t status);
  * grid_dim^3 volume: a status word, one 32-bit offset mask per 128-row tile,
  * and the lookup table -- a direct-address table of batch * grid_dim^3 int32
  * cells when that is at most 64 MB, else an open-addressing hash table of at
- * least 2N slots (8 bytes each, 12 with batch > 4 or grid_dim > 1024).
- * Host-only, no CUDA call.  Returns 0 for arguments subm3d_build_map() would
+ * least 2N slots (8 bytes each, 12 with batch > 4 or grid_dim > 1024) -- and
+ * the x-run layout of subm3d_forward_map(): per-1024-row run counts, a header,
+ * a position table of 3N int32 (rounded up) and an E index table of
+ * 9 x 260 int32 per 256 positions (~110 bytes per voxel).  Host-only, no CUDA
+ * call.  Returns 0 for arguments subm3d_build_map() would
  * reject (N < 0, grid_dim < 1 or > 65535, batch < 1 or > 65535).
  */
 SUBM3D_API size_t subm3d_map_workspace_bytes(int64_t n, int32_t grid_dim, int32_t batch);
@@ -107,7 +110,9 @@ SUBM3D_API size_t subm3d_map_workspace_bytes(int64_t n, int32_t grid_dim, int32_
  * The map is bit-identical to the plain definition for every valid input and
  * does not depend on the hash layout.  Coordinates outside the volume or
  * repeated are reported by subm3d_map_status(); until it returns SUBM3D_OK the
- * contents of nbr are unspecified.  Enqueues 3 kernels; no allocation.
+ * contents of nbr are unspecified.  Besides nbr and the tile masks the build
+ * writes the x-run position layout that subm3d_forward_map() uses.  Enqueues 7
+ * kernels; no allocation.
  * Testing knobs, read from the environment by this function and by
  * subm3d_map_workspace_bytes() alike: SUBM3D_MAP_KIND=hash selects the hash
  * table even where the direct table fits; SUBM3D_TABLE_CAPACITY=<slots> caps
@@ -203,6 +208,34 @@ SUBM3D_API subm3d_status subm3d_forward(const int32_t* nbr, const uint32_t* tile
 SUBM3D_API subm3d_status subm3d_build_map_noalloc(const int32_t* coords, int64_t n,
                                                   int32_t grid_dim, int32_t batch, int32_t* nbr,
                                                   uint32_t* tile_mask, void* stream);
+
+/*
+ * Forward of one layer over a built map -- the same op and arguments as
+ * subm3d_forward(), with N, nbr and the masks taken from the map.  For bf16
+ * with Cin a multiple of 64 it runs the x-run kernel, which uses the map's
+ * position layout: voxels on a line of positions in row order, two pad
+ * positions before every run of x-adjacent voxels, tiles of 256 positions,
+ * and per tile and (dz, dy) one gathered tile of feature rows whose rows
+ * p-1, p, p+1 are the dx = -1, 0, +1 neighbours of the voxel at position p;
+ * the three offsets of a (dz, dy) pair share that tile through row-shifted
+ * tensor-core operands, so ~3x fewer feature rows are gathered.  Other shapes
+ * and fp32 run subm3d_forward().  Errors as subm3d_forward().
+ */
+SUBM3D_API subm3d_status subm3d_forward_map(const subm3d_map* map, const void* feats,
+                                            const void* weight, void* out, int32_t cin,
+                                            int32_t cout, subm3d_dtype dtype, int32_t flip,
+                                            subm3d_act act, void* stream);
+
+/*
+ * Device pointers into the map's x-run layout, for tests and tools: the
+ * position table (int32, one entry per position: row * 4 + tag, tag 0 voxel,
+ * 1 left pad of that row's voxel, 2 right pad, -1 empty), the E index table
+ * (int32 [tiles][9][260]: entry i of (tile, dz-dy) is the feature row of
+ * gathered row i-1, or -1) and a 4-int header [runs, tiles, positions, 0].
+ * Valid once the build has completed on its stream.  Host-only.
+ */
+SUBM3D_API subm3d_status subm3d_map_run_layout(const subm3d_map* map, const int32_t** pos,
+                                               const int32_t** etable, const int32_t** header);
 
 /*
  * Synchronizes `stream`, then reads and clears the library's device error word

@@ -60,6 +60,10 @@ def _load() -> ctypes.CDLL:
                                           ctypes.c_int, vp]),
         "subm3d_device_status": (ctypes.c_int, [vp]),
         "subm3d_build_map_noalloc": (ctypes.c_int, [vp, i64, i32, i32, vp, vp, vp]),
+        "subm3d_forward_map": (ctypes.c_int, [vp, vp, vp, vp, i32, i32, ctypes.c_int, i32,
+                                              ctypes.c_int, vp]),
+        "subm3d_map_run_layout": (ctypes.c_int, [vp, ctypes.POINTER(vp), ctypes.POINTER(vp),
+                                                 ctypes.POINTER(vp)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -168,6 +172,24 @@ def subm3d_forward(nbr, tile_mask, n: int, feats, weight, out, cin: int, cout: i
                             _ptr(out), int(cin), int(cout), int(dtype), 1 if flip else 0,
                             int(act), _stream(stream))
     _check(st, "subm3d_forward")
+
+
+def subm3d_forward_map(handle: MapHandle, feats, weight, out, cin: int, cout: int, dtype: int,
+                       flip: bool, act: int, stream=None) -> None:
+    """Enqueue one layer's forward over a built map (x-run kernel for bf16 with
+    Cin % 64 == 0); raises Subm3dError on an argument error."""
+    st = lib.subm3d_forward_map(handle.ptr, _ptr(feats), _ptr(weight), _ptr(out), int(cin),
+                                int(cout), int(dtype), 1 if flip else 0, int(act),
+                                _stream(stream))
+    _check(st, "subm3d_forward_map")
+
+
+def subm3d_map_run_layout(handle: MapHandle):
+    """Device pointers (position table, E index table, header) of the map."""
+    pos, et, hdr = ctypes.c_void_p(), ctypes.c_void_p(), ctypes.c_void_p()
+    _check(lib.subm3d_map_run_layout(handle.ptr, ctypes.byref(pos), ctypes.byref(et),
+                                     ctypes.byref(hdr)), "subm3d_map_run_layout")
+    return int(pos.value), int(et.value), int(hdr.value)
 
 
 def subm3d_device_status(stream=None) -> int:

@@ -26,7 +26,21 @@ constexpr size_t kDirectTableMaxBytes = size_t(64) << 20;
 struct MapOptions {
   bool force_hash = false;
   uint64_t forced_capacity = 0;  // a power of two, or 0
+  bool run_layout = true;        // also build the x-run layout (subm3d_forward_map)
 };
+
+// x-run position layout used by the run-padded forward.  Voxels are laid out
+// in row order on a line of positions; every run of x-adjacent voxels (same
+// b, z, y; consecutive x and consecutive rows) is preceded by two pad
+// positions: the right neighbour slot of the previous run and the left
+// neighbour slot of this one.  Positions are cut into tiles of kPosTile.
+constexpr int kPosTile = 256;
+// Row stride (int32) of the E index table: for a tile and an offset pair
+// (dz, dy), entries 0..257 are the feature rows of positions -1..256.
+constexpr int kEtStride = 260;
+constexpr int kRunBlock = 1024;  // voxels per block of the run-count scan
+// Tags of a position-table entry (row * 4 + tag); -1 is an empty position.
+constexpr int kPosVoxel = 0, kPosLeftPad = 1, kPosRightPad = 2;
 
 // Placement of the map build's pieces inside the caller's workspace.
 struct MapLayout {
@@ -39,6 +53,15 @@ struct MapLayout {
   size_t table_off = 0;     // direct: int32 [cells]; hash: uint64 [capacity] (slots or keys)
   size_t table_bytes = 0;   // bytes of the table (a multiple of 16)
   size_t rows_off = 0;      // hash, wide keys only: int32 rows [capacity]
+  // run layout (all kinds)
+  size_t runcnt_off = 0;    // int32 [n_run_blocks]: run starts per block, then offsets
+  size_t hdr_off = 0;       // int32 [4]: runs, position tiles, positions, 0
+  size_t pos_off = 0;       // int32 [pos_max]: position table (row * 4 + tag, or -1)
+  size_t pos_bytes = 0;
+  size_t et_off = 0;        // int32 [ptile_max][9][kEtStride]: E index table
+  int64_t n_run_blocks = 0;
+  int64_t pos_max = 0;      // positions reserved: 3N rounded up to whole tiles
+  int64_t ptile_max = 0;
   size_t total = 0;         // bytes
   int64_t n_tiles = 0;
 };
@@ -63,5 +86,13 @@ cudaError_t launch_forward_bf16(const int32_t* nbr, const uint32_t* tile_mask, i
                                 const void* feats, const void* weight, void* out, int32_t cin,
                                 int32_t cout, int32_t flip, int32_t act, int32_t* err_word,
                                 cudaStream_t stream);
+
+// bf16 forward over the x-run position layout (forward_bf16_runs_sm100.cu);
+// Cin a multiple of 64, Cout a multiple of 16.
+cudaError_t launch_forward_bf16_runs(const int32_t* pos, const int32_t* etable,
+                                     const int32_t* header, int64_t max_tiles, const void* feats,
+                                     const void* weight, void* out, int32_t cin, int32_t cout,
+                                     int32_t flip, int32_t act, int32_t* err_word,
+                                     cudaStream_t stream);
 
 }  // namespace subm3d

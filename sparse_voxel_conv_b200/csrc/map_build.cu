@@ -78,12 +78,14 @@ __device__ __forceinline__ int64_t cell_of(int b, int z, int y, int x, int grid)
   return ((static_cast<int64_t>(b) * grid + z) * grid + y) * grid + x;
 }
 
-// Fills `words16` 16-byte words of the table with all-ones and zeroes the status word.
-__global__ void map_init(uint4* table, size_t words16, uint32_t* status) {
+// Fills two regions (`words16a`, `words16b` 16-byte words) with all-ones --
+// the lookup table and the position table -- and zeroes the status word.
+__global__ void map_init(uint4* a, size_t words16a, uint4* b, size_t words16b, uint32_t* status) {
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   const size_t t0 = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const uint4 ones = make_uint4(~0u, ~0u, ~0u, ~0u);
-  for (size_t t = t0; t < words16; t += stride) table[t] = ones;
+  for (size_t t = t0; t < words16a; t += stride) a[t] = ones;
+  for (size_t t = t0; t < words16b; t += stride) b[t] = ones;
   if (t0 == 0) *status = 0u;
 }
 
@@ -238,6 +240,151 @@ __global__ void __launch_bounds__(kTileRows)
   }
 }
 
+// ----------------------------------------------------------- run layout ----
+// A voxel starts a run unless the previous row is its x-1 neighbour (same b, z,
+// y and x one less).
+
+__device__ __forceinline__ bool run_start(const int4* coords, int64_t v) {
+  if (v == 0) return true;
+  const int4 p = __ldg(coords + v - 1);
+  const int4 c = __ldg(coords + v);
+  return !(p.x == c.x && p.y == c.y && p.z == c.z && p.w + 1 == c.w);
+}
+
+// Run starts per block of kRunBlock rows.
+__global__ void __launch_bounds__(256) map_run_count(const int4* __restrict__ coords, int64_t n,
+                                                     int32_t* __restrict__ cnt) {
+  __shared__ int32_t s_sum[8];
+  int32_t c = 0;
+  for (int i = 0; i < kRunBlock / 256; ++i) {
+    const int64_t v = static_cast<int64_t>(blockIdx.x) * kRunBlock + i * 256 + threadIdx.x;
+    if (v < n && run_start(coords, v)) ++c;
+  }
+  c = __reduce_add_sync(0xFFFFFFFFu, c);
+  if ((threadIdx.x & 31) == 0) s_sum[threadIdx.x >> 5] = c;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int32_t t = 0;
+    for (int w = 0; w < 8; ++w) t += s_sum[w];
+    cnt[blockIdx.x] = t;
+  }
+}
+
+// Exclusive scan of the per-block run counts (one block), and the header:
+// hdr[0] = runs, hdr[1] = position tiles, hdr[2] = positions.
+__global__ void __launch_bounds__(1024) map_run_scan(int32_t* __restrict__ cnt, int64_t n_blocks,
+                                                     int64_t n, int32_t* __restrict__ hdr) {
+  __shared__ int32_t s_warp[32];
+  __shared__ int64_t s_carry;
+  if (threadIdx.x == 0) s_carry = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int64_t base = 0; base < n_blocks; base += 1024) {
+    const int64_t i = base + threadIdx.x;
+    const int32_t x = i < n_blocks ? cnt[i] : 0;
+    int32_t incl = x;
+    for (int d = 1; d < 32; d <<= 1) {
+      const int32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+      if (lane >= d) incl += y;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int32_t w = s_warp[lane];
+      for (int d = 1; d < 32; d <<= 1) {
+        const int32_t y = __shfl_up_sync(0xFFFFFFFFu, w, d);
+        if (lane >= d) w += y;
+      }
+      s_warp[lane] = w;  // inclusive over warps
+    }
+    __syncthreads();
+    const int32_t before = (warp > 0 ? s_warp[warp - 1] : 0) + incl - x;
+    const int64_t carry = s_carry;
+    if (i < n_blocks) cnt[i] = static_cast<int32_t>(carry + before);
+    __syncthreads();
+    if (threadIdx.x == 0) s_carry = carry + s_warp[31];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const int64_t runs = s_carry;
+    const int64_t positions = n + 2 * runs;
+    hdr[0] = static_cast<int32_t>(runs);
+    hdr[1] = static_cast<int32_t>((positions + kPosTile - 1) / kPosTile);
+    hdr[2] = static_cast<int32_t>(positions);
+    hdr[3] = 0;
+  }
+}
+
+// Places every voxel v at position v + 2 R(v), R(v) = run starts among rows
+// 0..v, with the left-pad slot before a run's first voxel and the right-pad
+// slot after its last.  Each thread handles 4 consecutive rows.
+__global__ void __launch_bounds__(256) map_run_place(const int4* __restrict__ coords, int64_t n,
+                                                     const int32_t* __restrict__ blk_off,
+                                                     int32_t* __restrict__ pos) {
+  __shared__ int32_t s_warp[8];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t v0 = static_cast<int64_t>(blockIdx.x) * kRunBlock + 4 * threadIdx.x;
+  bool rs[5];
+#pragma unroll
+  for (int i = 0; i < 5; ++i) rs[i] = (v0 + i < n) ? run_start(coords, v0 + i) : true;
+  int32_t local = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) local += (v0 + i < n && rs[i]) ? 1 : 0;
+  int32_t incl = local;
+  for (int d = 1; d < 32; d <<= 1) {
+    const int32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+    if (lane >= d) incl += y;
+  }
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  int32_t warp_before = 0;
+  for (int w = 0; w < warp; ++w) warp_before += s_warp[w];
+  int64_t r = blk_off[blockIdx.x] + warp_before + incl - local;  // run starts before v0
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t v = v0 + i;
+    if (v >= n) break;
+    if (rs[i]) ++r;
+    const int64_t p = v + 2 * r;
+    pos[p] = static_cast<int32_t>(v * 4 + kPosVoxel);
+    if (rs[i]) pos[p - 1] = static_cast<int32_t>(v * 4 + kPosLeftPad);
+    if (v + 1 == n || rs[i + 1]) pos[p + 1] = static_cast<int32_t>(v * 4 + kPosRightPad);
+  }
+}
+
+// E index table: for position tile t and offset pair (dz, dy), entry i is the
+// feature row of E row i-1: a voxel position takes its (dz, dy, 0) neighbour,
+// a left pad its voxel's (dz, dy, -1) neighbour, a right pad the (dz, dy, +1)
+// one; entry 0 (row -1) and entry 257 (row 256) are the (dz, dy, -1) and
+// (dz, dy, +1) neighbours of the voxels at positions 0 and 255.  So for the
+// voxel at position p, E rows p-1, p, p+1 hold its dx = -1, 0, +1 neighbours.
+__global__ void __launch_bounds__(kEtStride) map_etable(const int32_t* __restrict__ pos,
+                                                         const int32_t* __restrict__ nbr,
+                                                         const int32_t* __restrict__ hdr,
+                                                         int32_t* __restrict__ et) {
+  const int64_t t = blockIdx.x;
+  if (t >= hdr[1]) return;
+  const int i = threadIdx.x;  // 0 .. kEtStride-1
+  int64_t v = -1;
+  int dx = 0;
+  if (i == 0 || i == 257) {
+    const int32_t e = pos[t * kPosTile + (i == 0 ? 0 : kPosTile - 1)];
+    if (e >= 0 && (e & 3) == kPosVoxel) {
+      v = e >> 2;
+      dx = i == 0 ? -1 : 1;
+    }
+  } else if (i < 257) {
+    const int32_t e = pos[t * kPosTile + i - 1];
+    if (e >= 0) {
+      v = e >> 2;
+      dx = (e & 3) == kPosLeftPad ? -1 : ((e & 3) == kPosRightPad ? 1 : 0);
+    }
+  }
+#pragma unroll
+  for (int dzdy = 0; dzdy < 9; ++dzdy)
+    et[(t * 9 + dzdy) * kEtStride + i] = v >= 0 ? __ldg(nbr + v * kKvol + 3 * dzdy + dx + 1) : -1;
+}
+
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 }  // namespace
@@ -265,15 +412,31 @@ bool map_layout(int64_t n, int32_t grid_dim, int32_t batch, const MapOptions& op
   lay.status_off = 0;
   lay.mask_off = 256;
   lay.table_off = align_up(lay.mask_off + static_cast<size_t>(lay.n_tiles) * 4, 256);
+  size_t end = 0;
   if (lay.kind == MapKind::kDirect) {
     lay.table_bytes = align_up(lay.cells * 4, 256);
     lay.rows_off = lay.table_off + lay.table_bytes;
-    lay.total = lay.rows_off;
+    end = lay.rows_off;
   } else {
     lay.table_bytes = cap * 8;
     lay.rows_off = align_up(lay.table_off + lay.table_bytes, 256);
-    lay.total = lay.compact ? lay.rows_off : align_up(lay.rows_off + cap * 4, 256);
+    end = lay.compact ? lay.rows_off : align_up(lay.rows_off + cap * 4, 256);
   }
+  if (!opt.run_layout) {  // nbr and tile masks only
+    lay.runcnt_off = lay.hdr_off = lay.pos_off = lay.et_off = end;
+    lay.total = end;
+    *out = lay;
+    return true;
+  }
+  lay.n_run_blocks = (n + kRunBlock - 1) / kRunBlock;
+  lay.pos_max = static_cast<int64_t>(align_up(static_cast<size_t>(3 * n), kPosTile)) + kPosTile;
+  lay.ptile_max = lay.pos_max / kPosTile;
+  lay.runcnt_off = end;
+  lay.hdr_off = align_up(lay.runcnt_off + static_cast<size_t>(lay.n_run_blocks) * 4, 256);
+  lay.pos_off = lay.hdr_off + 256;
+  lay.pos_bytes = static_cast<size_t>(lay.pos_max) * 4;
+  lay.et_off = align_up(lay.pos_off + lay.pos_bytes, 256);
+  lay.total = align_up(lay.et_off + static_cast<size_t>(lay.ptile_max) * 9 * kEtStride * 4, 256);
   *out = lay;
   return true;
 }
@@ -286,12 +449,16 @@ cudaError_t launch_map_build(const int32_t* coords, int64_t n, int32_t grid_dim,
   auto* mask = reinterpret_cast<uint32_t*>(ws + lay.mask_off);
   auto* table = ws + lay.table_off;
   const size_t words16 = lay.table_bytes / 16;
+  const size_t pos_words16 = lay.pos_bytes / 16;
+  auto* pos = reinterpret_cast<int32_t*>(ws + lay.pos_off);
   {
-    size_t blocks = (words16 + 255) / 256;
+    const size_t work = words16 > pos_words16 ? words16 : pos_words16;
+    size_t blocks = (work + 255) / 256;
     if (blocks > 148 * 8) blocks = 148 * 8;
     if (blocks == 0) blocks = 1;
-    map_init<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(reinterpret_cast<uint4*>(table),
-                                                               words16, status);
+    map_init<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        reinterpret_cast<uint4*>(table), words16, reinterpret_cast<uint4*>(pos), pos_words16,
+        status);
   }
   if (n == 0) return cudaGetLastError();
   const auto* c4 = reinterpret_cast<const int4*>(coords);
@@ -321,6 +488,16 @@ cudaError_t launch_map_build(const int32_t* coords, int64_t n, int32_t grid_dim,
     map_query<Kind::kWide><<<q_blocks, kTileRows, 0, stream>>>(c4, n, grid_dim, batch, t, nbr,
                                                                mask, status);
   }
+  if (lay.ptile_max == 0) return cudaGetLastError();
+  // x-run position layout and E index table for the run-padded forward
+  auto* runcnt = reinterpret_cast<int32_t*>(ws + lay.runcnt_off);
+  auto* hdr = reinterpret_cast<int32_t*>(ws + lay.hdr_off);
+  auto* et = reinterpret_cast<int32_t*>(ws + lay.et_off);
+  const unsigned rblocks = static_cast<unsigned>(lay.n_run_blocks);
+  map_run_count<<<rblocks, 256, 0, stream>>>(c4, n, runcnt);
+  map_run_scan<<<1, 1024, 0, stream>>>(runcnt, lay.n_run_blocks, n, hdr);
+  map_run_place<<<rblocks, 256, 0, stream>>>(c4, n, runcnt, pos);
+  map_etable<<<static_cast<unsigned>(lay.ptile_max), kEtStride, 0, stream>>>(pos, nbr, hdr, et);
   return cudaGetLastError();
 }
 

@@ -71,6 +71,7 @@ subm3d_status subm3d_build_map_noalloc(const int32_t* coords, int64_t n, int32_t
   if (n > static_cast<int64_t>(kMaxVoxels)) return SUBM3D_E_UNSUPPORTED;  // beyond the scratch
   subm3d::MapOptions opt;
   opt.force_hash = true;  // the hash table's size depends on N only, never on the volume
+  opt.run_layout = false;  // nbr and tile masks are all subm3d_forward() needs
   subm3d::MapLayout lay;
   if (!subm3d::map_layout(n, grid_dim, batch, opt, &lay))
     return (grid_dim < 1 || batch < 1) ? SUBM3D_E_INVALID : SUBM3D_E_UNSUPPORTED;

@@ -18,6 +18,10 @@ struct subm3d_map {
   const int32_t* nbr;
   const uint32_t* tile_mask;
   const uint32_t* status_word;
+  const int32_t* pos;     // x-run position table
+  const int32_t* et;      // E index table
+  const int32_t* hdr;     // [runs, position tiles, positions, 0]
+  int64_t ptile_max;      // position tiles reserved in the workspace
   int64_t n;
   int32_t grid_dim;
   int32_t batch;
@@ -124,6 +128,10 @@ subm3d_status subm3d_build_map(const int32_t* coords, int64_t n, int32_t grid_di
   h->nbr = nbr;
   h->tile_mask = reinterpret_cast<const uint32_t*>(ws + lay.mask_off);
   h->status_word = reinterpret_cast<const uint32_t*>(ws + lay.status_off);
+  h->pos = reinterpret_cast<const int32_t*>(ws + lay.pos_off);
+  h->et = reinterpret_cast<const int32_t*>(ws + lay.et_off);
+  h->hdr = reinterpret_cast<const int32_t*>(ws + lay.hdr_off);
+  h->ptile_max = lay.ptile_max;
   h->n = n;
   h->grid_dim = grid_dim;
   h->batch = batch;
@@ -196,6 +204,42 @@ subm3d_status subm3d_forward(const int32_t* nbr, const uint32_t* tile_mask, int6
   if (!err) return SUBM3D_E_CUDA;
   const cudaError_t e = subm3d::launch_forward_bf16(nbr, tile_mask, n, feats, weight, out, cin,
                                                     cout, flip01, act01, err, s);
+  if (e == cudaErrorNotSupported) return SUBM3D_E_UNSUPPORTED;
+  return e == cudaSuccess ? SUBM3D_OK : SUBM3D_E_CUDA;
+}
+
+subm3d_status subm3d_map_run_layout(const subm3d_map* map, const int32_t** pos,
+                                    const int32_t** etable, const int32_t** header) {
+  if (!map || !pos || !etable || !header) return SUBM3D_E_INVALID;
+  *pos = map->pos;
+  *etable = map->et;
+  *header = map->hdr;
+  return SUBM3D_OK;
+}
+
+subm3d_status subm3d_forward_map(const subm3d_map* map, const void* feats, const void* weight,
+                                 void* out, int32_t cin, int32_t cout, subm3d_dtype dtype,
+                                 int32_t flip, subm3d_act act, void* stream) {
+  if (!map) return SUBM3D_E_INVALID;
+  const int64_t n = map->n;
+  const bool runs = dtype == SUBM3D_BF16 && n > 0 && cin % 64 == 0 && cout % 16 == 0 &&
+                    feats && weight && out && aligned(feats, 16) && aligned(weight, 16) &&
+                    aligned(out, 16) && (act == SUBM3D_ACT_NONE || act == SUBM3D_ACT_GELU);
+  if (!runs)
+    return subm3d_forward(map->nbr, map->tile_mask, n, feats, weight, out, cin, cout, dtype, flip,
+                          act, stream);
+  const auto* fb = static_cast<const uint8_t*>(feats);
+  const auto* ob = static_cast<const uint8_t*>(out);
+  if (fb < ob + static_cast<size_t>(n) * cout * 2 && ob < fb + static_cast<size_t>(n) * cin * 2)
+    return SUBM3D_E_INVALID;  // out overlaps feats
+  const int sm100 = device_is_sm100(nullptr);
+  if (sm100 < 0) return SUBM3D_E_CUDA;
+  if (sm100 == 0) return SUBM3D_E_UNSUPPORTED;
+  int32_t* err = device_error_word();
+  if (!err) return SUBM3D_E_CUDA;
+  const cudaError_t e = subm3d::launch_forward_bf16_runs(
+      map->pos, map->et, map->hdr, map->ptile_max, feats, weight, out, cin, cout, flip ? 1 : 0,
+      act == SUBM3D_ACT_GELU ? 1 : 0, err, static_cast<cudaStream_t>(stream));
   if (e == cudaErrorNotSupported) return SUBM3D_E_UNSUPPORTED;
   return e == cudaSuccess ? SUBM3D_OK : SUBM3D_E_CUDA;
 }

@@ -76,11 +76,14 @@ def tile_mask_tensor(h: MapHandle) -> torch.Tensor:
 
 def forward(h: MapHandle, feats: torch.Tensor, weight: torch.Tensor, flip: bool = False,
             act: str | None = None, out: torch.Tensor | None = None, stream=None,
-            use_tile_mask: bool = True) -> torch.Tensor:
+            use_tile_mask: bool = True, kernel: str = "auto") -> torch.Tensor:
     """One SubMConv3d layer: out[i] = act(sum_k Wf[:,k,:] . feats[nbr[i,k]]).
 
     feats: [N, Cin] float32 or bfloat16; weight: KRSC [Cout, 3, 3, 3, Cin] (or
     [Cout, 27, Cin]) of the same dtype.  Returns [N, Cout] of that dtype.
+    kernel: "auto" runs subm3d_forward_map (the x-run kernel for bf16 with
+    Cin % 64 == 0); "gather" runs subm3d_forward on nbr and the tile masks
+    (use_tile_mask=False: no masks).
     """
     if feats.dtype not in _DTYPES:
         raise ValueError(f"unsupported feature dtype {feats.dtype}")
@@ -94,10 +97,29 @@ def forward(h: MapHandle, feats: torch.Tensor, weight: torch.Tensor, flip: bool 
         raise ValueError("weight must be KRSC [Cout, 3, 3, 3, Cin]")
     if out is None:
         out = torch.empty((n, cout), dtype=feats.dtype, device=feats.device)
+    if kernel == "auto" and use_tile_mask:
+        _abi.subm3d_forward_map(h, feats, weight, out, cin, cout, _DTYPES[feats.dtype], flip,
+                                _ACTS[act], stream)
+        return out
+    if kernel not in ("auto", "gather"):
+        raise ValueError(f"unknown kernel {kernel!r}")
     mask_ptr = _abi.subm3d_map_tile_mask(h) if use_tile_mask else None
     _abi.subm3d_forward(h.nbr, mask_ptr, n, feats, weight, out, cin, cout, _DTYPES[feats.dtype],
                         flip, _ACTS[act], stream)
     return out
+
+
+def run_layout_tensors(h: MapHandle):
+    """(position table, E index table [tiles, 9, 260], header) as int32 views
+    of the map's workspace; call after the build has completed."""
+    pos_p, et_p, hdr_p = _abi.subm3d_map_run_layout(h)
+    base = h.workspace.data_ptr()
+    ws = h.workspace
+    hdr = ws[hdr_p - base:hdr_p - base + 16].view(torch.int32)
+    tiles = int(hdr[1].item())
+    pos = ws[pos_p - base:pos_p - base + 4 * 256 * tiles].view(torch.int32)
+    et = ws[et_p - base:et_p - base + 4 * tiles * 9 * 260].view(torch.int32).view(tiles, 9, 260)
+    return pos, et, hdr
 
 
 class SparseTensor:

@@ -43,6 +43,20 @@ def test_version_and_strings(abi):
     assert abi.subm3d_status_string(99) == "unknown status"
 
 
+def _expected_ws(n, table_bytes):
+    """Workspace layout: 256-B status block, tile masks, lookup table, run
+    counts, 256-B header, position table (3N rounded to 256, + 256), E index
+    table (one [9, 260] int32 block per 256 positions); 256-B aligned parts."""
+    up = lambda v: (v + 255) // 256 * 256
+    head = up(256 + 4 * ((n + 127) // 128))
+    runcnt = 4 * ((n + 1023) // 1024)
+    pos_max = up(3 * n) + 256
+    after_table = up(head + table_bytes)
+    pos_off = up(after_table + runcnt) + 256
+    et_off = up(pos_off + 4 * pos_max)
+    return up(et_off + (pos_max // 256) * 9 * 260 * 4)
+
+
 def test_workspace_bytes(abi, monkeypatch):
     monkeypatch.delenv("SUBM3D_MAP_KIND", raising=False)
     monkeypatch.delenv("SUBM3D_TABLE_CAPACITY", raising=False)
@@ -50,17 +64,16 @@ def test_workspace_bytes(abi, monkeypatch):
     assert f(-1, 16, 1) == 0 and f(10, 0, 1) == 0 and f(10, 16, 0) == 0
     assert f(10, 70000, 1) == 0 and f(10, 16, 70000) == 0
     n = 329839
-    head = 256 + 4 * ((n + 127) // 128)
     # direct table: one int32 per cell of a volume up to 64 MB
-    assert head + 4 * 128 ** 3 <= f(n, 128, 1) < head + 4 * 128 ** 3 + 1024
-    assert head + 4 * 256 ** 3 <= f(n, 256, 1) < head + 4 * 256 ** 3 + 1024
+    assert f(n, 128, 1) == _expected_ws(n, 4 * 128 ** 3)
+    assert f(n, 256, 1) == _expected_ws(n, 4 * 256 ** 3)
     # larger volumes: hash table, 8-byte slots, capacity max(1024, pow2 >= 2N)
-    assert head + 8 * (1 << 20) <= f(n, 512, 1) < head + 8 * (1 << 20) + 1024
+    assert f(n, 512, 1) == _expected_ws(n, 8 * (1 << 20))
     # wide keys (batch > 4 or grid > 1024) add a 4-byte row array
-    assert f(n, 2048, 1) >= head + 12 * (1 << 20)
+    assert f(n, 2048, 1) == _expected_ws(n, 12 * (1 << 20))
     monkeypatch.setenv("SUBM3D_MAP_KIND", "hash")
-    assert head + 8 * (1 << 20) <= f(n, 128, 1) < head + 8 * (1 << 20) + 1024
-    assert f(n, 128, 5) >= head + 12 * (1 << 20)
+    assert f(n, 128, 1) == _expected_ws(n, 8 * (1 << 20))
+    assert f(n, 128, 5) == _expected_ws(n, 12 * (1 << 20))
     assert f(0, 16, 1) > 0
 
 

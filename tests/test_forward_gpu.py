@@ -212,3 +212,21 @@ def test_bf16_stack_end_to_end_small(S):
         ref = C.forward(nbr, ref, np.asarray(w, np.float64), act="gelu" if l < 3 else None,
                         round_to_bf16=True)
     assert_close(st.feats.float().cpu().numpy(), ref, RTOL_BF16, "stack e2e")
+
+
+@pytest.mark.parametrize("name", ["shell_bf16", "headline"])
+@pytest.mark.parametrize("flip", [False, True])
+def test_bf16_both_kernels_agree_with_oracle(S, name, flip):
+    """The x-run kernel (subm3d_forward_map) and the per-offset gather kernel
+    (subm3d_forward) on the same map and inputs, both against the oracle."""
+    wl = WL.make_workload(name)
+    x, w = wl.features(), wl.weights()[0]
+    h = S.build_map(torch.from_numpy(wl.coords).cuda(), wl.grid_dim, wl.batch)
+    xt = torch.from_numpy(x).cuda().to(torch.bfloat16)
+    wt = torch.from_numpy(w).cuda().to(torch.bfloat16)
+    rows = sample_rows(wl.n, 6000, seed=4)
+    ref = _oracle(wl.coords, wl.grid_dim, wl.batch, x, w, flip=flip, bf16_out=True, rows=rows)
+    for kernel in ("auto", "gather"):
+        y = S.forward(h, xt, wt, flip=flip, kernel=kernel).float().cpu().numpy()
+        assert S._abi.subm3d_device_status() == 0
+        assert_close(y[rows], ref, RTOL_BF16, f"{name} {kernel} flip={flip}")

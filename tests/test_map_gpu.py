@@ -125,3 +125,27 @@ def test_map_async_status_and_reuse(S):
     nbr = torch.empty((c2.shape[0], 27), dtype=torch.int32, device="cuda")
     h2 = S.build_map(c2, 16, 1, nbr=nbr, workspace=h1.workspace)
     assert np.array_equal(h2.nbr.cpu().numpy(), C.build_map(WL.tiny_coords(), 16, 1))
+
+
+@pytest.mark.parametrize("name", ["tiny", "shell", "headline", "batched"])
+def test_run_layout_invariant(S, kind, name):
+    """Every voxel sits at one position p of the x-run layout, and for each of
+    its 27 offsets (dz, dy, dx) the E index entry of (tile, dz-dy) at row p+dx
+    is its neighbour nbr[v][k] -- the property the x-run forward relies on."""
+    wl = WL.make_workload(name)
+    h = S.build_map(torch.from_numpy(wl.coords).cuda(), wl.grid_dim, wl.batch)
+    pos, et, hdr = (t.cpu().numpy() for t in S.run_layout_tensors(h))
+    ref = C.build_map(wl.coords, wl.grid_dim, wl.batch)
+    n = wl.n
+    c = wl.coords.astype(np.int64)
+    same = (c[1:, 0] == c[:-1, 0]) & (c[1:, 1] == c[:-1, 1]) & (c[1:, 2] == c[:-1, 2]) & \
+        (c[1:, 3] == c[:-1, 3] + 1)
+    runs = int((~same).sum()) + 1
+    assert hdr[0] == runs and hdr[2] == n + 2 * runs and hdr[1] == (n + 2 * runs + 255) // 256
+    voxel_pos = np.nonzero((pos >= 0) & ((pos & 3) == 0))[0]
+    assert np.array_equal(pos[voxel_pos] >> 2, np.arange(n))      # every row once, in order
+    tile, local = voxel_pos // 256, voxel_pos % 256
+    for k in range(27):
+        dzdy, dx = k // 3, k % 3 - 1
+        got = et[tile, dzdy, local + dx + 1]
+        assert np.array_equal(got, ref[:, k]), f"offset {k}"

@@ -37,9 +37,9 @@ sys.path.insert(0, ROOT)
 METRIC = "SubMConv3d fwd voxels/s and TFLOP/s at 128^3/128ch bf16; % of B200 roofline"
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# Kernels one map build launches: table init, insert, query, and the x-run
-# position layout (run count, run scan, placement, E index table).
-MAP_LAUNCHES = 7
+# Kernels one map build launches: table init, insert, and the query, which
+# also lays out the x-run positions and the E index table.
+MAP_LAUNCHES = 3
 
 # Algorithmic bytes of the map build per voxel: int32 (b,z,y,x) in + int32 [27] out.
 MAP_BYTES_PER_VOXEL = 16 + 27 * 4

@@ -82,9 +82,10 @@ SUBM3D_API const char* subm3d_status_string(int32_t status);
  * and the lookup table -- a direct-address table of batch * grid_dim^3 int32
  * cells when that is at most 64 MB, else an open-addressing hash table of at
  * least 2N slots (8 bytes each, 12 with batch > 4 or grid_dim > 1024) -- and
- * the x-run layout of subm3d_forward_map(): per-1024-row run counts, a header,
- * a position table of 3N int32 (rounded up) and an E index table of
- * 9 x 260 int32 per 256 positions (~110 bytes per voxel).  Host-only, no CUDA
+ * for N < 2^29 the x-run layout of subm3d_forward_map(): one 8-byte scan word
+ * per 128-row tile, a header, a position table of 3N int32 (rounded up) and an
+ * E index table of 9 x 260 int32 per 256 positions (~110 bytes per voxel).
+ * Host-only, no CUDA
  * call.  Returns 0 for arguments subm3d_build_map() would
  * reject (N < 0, grid_dim < 1 or > 65535, batch < 1 or > 65535).
  */
@@ -111,8 +112,10 @@ SUBM3D_API size_t subm3d_map_workspace_bytes(int64_t n, int32_t grid_dim, int32_
  * does not depend on the hash layout.  Coordinates outside the volume or
  * repeated are reported by subm3d_map_status(); until it returns SUBM3D_OK the
  * contents of nbr are unspecified.  Besides nbr and the tile masks the build
- * writes the x-run position layout that subm3d_forward_map() uses.  Enqueues 7
- * kernels; no allocation.
+ * writes, for N < 2^29, the x-run position layout that subm3d_forward_map()
+ * uses; the query kernel's tiles take their run offsets from one another by a
+ * single-pass scan whose waits are bounded (SUBM3D_E_TIMEOUT if one runs out).
+ * Enqueues 3 kernels; no allocation.
  * Testing knobs, read from the environment by this function and by
  * subm3d_map_workspace_bytes() alike: SUBM3D_MAP_KIND=hash selects the hash
  * table even where the direct table fits; SUBM3D_TABLE_CAPACITY=<slots> caps
@@ -125,8 +128,9 @@ SUBM3D_API subm3d_status subm3d_build_map(const int32_t* coords, int64_t n, int3
 
 /*
  * Synchronizes the map's stream and returns the device-detected status of the
- * build: SUBM3D_OK, SUBM3D_E_RANGE, SUBM3D_E_DUPLICATE or SUBM3D_E_TABLE_FULL
- * (first in that order of precedence), or SUBM3D_E_CUDA.  Blocking.
+ * build: SUBM3D_OK, SUBM3D_E_RANGE, SUBM3D_E_DUPLICATE, SUBM3D_E_TABLE_FULL or
+ * SUBM3D_E_TIMEOUT (first in that order of precedence), or SUBM3D_E_CUDA.
+ * Blocking.
  */
 SUBM3D_API subm3d_status subm3d_map_status(const subm3d_map* map);
 
@@ -212,7 +216,8 @@ SUBM3D_API subm3d_status subm3d_build_map_noalloc(const int32_t* coords, int64_t
 /*
  * Forward of one layer over a built map -- the same op and arguments as
  * subm3d_forward(), with N, nbr and the masks taken from the map.  For bf16
- * with Cin a multiple of 64 it runs the x-run kernel, which uses the map's
+ * with Cin a multiple of 64 (and a map of N < 2^29) it runs the x-run kernel,
+ * which uses the map's
  * position layout: voxels on a line of positions in row order, two pad
  * positions before every run of x-adjacent voxels, tiles of 256 positions,
  * and per tile and (dz, dy) one gathered tile of feature rows whose rows
@@ -233,6 +238,7 @@ SUBM3D_API subm3d_status subm3d_forward_map(const subm3d_map* map, const void* f
  * (int32 [tiles][9][260]: entry i of (tile, dz-dy) is the feature row of
  * gathered row i-1, or -1) and a 4-int header [runs, tiles, positions, 0].
  * Valid once the build has completed on its stream.  Host-only.
+ * SUBM3D_E_UNSUPPORTED when the map has no run layout (N >= 2^29).
  */
 SUBM3D_API subm3d_status subm3d_map_run_layout(const subm3d_map* map, const int32_t** pos,
                                                const int32_t** etable, const int32_t** header);

@@ -12,6 +12,7 @@ namespace subm3d {
 constexpr uint32_t kErrRange = 1u;
 constexpr uint32_t kErrDuplicate = 2u;
 constexpr uint32_t kErrTableFull = 4u;
+constexpr uint32_t kErrTimeout = 8u;  // a bounded wait of the run-offset scan ran out
 
 constexpr int kTileRows = 128;  // rows per tile-mask word
 constexpr int kKvol = 27;
@@ -38,7 +39,9 @@ constexpr int kPosTile = 256;
 // Row stride (int32) of the E index table: for a tile and an offset pair
 // (dz, dy), entries 0..257 are the feature rows of positions -1..256.
 constexpr int kEtStride = 260;
-constexpr int kRunBlock = 1024;  // voxels per block of the run-count scan
+// The run layout is built for N < 2^29, so that positions (< 3N + 512) and
+// position-table entries (row * 4 + tag) fit int32; larger maps go without it.
+constexpr int64_t kRunLayoutMaxRows = int64_t(1) << 29;
 // Tags of a position-table entry (row * 4 + tag); -1 is an empty position.
 constexpr int kPosVoxel = 0, kPosLeftPad = 1, kPosRightPad = 2;
 
@@ -54,12 +57,11 @@ struct MapLayout {
   size_t table_bytes = 0;   // bytes of the table (a multiple of 16)
   size_t rows_off = 0;      // hash, wide keys only: int32 rows [capacity]
   // run layout (all kinds)
-  size_t runcnt_off = 0;    // int32 [n_run_blocks]: run starts per block, then offsets
-  size_t hdr_off = 0;       // int32 [4]: runs, position tiles, positions, 0
+  size_t lb_off = 0;        // uint64 [n_tiles]: run-offset scan words of the query tiles
+  size_t hdr_off = 0;       // int32 [8]: runs, position tiles, positions, 0, tile ticket
   size_t pos_off = 0;       // int32 [pos_max]: position table (row * 4 + tag, or -1)
   size_t pos_bytes = 0;
   size_t et_off = 0;        // int32 [ptile_max][9][kEtStride]: E index table
-  int64_t n_run_blocks = 0;
   int64_t pos_max = 0;      // positions reserved: 3N rounded up to whole tiles
   int64_t ptile_max = 0;
   size_t total = 0;         // bytes
@@ -70,7 +72,8 @@ struct MapLayout {
 bool map_layout(int64_t n, int32_t grid_dim, int32_t batch, const MapOptions& opt,
                 MapLayout* out);
 
-// Enqueues the three map-build kernels on `stream`.  Returns the launch error.
+// Enqueues the three map-build kernels (init, insert, query) on `stream`.
+// Returns the launch error.
 cudaError_t launch_map_build(const int32_t* coords, int64_t n, int32_t grid_dim, int32_t batch,
                              int32_t* nbr, void* workspace, const MapLayout& lay,
                              cudaStream_t stream);

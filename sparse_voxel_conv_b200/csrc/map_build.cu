@@ -24,7 +24,7 @@
 // voxel: 16-byte coordinate load, range check, insert), map_query (one block
 // per 128-row tile, one thread per voxel: 27 lookups into shared memory, then
 // the [128, 27] block and the tile's offset mask are written with coalesced
-// stores; no atomics on the output).
+// stores; no atomics on the output; and the tile's share of the x-run layout).
 #include <cuda_runtime.h>
 
 #include "internal.h"
@@ -79,14 +79,20 @@ __device__ __forceinline__ int64_t cell_of(int b, int z, int y, int x, int grid)
 }
 
 // Fills two regions (`words16a`, `words16b` 16-byte words) with all-ones --
-// the lookup table and the position table -- and zeroes the status word.
-__global__ void map_init(uint4* a, size_t words16a, uint4* b, size_t words16b, uint32_t* status) {
+// the lookup table and the run layout's look-back words -- and zeroes the
+// status word and the run layout's header (when there is one).
+__global__ void map_init(uint4* a, size_t words16a, uint4* b, size_t words16b, uint32_t* status,
+                         int32_t* hdr) {
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   const size_t t0 = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const uint4 ones = make_uint4(~0u, ~0u, ~0u, ~0u);
   for (size_t t = t0; t < words16a; t += stride) a[t] = ones;
   for (size_t t = t0; t < words16b; t += stride) b[t] = ones;
-  if (t0 == 0) *status = 0u;
+  if (t0 == 0) {
+    *status = 0u;
+    if (hdr)
+      for (int k = 0; k < 8; ++k) hdr[k] = 0;
+  }
 }
 
 __global__ void map_insert_direct(const int4* __restrict__ coords, int64_t n, int grid, int batch,
@@ -191,18 +197,125 @@ __device__ __forceinline__ int32_t lookup(const Tables& t, int b, int z, int y, 
   }
 }
 
-template <Kind K>
+// ----------------------------------------------------------- run layout ----
+// The query kernel also lays out the x-run positions.  Row v starts a run
+// unless row v-1 is its x-1 neighbour (same b, z, y and x one less).  With
+// R(v) the run starts among rows 0..v, voxel v sits at position v + 2 R(v), its
+// run's left pad (when v starts the run) at the position before, the right pad
+// (when v ends it) at the one after.  R needs a count across tiles: every tile
+// publishes its own run-start count as soon as its coordinates are loaded, and
+// after its lookups takes the sum over the earlier tiles by decoupled look-back
+// (Merrill and Garland, "Single-pass Parallel Prefix Scan with Decoupled
+// Look-back", NVIDIA 2016): walk back over the preceding tiles' words, adding
+// their counts, until one that already holds an inclusive prefix.  Tiles take
+// their index from a ticket counter, so every tile waited for has started, and
+// every wait is bounded (2 s on the global timer, then kErrTimeout).
+
+static_assert(kPosTile == 256, "et_store splits positions with shifts by 8");
+
+struct RunOut {
+  unsigned long long* lb;  // [n_tiles] look-back words, all-ones = not published
+  int32_t* hdr;            // [8]: runs, position tiles, positions, 0, tile ticket
+  int32_t* pos;            // position table
+  int32_t* et;             // E index table
+};
+
+// Look-back word: flag in bits [62, 64), run-start count in bits [0, 32).
+constexpr unsigned long long kLbAggregate = 1ull << 62;
+constexpr unsigned long long kLbInclusive = 2ull << 62;
+constexpr unsigned long long kLbNotReady = ~0ull;
+constexpr uint64_t kLookbackLimitNs = 2000000000ull;
+
+__device__ __forceinline__ void lb_store(unsigned long long* w, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(w), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long lb_load(const unsigned long long* w) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(w) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Run starts in the tiles before `tile`, by one full warp; -1 when a wait ran out.
+__device__ int64_t lookback(const unsigned long long* lb, int64_t tile) {
+  const int lane = threadIdx.x & 31;
+  uint32_t sum = 0;
+  const uint64_t t0 = global_ns();
+  for (int64_t base = tile - 1; base >= 0; base -= 32) {
+    const int64_t j = base - lane;  // lane 0 reads the nearest predecessor
+    // before tile 0 the prefix is 0: an inclusive word with count 0
+    unsigned long long w = j >= 0 ? lb_load(lb + j) : kLbInclusive;
+    while (__any_sync(0xFFFFFFFFu, w == kLbNotReady)) {
+      if (__shfl_sync(0xFFFFFFFFu, global_ns() - t0 > kLookbackLimitNs ? 1 : 0, 0)) return -1;
+      __nanosleep(64);
+      if (w == kLbNotReady) w = lb_load(lb + j);
+    }
+    const uint32_t incl = __ballot_sync(0xFFFFFFFFu, (w >> 62) == 2u);
+    const int stop = incl ? __ffs(incl) - 1 : 31;
+    sum += __reduce_add_sync(0xFFFFFFFFu, lane <= stop ? static_cast<uint32_t>(w) : 0u);
+    if (incl) break;
+  }
+  return sum;
+}
+
+__device__ __forceinline__ bool x_next(int4 a, int4 b) {  // b is a's x+1 neighbour
+  return a.x == b.x && a.y == b.y && a.z == b.z && a.w + 1 == b.w;
+}
+
+// E row q of offset pair dzdy: entry (q mod 256) + 1 of tile q / 256, and the
+// copies a tile keeps of its edge rows' outer neighbours (entry 0 of the next
+// tile is row 255 of this one; entry 257 of the previous tile is row 0).
+__device__ __forceinline__ void et_store(int32_t* et, int64_t q, int dzdy, int32_t v) {
+  const int64_t t = q >> 8;
+  const int i = static_cast<int>(q & 255);
+  et[(t * 9 + dzdy) * kEtStride + i + 1] = v;
+  if (i == kPosTile - 1) et[((t + 1) * 9 + dzdy) * kEtStride] = v;
+  if (i == 0 && t > 0) et[((t - 1) * 9 + dzdy) * kEtStride + kPosTile + 1] = v;
+}
+
+// One block per 128-row tile, one thread per voxel: 27 lookups into shared
+// memory, then the [128, 27] nbr block and the tile's offset mask with
+// coalesced stores.  With RUNS, also the tile's positions and E index entries.
+template <Kind K, bool RUNS>
 __global__ void __launch_bounds__(kTileRows)
     map_query(const int4* __restrict__ coords, int64_t n, int grid, int batch, Tables t,
-              int32_t* __restrict__ nbr, uint32_t* __restrict__ tile_mask, uint32_t* status) {
+              int32_t* __restrict__ nbr, uint32_t* __restrict__ tile_mask, uint32_t* status,
+              RunOut ro) {
   __shared__ __align__(16) int32_t s_nbr[kTileRows * kKvol];
   __shared__ uint32_t s_bits[kTileRows / 32];
+  __shared__ uint32_t s_starts[kTileRows / 32];  // run-start ballot of each warp
+  __shared__ int64_t s_tile, s_excl, s_end;
   const int r = threadIdx.x;
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kTileRows;
+  const int lane = r & 31, warp = r >> 5;
+  int64_t tile = blockIdx.x;
+  if constexpr (RUNS) {
+    if (r == 0) s_tile = atomicAdd(reinterpret_cast<unsigned int*>(ro.hdr + 4), 1u);
+    __syncthreads();
+    tile = s_tile;
+  }
+  const int64_t row0 = tile * kTileRows;
   const int64_t i = row0 + r;
+  int4 c = make_int4(-1, -1, -1, -1);
+  if (i < n) c = __ldg(coords + i);
+  bool starts = false, ends = false;
+  uint32_t agg = 0;
+  if constexpr (RUNS) {
+    if (i < n) {
+      starts = i == 0 || !x_next(__ldg(coords + i - 1), c);
+      ends = i == n - 1 || !x_next(c, __ldg(coords + i + 1));
+    }
+    const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, starts);
+    if (lane == 0) s_starts[warp] = ballot;
+    __syncthreads();
+    agg = __popc(s_starts[0]) + __popc(s_starts[1]) + __popc(s_starts[2]) + __popc(s_starts[3]);
+    if (r == 0) lb_store(ro.lb + tile, (tile == 0 ? kLbInclusive : kLbAggregate) | agg);
+  }
   uint32_t bits = 0u;
   if (i < n) {
-    const int4 c = __ldg(coords + i);
     if (in_volume(c, grid, batch)) {
 #pragma unroll
       for (int k = 0; k < kKvol; ++k) {
@@ -225,9 +338,9 @@ __global__ void __launch_bounds__(kTileRows)
     }
   }
   bits = __reduce_or_sync(0xFFFFFFFFu, bits);
-  if ((r & 31) == 0) s_bits[r >> 5] = bits;
+  if (lane == 0) s_bits[warp] = bits;
   __syncthreads();
-  if (r == 0) tile_mask[blockIdx.x] = s_bits[0] | s_bits[1] | s_bits[2] | s_bits[3];
+  if (r == 0) tile_mask[tile] = s_bits[0] | s_bits[1] | s_bits[2] | s_bits[3];
   const int rows = static_cast<int>(n - row0 < kTileRows ? n - row0 : kTileRows);
   int32_t* dst = nbr + row0 * kKvol;
   if (rows == kTileRows) {
@@ -238,151 +351,65 @@ __global__ void __launch_bounds__(kTileRows)
   } else {
     for (int e = r; e < rows * kKvol; e += kTileRows) dst[e] = s_nbr[e];
   }
-}
-
-// ----------------------------------------------------------- run layout ----
-// A voxel starts a run unless the previous row is its x-1 neighbour (same b, z,
-// y and x one less).
-
-__device__ __forceinline__ bool run_start(const int4* coords, int64_t v) {
-  if (v == 0) return true;
-  const int4 p = __ldg(coords + v - 1);
-  const int4 c = __ldg(coords + v);
-  return !(p.x == c.x && p.y == c.y && p.z == c.z && p.w + 1 == c.w);
-}
-
-// Run starts per block of kRunBlock rows.
-__global__ void __launch_bounds__(256) map_run_count(const int4* __restrict__ coords, int64_t n,
-                                                     int32_t* __restrict__ cnt) {
-  __shared__ int32_t s_sum[8];
-  int32_t c = 0;
-  for (int i = 0; i < kRunBlock / 256; ++i) {
-    const int64_t v = static_cast<int64_t>(blockIdx.x) * kRunBlock + i * 256 + threadIdx.x;
-    if (v < n && run_start(coords, v)) ++c;
-  }
-  c = __reduce_add_sync(0xFFFFFFFFu, c);
-  if ((threadIdx.x & 31) == 0) s_sum[threadIdx.x >> 5] = c;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int32_t t = 0;
-    for (int w = 0; w < 8; ++w) t += s_sum[w];
-    cnt[blockIdx.x] = t;
-  }
-}
-
-// Exclusive scan of the per-block run counts (one block), and the header:
-// hdr[0] = runs, hdr[1] = position tiles, hdr[2] = positions.
-__global__ void __launch_bounds__(1024) map_run_scan(int32_t* __restrict__ cnt, int64_t n_blocks,
-                                                     int64_t n, int32_t* __restrict__ hdr) {
-  __shared__ int32_t s_warp[32];
-  __shared__ int64_t s_carry;
-  if (threadIdx.x == 0) s_carry = 0;
-  __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int64_t base = 0; base < n_blocks; base += 1024) {
-    const int64_t i = base + threadIdx.x;
-    const int32_t x = i < n_blocks ? cnt[i] : 0;
-    int32_t incl = x;
-    for (int d = 1; d < 32; d <<= 1) {
-      const int32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-      if (lane >= d) incl += y;
+  if constexpr (!RUNS) return;
+  if (warp == 0) {
+    const int64_t excl = tile == 0 ? 0 : lookback(ro.lb, tile);
+    if (lane == 0) {
+      if (excl < 0)
+        atomicOr(status, kErrTimeout);
+      else if (tile > 0)
+        lb_store(ro.lb + tile, kLbInclusive | static_cast<uint32_t>(excl + agg));
+      s_excl = excl;
     }
-    if (lane == 31) s_warp[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-      int32_t w = s_warp[lane];
-      for (int d = 1; d < 32; d <<= 1) {
-        const int32_t y = __shfl_up_sync(0xFFFFFFFFu, w, d);
-        if (lane >= d) w += y;
+  }
+  __syncthreads();
+  const int64_t excl = s_excl;
+  if (excl < 0) return;
+  int64_t runs = excl;  // run starts among rows 0..i
+  for (int w = 0; w < warp; ++w) runs += __popc(s_starts[w]);
+  runs += __popc(s_starts[warp] & (0xFFFFFFFFu >> (31 - lane)));
+  if (i < n) {
+    const int64_t p = i + 2 * runs;
+    const int32_t tag = static_cast<int32_t>(i * 4);
+    ro.pos[p] = tag + kPosVoxel;
+    if (starts) ro.pos[p - 1] = tag + kPosLeftPad;
+    if (ends) ro.pos[p + 1] = tag + kPosRightPad;
+    const int32_t* nb = s_nbr + r * kKvol;
+#pragma unroll
+    for (int dzdy = 0; dzdy < 9; ++dzdy) {
+      et_store(ro.et, p, dzdy, nb[3 * dzdy + 1]);
+      if (starts) et_store(ro.et, p - 1, dzdy, nb[3 * dzdy]);
+      if (ends) et_store(ro.et, p + 1, dzdy, nb[3 * dzdy + 2]);
+    }
+    if (i == 0) {  // position 0 (the absent right pad before the first run) and row -1
+      ro.pos[0] = -1;
+#pragma unroll
+      for (int dzdy = 0; dzdy < 9; ++dzdy) {
+        ro.et[dzdy * kEtStride] = -1;
+        ro.et[dzdy * kEtStride + 1] = -1;
       }
-      s_warp[lane] = w;  // inclusive over warps
     }
+    if (i == n - 1) s_end = p + 2;  // one past the last run's right pad
+  }
+  if (row0 + kTileRows >= n) {  // the tile of row n-1: header, and the line's tail
     __syncthreads();
-    const int32_t before = (warp > 0 ? s_warp[warp - 1] : 0) + incl - x;
-    const int64_t carry = s_carry;
-    if (i < n_blocks) cnt[i] = static_cast<int32_t>(carry + before);
-    __syncthreads();
-    if (threadIdx.x == 0) s_carry = carry + s_warp[31];
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) {
-    const int64_t runs = s_carry;
-    const int64_t positions = n + 2 * runs;
-    hdr[0] = static_cast<int32_t>(runs);
-    hdr[1] = static_cast<int32_t>((positions + kPosTile - 1) / kPosTile);
-    hdr[2] = static_cast<int32_t>(positions);
-    hdr[3] = 0;
-  }
-}
-
-// Places every voxel v at position v + 2 R(v), R(v) = run starts among rows
-// 0..v, with the left-pad slot before a run's first voxel and the right-pad
-// slot after its last.  Each thread handles 4 consecutive rows.
-__global__ void __launch_bounds__(256) map_run_place(const int4* __restrict__ coords, int64_t n,
-                                                     const int32_t* __restrict__ blk_off,
-                                                     int32_t* __restrict__ pos) {
-  __shared__ int32_t s_warp[8];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t v0 = static_cast<int64_t>(blockIdx.x) * kRunBlock + 4 * threadIdx.x;
-  bool rs[5];
-#pragma unroll
-  for (int i = 0; i < 5; ++i) rs[i] = (v0 + i < n) ? run_start(coords, v0 + i) : true;
-  int32_t local = 0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) local += (v0 + i < n && rs[i]) ? 1 : 0;
-  int32_t incl = local;
-  for (int d = 1; d < 32; d <<= 1) {
-    const int32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-    if (lane >= d) incl += y;
-  }
-  if (lane == 31) s_warp[warp] = incl;
-  __syncthreads();
-  int32_t warp_before = 0;
-  for (int w = 0; w < warp; ++w) warp_before += s_warp[w];
-  int64_t r = blk_off[blockIdx.x] + warp_before + incl - local;  // run starts before v0
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int64_t v = v0 + i;
-    if (v >= n) break;
-    if (rs[i]) ++r;
-    const int64_t p = v + 2 * r;
-    pos[p] = static_cast<int32_t>(v * 4 + kPosVoxel);
-    if (rs[i]) pos[p - 1] = static_cast<int32_t>(v * 4 + kPosLeftPad);
-    if (v + 1 == n || rs[i + 1]) pos[p + 1] = static_cast<int32_t>(v * 4 + kPosRightPad);
-  }
-}
-
-// E index table: for position tile t and offset pair (dz, dy), entry i is the
-// feature row of E row i-1: a voxel position takes its (dz, dy, 0) neighbour,
-// a left pad its voxel's (dz, dy, -1) neighbour, a right pad the (dz, dy, +1)
-// one; entry 0 (row -1) and entry 257 (row 256) are the (dz, dy, -1) and
-// (dz, dy, +1) neighbours of the voxels at positions 0 and 255.  So for the
-// voxel at position p, E rows p-1, p, p+1 hold its dx = -1, 0, +1 neighbours.
-__global__ void __launch_bounds__(kEtStride) map_etable(const int32_t* __restrict__ pos,
-                                                         const int32_t* __restrict__ nbr,
-                                                         const int32_t* __restrict__ hdr,
-                                                         int32_t* __restrict__ et) {
-  const int64_t t = blockIdx.x;
-  if (t >= hdr[1]) return;
-  const int i = threadIdx.x;  // 0 .. kEtStride-1
-  int64_t v = -1;
-  int dx = 0;
-  if (i == 0 || i == 257) {
-    const int32_t e = pos[t * kPosTile + (i == 0 ? 0 : kPosTile - 1)];
-    if (e >= 0 && (e & 3) == kPosVoxel) {
-      v = e >> 2;
-      dx = i == 0 ? -1 : 1;
+    // positions up to the last voxel: N + 2 runs; the last right pad is not counted,
+    // as its only reader, row 256 of its voxel's tile, holds a copy of it
+    const int64_t end = s_end;
+    const int64_t positions = end - 1;
+    const int64_t ptiles = (positions + kPosTile - 1) / kPosTile;
+    if (r == 0) {
+      ro.hdr[0] = static_cast<int32_t>(excl + agg);
+      ro.hdr[1] = static_cast<int32_t>(ptiles);
+      ro.hdr[2] = static_cast<int32_t>(positions);
+      ro.hdr[3] = 0;
     }
-  } else if (i < 257) {
-    const int32_t e = pos[t * kPosTile + i - 1];
-    if (e >= 0) {
-      v = e >> 2;
-      dx = (e & 3) == kPosLeftPad ? -1 : ((e & 3) == kPosRightPad ? 1 : 0);
+    for (int64_t q = end + r; q <= ptiles * kPosTile; q += kTileRows) {
+      if (q < ptiles * kPosTile) ro.pos[q] = -1;
+#pragma unroll
+      for (int dzdy = 0; dzdy < 9; ++dzdy) et_store(ro.et, q, dzdy, -1);
     }
   }
-#pragma unroll
-  for (int dzdy = 0; dzdy < 9; ++dzdy)
-    et[(t * 9 + dzdy) * kEtStride + i] = v >= 0 ? __ldg(nbr + v * kKvol + 3 * dzdy + dx + 1) : -1;
 }
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -422,17 +449,16 @@ bool map_layout(int64_t n, int32_t grid_dim, int32_t batch, const MapOptions& op
     lay.rows_off = align_up(lay.table_off + lay.table_bytes, 256);
     end = lay.compact ? lay.rows_off : align_up(lay.rows_off + cap * 4, 256);
   }
-  if (!opt.run_layout) {  // nbr and tile masks only
-    lay.runcnt_off = lay.hdr_off = lay.pos_off = lay.et_off = end;
+  if (!opt.run_layout || n >= kRunLayoutMaxRows) {  // nbr and tile masks only
+    lay.lb_off = lay.hdr_off = lay.pos_off = lay.et_off = end;
     lay.total = end;
     *out = lay;
     return true;
   }
-  lay.n_run_blocks = (n + kRunBlock - 1) / kRunBlock;
   lay.pos_max = static_cast<int64_t>(align_up(static_cast<size_t>(3 * n), kPosTile)) + kPosTile;
   lay.ptile_max = lay.pos_max / kPosTile;
-  lay.runcnt_off = end;
-  lay.hdr_off = align_up(lay.runcnt_off + static_cast<size_t>(lay.n_run_blocks) * 4, 256);
+  lay.lb_off = end;
+  lay.hdr_off = align_up(lay.lb_off + static_cast<size_t>(lay.n_tiles) * 8, 256);
   lay.pos_off = lay.hdr_off + 256;
   lay.pos_bytes = static_cast<size_t>(lay.pos_max) * 4;
   lay.et_off = align_up(lay.pos_off + lay.pos_bytes, 256);
@@ -441,6 +467,22 @@ bool map_layout(int64_t n, int32_t grid_dim, int32_t batch, const MapOptions& op
   return true;
 }
 
+namespace {
+
+template <Kind K>
+void launch_query(unsigned blocks, bool runs, const int4* c4, int64_t n, int grid, int batch,
+                  const Tables& t, int32_t* nbr, uint32_t* mask, uint32_t* status,
+                  const RunOut& ro, cudaStream_t stream) {
+  if (runs)
+    map_query<K, true><<<blocks, kTileRows, 0, stream>>>(c4, n, grid, batch, t, nbr, mask, status,
+                                                         ro);
+  else
+    map_query<K, false><<<blocks, kTileRows, 0, stream>>>(c4, n, grid, batch, t, nbr, mask,
+                                                          status, ro);
+}
+
+}  // namespace
+
 cudaError_t launch_map_build(const int32_t* coords, int64_t n, int32_t grid_dim, int32_t batch,
                              int32_t* nbr, void* workspace, const MapLayout& lay,
                              cudaStream_t stream) {
@@ -448,17 +490,24 @@ cudaError_t launch_map_build(const int32_t* coords, int64_t n, int32_t grid_dim,
   auto* status = reinterpret_cast<uint32_t*>(ws + lay.status_off);
   auto* mask = reinterpret_cast<uint32_t*>(ws + lay.mask_off);
   auto* table = ws + lay.table_off;
+  const bool runs = lay.ptile_max > 0;
+  RunOut ro{};
+  if (runs) {
+    ro.lb = reinterpret_cast<unsigned long long*>(ws + lay.lb_off);
+    ro.hdr = reinterpret_cast<int32_t*>(ws + lay.hdr_off);
+    ro.pos = reinterpret_cast<int32_t*>(ws + lay.pos_off);
+    ro.et = reinterpret_cast<int32_t*>(ws + lay.et_off);
+  }
   const size_t words16 = lay.table_bytes / 16;
-  const size_t pos_words16 = lay.pos_bytes / 16;
-  auto* pos = reinterpret_cast<int32_t*>(ws + lay.pos_off);
+  const size_t lb_words16 = runs ? (static_cast<size_t>(lay.n_tiles) * 8 + 15) / 16 : 0;
   {
-    const size_t work = words16 > pos_words16 ? words16 : pos_words16;
+    const size_t work = words16 > lb_words16 ? words16 : lb_words16;
     size_t blocks = (work + 255) / 256;
     if (blocks > 148 * 8) blocks = 148 * 8;
     if (blocks == 0) blocks = 1;
     map_init<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-        reinterpret_cast<uint4*>(table), words16, reinterpret_cast<uint4*>(pos), pos_words16,
-        status);
+        reinterpret_cast<uint4*>(table), words16, reinterpret_cast<uint4*>(ro.lb), lb_words16,
+        status, ro.hdr);
   }
   if (n == 0) return cudaGetLastError();
   const auto* c4 = reinterpret_cast<const int4*>(coords);
@@ -470,14 +519,14 @@ cudaError_t launch_map_build(const int32_t* coords, int64_t n, int32_t grid_dim,
     t.cells = reinterpret_cast<const int32_t*>(table);
     map_insert_direct<<<ins_blocks, 256, 0, stream>>>(c4, n, grid_dim, batch,
                                                       reinterpret_cast<int32_t*>(table), status);
-    map_query<Kind::kDirect><<<q_blocks, kTileRows, 0, stream>>>(c4, n, grid_dim, batch, t, nbr,
-                                                                 mask, status);
+    launch_query<Kind::kDirect>(q_blocks, runs, c4, n, grid_dim, batch, t, nbr, mask, status, ro,
+                                stream);
   } else if (lay.compact) {
     t.table = reinterpret_cast<const unsigned long long*>(table);
     map_insert_compact<<<ins_blocks, 256, 0, stream>>>(
         c4, n, grid_dim, batch, reinterpret_cast<unsigned long long*>(table), t.capmask, status);
-    map_query<Kind::kCompact><<<q_blocks, kTileRows, 0, stream>>>(c4, n, grid_dim, batch, t, nbr,
-                                                                  mask, status);
+    launch_query<Kind::kCompact>(q_blocks, runs, c4, n, grid_dim, batch, t, nbr, mask, status,
+                                 ro, stream);
   } else {
     auto* rows = reinterpret_cast<int32_t*>(ws + lay.rows_off);
     t.table = reinterpret_cast<const unsigned long long*>(table);
@@ -485,19 +534,9 @@ cudaError_t launch_map_build(const int32_t* coords, int64_t n, int32_t grid_dim,
     map_insert_wide<<<ins_blocks, 256, 0, stream>>>(c4, n, grid_dim, batch,
                                                     reinterpret_cast<unsigned long long*>(table),
                                                     rows, t.capmask, status);
-    map_query<Kind::kWide><<<q_blocks, kTileRows, 0, stream>>>(c4, n, grid_dim, batch, t, nbr,
-                                                               mask, status);
+    launch_query<Kind::kWide>(q_blocks, runs, c4, n, grid_dim, batch, t, nbr, mask, status, ro,
+                              stream);
   }
-  if (lay.ptile_max == 0) return cudaGetLastError();
-  // x-run position layout and E index table for the run-padded forward
-  auto* runcnt = reinterpret_cast<int32_t*>(ws + lay.runcnt_off);
-  auto* hdr = reinterpret_cast<int32_t*>(ws + lay.hdr_off);
-  auto* et = reinterpret_cast<int32_t*>(ws + lay.et_off);
-  const unsigned rblocks = static_cast<unsigned>(lay.n_run_blocks);
-  map_run_count<<<rblocks, 256, 0, stream>>>(c4, n, runcnt);
-  map_run_scan<<<1, 1024, 0, stream>>>(runcnt, lay.n_run_blocks, n, hdr);
-  map_run_place<<<rblocks, 256, 0, stream>>>(c4, n, runcnt, pos);
-  map_etable<<<static_cast<unsigned>(lay.ptile_max), kEtStride, 0, stream>>>(pos, nbr, hdr, et);
   return cudaGetLastError();
 }
 

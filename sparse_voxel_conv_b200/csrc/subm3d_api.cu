@@ -128,9 +128,10 @@ subm3d_status subm3d_build_map(const int32_t* coords, int64_t n, int32_t grid_di
   h->nbr = nbr;
   h->tile_mask = reinterpret_cast<const uint32_t*>(ws + lay.mask_off);
   h->status_word = reinterpret_cast<const uint32_t*>(ws + lay.status_off);
-  h->pos = reinterpret_cast<const int32_t*>(ws + lay.pos_off);
-  h->et = reinterpret_cast<const int32_t*>(ws + lay.et_off);
-  h->hdr = reinterpret_cast<const int32_t*>(ws + lay.hdr_off);
+  const bool runs = lay.ptile_max > 0;
+  h->pos = runs ? reinterpret_cast<const int32_t*>(ws + lay.pos_off) : nullptr;
+  h->et = runs ? reinterpret_cast<const int32_t*>(ws + lay.et_off) : nullptr;
+  h->hdr = runs ? reinterpret_cast<const int32_t*>(ws + lay.hdr_off) : nullptr;
   h->ptile_max = lay.ptile_max;
   h->n = n;
   h->grid_dim = grid_dim;
@@ -155,6 +156,7 @@ subm3d_status subm3d_map_status(const subm3d_map* map) {
   if (word & subm3d::kErrRange) return SUBM3D_E_RANGE;
   if (word & subm3d::kErrDuplicate) return SUBM3D_E_DUPLICATE;
   if (word & subm3d::kErrTableFull) return SUBM3D_E_TABLE_FULL;
+  if (word & subm3d::kErrTimeout) return SUBM3D_E_TIMEOUT;
   return SUBM3D_OK;
 }
 
@@ -211,6 +213,7 @@ subm3d_status subm3d_forward(const int32_t* nbr, const uint32_t* tile_mask, int6
 subm3d_status subm3d_map_run_layout(const subm3d_map* map, const int32_t** pos,
                                     const int32_t** etable, const int32_t** header) {
   if (!map || !pos || !etable || !header) return SUBM3D_E_INVALID;
+  if (!map->pos) return SUBM3D_E_UNSUPPORTED;
   *pos = map->pos;
   *etable = map->et;
   *header = map->hdr;
@@ -222,7 +225,7 @@ subm3d_status subm3d_forward_map(const subm3d_map* map, const void* feats, const
                                  int32_t flip, subm3d_act act, void* stream) {
   if (!map) return SUBM3D_E_INVALID;
   const int64_t n = map->n;
-  const bool runs = dtype == SUBM3D_BF16 && n > 0 && cin % 64 == 0 && cout % 16 == 0 &&
+  const bool runs = map->pos && dtype == SUBM3D_BF16 && n > 0 && cin % 64 == 0 && cout % 16 == 0 &&
                     feats && weight && out && aligned(feats, 16) && aligned(weight, 16) &&
                     aligned(out, 16) && (act == SUBM3D_ACT_NONE || act == SUBM3D_ACT_GELU);
   if (!runs)

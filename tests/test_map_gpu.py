@@ -127,25 +127,62 @@ def test_map_async_status_and_reuse(S):
     assert np.array_equal(h2.nbr.cpu().numpy(), C.build_map(WL.tiny_coords(), 16, 1))
 
 
-@pytest.mark.parametrize("name", ["tiny", "shell", "headline", "batched"])
-def test_run_layout_invariant(S, kind, name):
-    """Every voxel sits at one position p of the x-run layout, and for each of
-    its 27 offsets (dz, dy, dx) the E index entry of (tile, dz-dy) at row p+dx
-    is its neighbour nbr[v][k] -- the property the x-run forward relies on."""
-    wl = WL.make_workload(name)
-    h = S.build_map(torch.from_numpy(wl.coords).cuda(), wl.grid_dim, wl.batch)
+def _check_run_layout(S, coords, grid, batch):
+    """Every voxel sits at one position p of the x-run layout, its run's pads
+    beside it, and for each of its 27 offsets (dz, dy, dx) the E index entry of
+    (tile, dz-dy) at row p+dx is its neighbour nbr[v][k] -- the property the
+    x-run forward relies on.  Every other entry of the used tiles is empty or
+    a valid row, so no gather can leave the feature array."""
+    coords = np.ascontiguousarray(coords, dtype=np.int32)
+    h = S.build_map(torch.from_numpy(coords).cuda(), grid, batch)
     pos, et, hdr = (t.cpu().numpy() for t in S.run_layout_tensors(h))
-    ref = C.build_map(wl.coords, wl.grid_dim, wl.batch)
-    n = wl.n
-    c = wl.coords.astype(np.int64)
+    ref = C.build_map(coords, grid, batch)
+    n = coords.shape[0]
+    c = coords.astype(np.int64)
     same = (c[1:, 0] == c[:-1, 0]) & (c[1:, 1] == c[:-1, 1]) & (c[1:, 2] == c[:-1, 2]) & \
         (c[1:, 3] == c[:-1, 3] + 1)
-    runs = int((~same).sum()) + 1
-    assert hdr[0] == runs and hdr[2] == n + 2 * runs and hdr[1] == (n + 2 * runs + 255) // 256
+    starts = np.concatenate([[True], ~same])
+    ends = np.concatenate([~same, [True]])
+    runs = int(starts.sum())
+    positions = n + 2 * runs
+    assert hdr[0] == runs and hdr[2] == positions and hdr[1] == (positions + 255) // 256
+    assert pos.shape[0] == 256 * hdr[1] and et.shape == (hdr[1], 9, 260)
     voxel_pos = np.nonzero((pos >= 0) & ((pos & 3) == 0))[0]
     assert np.array_equal(pos[voxel_pos] >> 2, np.arange(n))      # every row once, in order
+    assert np.array_equal(voxel_pos, np.arange(n) + 2 * np.cumsum(starts))
+    left = np.nonzero((pos >= 0) & ((pos & 3) == 1))[0]
+    assert np.array_equal(left + 1, voxel_pos[starts]) and np.array_equal(pos[left] >> 2,
+                                                                           np.nonzero(starts)[0])
+    right = np.nonzero((pos >= 0) & ((pos & 3) == 2))[0]
+    inside = voxel_pos[ends] + 1 < pos.shape[0]          # the last right pad may sit past the tiles
+    assert np.array_equal(right, (voxel_pos[ends] + 1)[inside])
+    assert pos[0] == -1 and (pos[positions + 1:] == -1).all()
+    assert ((pos >= 0) | (pos == -1)).all()
+    assert (et[:, :, :258] >= -1).all() and (et[:, :, :258] < n).all()
     tile, local = voxel_pos // 256, voxel_pos % 256
     for k in range(27):
         dzdy, dx = k // 3, k % 3 - 1
         got = et[tile, dzdy, local + dx + 1]
         assert np.array_equal(got, ref[:, k]), f"offset {k}"
+
+
+@pytest.mark.parametrize("name", ["tiny", "shell", "headline", "batched"])
+def test_run_layout_invariant(S, kind, name):
+    wl = WL.make_workload(name)
+    _check_run_layout(S, wl.coords, wl.grid_dim, wl.batch)
+
+
+def test_run_layout_edges(S, kind):
+    """Tiny maps, a last tile ending on a position-tile boundary (one run of
+    252 to 255 voxels puts the last right pad at 255, 256 or beyond), and
+    random row order (short runs, many pads)."""
+    rng = np.random.default_rng(17)
+    for n in (1, 2, 127, 128, 129, 300):
+        cells = rng.choice(8 ** 3, n, replace=False)
+        zyx = np.stack(np.unravel_index(np.sort(cells), (8, 8, 8)), 1)
+        _check_run_layout(S, np.concatenate([np.zeros((n, 1), np.int64), zyx], 1), 8, 1)
+    for length in (252, 253, 254, 255, 510, 511):
+        line = np.array([[0, 3, 5, x] for x in range(length)])
+        _check_run_layout(S, line, 512, 1)
+    wl = WL.make_workload("shell")
+    _check_run_layout(S, wl.coords[WL.permute_rows(wl.n, 5)], wl.grid_dim, wl.batch)

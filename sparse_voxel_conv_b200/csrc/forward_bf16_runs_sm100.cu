@@ -179,9 +179,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int64_t n_tiles = __ldg(a.hdr + 1);
-  const int64_t n_units = n_tiles * a.n_oblocks;
-
   if (threadIdx.x == 0) {
     for (int s = 0; s < SE; ++s) {
       mbar_init(&e_full[s], GATHER_THREADS);  // every gather thread's cp.async arrive
@@ -208,6 +205,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // the setup above overlaps the map build's tail; global reads start here
+  const int64_t n_tiles = __ldg(a.hdr + 1);
+  const int64_t n_units = n_tiles * a.n_oblocks;
 
   if (warp >= GATHER_WARP0 && warp < GATHER_WARP0 + NUM_GATHER_WARPS) {
     // ---------------------------------------------------------- gather ----
@@ -468,10 +468,10 @@ cudaError_t launch_forward_bf16_runs(const int32_t* pos, const int32_t* etable,
   const int64_t units = max_tiles * a.n_oblocks;
   const unsigned grid = static_cast<unsigned>(units < num_sms ? units : num_sms);
   if (act)
-    subm3d_fwd_bf16_runs_sm100<true><<<grid, NUM_THREADS, plan.bytes, stream>>>(wmap, a);
-  else
-    subm3d_fwd_bf16_runs_sm100<false><<<grid, NUM_THREADS, plan.bytes, stream>>>(wmap, a);
-  return cudaGetLastError();
+    return launch_pdl(subm3d_fwd_bf16_runs_sm100<true>, grid, NUM_THREADS, plan.bytes, stream,
+                      wmap, a);
+  return launch_pdl(subm3d_fwd_bf16_runs_sm100<false>, grid, NUM_THREADS, plan.bytes, stream,
+                    wmap, a);
 }
 
 }  // namespace subm3d

@@ -4,9 +4,38 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 #include <cuda_runtime.h>
 
 namespace subm3d {
+
+// Programmatic dependent launch.  The library's kernels are launched with the
+// programmatic-serialization attribute, so a kernel may be scheduled while the
+// previous kernel on the stream is finishing; every such kernel executes
+// pdl_wait() (griddepcontrol.wait: until the preceding grid has completed and
+// its writes are visible) before its first global-memory access, and the map
+// kernels call pdl_trigger() to let the next kernel be scheduled early.  The
+// wait is a no-op for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Bits of the map build's device status word.
 constexpr uint32_t kErrRange = 1u;

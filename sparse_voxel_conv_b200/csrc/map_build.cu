@@ -83,6 +83,8 @@ __device__ __forceinline__ int64_t cell_of(int b, int z, int y, int x, int grid)
 // status word and the run layout's header (when there is one).
 __global__ void map_init(uint4* a, size_t words16a, uint4* b, size_t words16b, uint32_t* status,
                          int32_t* hdr) {
+  pdl_wait();
+  pdl_trigger();
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   const size_t t0 = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const uint4 ones = make_uint4(~0u, ~0u, ~0u, ~0u);
@@ -97,6 +99,8 @@ __global__ void map_init(uint4* a, size_t words16a, uint4* b, size_t words16b, u
 
 __global__ void map_insert_direct(const int4* __restrict__ coords, int64_t n, int grid, int batch,
                                   int32_t* __restrict__ cells, uint32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= n) return;
   const int4 c = __ldg(coords + i);
@@ -110,6 +114,8 @@ __global__ void map_insert_direct(const int4* __restrict__ coords, int64_t n, in
 __global__ void map_insert_compact(const int4* __restrict__ coords, int64_t n, int grid, int batch,
                                    unsigned long long* __restrict__ table, uint32_t capmask,
                                    uint32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= n) return;
   const int4 c = __ldg(coords + i);
@@ -136,6 +142,8 @@ __global__ void map_insert_compact(const int4* __restrict__ coords, int64_t n, i
 __global__ void map_insert_wide(const int4* __restrict__ coords, int64_t n, int grid, int batch,
                                 unsigned long long* __restrict__ keys, int32_t* __restrict__ rows,
                                 uint32_t capmask, uint32_t* status) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= n) return;
   const int4 c = __ldg(coords + i);
@@ -211,7 +219,7 @@ __device__ __forceinline__ int32_t lookup(const Tables& t, int b, int z, int y, 
 // their index from a ticket counter, so every tile waited for has started, and
 // every wait is bounded (2 s on the global timer, then kErrTimeout).
 
-static_assert(kPosTile == 256, "et_store splits positions with shifts by 8");
+static_assert(kPosTile == 256, "et_store_row splits positions with shifts by 8");
 
 struct RunOut {
   unsigned long long* lb;  // [n_tiles] look-back words, all-ones = not published
@@ -266,15 +274,22 @@ __device__ __forceinline__ bool x_next(int4 a, int4 b) {  // b is a's x+1 neighb
   return a.x == b.x && a.y == b.y && a.z == b.z && a.w + 1 == b.w;
 }
 
-// E row q of offset pair dzdy: entry (q mod 256) + 1 of tile q / 256, and the
-// copies a tile keeps of its edge rows' outer neighbours (entry 0 of the next
+// E row q of offset pair dzdy is entry (q mod 256) + 1 of tile q / 256; a tile
+// also keeps copies of its edge rows' outer neighbours (entry 0 of the next
 // tile is row 255 of this one; entry 257 of the previous tile is row 0).
-__device__ __forceinline__ void et_store(int32_t* et, int64_t q, int dzdy, int32_t v) {
+// Writes E row q for all 9 pairs, the value of pair dzdy being v[3 * dzdy].
+__device__ __forceinline__ void et_store_row(int32_t* et, int64_t q, const int32_t* v) {
   const int64_t t = q >> 8;
   const int i = static_cast<int>(q & 255);
-  et[(t * 9 + dzdy) * kEtStride + i + 1] = v;
-  if (i == kPosTile - 1) et[((t + 1) * 9 + dzdy) * kEtStride] = v;
-  if (i == 0 && t > 0) et[((t - 1) * 9 + dzdy) * kEtStride + kPosTile + 1] = v;
+  int32_t* b = et + t * (9 * kEtStride) + i + 1;
+#pragma unroll
+  for (int dzdy = 0; dzdy < 9; ++dzdy) b[dzdy * kEtStride] = v[3 * dzdy];
+  if (i == kPosTile - 1 || (i == 0 && t > 0)) {  // one row in 128
+    int32_t* h = i == 0 ? et + (t - 1) * (9 * kEtStride) + kPosTile + 1
+                        : et + (t + 1) * (9 * kEtStride);
+#pragma unroll
+    for (int dzdy = 0; dzdy < 9; ++dzdy) h[dzdy * kEtStride] = v[3 * dzdy];
+  }
 }
 
 // One block per 128-row tile, one thread per voxel: 27 lookups into shared
@@ -291,6 +306,8 @@ __global__ void __launch_bounds__(kTileRows)
   __shared__ int64_t s_tile, s_excl, s_end;
   const int r = threadIdx.x;
   const int lane = r & 31, warp = r >> 5;
+  pdl_wait();
+  pdl_trigger();
   int64_t tile = blockIdx.x;
   if constexpr (RUNS) {
     if (r == 0) s_tile = atomicAdd(reinterpret_cast<unsigned int*>(ro.hdr + 4), 1u);
@@ -317,21 +334,45 @@ __global__ void __launch_bounds__(kTileRows)
   uint32_t bits = 0u;
   if (i < n) {
     if (in_volume(c, grid, batch)) {
+      if constexpr (K == Kind::kDirect) {
+        // the direct table has < 2^24 cells: int32 cell indices.  The 9 (dz, dy)
+        // rows are base pointers; dx = -1, 0, +1 are the cells before and after.
+        const int32_t g = grid, g2 = grid * grid;
+        const int32_t* centre = t.cells + (((c.x * g + c.y) * g + c.z) * g + c.w);
+        const bool vz[3] = {c.y > 0, true, c.y < g - 1};
+        const bool vy[3] = {c.z > 0, true, c.z < g - 1};
+        const bool vx[3] = {c.w > 0, true, c.w < g - 1};
 #pragma unroll
-      for (int k = 0; k < kKvol; ++k) {
-        const int z = c.y + k / 9 - 1;
-        const int y = c.z + (k / 3) % 3 - 1;
-        const int x = c.w + k % 3 - 1;
-        int32_t found = -1;
-        if (static_cast<unsigned>(z) < static_cast<unsigned>(grid) &&
-            static_cast<unsigned>(y) < static_cast<unsigned>(grid) &&
-            static_cast<unsigned>(x) < static_cast<unsigned>(grid))
-          found = lookup<K>(t, c.x, z, y, x, grid);
-        s_nbr[r * kKvol + k] = found;
-        bits |= (found >= 0 ? 1u : 0u) << k;
+        for (int dz = 0; dz < 3; ++dz) {
+#pragma unroll
+          for (int dy = 0; dy < 3; ++dy) {
+            const int32_t* row = centre + (dz - 1) * g2 + (dy - 1) * g;
+#pragma unroll
+            for (int dx = 0; dx < 3; ++dx) {
+              const int k = dz * 9 + dy * 3 + dx;
+              const int32_t found = (vz[dz] && vy[dy] && vx[dx]) ? __ldg(row + dx - 1) : -1;
+              s_nbr[r * kKvol + k] = found;
+              bits |= (found >= 0 ? 1u : 0u) << k;
+            }
+          }
+        }
+        if (s_nbr[r * kKvol + 13] != static_cast<int32_t>(i))
+          atomicOr(status, kErrDuplicate);  // another row owns this voxel's cell
+      } else {
+#pragma unroll
+        for (int k = 0; k < kKvol; ++k) {
+          const int z = c.y + k / 9 - 1;
+          const int y = c.z + (k / 3) % 3 - 1;
+          const int x = c.w + k % 3 - 1;
+          int32_t found = -1;
+          if (static_cast<unsigned>(z) < static_cast<unsigned>(grid) &&
+              static_cast<unsigned>(y) < static_cast<unsigned>(grid) &&
+              static_cast<unsigned>(x) < static_cast<unsigned>(grid))
+            found = lookup<K>(t, c.x, z, y, x, grid);
+          s_nbr[r * kKvol + k] = found;
+          bits |= (found >= 0 ? 1u : 0u) << k;
+        }
       }
-      if (K == Kind::kDirect && s_nbr[r * kKvol + 13] != static_cast<int32_t>(i))
-        atomicOr(status, kErrDuplicate);  // another row owns this voxel's cell
     } else {
 #pragma unroll
       for (int k = 0; k < kKvol; ++k) s_nbr[r * kKvol + k] = -1;
@@ -374,13 +415,10 @@ __global__ void __launch_bounds__(kTileRows)
     ro.pos[p] = tag + kPosVoxel;
     if (starts) ro.pos[p - 1] = tag + kPosLeftPad;
     if (ends) ro.pos[p + 1] = tag + kPosRightPad;
-    const int32_t* nb = s_nbr + r * kKvol;
-#pragma unroll
-    for (int dzdy = 0; dzdy < 9; ++dzdy) {
-      et_store(ro.et, p, dzdy, nb[3 * dzdy + 1]);
-      if (starts) et_store(ro.et, p - 1, dzdy, nb[3 * dzdy]);
-      if (ends) et_store(ro.et, p + 1, dzdy, nb[3 * dzdy + 2]);
-    }
+    const int32_t* nb = s_nbr + r * kKvol;  // nb[3 * dzdy + dx + 1]
+    et_store_row(ro.et, p, nb + 1);
+    if (starts) et_store_row(ro.et, p - 1, nb);
+    if (ends) et_store_row(ro.et, p + 1, nb + 2);
     if (i == 0) {  // position 0 (the absent right pad before the first run) and row -1
       ro.pos[0] = -1;
 #pragma unroll
@@ -404,10 +442,12 @@ __global__ void __launch_bounds__(kTileRows)
       ro.hdr[2] = static_cast<int32_t>(positions);
       ro.hdr[3] = 0;
     }
+    int32_t none[kKvol];
+#pragma unroll
+    for (int k = 0; k < kKvol; ++k) none[k] = -1;
     for (int64_t q = end + r; q <= ptiles * kPosTile; q += kTileRows) {
       if (q < ptiles * kPosTile) ro.pos[q] = -1;
-#pragma unroll
-      for (int dzdy = 0; dzdy < 9; ++dzdy) et_store(ro.et, q, dzdy, -1);
+      et_store_row(ro.et, q, none);
     }
   }
 }
@@ -474,11 +514,11 @@ void launch_query(unsigned blocks, bool runs, const int4* c4, int64_t n, int gri
                   const Tables& t, int32_t* nbr, uint32_t* mask, uint32_t* status,
                   const RunOut& ro, cudaStream_t stream) {
   if (runs)
-    map_query<K, true><<<blocks, kTileRows, 0, stream>>>(c4, n, grid, batch, t, nbr, mask, status,
-                                                         ro);
+    launch_pdl(map_query<K, true>, blocks, kTileRows, 0, stream, c4, n, grid, batch, t, nbr, mask,
+               status, ro);
   else
-    map_query<K, false><<<blocks, kTileRows, 0, stream>>>(c4, n, grid, batch, t, nbr, mask,
-                                                          status, ro);
+    launch_pdl(map_query<K, false>, blocks, kTileRows, 0, stream, c4, n, grid, batch, t, nbr,
+               mask, status, ro);
 }
 
 }  // namespace
@@ -505,9 +545,9 @@ cudaError_t launch_map_build(const int32_t* coords, int64_t n, int32_t grid_dim,
     size_t blocks = (work + 255) / 256;
     if (blocks > 148 * 8) blocks = 148 * 8;
     if (blocks == 0) blocks = 1;
-    map_init<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-        reinterpret_cast<uint4*>(table), words16, reinterpret_cast<uint4*>(ro.lb), lb_words16,
-        status, ro.hdr);
+    launch_pdl(map_init, static_cast<unsigned>(blocks), 256, 0, stream,
+               reinterpret_cast<uint4*>(table), words16, reinterpret_cast<uint4*>(ro.lb),
+               lb_words16, status, ro.hdr);
   }
   if (n == 0) return cudaGetLastError();
   const auto* c4 = reinterpret_cast<const int4*>(coords);
@@ -517,23 +557,22 @@ cudaError_t launch_map_build(const int32_t* coords, int64_t n, int32_t grid_dim,
   t.capmask = static_cast<uint32_t>(lay.capacity - 1);
   if (lay.kind == MapKind::kDirect) {
     t.cells = reinterpret_cast<const int32_t*>(table);
-    map_insert_direct<<<ins_blocks, 256, 0, stream>>>(c4, n, grid_dim, batch,
-                                                      reinterpret_cast<int32_t*>(table), status);
+    launch_pdl(map_insert_direct, ins_blocks, 256, 0, stream, c4, n, grid_dim, batch,
+               reinterpret_cast<int32_t*>(table), status);
     launch_query<Kind::kDirect>(q_blocks, runs, c4, n, grid_dim, batch, t, nbr, mask, status, ro,
                                 stream);
   } else if (lay.compact) {
     t.table = reinterpret_cast<const unsigned long long*>(table);
-    map_insert_compact<<<ins_blocks, 256, 0, stream>>>(
-        c4, n, grid_dim, batch, reinterpret_cast<unsigned long long*>(table), t.capmask, status);
+    launch_pdl(map_insert_compact, ins_blocks, 256, 0, stream, c4, n, grid_dim, batch,
+               reinterpret_cast<unsigned long long*>(table), t.capmask, status);
     launch_query<Kind::kCompact>(q_blocks, runs, c4, n, grid_dim, batch, t, nbr, mask, status,
                                  ro, stream);
   } else {
     auto* rows = reinterpret_cast<int32_t*>(ws + lay.rows_off);
     t.table = reinterpret_cast<const unsigned long long*>(table);
     t.rows = rows;
-    map_insert_wide<<<ins_blocks, 256, 0, stream>>>(c4, n, grid_dim, batch,
-                                                    reinterpret_cast<unsigned long long*>(table),
-                                                    rows, t.capmask, status);
+    launch_pdl(map_insert_wide, ins_blocks, 256, 0, stream, c4, n, grid_dim, batch,
+               reinterpret_cast<unsigned long long*>(table), rows, t.capmask, status);
     launch_query<Kind::kWide>(q_blocks, runs, c4, n, grid_dim, batch, t, nbr, mask, status, ro,
                               stream);
   }

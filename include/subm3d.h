@@ -82,9 +82,10 @@ SUBM3D_API const char* subm3d_status_string(int32_t status);
  * and the lookup table -- a direct-address table of batch * grid_dim^3 int32
  * cells when that is at most 64 MB, else an open-addressing hash table of at
  * least 2N slots (8 bytes each, 12 with batch > 4 or grid_dim > 1024) -- and
- * for N < 2^29 the x-run layout of subm3d_forward_map(): one 8-byte scan word
- * per 128-row tile, a header, a position table of 3N int32 (rounded up) and an
- * E index table of 9 x 260 int32 per 256 positions (~110 bytes per voxel).
+ * for N < 2^29 the x-run layout of subm3d_forward_map(): run-start counts (an
+ * int32 per 128-row tile and per 128 tiles), a header, a position table of 3N
+ * int32 (rounded up) and an E index table of 9 x 260 int32 per 256 positions
+ * (~110 bytes per voxel).
  * Host-only, no CUDA
  * call.  Returns 0 for arguments subm3d_build_map() would
  * reject (N < 0, grid_dim < 1 or > 65535, batch < 1 or > 65535).
@@ -113,9 +114,7 @@ SUBM3D_API size_t subm3d_map_workspace_bytes(int64_t n, int32_t grid_dim, int32_
  * repeated are reported by subm3d_map_status(); until it returns SUBM3D_OK the
  * contents of nbr are unspecified.  Besides nbr and the tile masks the build
  * writes, for N < 2^29, the x-run position layout that subm3d_forward_map()
- * uses; the query kernel's tiles take their run offsets from one another by a
- * single-pass scan whose waits are bounded (SUBM3D_E_TIMEOUT if one runs out).
- * Enqueues 3 kernels; no allocation.
+ * uses.  Enqueues 3 kernels; no allocation.
  * Testing knobs, read from the environment by this function and by
  * subm3d_map_workspace_bytes() alike: SUBM3D_MAP_KIND=hash selects the hash
  * table even where the direct table fits; SUBM3D_TABLE_CAPACITY=<slots> caps
@@ -128,9 +127,8 @@ SUBM3D_API subm3d_status subm3d_build_map(const int32_t* coords, int64_t n, int3
 
 /*
  * Synchronizes the map's stream and returns the device-detected status of the
- * build: SUBM3D_OK, SUBM3D_E_RANGE, SUBM3D_E_DUPLICATE, SUBM3D_E_TABLE_FULL or
- * SUBM3D_E_TIMEOUT (first in that order of precedence), or SUBM3D_E_CUDA.
- * Blocking.
+ * build: SUBM3D_OK, SUBM3D_E_RANGE, SUBM3D_E_DUPLICATE or SUBM3D_E_TABLE_FULL
+ * (first in that order of precedence), or SUBM3D_E_CUDA.  Blocking.
  */
 SUBM3D_API subm3d_status subm3d_map_status(const subm3d_map* map);
 

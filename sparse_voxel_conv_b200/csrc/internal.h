@@ -41,7 +41,6 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 constexpr uint32_t kErrRange = 1u;
 constexpr uint32_t kErrDuplicate = 2u;
 constexpr uint32_t kErrTableFull = 4u;
-constexpr uint32_t kErrTimeout = 8u;  // a bounded wait of the run-offset scan ran out
 
 constexpr int kTileRows = 128;  // rows per tile-mask word
 constexpr int kKvol = 27;
@@ -86,8 +85,9 @@ struct MapLayout {
   size_t table_bytes = 0;   // bytes of the table (a multiple of 16)
   size_t rows_off = 0;      // hash, wide keys only: int32 rows [capacity]
   // run layout (all kinds)
-  size_t lb_off = 0;        // uint64 [n_tiles]: run-offset scan words of the query tiles
-  size_t hdr_off = 0;       // int32 [8]: runs, position tiles, positions, 0, tile ticket
+  size_t cnt_off = 0;       // int32 [n_tiles]: run starts per 128-row tile
+  size_t sb_off = 0;        // int32 [ceil(n_tiles / 128)]: run starts per superblock
+  size_t hdr_off = 0;       // int32 [4]: runs, position tiles, positions, 0
   size_t pos_off = 0;       // int32 [pos_max]: position table (row * 4 + tag, or -1)
   size_t pos_bytes = 0;
   size_t et_off = 0;        // int32 [ptile_max][9][kEtStride]: E index table

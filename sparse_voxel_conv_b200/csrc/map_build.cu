@@ -78,10 +78,10 @@ __device__ __forceinline__ int64_t cell_of(int b, int z, int y, int x, int grid)
   return ((static_cast<int64_t>(b) * grid + z) * grid + y) * grid + x;
 }
 
-// Fills two regions (`words16a`, `words16b` 16-byte words) with all-ones --
-// the lookup table and the run layout's look-back words -- and zeroes the
-// status word and the run layout's header (when there is one).
-__global__ void map_init(uint4* a, size_t words16a, uint4* b, size_t words16b, uint32_t* status,
+// Fills the lookup table (`words16a` 16-byte words) with all-ones, zeroes the
+// run layout's superblock sums (`words16z` words), the status word and the
+// run layout's header (when there is one).
+__global__ void map_init(uint4* a, size_t words16a, uint4* z, size_t words16z, uint32_t* status,
                          int32_t* hdr) {
   pdl_wait();
   pdl_trigger();
@@ -89,21 +89,71 @@ __global__ void map_init(uint4* a, size_t words16a, uint4* b, size_t words16b, u
   const size_t t0 = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const uint4 ones = make_uint4(~0u, ~0u, ~0u, ~0u);
   for (size_t t = t0; t < words16a; t += stride) a[t] = ones;
-  for (size_t t = t0; t < words16b; t += stride) b[t] = ones;
+  for (size_t t = t0; t < words16z; t += stride) z[t] = make_uint4(0u, 0u, 0u, 0u);
   if (t0 == 0) {
     *status = 0u;
     if (hdr)
-      for (int k = 0; k < 8; ++k) hdr[k] = 0;
+      for (int k = 0; k < 4; ++k) hdr[k] = 0;
+  }
+}
+
+// ----------------------------------------------------- run-start counts ----
+// A voxel starts a run unless the previous row is its x-1 neighbour (same b, z,
+// y and x one less).  The insert kernels (256 rows per block = two 128-row
+// tiles) count run starts per tile and add the block's total to its superblock
+// (128 tiles) sum; the query tile then finds the run starts before it by
+// summing the superblock sums before its superblock and the tile counts before
+// it within its superblock -- at most N / 16384 + 127 loads, no waits.
+
+constexpr int kInsertThreads = 2 * kTileRows;
+constexpr int kSuperTiles = 128;
+
+struct RunCount {
+  int32_t* cnt;  // [n_tiles] run starts per 128-row tile (nullptr: no run layout)
+  int32_t* sb;   // [ceil(n_tiles / 128)] run starts per superblock, zeroed by map_init
+};
+
+__device__ __forceinline__ bool x_next(int4 a, int4 b) {  // b is a's x+1 neighbour
+  return a.x == b.x && a.y == b.y && a.z == b.z && a.w + 1 == b.w;
+}
+
+// Called by all kInsertThreads threads of an insert block; c = coords[i] for i < n.
+__device__ __forceinline__ void count_run_starts(const int4* __restrict__ coords, int64_t n,
+                                                 int64_t i, int4 c, const RunCount& rc) {
+  __shared__ int32_t s_cnt[kInsertThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int4 prev;
+  prev.x = __shfl_up_sync(0xFFFFFFFFu, c.x, 1);
+  prev.y = __shfl_up_sync(0xFFFFFFFFu, c.y, 1);
+  prev.z = __shfl_up_sync(0xFFFFFFFFu, c.z, 1);
+  prev.w = __shfl_up_sync(0xFFFFFFFFu, c.w, 1);
+  if (lane == 0 && i > 0 && i < n) prev = __ldg(coords + i - 1);
+  const bool starts = i < n && (i == 0 || !x_next(prev, c));
+  const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, starts);
+  if (lane == 0) s_cnt[warp] = __popc(ballot);
+  __syncthreads();
+  if (threadIdx.x < 2) {
+    const int h = threadIdx.x * 4;
+    const int64_t tile = static_cast<int64_t>(blockIdx.x) * 2 + threadIdx.x;
+    if (tile * kTileRows < n) rc.cnt[tile] = s_cnt[h] + s_cnt[h + 1] + s_cnt[h + 2] + s_cnt[h + 3];
+  }
+  if (threadIdx.x == 0) {
+    int32_t total = 0;
+#pragma unroll
+    for (int w = 0; w < kInsertThreads / 32; ++w) total += s_cnt[w];
+    if (total) atomicAdd(rc.sb + (static_cast<int64_t>(blockIdx.x) * 2) / kSuperTiles, total);
   }
 }
 
 __global__ void map_insert_direct(const int4* __restrict__ coords, int64_t n, int grid, int batch,
-                                  int32_t* __restrict__ cells, uint32_t* status) {
+                                  int32_t* __restrict__ cells, uint32_t* status,
+                                  RunCount rc) {
   pdl_wait();
   pdl_trigger();
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int4 c = i < n ? __ldg(coords + i) : make_int4(-1, -1, -1, -1);
+  if (rc.cnt) count_run_starts(coords, n, i, c, rc);
   if (i >= n) return;
-  const int4 c = __ldg(coords + i);
   if (!in_volume(c, grid, batch)) {
     atomicOr(status, kErrRange);
     return;
@@ -113,12 +163,13 @@ __global__ void map_insert_direct(const int4* __restrict__ coords, int64_t n, in
 
 __global__ void map_insert_compact(const int4* __restrict__ coords, int64_t n, int grid, int batch,
                                    unsigned long long* __restrict__ table, uint32_t capmask,
-                                   uint32_t* status) {
+                                   uint32_t* status, RunCount rc) {
   pdl_wait();
   pdl_trigger();
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int4 c = i < n ? __ldg(coords + i) : make_int4(-1, -1, -1, -1);
+  if (rc.cnt) count_run_starts(coords, n, i, c, rc);
   if (i >= n) return;
-  const int4 c = __ldg(coords + i);
   if (!in_volume(c, grid, batch)) {
     atomicOr(status, kErrRange);
     return;
@@ -141,12 +192,13 @@ __global__ void map_insert_compact(const int4* __restrict__ coords, int64_t n, i
 
 __global__ void map_insert_wide(const int4* __restrict__ coords, int64_t n, int grid, int batch,
                                 unsigned long long* __restrict__ keys, int32_t* __restrict__ rows,
-                                uint32_t capmask, uint32_t* status) {
+                                uint32_t capmask, uint32_t* status, RunCount rc) {
   pdl_wait();
   pdl_trigger();
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int4 c = i < n ? __ldg(coords + i) : make_int4(-1, -1, -1, -1);
+  if (rc.cnt) count_run_starts(coords, n, i, c, rc);
   if (i >= n) return;
-  const int4 c = __ldg(coords + i);
   if (!in_volume(c, grid, batch)) {
     atomicOr(status, kErrRange);
     return;
@@ -206,73 +258,21 @@ __device__ __forceinline__ int32_t lookup(const Tables& t, int b, int z, int y, 
 }
 
 // ----------------------------------------------------------- run layout ----
-// The query kernel also lays out the x-run positions.  Row v starts a run
-// unless row v-1 is its x-1 neighbour (same b, z, y and x one less).  With
-// R(v) the run starts among rows 0..v, voxel v sits at position v + 2 R(v), its
-// run's left pad (when v starts the run) at the position before, the right pad
-// (when v ends it) at the one after.  R needs a count across tiles: every tile
-// publishes its own run-start count as soon as its coordinates are loaded, and
-// after its lookups takes the sum over the earlier tiles by decoupled look-back
-// (Merrill and Garland, "Single-pass Parallel Prefix Scan with Decoupled
-// Look-back", NVIDIA 2016): walk back over the preceding tiles' words, adding
-// their counts, until one that already holds an inclusive prefix.  Tiles take
-// their index from a ticket counter, so every tile waited for has started, and
-// every wait is bounded (2 s on the global timer, then kErrTimeout).
+// The query kernel also lays out the x-run positions: with R(v) the run starts
+// among rows 0..v, voxel v sits at position v + 2 R(v), its run's left pad (when
+// v starts the run) at the position before, the right pad (when v ends it) at
+// the one after.
 
 static_assert(kPosTile == 256, "et_store_row splits positions with shifts by 8");
+static_assert(kInsertThreads == 256 && kSuperTiles % 2 == 0, "insert block = two query tiles");
 
 struct RunOut {
-  unsigned long long* lb;  // [n_tiles] look-back words, all-ones = not published
-  int32_t* hdr;            // [8]: runs, position tiles, positions, 0, tile ticket
-  int32_t* pos;            // position table
-  int32_t* et;             // E index table
+  const int32_t* cnt;  // run starts per 128-row tile (insert kernel)
+  const int32_t* sb;   // run starts per superblock of 128 tiles (insert kernel)
+  int32_t* hdr;        // [4]: runs, position tiles, positions, 0
+  int32_t* pos;        // position table
+  int32_t* et;         // E index table
 };
-
-// Look-back word: flag in bits [62, 64), run-start count in bits [0, 32).
-constexpr unsigned long long kLbAggregate = 1ull << 62;
-constexpr unsigned long long kLbInclusive = 2ull << 62;
-constexpr unsigned long long kLbNotReady = ~0ull;
-constexpr uint64_t kLookbackLimitNs = 2000000000ull;
-
-__device__ __forceinline__ void lb_store(unsigned long long* w, unsigned long long v) {
-  asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(w), "l"(v) : "memory");
-}
-__device__ __forceinline__ unsigned long long lb_load(const unsigned long long* w) {
-  unsigned long long v;
-  asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(w) : "memory");
-  return v;
-}
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-// Run starts in the tiles before `tile`, by one full warp; -1 when a wait ran out.
-__device__ int64_t lookback(const unsigned long long* lb, int64_t tile) {
-  const int lane = threadIdx.x & 31;
-  uint32_t sum = 0;
-  const uint64_t t0 = global_ns();
-  for (int64_t base = tile - 1; base >= 0; base -= 32) {
-    const int64_t j = base - lane;  // lane 0 reads the nearest predecessor
-    // before tile 0 the prefix is 0: an inclusive word with count 0
-    unsigned long long w = j >= 0 ? lb_load(lb + j) : kLbInclusive;
-    while (__any_sync(0xFFFFFFFFu, w == kLbNotReady)) {
-      if (__shfl_sync(0xFFFFFFFFu, global_ns() - t0 > kLookbackLimitNs ? 1 : 0, 0)) return -1;
-      __nanosleep(64);
-      if (w == kLbNotReady) w = lb_load(lb + j);
-    }
-    const uint32_t incl = __ballot_sync(0xFFFFFFFFu, (w >> 62) == 2u);
-    const int stop = incl ? __ffs(incl) - 1 : 31;
-    sum += __reduce_add_sync(0xFFFFFFFFu, lane <= stop ? static_cast<uint32_t>(w) : 0u);
-    if (incl) break;
-  }
-  return sum;
-}
-
-__device__ __forceinline__ bool x_next(int4 a, int4 b) {  // b is a's x+1 neighbour
-  return a.x == b.x && a.y == b.y && a.z == b.z && a.w + 1 == b.w;
-}
 
 // E row q of offset pair dzdy is entry (q mod 256) + 1 of tile q / 256; a tile
 // also keeps copies of its edge rows' outer neighbours (entry 0 of the next
@@ -303,33 +303,33 @@ __global__ void __launch_bounds__(kTileRows)
   __shared__ __align__(16) int32_t s_nbr[kTileRows * kKvol];
   __shared__ uint32_t s_bits[kTileRows / 32];
   __shared__ uint32_t s_starts[kTileRows / 32];  // run-start ballot of each warp
-  __shared__ int64_t s_tile, s_excl, s_end;
+  __shared__ int32_t s_before[kTileRows / 32];   // partial sums of the run starts before the tile
+  __shared__ int64_t s_end;
   const int r = threadIdx.x;
   const int lane = r & 31, warp = r >> 5;
   pdl_wait();
   pdl_trigger();
-  int64_t tile = blockIdx.x;
-  if constexpr (RUNS) {
-    if (r == 0) s_tile = atomicAdd(reinterpret_cast<unsigned int*>(ro.hdr + 4), 1u);
-    __syncthreads();
-    tile = s_tile;
-  }
+  const int64_t tile = blockIdx.x;
   const int64_t row0 = tile * kTileRows;
   const int64_t i = row0 + r;
   int4 c = make_int4(-1, -1, -1, -1);
   if (i < n) c = __ldg(coords + i);
   bool starts = false, ends = false;
-  uint32_t agg = 0;
   if constexpr (RUNS) {
     if (i < n) {
       starts = i == 0 || !x_next(__ldg(coords + i - 1), c);
       ends = i == n - 1 || !x_next(c, __ldg(coords + i + 1));
     }
+    const int64_t sb = tile / kSuperTiles;
+    int32_t part = 0;
+    for (int64_t j = r; j < sb; j += kTileRows) part += __ldg(ro.sb + j);
+    for (int64_t j = sb * kSuperTiles + r; j < tile; j += kTileRows) part += __ldg(ro.cnt + j);
+    part = __reduce_add_sync(0xFFFFFFFFu, part);
     const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, starts);
-    if (lane == 0) s_starts[warp] = ballot;
-    __syncthreads();
-    agg = __popc(s_starts[0]) + __popc(s_starts[1]) + __popc(s_starts[2]) + __popc(s_starts[3]);
-    if (r == 0) lb_store(ro.lb + tile, (tile == 0 ? kLbInclusive : kLbAggregate) | agg);
+    if (lane == 0) {
+      s_starts[warp] = ballot;
+      s_before[warp] = part;
+    }
   }
   uint32_t bits = 0u;
   if (i < n) {
@@ -393,19 +393,10 @@ __global__ void __launch_bounds__(kTileRows)
     for (int e = r; e < rows * kKvol; e += kTileRows) dst[e] = s_nbr[e];
   }
   if constexpr (!RUNS) return;
-  if (warp == 0) {
-    const int64_t excl = tile == 0 ? 0 : lookback(ro.lb, tile);
-    if (lane == 0) {
-      if (excl < 0)
-        atomicOr(status, kErrTimeout);
-      else if (tile > 0)
-        lb_store(ro.lb + tile, kLbInclusive | static_cast<uint32_t>(excl + agg));
-      s_excl = excl;
-    }
-  }
-  __syncthreads();
-  const int64_t excl = s_excl;
-  if (excl < 0) return;
+  // (the __syncthreads above also published s_starts and s_before)
+  const int64_t excl = static_cast<int64_t>(s_before[0]) + s_before[1] + s_before[2] + s_before[3];
+  const uint32_t agg = __popc(s_starts[0]) + __popc(s_starts[1]) + __popc(s_starts[2]) +
+                       __popc(s_starts[3]);
   int64_t runs = excl;  // run starts among rows 0..i
   for (int w = 0; w < warp; ++w) runs += __popc(s_starts[w]);
   runs += __popc(s_starts[warp] & (0xFFFFFFFFu >> (31 - lane)));
@@ -490,15 +481,17 @@ bool map_layout(int64_t n, int32_t grid_dim, int32_t batch, const MapOptions& op
     end = lay.compact ? lay.rows_off : align_up(lay.rows_off + cap * 4, 256);
   }
   if (!opt.run_layout || n >= kRunLayoutMaxRows) {  // nbr and tile masks only
-    lay.lb_off = lay.hdr_off = lay.pos_off = lay.et_off = end;
+    lay.cnt_off = lay.sb_off = lay.hdr_off = lay.pos_off = lay.et_off = end;
     lay.total = end;
     *out = lay;
     return true;
   }
   lay.pos_max = static_cast<int64_t>(align_up(static_cast<size_t>(3 * n), kPosTile)) + kPosTile;
   lay.ptile_max = lay.pos_max / kPosTile;
-  lay.lb_off = end;
-  lay.hdr_off = align_up(lay.lb_off + static_cast<size_t>(lay.n_tiles) * 8, 256);
+  lay.cnt_off = end;
+  lay.sb_off = align_up(lay.cnt_off + static_cast<size_t>(lay.n_tiles) * 4, 256);
+  const int64_t n_super = (lay.n_tiles + kSuperTiles - 1) / kSuperTiles;
+  lay.hdr_off = align_up(lay.sb_off + static_cast<size_t>(n_super) * 4, 256);
   lay.pos_off = lay.hdr_off + 256;
   lay.pos_bytes = static_cast<size_t>(lay.pos_max) * 4;
   lay.et_off = align_up(lay.pos_off + lay.pos_bytes, 256);
@@ -532,47 +525,52 @@ cudaError_t launch_map_build(const int32_t* coords, int64_t n, int32_t grid_dim,
   auto* table = ws + lay.table_off;
   const bool runs = lay.ptile_max > 0;
   RunOut ro{};
+  RunCount rc{};
+  size_t sb_words16 = 0;
   if (runs) {
-    ro.lb = reinterpret_cast<unsigned long long*>(ws + lay.lb_off);
+    rc.cnt = reinterpret_cast<int32_t*>(ws + lay.cnt_off);
+    rc.sb = reinterpret_cast<int32_t*>(ws + lay.sb_off);
+    ro.cnt = rc.cnt;
+    ro.sb = rc.sb;
     ro.hdr = reinterpret_cast<int32_t*>(ws + lay.hdr_off);
     ro.pos = reinterpret_cast<int32_t*>(ws + lay.pos_off);
     ro.et = reinterpret_cast<int32_t*>(ws + lay.et_off);
+    sb_words16 = (lay.hdr_off - lay.sb_off) / 16;  // the 256-byte aligned superblock region
   }
   const size_t words16 = lay.table_bytes / 16;
-  const size_t lb_words16 = runs ? (static_cast<size_t>(lay.n_tiles) * 8 + 15) / 16 : 0;
   {
-    const size_t work = words16 > lb_words16 ? words16 : lb_words16;
+    const size_t work = words16 > sb_words16 ? words16 : sb_words16;
     size_t blocks = (work + 255) / 256;
     if (blocks > 148 * 8) blocks = 148 * 8;
     if (blocks == 0) blocks = 1;
     launch_pdl(map_init, static_cast<unsigned>(blocks), 256, 0, stream,
-               reinterpret_cast<uint4*>(table), words16, reinterpret_cast<uint4*>(ro.lb),
-               lb_words16, status, ro.hdr);
+               reinterpret_cast<uint4*>(table), words16, reinterpret_cast<uint4*>(rc.sb),
+               sb_words16, status, ro.hdr);
   }
   if (n == 0) return cudaGetLastError();
   const auto* c4 = reinterpret_cast<const int4*>(coords);
-  const unsigned ins_blocks = static_cast<unsigned>((n + 255) / 256);
+  const unsigned ins_blocks = static_cast<unsigned>((n + kInsertThreads - 1) / kInsertThreads);
   const unsigned q_blocks = static_cast<unsigned>(lay.n_tiles);
   Tables t{};
   t.capmask = static_cast<uint32_t>(lay.capacity - 1);
   if (lay.kind == MapKind::kDirect) {
     t.cells = reinterpret_cast<const int32_t*>(table);
-    launch_pdl(map_insert_direct, ins_blocks, 256, 0, stream, c4, n, grid_dim, batch,
-               reinterpret_cast<int32_t*>(table), status);
+    launch_pdl(map_insert_direct, ins_blocks, kInsertThreads, 0, stream, c4, n, grid_dim, batch,
+               reinterpret_cast<int32_t*>(table), status, rc);
     launch_query<Kind::kDirect>(q_blocks, runs, c4, n, grid_dim, batch, t, nbr, mask, status, ro,
                                 stream);
   } else if (lay.compact) {
     t.table = reinterpret_cast<const unsigned long long*>(table);
-    launch_pdl(map_insert_compact, ins_blocks, 256, 0, stream, c4, n, grid_dim, batch,
-               reinterpret_cast<unsigned long long*>(table), t.capmask, status);
+    launch_pdl(map_insert_compact, ins_blocks, kInsertThreads, 0, stream, c4, n, grid_dim, batch,
+               reinterpret_cast<unsigned long long*>(table), t.capmask, status, rc);
     launch_query<Kind::kCompact>(q_blocks, runs, c4, n, grid_dim, batch, t, nbr, mask, status,
                                  ro, stream);
   } else {
     auto* rows = reinterpret_cast<int32_t*>(ws + lay.rows_off);
     t.table = reinterpret_cast<const unsigned long long*>(table);
     t.rows = rows;
-    launch_pdl(map_insert_wide, ins_blocks, 256, 0, stream, c4, n, grid_dim, batch,
-               reinterpret_cast<unsigned long long*>(table), rows, t.capmask, status);
+    launch_pdl(map_insert_wide, ins_blocks, kInsertThreads, 0, stream, c4, n, grid_dim, batch,
+               reinterpret_cast<unsigned long long*>(table), rows, t.capmask, status, rc);
     launch_query<Kind::kWide>(q_blocks, runs, c4, n, grid_dim, batch, t, nbr, mask, status, ro,
                               stream);
   }

@@ -156,7 +156,6 @@ subm3d_status subm3d_map_status(const subm3d_map* map) {
   if (word & subm3d::kErrRange) return SUBM3D_E_RANGE;
   if (word & subm3d::kErrDuplicate) return SUBM3D_E_DUPLICATE;
   if (word & subm3d::kErrTableFull) return SUBM3D_E_TABLE_FULL;
-  if (word & subm3d::kErrTimeout) return SUBM3D_E_TIMEOUT;
   return SUBM3D_OK;
 }
 

@@ -44,16 +44,16 @@ def test_version_and_strings(abi):
 
 
 def _expected_ws(n, table_bytes):
-    """Workspace layout: 256-B status block, tile masks, lookup table, one
-    8-byte run-scan word per 128-row tile, 256-B header, position table (3N
-    rounded to 256, + 256), E index table (one [9, 260] int32 block per 256
-    positions); 256-B aligned parts."""
+    """Workspace layout: 256-B status block, tile masks, lookup table, run-start
+    counts (one int32 per 128-row tile, one per 128 tiles), 256-B header,
+    position table (3N rounded to 256, + 256), E index table (one [9, 260]
+    int32 block per 256 positions); 256-B aligned parts."""
     up = lambda v: (v + 255) // 256 * 256
     head = up(256 + 4 * ((n + 127) // 128))
-    lb = 8 * ((n + 127) // 128)
+    tiles = (n + 127) // 128
     pos_max = up(3 * n) + 256
     after_table = up(head + table_bytes)
-    pos_off = up(after_table + lb) + 256
+    pos_off = up(up(after_table + 4 * tiles) + 4 * ((tiles + 127) // 128)) + 256
     et_off = up(pos_off + 4 * pos_max)
     return up(et_off + (pos_max // 256) * 9 * 260 * 4)
 

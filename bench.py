@@ -164,6 +164,62 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def _time_ms(fn, flush, reps=5, warm=2):
+    """Median CUDA-event time of fn() over `reps` calls, L2 flushed before each."""
+    import torch
+    for _ in range(warm):
+        fn()
+    ts = []
+    for _ in range(reps):
+        flush.fill_(7)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts)
+
+
+def fp32_forward_line(h, feats_f32, w_f32, flops, flush, sm_mhz):
+    """The fp32 path (CUDA-core FMA) on the same map, against the FP32 peak
+    SMs x 128 lanes x 2 flop x SM clock."""
+    import torch
+    import sparse_voxel_conv_b200 as S
+    out = torch.empty((h.n, w_f32.shape[0]), dtype=torch.float32, device=feats_f32.device)
+    ms = _time_ms(lambda: S.forward(h, feats_f32, w_f32, out=out), flush)
+    sms = torch.cuda.get_device_properties(feats_f32.device).multi_processor_count
+    peak = sms * 128 * 2 * sm_mhz * 1e6 / 1e12
+    achieved = flops / (ms / 1e3) / 1e12
+    return {"bound": "alu", "ms": ms, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak,
+            "peak_source": f"{sms} SMs x 128 FP32 lanes x 2 x {sm_mhz:.0f} MHz"}
+
+
+def per_offset_context(h, feats, weight, flush):
+    """The pages' "obvious per-offset loop" in torch on this GPU, as context:
+    27 x (index_select + matmul + index_add_) over this library's nbr, fp32
+    accumulation.  Not part of the timed step."""
+    import torch
+    nbr = h.nbr.long()
+    cout = weight.shape[0]
+    w = weight.reshape(cout, 27, -1)
+    acc = torch.empty((h.n, cout), dtype=torch.float32, device=feats.device)
+    rows = [(nbr[:, k] >= 0).nonzero().squeeze(1) for k in range(27)]
+    src = [nbr[r, k] for k, r in enumerate(rows)]
+
+    def loop():
+        acc.zero_()
+        for k in range(27):
+            part = feats.index_select(0, src[k]) @ w[:, k, :].t()
+            acc.index_add_(0, rows[k], part.float())
+        return acc.to(feats.dtype)
+
+    ms = _time_ms(loop, flush, reps=3, warm=1)
+    return {"ms": ms, "what": "27 x (index_select + bf16 matmul + index_add_) in torch, "
+            "fp32 accumulation, indices precomputed from this library's nbr"}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -325,6 +381,14 @@ def run_ours(args):
             "gpu_launches": (MAP_LAUNCHES + 1) * K,
             "clocks": clocks,
         }
+        if world == 1 and not args.no_context:
+            h_ctx = step()
+            torch.cuda.synchronize()
+            flops_alg = 2.0 * nnz_total * cin * cout
+            line["fp32_forward"] = fp32_forward_line(
+                h_ctx, feats.float(), weight.float(), flops_alg, flush,
+                float(clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965.0))
+            line["context_per_offset_torch"] = per_offset_context(h_ctx, feats, weight, flush)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl, args.cpu_rows)
         print(json.dumps(line), flush=True)
@@ -413,6 +477,8 @@ def main():
     ap.add_argument("--workload", default="headline", choices=["headline", "dense", "shell_bf16"])
     ap.add_argument("--cpu-rows", type=int, default=40000)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-context", action="store_true",
+                    help="skip the fp32-path and per-offset-loop context measurements")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

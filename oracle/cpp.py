@@ -46,6 +46,7 @@ def load():
                                        ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                        ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p]
         lib.oracle_gelu.argtypes = [ctypes.c_void_p, ctypes.c_int64]
+        lib.oracle_silu.argtypes = [ctypes.c_void_p, ctypes.c_int64]
         lib.oracle_round_bf16.argtypes = [ctypes.c_void_p, ctypes.c_int64]
         del i64p
         _lib = lib
@@ -72,8 +73,9 @@ def build_map(coords, grid_dim: int, batch: int = 1) -> np.ndarray:
 
 
 def forward(nbr, x, w, flip: bool = False, act: str | None = None,
-            round_to_bf16: bool = False, rows=None) -> np.ndarray:
-    """fp64 forward over all rows or a subset (see oracle_forward)."""
+            round_to_bf16: bool = False, rows=None, bias=None, residual=None) -> np.ndarray:
+    """fp64 forward over all rows or a subset (see oracle_forward), then the
+    epilogue act(sum + bias) + residual and an optional bf16 rounding."""
     nbr = np.ascontiguousarray(nbr, np.int32)
     x = np.ascontiguousarray(x, np.float64)
     w = np.ascontiguousarray(w, np.float64)
@@ -88,10 +90,17 @@ def forward(nbr, x, w, flip: bool = False, act: str | None = None,
     out = np.empty((n_rows, cout), np.float64)
     load().oracle_forward(nbr.ctypes.data, x.ctypes.data, w.ctypes.data, cin, cout,
                           1 if flip else 0, rows_ptr, n_rows, out.ctypes.data)
+    if bias is not None:
+        out += np.asarray(bias, np.float64)[None, :]
     if act == "gelu":
         load().oracle_gelu(out.ctypes.data, out.size)
+    elif act == "silu":
+        load().oracle_silu(out.ctypes.data, out.size)
     elif act is not None:
         raise ValueError(f"unknown activation {act!r}")
+    if residual is not None:
+        res = np.asarray(residual, np.float64)
+        out += res if rows_arr is None else res[rows_arr]
     if round_to_bf16:
         load().oracle_round_bf16(out.ctypes.data, out.size)
     return out
@@ -100,6 +109,12 @@ def forward(nbr, x, w, flip: bool = False, act: str | None = None,
 def gelu(v) -> np.ndarray:
     v = np.array(v, np.float64, copy=True, order="C")
     load().oracle_gelu(v.ctypes.data, v.size)
+    return v
+
+
+def silu(v) -> np.ndarray:
+    v = np.array(v, np.float64, copy=True, order="C")
+    load().oracle_silu(v.ctypes.data, v.size)
     return v
 
 

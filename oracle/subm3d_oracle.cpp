@@ -106,6 +106,11 @@ void oracle_gelu(double* v, int64_t n) {
   for (int64_t i = 0; i < n; ++i) v[i] = 0.5 * v[i] * (1.0 + std::erf(v[i] / std::sqrt(2.0)));
 }
 
+// SiLU in place: v <- v * sigmoid(v) = v / (1 + exp(-v)).
+void oracle_silu(double* v, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) v[i] = v[i] / (1.0 + std::exp(-v[i]));
+}
+
 // Round in place to the nearest bfloat16 value, ties to even.  bfloat16 keeps
 // 8 significant bits and float32's exponent range (normal numbers down to
 // 2^-126, subnormal spacing 2^-133, largest finite (2 - 2^-7) * 2^127).

@@ -27,7 +27,7 @@ import math
 
 import numpy as np
 
-__all__ = ["OFFSETS", "OracleError", "build_map", "forward", "gelu", "round_bf16",
+__all__ = ["OFFSETS", "OracleError", "build_map", "forward", "gelu", "silu", "round_bf16",
            "brute_force_map"]
 
 # (dz, dy, dx) for k = 0..26, kz-major: dz slowest, dx fastest.
@@ -72,13 +72,16 @@ def brute_force_map(coords) -> np.ndarray:
 
 
 def forward(nbr, x, w, flip: bool = False, act: str | None = None,
-            round_to_bf16: bool = False, rows=None) -> np.ndarray:
-    """out[i] = sum_k Wf[:, k, :] @ x[nbr[i, k]] over nbr[i, k] != -1, in fp64.
+            round_to_bf16: bool = False, rows=None, bias=None, residual=None) -> np.ndarray:
+    """out[i] = act(sum_k Wf[:, k, :] @ x[nbr[i, k]] + bias) + residual[i], in fp64.
 
-    x: [N, Cin]; w: KRSC [Cout, 3, 3, 3, Cin] (or [Cout, 27, Cin]).
-    Wf[:, k] = w[:, k] (correlation) or w[:, 26 - k] (flip).
-    act: None or "gelu" (exact erf form), applied to the fp64 sum.
-    round_to_bf16: round the result to bf16 (RNE) as a bf16 output would be.
+    The sum runs over nbr[i, k] != -1.  x: [N, Cin]; w: KRSC [Cout, 3, 3, 3, Cin]
+    (or [Cout, 27, Cin]).  Wf[:, k] = w[:, k] (correlation) or w[:, 26 - k] (flip).
+    bias: optional [Cout], added to the sum.  act: None, "gelu" (exact erf form)
+    or "silu" (v * sigmoid(v)), applied after the bias.  residual: optional
+    [N, Cout], added after the activation -- the epilogue of a sparse residual
+    block's second convolution (conv + bias + skip).
+    round_to_bf16: round the result to bf16 (RNE) once, as a bf16 output would be.
     rows: optional subset of output rows (the result then has len(rows) rows).
     """
     nbr = np.asarray(nbr)
@@ -97,10 +100,16 @@ def forward(nbr, x, w, flip: bool = False, act: str | None = None,
             kw = 26 - k if flip else k
             acc += w27[:, kw, :] @ x[j]
         out[p] = acc
+    if bias is not None:
+        out = out + np.asarray(bias, np.float64)[None, :]
     if act == "gelu":
         out = gelu(out)
+    elif act == "silu":
+        out = silu(out)
     elif act is not None:
         raise ValueError(f"unknown activation {act!r}")
+    if residual is not None:
+        out = out + np.asarray(residual, np.float64)[list(rows)]
     if round_to_bf16:
         out = round_bf16(out)
     return out
@@ -111,6 +120,13 @@ def gelu(v) -> np.ndarray:
     v = np.asarray(v, np.float64)
     erf = np.vectorize(math.erf, otypes=[np.float64])
     return 0.5 * v * (1.0 + erf(v / math.sqrt(2.0)))
+
+
+def silu(v) -> np.ndarray:
+    """SiLU, v * sigmoid(v) = v / (1 + exp(-v)), element-wise in fp64."""
+    v = np.asarray(v, np.float64)
+    with np.errstate(over="ignore"):
+        return v / (1.0 + np.exp(-v))
 
 
 def round_bf16(v) -> np.ndarray:

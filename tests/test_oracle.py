@@ -373,3 +373,69 @@ def test_workload_sizes():
     for c in (WL.tiny_coords(), WL.shell_coords()):
         keys = [tuple(r) for r in c.tolist()]
         assert keys == sorted(keys) and len(set(keys)) == len(keys)
+
+
+# -------------------------------------------- fused residual-block epilogue ---
+
+def _dense_block(c, x, w, bias, residual, g, batch, flip, act):
+    """torch's dense Conv3d with its own bias argument, torch's activation, then
+    the residual: the epilogue act(conv + bias) + residual on a full grid."""
+    cin = x.shape[1]
+    xd = torch.zeros(batch, cin, g, g, g, dtype=torch.float64)
+    ct = torch.from_numpy(c.astype(np.int64))
+    xd[ct[:, 0], :, ct[:, 1], ct[:, 2], ct[:, 3]] = torch.from_numpy(x)
+    wt = torch.from_numpy(w).permute(0, 4, 1, 2, 3)
+    if flip:
+        wt = wt.flip(2, 3, 4)
+    yd = F.conv3d(xd, wt, bias=torch.from_numpy(bias), padding=1)
+    y = yd[ct[:, 0], :, ct[:, 1], ct[:, 2], ct[:, 3]]
+    y = {"gelu": F.gelu, "silu": F.silu, None: lambda t: t}[act](y)
+    return (y + torch.from_numpy(residual)).numpy()
+
+
+@pytest.mark.parametrize("orc", ORACLES)
+@pytest.mark.parametrize("act", [None, "gelu", "silu"])
+@pytest.mark.parametrize("flip", [False, True])
+def test_block_epilogue_equals_dense_conv3d_bias_act_residual(orc, act, flip):
+    g, batch, cin, cout = 5, 2, 3, 4
+    c, x, w = _dense_case(g, batch, cin, cout, seed=11)
+    rng = np.random.default_rng(12)
+    bias = rng.standard_normal(cout)
+    residual = rng.standard_normal((c.shape[0], cout))
+    nbr = orc.build_map(c, g, batch)
+    out = orc.forward(nbr, x, w, flip=flip, act=act, bias=bias, residual=residual)
+    ref = _dense_block(c, x, w, bias, residual, g, batch, flip, act)
+    assert np.max(np.abs(out - ref)) <= 1e-12 * max(1.0, np.max(np.abs(ref)))
+    # the residual enters after the activation and the bias before it
+    if act is not None:
+        no_res = orc.forward(nbr, x, w, flip=flip, act=act, bias=bias)
+        assert np.max(np.abs(out - no_res - residual)) <= 1e-12
+
+
+def test_block_epilogue_rows_and_bf16_rounding_once():
+    wl = WL.make_workload("tiny")
+    nbr = C.build_map(wl.coords, wl.grid_dim)
+    x = wl.features().astype(np.float64)
+    w = wl.weights()[0].astype(np.float64)
+    rng = np.random.default_rng(3)
+    bias = rng.standard_normal(w.shape[0])
+    res = rng.standard_normal((wl.n, w.shape[0]))
+    full = C.forward(nbr, x, w, act="silu", bias=bias, residual=res)
+    rows = np.array([0, 5, 77, wl.n - 1])
+    part = C.forward(nbr, x, w, act="silu", bias=bias, residual=res, rows=rows)
+    assert np.array_equal(part, full[rows])
+    # the Python oracle agrees, and bf16 rounding is applied once, at the end
+    py = P.forward(nbr, x, w, act="silu", bias=bias, residual=res, rows=rows, round_to_bf16=True)
+    assert np.array_equal(py, P.round_bf16(full[rows]))
+
+
+@pytest.mark.parametrize("orc", [P, C])
+def test_silu_closed_forms_and_torch(orc):
+    v = np.linspace(-30.0, 30.0, 4001)
+    got = orc.silu(v)
+    ref = F.silu(torch.from_numpy(v)).numpy()
+    assert np.max(np.abs(got - ref)) <= 1e-14 * np.max(np.abs(ref))
+    assert orc.silu(np.array([0.0]))[0] == 0.0
+    # silu(v) - silu(-v) = v (sigmoid(v) + sigmoid(-v) = 1), and silu(1) = 1/(1+e^-1)
+    assert np.max(np.abs(orc.silu(v) - orc.silu(-v) - v)) <= 1e-13
+    assert abs(orc.silu(np.array([1.0]))[0] - 1.0 / (1.0 + math.exp(-1.0))) < 1e-15

@@ -220,6 +220,24 @@ def per_offset_context(h, feats, weight, flush):
             "fp32 accumulation, indices precomputed from this library's nbr"}
 
 
+def fused_epilogue_line(h, feats, weight, flops, flush, peak_tf, plain_ms):
+    """The residual-block epilogue fused into the headline forward:
+    out = silu(conv + bias) + residual, against the same tensor-core peak."""
+    import torch
+    import sparse_voxel_conv_b200 as S
+    cout = weight.shape[0]
+    bias = torch.linspace(-0.5, 0.5, cout, device=feats.device).to(feats.dtype)
+    res = torch.empty((h.n, cout), dtype=feats.dtype, device=feats.device).normal_()
+    out = torch.empty_like(res)
+    ms = _time_ms(lambda: S.forward(h, feats, weight, act="silu", bias=bias, residual=res,
+                                    out=out), flush)
+    achieved = flops / (ms / 1e3) / 1e12
+    return {"what": "silu(conv + bias) + residual in the forward's epilogue",
+            "ms": ms, "plain_forward_ms": plain_ms, "achieved": achieved, "peak": peak_tf,
+            "unit": "TFLOP/s", "frac": achieved / peak_tf,
+            "extra_bytes": int(h.n) * cout * feats.element_size()}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -388,6 +406,8 @@ def run_ours(args):
             line["fp32_forward"] = fp32_forward_line(
                 h_ctx, feats.float(), weight.float(), flops_alg, flush,
                 float(clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965.0))
+            line["fused_epilogue"] = fused_epilogue_line(h_ctx, feats, weight, flops_alg, flush,
+                                                         peak_tf, fwd_avg_s * 1e3)
             line["context_per_offset_torch"] = per_offset_context(h_ctx, feats, weight, flush)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl, args.cpu_rows)

@@ -65,7 +65,7 @@ typedef enum {
 } subm3d_status;
 
 typedef enum { SUBM3D_F32 = 0, SUBM3D_BF16 = 1 } subm3d_dtype;
-typedef enum { SUBM3D_ACT_NONE = 0, SUBM3D_ACT_GELU = 1 } subm3d_act;
+typedef enum { SUBM3D_ACT_NONE = 0, SUBM3D_ACT_GELU = 1, SUBM3D_ACT_SILU = 2 } subm3d_act;
 
 /* Opaque handle of a built neighbour map (host memory; see subm3d_build_map). */
 typedef struct subm3d_map subm3d_map;
@@ -160,7 +160,9 @@ SUBM3D_API void subm3d_map_destroy(subm3d_map* map);
  *   dtype      SUBM3D_BF16: bf16 feats/weight/out, fp32 accumulation on the tensor
  *              cores, Cin and Cout multiples of 16 (else SUBM3D_E_UNSUPPORTED).
  *              SUBM3D_F32: fp32 throughout on CUDA-core FMA, any Cin, Cout >= 1.
- *   act        SUBM3D_ACT_NONE, or SUBM3D_ACT_GELU (exact erf form) on the fp32 sum.
+ *   act        SUBM3D_ACT_NONE, SUBM3D_ACT_GELU (exact erf form) or SUBM3D_ACT_SILU
+ *              (v * sigmoid(v)) on the fp32 sum; a bf16 output is rounded once,
+ *              after the activation.
  *
  * The forward never fails on data.  SUBM3D_E_UNSUPPORTED is also returned when
  * the current device is not sm_100.  A bounded device-side wait that runs out
@@ -215,8 +217,7 @@ SUBM3D_API subm3d_status subm3d_build_map_noalloc(const int32_t* coords, int64_t
  * Forward of one layer over a built map -- the same op and arguments as
  * subm3d_forward(), with N, nbr and the masks taken from the map.  For bf16
  * with Cin a multiple of 64 (and a map of N < 2^29) it runs the x-run kernel,
- * which uses the map's
- * position layout: voxels on a line of positions in row order, two pad
+ * which uses the map's position layout: voxels on a line of positions in row order, two pad
  * positions before every run of x-adjacent voxels, tiles of 256 positions,
  * and per tile and (dz, dy) one gathered tile of feature rows whose rows
  * p-1, p, p+1 are the dx = -1, 0, +1 neighbours of the voxel at position p;
@@ -228,6 +229,32 @@ SUBM3D_API subm3d_status subm3d_forward_map(const subm3d_map* map, const void* f
                                             const void* weight, void* out, int32_t cin,
                                             int32_t cout, subm3d_dtype dtype, int32_t flip,
                                             subm3d_act act, void* stream);
+
+/*
+ * One layer with the epilogue of a sparse residual block fused into its store:
+ *
+ *   out[i] = act( sum_k Wf[:, k, :] . feats[nbr[i][k]] + bias ) + residual[i]
+ *
+ * -- the first convolution of a block takes a bias and an activation, the
+ * second a bias and the block's skip input as residual, both on one map.  The
+ * pages define the convolution only; this epilogue is the plain reading of
+ * "conv + bias, activation, skip add" for the decoders' residual blocks.
+ *
+ *   bias      (device) [Cout] in the feature dtype, or NULL.  Added to the fp32
+ *             sum before the activation.  2-byte aligned (bf16) / 4 (fp32).
+ *   residual  (device) [N, Cout] in the feature dtype, or NULL.  Added after the
+ *             activation, before the single rounding of a bf16 output.  It may
+ *             be `out` itself (an in-place skip add) or overlap feats; a partial
+ *             overlap with out is SUBM3D_E_INVALID.  16-byte aligned (bf16,
+ *             else SUBM3D_E_UNSUPPORTED) / 4-byte (fp32, else E_INVALID).
+ *
+ * Everything else -- arguments, kernels chosen, errors -- as subm3d_forward_map().
+ */
+SUBM3D_API subm3d_status subm3d_forward_fused(const subm3d_map* map, const void* feats,
+                                              const void* weight, const void* bias,
+                                              const void* residual, void* out, int32_t cin,
+                                              int32_t cout, subm3d_dtype dtype, int32_t flip,
+                                              subm3d_act act, void* stream);
 
 /*
  * Device pointers into the map's x-run layout, for tests and tools: the

@@ -28,6 +28,7 @@ SUBM3D_F32 = 0
 SUBM3D_BF16 = 1
 SUBM3D_ACT_NONE = 0
 SUBM3D_ACT_GELU = 1
+SUBM3D_ACT_SILU = 2
 SUBM3D_KVOL = 27
 SUBM3D_TILE_ROWS = 128
 
@@ -64,6 +65,8 @@ def _load() -> ctypes.CDLL:
                                               ctypes.c_int, vp]),
         "subm3d_map_run_layout": (ctypes.c_int, [vp, ctypes.POINTER(vp), ctypes.POINTER(vp),
                                                  ctypes.POINTER(vp)]),
+        "subm3d_forward_fused": (ctypes.c_int, [vp, vp, vp, vp, vp, vp, i32, i32, ctypes.c_int,
+                                                i32, ctypes.c_int, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -182,6 +185,17 @@ def subm3d_forward_map(handle: MapHandle, feats, weight, out, cin: int, cout: in
                                 int(cout), int(dtype), 1 if flip else 0, int(act),
                                 _stream(stream))
     _check(st, "subm3d_forward_map")
+
+
+def subm3d_forward_fused(handle: MapHandle, feats, weight, bias, residual, out, cin: int,
+                         cout: int, dtype: int, flip: bool, act: int, stream=None) -> None:
+    """Enqueue one layer with the residual-block epilogue act(conv + bias) +
+    residual (bias / residual may be None); raises Subm3dError on an argument
+    error."""
+    st = lib.subm3d_forward_fused(handle.ptr, _ptr(feats), _ptr(weight), _ptr(bias),
+                                  _ptr(residual), _ptr(out), int(cin), int(cout), int(dtype),
+                                  1 if flip else 0, int(act), _stream(stream))
+    _check(st, "subm3d_forward_fused")
 
 
 def subm3d_map_run_layout(handle: MapHandle):

@@ -1,0 +1,149 @@
+// Epilogue arithmetic shared by the forward kernels:
+//   out = act(acc + bias) + residual,
+// bias added to the fp32 accumulator, then the activation, then the residual,
+// and a bf16 output rounded once (round to nearest even) at the end.  The
+// epilogue of a sparse residual block: the first convolution takes a bias and
+// an activation, the second a bias and the block's skip input as residual.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace subm3d {
+
+template <int ACT>
+__device__ __forceinline__ float activate(float v) {
+  if constexpr (ACT == kActGelu) {
+    return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f));  // exact erf form
+  } else if constexpr (ACT == kActSilu) {
+    // v * sigmoid(v) with the fast exponential and the fast divide (a few ulp,
+    // well inside both paths' bars); for v -> -inf the divisor overflows to inf
+    // and the quotient is -0
+    return __fdividef(v, 1.0f + __expf(-v));
+  } else {
+    return v;
+  }
+}
+
+// Eight fp32 values + an optional bf16 residual chunk -> eight bf16 (one rounding).
+__device__ __forceinline__ uint4 finish_bf16x8(const float (&f)[8], bool has_residual,
+                                               uint4 r) {
+  float g[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) g[j] = f[j];
+  if (has_residual) {
+    const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      g[2 * j] += __uint_as_float(rw[j] << 16);
+      g[2 * j + 1] += __uint_as_float(rw[j] & 0xFFFF0000u);
+    }
+  }
+  uint32_t w[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(g[2 * j], g[2 * j + 1]);
+    w[j] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Bytes of fp32 staging one bf16 epilogue warp needs: 32 positions x 32 channels.
+constexpr int kEpiWarpStageBytes = 32 * 32 * 4;
+
+// The epilogue of one 256-position accumulator by one warp: its 32 channels
+// (TMEM lanes; lane = channel o_warp + lane) in 8 chunks of 32 positions.  Per
+// chunk the fp32 values (bias, activation) go to the warp's staging area
+// (`stage`, kEpiWarpStageBytes; a position's 128-byte row has its 16-byte halves
+// swapped at odd positions, so the reads below are free of bank conflicts),
+// then each lane takes 8 channels of one position, adds the residual and
+// stores 16 bytes.  The output row of position j is pos[j] >> 2 when pos[j] is
+// a voxel entry (POS: the x-run layout; pads and empty positions are dropped),
+// else row0 + j below n.  Latency is hidden by prefetching: position entries
+// two chunks ahead and each chunk's residual rows one chunk ahead, so they load
+// while the previous chunk is staged.  The chunk loop stays rolled: an
+// unrolled one inlines 256 activations and slows every warp of the kernel.
+template <int ACT, bool POS>
+__device__ __forceinline__ void epilogue_tile_bf16(uint32_t taddr, float bias_v, uint32_t stage,
+                                                   int lane, int o_warp, int cout,
+                                                   const int32_t* pos, int64_t row0, int64_t n,
+                                                   __nv_bfloat16* out,
+                                                   const __nv_bfloat16* residual) {
+  constexpr int kChunks = 8;
+  const int q = lane % 4;  // this lane's 8-channel group in the store phase
+  const int o = o_warp + q * 8;
+  const bool o_ok = o < cout;
+  // rows (int32: N < 2^31) of this lane's 4 store slots of chunk ci, -1 to skip;
+  // pe = the pos entry of position ci * 32 + lane (POS)
+  auto rows_of = [&](int ci, int32_t pe, int32_t (&r)[4]) {
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const int jj = p * 8 + lane / 4;
+      if constexpr (POS) {
+        const int32_t e = __shfl_sync(0xFFFFFFFFu, pe, jj);
+        r[p] = (e >= 0 && (e & 3) == kPosVoxel) ? (e >> 2) : -1;
+      } else {
+        const int64_t row = row0 + ci * 32 + jj;
+        r[p] = row < n ? static_cast<int32_t>(row) : -1;
+      }
+    }
+  };
+  auto load_res = [&](const int32_t (&r)[4], uint4 (&v)[4]) {
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+      v[p] = (residual && r[p] >= 0 && o_ok)
+                 ? *reinterpret_cast<const uint4*>(residual + static_cast<int64_t>(r[p]) * cout + o)
+                 : make_uint4(0u, 0u, 0u, 0u);
+  };
+  // chunk 0's rows and residual now, chunk 1's pos entry in flight
+  int32_t pe_next = POS ? __ldg(pos + 32 + lane) : 0;
+  int32_t rows[4];
+  uint4 res[4];
+  rows_of(0, POS ? __ldg(pos + lane) : 0, rows);
+  load_res(rows, res);
+#pragma unroll 1
+  for (int ci = 0; ci < kChunks; ++ci) {
+    uint32_t v[32];
+    tmem_ld_32x32b_x32(taddr + ci * 32, v);
+    int32_t rows_n[4];
+    uint4 res_n[4];
+    if (ci + 1 < kChunks) {  // next chunk's rows and residual (and the pos entry after it)
+      rows_of(ci + 1, pe_next, rows_n);
+      load_res(rows_n, res_n);
+      if (POS && ci + 2 < kChunks) pe_next = __ldg(pos + (ci + 2) * 32 + lane);
+    }
+    tmem_ld_wait();
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const float f = activate<ACT>(__uint_as_float(v[e]) + bias_v);
+      sts_u32(stage + e * 128 + ((lane * 4) ^ ((e & 1) << 4)), __float_as_uint(f));
+    }
+    __syncwarp();
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const int j = p * 8 + lane / 4;
+      const uint32_t rb = stage + j * 128;
+      const uint32_t sw = static_cast<uint32_t>(j & 1) << 4;
+      const uint4 lo = lds_16(rb + ((q * 32) ^ sw));
+      const uint4 hi = lds_16(rb + ((q * 32 + 16) ^ sw));
+      if (rows[p] >= 0 && o_ok) {
+        const float f[8] = {__uint_as_float(lo.x), __uint_as_float(lo.y), __uint_as_float(lo.z),
+                            __uint_as_float(lo.w), __uint_as_float(hi.x), __uint_as_float(hi.y),
+                            __uint_as_float(hi.z), __uint_as_float(hi.w)};
+        *reinterpret_cast<uint4*>(out + static_cast<int64_t>(rows[p]) * cout + o) =
+            finish_bf16x8(f, residual != nullptr, res[p]);
+      }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      rows[p] = rows_n[p];
+      res[p] = res_n[p];
+    }
+  }
+}
+
+}  // namespace subm3d

@@ -1,7 +1,7 @@
 // bf16 forward over the x-run position layout, sm_100a tensor cores.
 //
 // Same op as forward_bf16_sm100.cu: out[i] = act( sum_k Wf[:, k, :] .
-// x[nbr[i][k]] ), Wf[:, k] = W[:, k] or W[:, 26-k] (flip), KRSC weights
+// x[nbr[i][k]] + bias ) + residual[i], Wf[:, k] = W[:, k] or W[:, 26-k] (flip), KRSC weights
 // (lato.2_mrp_mlx, commit 97dcdfb54a message and CLAUDE.md "Key facts").
 //
 // The map build lays the voxels out on a line of positions in row order, with
@@ -36,9 +36,10 @@
 //       The 128-byte swizzle XORs with address bits [7,10) of each row's own
 //       address, so a view shifted by whole 128-byte rows in a 1024-aligned
 //       slot is the same swizzled layout: base offset 0, start + dx * 128.
-//   warps 0-3       epilogue of the other accumulator: tcgen05.ld, optional
-//       exact-erf GELU, bf16, a transpose through shared memory, and 16-byte
-//       stores to the rows of the voxel positions (pad columns are dropped).
+//   warps 0-3       epilogue of the other accumulator: tcgen05.ld, bias,
+//       activation (none, exact GELU, SiLU), a transpose through fp32 shared
+//       memory, the residual, one bf16 rounding and 16-byte stores to the rows
+//       of the voxel positions (pad columns are dropped).
 //
 // Every wait is bounded (ptx.cuh); a wait that runs out sets the library's
 // device error word, the CTA lets its copies land, frees TMEM and exits.
@@ -50,6 +51,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "epilogue.cuh"
 
 namespace subm3d {
 namespace {
@@ -70,7 +72,7 @@ constexpr int kERows = TP + 2;                                   // rows -1 .. 2
 constexpr uint32_t E_SLOT = ((kERows * ROW_BYTES + 1023) / 1024) * 1024;  // 33792
 constexpr uint32_t IDX_BYTES = kEtStride * 4;                  // 1040
 constexpr uint32_t A_SLOT = TO * ROW_BYTES;                      // 16384
-constexpr int kEpiStageBytes = NUM_EPI_WARPS * 32 * 64;
+constexpr int kEpiStageBytes = NUM_EPI_WARPS * kEpiWarpStageBytes;
 constexpr uint32_t kTmemCols = 2 * TP;
 
 struct RunArgs {
@@ -79,6 +81,8 @@ struct RunArgs {
   const int32_t* hdr;     // [runs, position tiles, positions, 0]
   const __nv_bfloat16* x;
   __nv_bfloat16* out;
+  const __nv_bfloat16* bias;      // [cout] or nullptr
+  const __nv_bfloat16* residual;  // [N, cout] or nullptr; may be `out`
   int32_t cin, cout, n_oblocks, n_kchunks, se, sw, flip;
   int32_t* err_word;
 };
@@ -147,11 +151,7 @@ struct Ring {
   }
 };
 
-__device__ __forceinline__ float gelu_erf(float v) {
-  return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f));
-}
-
-template <bool GELU>
+template <int ACT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     subm3d_fwd_bf16_runs_sm100(const __grid_constant__ CUtensorMap wmap, const RunArgs a) {
   constexpr int PPR = CHUNK / 8;                       // 16-byte pieces per row: 8
@@ -328,7 +328,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // --------------------------------------------------------- epilogue ----
-    const uint32_t stage = smem_u32(epi_s) + static_cast<uint32_t>(warp) * (32 * 64);
+    const uint32_t stage =
+        smem_u32(epi_s) + static_cast<uint32_t>(warp) * static_cast<uint32_t>(kEpiWarpStageBytes);
     int local = 0;
     for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x, ++local) {
       const int acc = local & 1;
@@ -336,34 +337,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const int64_t tile = u / a.n_oblocks;
       const int o_warp = static_cast<int>(u % a.n_oblocks) * TO + warp * 32;
+      const float bias_v =
+          (a.bias && o_warp + lane < a.cout) ? __bfloat162float(a.bias[o_warp + lane]) : 0.0f;
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(acc * TP);
-      const int32_t* pos = a.pos + tile * TP;
-#pragma unroll 1
-      for (int c0 = 0; c0 < TP; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(taddr + c0, v);  // lane = channel o_warp + lane, 32 positions
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          float f = __uint_as_float(v[e]);
-          if constexpr (GELU) f = gelu_erf(f);
-          const __nv_bfloat16 h = __float2bfloat16_rn(f);
-          sts_u16(stage + e * 64 + lane * 2, *reinterpret_cast<const uint16_t*>(&h));
-        }
-        __syncwarp();
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          const int vv = p * 8 + lane / 4;  // position within the 32
-          const int q = lane % 4;           // 8-channel group
-          const int32_t e = __ldg(pos + c0 + vv);
-          const uint4 val = lds_16(stage + vv * 64 + q * 16);
-          const int o = o_warp + q * 8;
-          if (e >= 0 && (e & 3) == kPosVoxel && o < a.cout)
-            *reinterpret_cast<uint4*>(a.out + static_cast<int64_t>(e >> 2) * a.cout + o) = val;
-        }
-        __syncwarp();
-      }
+      // voxel positions store to their row; pads and empty positions are dropped
+      epilogue_tile_bf16<ACT, true>(taddr, bias_v, stage, lane, o_warp, a.cout, a.pos + tile * TP,
+                                    0, 0, a.out, a.residual);
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
     }
@@ -403,8 +383,10 @@ cudaError_t device_setup(int device, int* num_sms) {
   if (device < 0 || device >= 64) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(mu);
   if (sms[device] == 0) {
-    const void* kernels[2] = {reinterpret_cast<const void*>(subm3d_fwd_bf16_runs_sm100<false>),
-                              reinterpret_cast<const void*>(subm3d_fwd_bf16_runs_sm100<true>)};
+    const void* kernels[3] = {
+        reinterpret_cast<const void*>(subm3d_fwd_bf16_runs_sm100<kActNone>),
+        reinterpret_cast<const void*>(subm3d_fwd_bf16_runs_sm100<kActGelu>),
+        reinterpret_cast<const void*>(subm3d_fwd_bf16_runs_sm100<kActSilu>)};
     for (const void* k : kernels) {
       const cudaError_t e =
           cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
@@ -424,7 +406,7 @@ cudaError_t device_setup(int device, int* num_sms) {
 cudaError_t launch_forward_bf16_runs(const int32_t* pos, const int32_t* etable,
                                      const int32_t* header, int64_t max_tiles, const void* feats,
                                      const void* weight, void* out, int32_t cin, int32_t cout,
-                                     int32_t flip, int32_t act, int32_t* err_word,
+                                     int32_t flip, const Epilogue& epi, int32_t* err_word,
                                      cudaStream_t stream) {
   EncodeTiledFn encode = encode_fn();
   if (!encode) return cudaErrorNotSupported;
@@ -462,15 +444,20 @@ cudaError_t launch_forward_bf16_runs(const int32_t* pos, const int32_t* etable,
   a.se = se;
   a.sw = sw;
   a.flip = flip;
+  a.bias = static_cast<const __nv_bfloat16*>(epi.bias);
+  a.residual = static_cast<const __nv_bfloat16*>(epi.residual);
   a.err_word = err_word;
   // the tile count lives on the device; launch for the largest possible count
   // and let each CTA read the actual one
   const int64_t units = max_tiles * a.n_oblocks;
   const unsigned grid = static_cast<unsigned>(units < num_sms ? units : num_sms);
-  if (act)
-    return launch_pdl(subm3d_fwd_bf16_runs_sm100<true>, grid, NUM_THREADS, plan.bytes, stream,
+  if (epi.act == kActGelu)
+    return launch_pdl(subm3d_fwd_bf16_runs_sm100<kActGelu>, grid, NUM_THREADS, plan.bytes, stream,
                       wmap, a);
-  return launch_pdl(subm3d_fwd_bf16_runs_sm100<false>, grid, NUM_THREADS, plan.bytes, stream,
+  if (epi.act == kActSilu)
+    return launch_pdl(subm3d_fwd_bf16_runs_sm100<kActSilu>, grid, NUM_THREADS, plan.bytes, stream,
+                      wmap, a);
+  return launch_pdl(subm3d_fwd_bf16_runs_sm100<kActNone>, grid, NUM_THREADS, plan.bytes, stream,
                     wmap, a);
 }
 

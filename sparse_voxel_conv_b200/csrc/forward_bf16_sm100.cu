@@ -1,6 +1,7 @@
 // bf16 forward of the submanifold 3x3x3 convolution on sm_100a tensor cores.
 //
-// out[i] = act( sum_k Wf[:, k, :] . x[nbr[i][k]] ) with Wf[:, k] = W[:, k]
+// out[i] = act( sum_k Wf[:, k, :] . x[nbr[i][k]] + bias ) + residual[i] with
+// Wf[:, k] = W[:, k]
 // (correlation) or W[:, 26-k] (flip), W in spconv's KRSC layout
 // [Cout, kz, ky, kx, Cin] (lato.2_mrp_mlx, commit 97dcdfb54a message and
 // CLAUDE.md "Key facts").  An implicit gather-GEMM: no scatter, no atomics,
@@ -35,9 +36,10 @@
 //   warp 12 (MMA)        TMEM allocation (512 columns: two accumulators); lane 0
 //       issues tcgen05.mma (M=128, N=256, K=16) and commits each stage back.
 //   warps 0-3 (epilogue) drain the other accumulator: warp w holds channels
-//       32w..32w+31; tcgen05.ld 32 voxels at a time, optional exact-erf GELU,
-//       bf16 round-to-nearest-even, a transpose through shared memory, and
-//       16-byte stores of whole 64-byte channel runs of each voxel's row.
+//       32w..32w+31; tcgen05.ld 32 voxels at a time, bias, activation (none,
+//       exact GELU, SiLU), a transpose through fp32 shared memory, the
+//       residual, one bf16 rounding (nearest even) and 16-byte stores of whole
+//       64-byte channel runs of each voxel's row (epilogue.cuh).
 //
 // Offsets with no neighbour anywhere in the tile (bit clear in both 128-row
 // mask words) are skipped.  Every wait is bounded (ptx.cuh); a wait that runs
@@ -51,6 +53,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "epilogue.cuh"
 
 namespace subm3d {
 namespace {
@@ -66,7 +69,7 @@ constexpr int NUM_THREADS = (TMA_WARP + 1) * 32;
 constexpr int GATHER_THREADS = NUM_GATHER_WARPS * 32;
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kNbrTileBytes = TV * kKvol * 4;             // 27648
-constexpr int kEpiStageBytes = NUM_EPI_WARPS * 32 * 64;  // 32 voxels x 32 channels bf16 per warp
+constexpr int kEpiStageBytes = NUM_EPI_WARPS * kEpiWarpStageBytes;  // fp32 staging per warp
 constexpr uint32_t kTmemCols = 2 * TV;
 constexpr uint32_t kCentreBit = 1u << 13;
 
@@ -76,7 +79,9 @@ struct FwdArgs {
   const __nv_bfloat16* x;
   int64_t n;
   __nv_bfloat16* out;
-  int32_t cin, cout, n_oblocks, n_kchunks, stages, flip, act;
+  const __nv_bfloat16* bias;      // [cout] or nullptr
+  const __nv_bfloat16* residual;  // [n, cout] or nullptr; may be `out`
+  int32_t cin, cout, n_oblocks, n_kchunks, stages, flip;
   int64_t n_tiles;
   int32_t* err_word;
 };
@@ -164,11 +169,7 @@ struct Steps {
   }
 };
 
-__device__ __forceinline__ float gelu_erf(float v) {
-  return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f));
-}
-
-template <int CHUNK, bool GELU>
+template <int CHUNK, int ACT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     subm3d_fwd_bf16_sm100(const __grid_constant__ CUtensorMap wmap, const FwdArgs a) {
   constexpr int ROW_BYTES = CHUNK * 2;  // 128, 64 or 32
@@ -366,7 +367,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // --------------------------------------------------------- epilogue ----
     const int64_t n_units = a.n_tiles * a.n_oblocks;
-    const uint32_t stage = smem_u32(epi_s) + static_cast<uint32_t>(warp) * (32 * 64);
+    const uint32_t stage =
+        smem_u32(epi_s) + static_cast<uint32_t>(warp) * static_cast<uint32_t>(kEpiWarpStageBytes);
     int local = 0;
     for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x, ++local) {
       const int acc = local & 1;
@@ -374,34 +376,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const int64_t row0 = (u / a.n_oblocks) * TV;
       const int o_warp = static_cast<int>(u % a.n_oblocks) * TO + warp * 32;  // this warp's channels
+      const float bias_v =
+          (a.bias && o_warp + lane < a.cout) ? __bfloat162float(a.bias[o_warp + lane]) : 0.0f;
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(acc * TV);
-#pragma unroll 1
-      for (int c0 = 0; c0 < TV; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(taddr + c0, v);  // lane = channel o_warp + lane, 32 voxels
-        tmem_ld_wait();
-        // transpose through shared memory: [voxel 0..31][channel 0..31] bf16
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          float f = __uint_as_float(v[e]);
-          if constexpr (GELU) f = gelu_erf(f);
-          const __nv_bfloat16 h = __float2bfloat16_rn(f);
-          sts_u16(stage + e * 64 + lane * 2, *reinterpret_cast<const uint16_t*>(&h));
-        }
-        __syncwarp();
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          const int vv = p * 8 + lane / 4;  // voxel within the 32
-          const int q = lane % 4;           // 8-channel group
-          const uint4 val = lds_16(stage + vv * 64 + q * 16);
-          const int64_t row = row0 + c0 + vv;
-          const int o = o_warp + q * 8;
-          if (row < a.n && o < a.cout)
-            *reinterpret_cast<uint4*>(a.out + row * a.cout + o) = val;
-        }
-        __syncwarp();
-      }
+      epilogue_tile_bf16<ACT, false>(taddr, bias_v, stage, lane, o_warp, a.cout, nullptr, row0,
+                                     a.n, a.out, a.residual);
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
     }
@@ -442,12 +422,16 @@ cudaError_t device_setup(int device, int* num_sms) {
   if (device < 0 || device >= 64) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(mu);
   if (sms[device] == 0) {
-    const void* kernels[6] = {reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<64, false>),
-                              reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<32, false>),
-                              reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<16, false>),
-                              reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<64, true>),
-                              reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<32, true>),
-                              reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<16, true>)};
+    const void* kernels[9] = {
+        reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<64, kActNone>),
+        reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<32, kActNone>),
+        reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<16, kActNone>),
+        reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<64, kActGelu>),
+        reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<32, kActGelu>),
+        reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<16, kActGelu>),
+        reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<64, kActSilu>),
+        reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<32, kActSilu>),
+        reinterpret_cast<const void*>(subm3d_fwd_bf16_sm100<16, kActSilu>)};
     for (const void* k : kernels) {
       const cudaError_t e =
           cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
@@ -466,7 +450,7 @@ cudaError_t device_setup(int device, int* num_sms) {
 
 cudaError_t launch_forward_bf16(const int32_t* nbr, const uint32_t* tile_mask, int64_t n,
                                 const void* feats, const void* weight, void* out, int32_t cin,
-                                int32_t cout, int32_t flip, int32_t act, int32_t* err_word,
+                                int32_t cout, int32_t flip, const Epilogue& epi, int32_t* err_word,
                                 cudaStream_t stream) {
   EncodeTiledFn encode = encode_fn();
   if (!encode) return cudaErrorNotSupported;
@@ -509,7 +493,8 @@ cudaError_t launch_forward_bf16(const int32_t* nbr, const uint32_t* tile_mask, i
   a.n_kchunks = cin / chunk;
   a.stages = stages;
   a.flip = flip;
-  a.act = act;
+  a.bias = static_cast<const __nv_bfloat16*>(epi.bias);
+  a.residual = static_cast<const __nv_bfloat16*>(epi.residual);
   a.n_tiles = (n + TV - 1) / TV;
   a.err_word = err_word;
   const int64_t units = a.n_tiles * a.n_oblocks;
@@ -517,12 +502,23 @@ cudaError_t launch_forward_bf16(const int32_t* nbr, const uint32_t* tile_mask, i
   auto launch = [&](auto kernel) {
     kernel<<<grid, NUM_THREADS, plan.bytes, stream>>>(wmap, a);
   };
+  auto by_act = [&](auto k_none, auto k_gelu, auto k_silu) {
+    if (epi.act == kActGelu)
+      launch(k_gelu);
+    else if (epi.act == kActSilu)
+      launch(k_silu);
+    else
+      launch(k_none);
+  };
   if (chunk == 64)
-    act ? launch(subm3d_fwd_bf16_sm100<64, true>) : launch(subm3d_fwd_bf16_sm100<64, false>);
+    by_act(subm3d_fwd_bf16_sm100<64, kActNone>, subm3d_fwd_bf16_sm100<64, kActGelu>,
+           subm3d_fwd_bf16_sm100<64, kActSilu>);
   else if (chunk == 32)
-    act ? launch(subm3d_fwd_bf16_sm100<32, true>) : launch(subm3d_fwd_bf16_sm100<32, false>);
+    by_act(subm3d_fwd_bf16_sm100<32, kActNone>, subm3d_fwd_bf16_sm100<32, kActGelu>,
+           subm3d_fwd_bf16_sm100<32, kActSilu>);
   else
-    act ? launch(subm3d_fwd_bf16_sm100<16, true>) : launch(subm3d_fwd_bf16_sm100<16, false>);
+    by_act(subm3d_fwd_bf16_sm100<16, kActNone>, subm3d_fwd_bf16_sm100<16, kActGelu>,
+           subm3d_fwd_bf16_sm100<16, kActSilu>);
   return cudaGetLastError();
 }
 

@@ -1,8 +1,8 @@
 // fp32 forward of the submanifold 3x3x3 convolution on CUDA-core FMA.
 //
-// out[i] = act( sum_k Wf[:, k, :] . x[nbr[i][k]] ), Wf[:, k] = W[:, k] or
-// W[:, 26-k] with flip (correlation / mirrored kernel, lato.2_mrp_mlx commit
-// 97dcdfb54a message).  Implicit gather-GEMM: a 64-row x 64-column output tile
+// out[i] = act( sum_k Wf[:, k, :] . x[nbr[i][k]] + bias ) + residual[i],
+// Wf[:, k] = W[:, k] or W[:, 26-k] with flip (correlation / mirrored kernel,
+// lato.2_mrp_mlx commit 97dcdfb54a message); bias and residual optional.  Implicit gather-GEMM: a 64-row x 64-column output tile
 // per block, 256 threads with a 4x4 register tile each.  For every offset the
 // tile needs, 16-channel slices of the 64 gathered input rows (zero where
 // nbr = -1) and of the weight slice are staged in shared memory and
@@ -13,6 +13,7 @@
 // 1e-5 relative tolerance over 27*Cin terms.
 #include <cuda_runtime.h>
 
+#include "epilogue.cuh"
 #include "internal.h"
 
 namespace subm3d {
@@ -20,14 +21,13 @@ namespace {
 
 constexpr int BM = 64, BN = 64, BK = 16, NT = 256;
 
-__device__ __forceinline__ float gelu_erf(float v) {
-  return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f));
-}
-
+// out may alias residual (an in-place residual add): neither is __restrict__.
+template <int ACT>
 __global__ void __launch_bounds__(NT)
     fwd_f32_kernel(const int32_t* __restrict__ nbr, const uint32_t* __restrict__ tile_mask,
                    int64_t n, const float* __restrict__ x, const float* __restrict__ w,
-                   float* __restrict__ out, int cin, int cout, int flip, int act) {
+                   float* out, int cin, int cout, int flip, const float* bias,
+                   const float* residual) {
   __shared__ int32_t s_nbr[BM * kKvol];
   __shared__ __align__(16) float s_a[BK][BM];
   __shared__ __align__(16) float s_b[BK][BN];
@@ -96,8 +96,9 @@ __global__ void __launch_bounds__(NT)
     for (int j = 0; j < 4; ++j) {
       const int o = col0 + tx * 4 + j;
       if (o >= cout) continue;
-      const float v = acc[i][j];
-      out[r * cout + o] = act ? gelu_erf(v) : v;
+      float v = activate<ACT>(acc[i][j] + (bias ? bias[o] : 0.0f));
+      if (residual) v += residual[r * cout + o];
+      out[r * cout + o] = v;
     }
   }
 }
@@ -106,11 +107,21 @@ __global__ void __launch_bounds__(NT)
 
 cudaError_t launch_forward_f32(const int32_t* nbr, const uint32_t* tile_mask, int64_t n,
                                const float* feats, const float* weight, float* out, int32_t cin,
-                               int32_t cout, int32_t flip, int32_t act, cudaStream_t stream) {
+                               int32_t cout, int32_t flip, const Epilogue& epi,
+                               cudaStream_t stream) {
   const dim3 grid(static_cast<unsigned>((n + BM - 1) / BM),
                   static_cast<unsigned>((cout + BN - 1) / BN));
-  fwd_f32_kernel<<<grid, NT, 0, stream>>>(nbr, tile_mask, n, feats, weight, out, cin, cout, flip,
-                                         act);
+  const auto* bias = static_cast<const float*>(epi.bias);
+  const auto* res = static_cast<const float*>(epi.residual);
+  if (epi.act == kActGelu)
+    fwd_f32_kernel<kActGelu><<<grid, NT, 0, stream>>>(nbr, tile_mask, n, feats, weight, out, cin,
+                                                      cout, flip, bias, res);
+  else if (epi.act == kActSilu)
+    fwd_f32_kernel<kActSilu><<<grid, NT, 0, stream>>>(nbr, tile_mask, n, feats, weight, out, cin,
+                                                      cout, flip, bias, res);
+  else
+    fwd_f32_kernel<kActNone><<<grid, NT, 0, stream>>>(nbr, tile_mask, n, feats, weight, out, cin,
+                                                      cout, flip, bias, res);
   return cudaGetLastError();
 }
 

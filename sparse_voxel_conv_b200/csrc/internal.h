@@ -107,24 +107,37 @@ cudaError_t launch_map_build(const int32_t* coords, int64_t n, int32_t grid_dim,
                              int32_t* nbr, void* workspace, const MapLayout& lay,
                              cudaStream_t stream);
 
+// Activation codes of the forward epilogue (the values of subm3d_act).
+enum : int { kActNone = 0, kActGelu = 1, kActSilu = 2 };
+
+// Epilogue of a forward: out = act(acc + bias) + residual (epilogue.cuh).
+// bias: [Cout] and residual: [N, Cout] in the feature dtype, each optional; act:
+// 0 none, 1 exact GELU, 2 SiLU.  residual may be `out` itself.
+struct Epilogue {
+  const void* bias = nullptr;
+  const void* residual = nullptr;
+  int32_t act = 0;
+};
+
 // fp32 forward on CUDA-core FMA.
 cudaError_t launch_forward_f32(const int32_t* nbr, const uint32_t* tile_mask, int64_t n,
                                const float* feats, const float* weight, float* out, int32_t cin,
-                               int32_t cout, int32_t flip, int32_t act, cudaStream_t stream);
+                               int32_t cout, int32_t flip, const Epilogue& epi,
+                               cudaStream_t stream);
 
 // bf16 forward on tcgen05 tensor cores (fp32 accumulation in TMEM).
 // err_word is the library's device error word (set when a bounded wait runs out).
 cudaError_t launch_forward_bf16(const int32_t* nbr, const uint32_t* tile_mask, int64_t n,
                                 const void* feats, const void* weight, void* out, int32_t cin,
-                                int32_t cout, int32_t flip, int32_t act, int32_t* err_word,
-                                cudaStream_t stream);
+                                int32_t cout, int32_t flip, const Epilogue& epi,
+                                int32_t* err_word, cudaStream_t stream);
 
 // bf16 forward over the x-run position layout (forward_bf16_runs_sm100.cu);
 // Cin a multiple of 64, Cout a multiple of 16.
 cudaError_t launch_forward_bf16_runs(const int32_t* pos, const int32_t* etable,
                                      const int32_t* header, int64_t max_tiles, const void* feats,
                                      const void* weight, void* out, int32_t cin, int32_t cout,
-                                     int32_t flip, int32_t act, int32_t* err_word,
+                                     int32_t flip, const Epilogue& epi, int32_t* err_word,
                                      cudaStream_t stream);
 
 }  // namespace subm3d

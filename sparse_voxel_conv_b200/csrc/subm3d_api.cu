@@ -166,47 +166,78 @@ const uint32_t* subm3d_map_tile_mask(const subm3d_map* map) {
 int64_t subm3d_map_size(const subm3d_map* map) { return map ? map->n : -1; }
 void subm3d_map_destroy(subm3d_map* map) { delete map; }
 
-subm3d_status subm3d_forward(const int32_t* nbr, const uint32_t* tile_mask, int64_t n,
-                             const void* feats, const void* weight, void* out, int32_t cin,
-                             int32_t cout, subm3d_dtype dtype, int32_t flip, subm3d_act act,
-                             void* stream) {
+namespace {
+
+bool overlaps(const void* p, size_t p_bytes, const void* q, size_t q_bytes) {
+  const auto* a = static_cast<const uint8_t*>(p);
+  const auto* b = static_cast<const uint8_t*>(q);
+  return a < b + q_bytes && b < a + p_bytes;
+}
+
+// The forward of every entry point: map may be null (nbr-only callers), in
+// which case the x-run kernel is not available.
+subm3d_status forward_impl(const subm3d_map* map, const int32_t* nbr, const uint32_t* tile_mask,
+                           int64_t n, const void* feats, const void* weight, const void* bias,
+                           const void* residual, void* out, int32_t cin, int32_t cout,
+                           subm3d_dtype dtype, int32_t flip, subm3d_act act, void* stream) {
   if (n < 0 || cin < 1 || cout < 1) return SUBM3D_E_INVALID;
   if (dtype != SUBM3D_F32 && dtype != SUBM3D_BF16) return SUBM3D_E_INVALID;
-  if (act != SUBM3D_ACT_NONE && act != SUBM3D_ACT_GELU) return SUBM3D_E_INVALID;
+  if (act != SUBM3D_ACT_NONE && act != SUBM3D_ACT_GELU && act != SUBM3D_ACT_SILU)
+    return SUBM3D_E_INVALID;
   if (n > 0 && (!nbr || !feats || !weight || !out)) return SUBM3D_E_INVALID;
   if (n >= 0x7FFFFFFFll) return SUBM3D_E_UNSUPPORTED;
   if (n == 0) return SUBM3D_OK;
   const size_t esz = dtype == SUBM3D_BF16 ? 2 : 4;
-  const auto* fb = static_cast<const uint8_t*>(feats);
-  const auto* ob = static_cast<const uint8_t*>(out);
-  if (fb < ob + static_cast<size_t>(n) * cout * esz && ob < fb + static_cast<size_t>(n) * cin * esz)
+  const size_t out_bytes = static_cast<size_t>(n) * cout * esz;
+  if (overlaps(feats, static_cast<size_t>(n) * cin * esz, out, out_bytes))
     return SUBM3D_E_INVALID;  // out overlaps feats
+  if (residual && residual != out && overlaps(residual, out_bytes, out, out_bytes))
+    return SUBM3D_E_INVALID;  // a residual partly overlapping out would race
   auto s = static_cast<cudaStream_t>(stream);
   const int flip01 = flip ? 1 : 0;
-  const int act01 = act == SUBM3D_ACT_GELU ? 1 : 0;
+  subm3d::Epilogue epi;
+  epi.bias = bias;
+  epi.residual = residual;
+  epi.act = act == SUBM3D_ACT_GELU ? subm3d::kActGelu
+                                   : (act == SUBM3D_ACT_SILU ? subm3d::kActSilu : subm3d::kActNone);
   if (dtype == SUBM3D_F32) {
     if (!aligned(nbr, 4) || !aligned(feats, 4) || !aligned(weight, 4) || !aligned(out, 4) ||
-        (tile_mask && !aligned(tile_mask, 4)))
+        (tile_mask && !aligned(tile_mask, 4)) || !aligned(bias, 4) || !aligned(residual, 4))
       return SUBM3D_E_INVALID;
     return subm3d::launch_forward_f32(nbr, tile_mask, n, static_cast<const float*>(feats),
                                       static_cast<const float*>(weight), static_cast<float*>(out),
-                                      cin, cout, flip01, act01, s) == cudaSuccess
+                                      cin, cout, flip01, epi, s) == cudaSuccess
                ? SUBM3D_OK
                : SUBM3D_E_CUDA;
   }
   if (cin % 16 != 0 || cout % 16 != 0) return SUBM3D_E_UNSUPPORTED;
   if (!aligned(nbr, 16) || !aligned(feats, 16) || !aligned(weight, 16) || !aligned(out, 16) ||
-      (tile_mask && !aligned(tile_mask, 4)))
+      (tile_mask && !aligned(tile_mask, 4)) || !aligned(bias, 2) || !aligned(residual, 16))
     return SUBM3D_E_UNSUPPORTED;
   const int sm100 = device_is_sm100(nullptr);
   if (sm100 < 0) return SUBM3D_E_CUDA;
   if (sm100 == 0) return SUBM3D_E_UNSUPPORTED;
   int32_t* err = device_error_word();
   if (!err) return SUBM3D_E_CUDA;
-  const cudaError_t e = subm3d::launch_forward_bf16(nbr, tile_mask, n, feats, weight, out, cin,
-                                                    cout, flip01, act01, err, s);
+  cudaError_t e;
+  if (map && map->pos && cin % 64 == 0)
+    e = subm3d::launch_forward_bf16_runs(map->pos, map->et, map->hdr, map->ptile_max, feats,
+                                         weight, out, cin, cout, flip01, epi, err, s);
+  else
+    e = subm3d::launch_forward_bf16(nbr, tile_mask, n, feats, weight, out, cin, cout, flip01, epi,
+                                    err, s);
   if (e == cudaErrorNotSupported) return SUBM3D_E_UNSUPPORTED;
   return e == cudaSuccess ? SUBM3D_OK : SUBM3D_E_CUDA;
+}
+
+}  // namespace
+
+subm3d_status subm3d_forward(const int32_t* nbr, const uint32_t* tile_mask, int64_t n,
+                             const void* feats, const void* weight, void* out, int32_t cin,
+                             int32_t cout, subm3d_dtype dtype, int32_t flip, subm3d_act act,
+                             void* stream) {
+  return forward_impl(nullptr, nbr, tile_mask, n, feats, weight, nullptr, nullptr, out, cin, cout,
+                      dtype, flip, act, stream);
 }
 
 subm3d_status subm3d_map_run_layout(const subm3d_map* map, const int32_t** pos,
@@ -223,27 +254,17 @@ subm3d_status subm3d_forward_map(const subm3d_map* map, const void* feats, const
                                  void* out, int32_t cin, int32_t cout, subm3d_dtype dtype,
                                  int32_t flip, subm3d_act act, void* stream) {
   if (!map) return SUBM3D_E_INVALID;
-  const int64_t n = map->n;
-  const bool runs = map->pos && dtype == SUBM3D_BF16 && n > 0 && cin % 64 == 0 && cout % 16 == 0 &&
-                    feats && weight && out && aligned(feats, 16) && aligned(weight, 16) &&
-                    aligned(out, 16) && (act == SUBM3D_ACT_NONE || act == SUBM3D_ACT_GELU);
-  if (!runs)
-    return subm3d_forward(map->nbr, map->tile_mask, n, feats, weight, out, cin, cout, dtype, flip,
-                          act, stream);
-  const auto* fb = static_cast<const uint8_t*>(feats);
-  const auto* ob = static_cast<const uint8_t*>(out);
-  if (fb < ob + static_cast<size_t>(n) * cout * 2 && ob < fb + static_cast<size_t>(n) * cin * 2)
-    return SUBM3D_E_INVALID;  // out overlaps feats
-  const int sm100 = device_is_sm100(nullptr);
-  if (sm100 < 0) return SUBM3D_E_CUDA;
-  if (sm100 == 0) return SUBM3D_E_UNSUPPORTED;
-  int32_t* err = device_error_word();
-  if (!err) return SUBM3D_E_CUDA;
-  const cudaError_t e = subm3d::launch_forward_bf16_runs(
-      map->pos, map->et, map->hdr, map->ptile_max, feats, weight, out, cin, cout, flip ? 1 : 0,
-      act == SUBM3D_ACT_GELU ? 1 : 0, err, static_cast<cudaStream_t>(stream));
-  if (e == cudaErrorNotSupported) return SUBM3D_E_UNSUPPORTED;
-  return e == cudaSuccess ? SUBM3D_OK : SUBM3D_E_CUDA;
+  return forward_impl(map, map->nbr, map->tile_mask, map->n, feats, weight, nullptr, nullptr, out,
+                      cin, cout, dtype, flip, act, stream);
+}
+
+subm3d_status subm3d_forward_fused(const subm3d_map* map, const void* feats, const void* weight,
+                                   const void* bias, const void* residual, void* out, int32_t cin,
+                                   int32_t cout, subm3d_dtype dtype, int32_t flip, subm3d_act act,
+                                   void* stream) {
+  if (!map) return SUBM3D_E_INVALID;
+  return forward_impl(map, map->nbr, map->tile_mask, map->n, feats, weight, bias, residual, out,
+                      cin, cout, dtype, flip, act, stream);
 }
 
 subm3d_status subm3d_device_status(void* stream) {

@@ -16,12 +16,14 @@ import torch
 from . import _abi
 from ._abi import Subm3dError
 
-__all__ = ["MapHandle", "build_map", "forward", "SparseTensor", "SubMConv3d", "Subm3dError"]
+__all__ = ["MapHandle", "build_map", "forward", "SparseTensor", "SubMConv3d", "SubMResBlock3d",
+           "Subm3dError"]
 
 MapHandle = _abi.MapHandle
 
 _DTYPES = {torch.float32: _abi.SUBM3D_F32, torch.bfloat16: _abi.SUBM3D_BF16}
-_ACTS = {None: _abi.SUBM3D_ACT_NONE, "none": _abi.SUBM3D_ACT_NONE, "gelu": _abi.SUBM3D_ACT_GELU}
+_ACTS = {None: _abi.SUBM3D_ACT_NONE, "none": _abi.SUBM3D_ACT_NONE, "gelu": _abi.SUBM3D_ACT_GELU,
+         "silu": _abi.SUBM3D_ACT_SILU}
 
 
 def _cuda_contig(t: torch.Tensor, name: str, dtype=None) -> torch.Tensor:
@@ -76,14 +78,17 @@ def tile_mask_tensor(h: MapHandle) -> torch.Tensor:
 
 def forward(h: MapHandle, feats: torch.Tensor, weight: torch.Tensor, flip: bool = False,
             act: str | None = None, out: torch.Tensor | None = None, stream=None,
-            use_tile_mask: bool = True, kernel: str = "auto") -> torch.Tensor:
-    """One SubMConv3d layer: out[i] = act(sum_k Wf[:,k,:] . feats[nbr[i,k]]).
+            use_tile_mask: bool = True, kernel: str = "auto", bias: torch.Tensor | None = None,
+            residual: torch.Tensor | None = None) -> torch.Tensor:
+    """One SubMConv3d layer: out[i] = act(sum_k Wf[:,k,:] . feats[nbr[i,k]] + bias) + residual[i].
 
     feats: [N, Cin] float32 or bfloat16; weight: KRSC [Cout, 3, 3, 3, Cin] (or
     [Cout, 27, Cin]) of the same dtype.  Returns [N, Cout] of that dtype.
-    kernel: "auto" runs subm3d_forward_map (the x-run kernel for bf16 with
+    act: None, "gelu" (exact erf form) or "silu".  bias: optional [Cout];
+    residual: optional [N, Cout] (may be `out`), both of the feature dtype.
+    kernel: "auto" runs subm3d_forward_fused (the x-run kernel for bf16 with
     Cin % 64 == 0); "gather" runs subm3d_forward on nbr and the tile masks
-    (use_tile_mask=False: no masks).
+    (use_tile_mask=False: no masks; no bias or residual there).
     """
     if feats.dtype not in _DTYPES:
         raise ValueError(f"unsupported feature dtype {feats.dtype}")
@@ -95,14 +100,24 @@ def forward(h: MapHandle, feats: torch.Tensor, weight: torch.Tensor, flip: bool 
     cout = weight.shape[0]
     if weight.numel() != cout * 27 * cin:
         raise ValueError("weight must be KRSC [Cout, 3, 3, 3, Cin]")
+    if bias is not None:
+        bias = _cuda_contig(bias, "bias", feats.dtype)
+        if bias.numel() != cout:
+            raise ValueError("bias must have Cout elements")
+    if residual is not None:
+        residual = _cuda_contig(residual, "residual", feats.dtype)
+        if tuple(residual.shape) != (n, cout):
+            raise ValueError("residual must have shape [N, Cout]")
     if out is None:
         out = torch.empty((n, cout), dtype=feats.dtype, device=feats.device)
     if kernel == "auto" and use_tile_mask:
-        _abi.subm3d_forward_map(h, feats, weight, out, cin, cout, _DTYPES[feats.dtype], flip,
-                                _ACTS[act], stream)
+        _abi.subm3d_forward_fused(h, feats, weight, bias, residual, out, cin, cout,
+                                  _DTYPES[feats.dtype], flip, _ACTS[act], stream)
         return out
     if kernel not in ("auto", "gather"):
         raise ValueError(f"unknown kernel {kernel!r}")
+    if bias is not None or residual is not None:
+        raise ValueError("bias and residual need kernel='auto'")
     mask_ptr = _abi.subm3d_map_tile_mask(h) if use_tile_mask else None
     _abi.subm3d_forward(h.nbr, mask_ptr, n, feats, weight, out, cin, cout, _DTYPES[feats.dtype],
                         flip, _ACTS[act], stream)
@@ -155,13 +170,14 @@ class SubMConv3d(torch.nn.Module):
 
     The weight is a KRSC parameter [Cout, 3, 3, 3, Cin].  Layers sharing an
     indice_key reuse one neighbour map per SparseTensor coordinate set.
-    flip selects the mirrored kernel; act=None or "gelu" (exact erf form).
-    No bias: the pages' op has none.
+    flip selects the mirrored kernel; act=None, "gelu" (exact erf form) or
+    "silu".  bias=True adds a [Cout] bias before the activation (the pages'
+    op has none; the residual blocks' convolutions do).
     """
 
     def __init__(self, in_channels: int, out_channels: int, indice_key: str = "subm0",
                  flip: bool = False, act: str | None = None, dtype=torch.bfloat16,
-                 device=None):
+                 device=None, bias: bool = False):
         super().__init__()
         self.in_channels = in_channels
         self.out_channels = out_channels
@@ -171,8 +187,37 @@ class SubMConv3d(torch.nn.Module):
         w = torch.empty((out_channels, 3, 3, 3, in_channels), dtype=torch.float32)
         w.normal_(0.0, 1.0 / math.sqrt(27.0 * in_channels))
         self.weight = torch.nn.Parameter(w.to(dtype=dtype, device=device), requires_grad=False)
+        if bias:
+            b = torch.empty(out_channels, dtype=torch.float32).normal_(0.0, 0.1)
+            self.bias = torch.nn.Parameter(b.to(dtype=dtype, device=device), requires_grad=False)
+        else:
+            self.bias = None
+
+    def forward(self, x: SparseTensor, residual: torch.Tensor | None = None) -> SparseTensor:
+        h = x.get_map(self.indice_key)
+        y = forward(h, x.feats, self.weight, flip=self.flip, act=self.act, bias=self.bias,
+                    residual=residual)
+        return x.replace(y)
+
+
+class SubMResBlock3d(torch.nn.Module):
+    """Two submanifold convolutions on one neighbour map with the residual
+    block's epilogues fused into their stores:
+
+        h   = act(conv1(x) + b1)
+        out = conv2(h) + b2 + x
+
+    Both convolutions share `indice_key`, so the map is built once per
+    coordinate set; no separate bias, activation or add kernel runs.
+    """
+
+    def __init__(self, channels: int, indice_key: str = "subm0", act: str = "silu",
+                 dtype=torch.bfloat16, device=None):
+        super().__init__()
+        self.conv1 = SubMConv3d(channels, channels, indice_key, act=act, dtype=dtype,
+                                device=device, bias=True)
+        self.conv2 = SubMConv3d(channels, channels, indice_key, act=None, dtype=dtype,
+                                device=device, bias=True)
 
     def forward(self, x: SparseTensor) -> SparseTensor:
-        h = x.get_map(self.indice_key)
-        y = forward(h, x.feats, self.weight, flip=self.flip, act=self.act)
-        return x.replace(y)
+        return self.conv2(self.conv1(x), residual=x.feats)

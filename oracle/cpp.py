@@ -45,6 +45,14 @@ def load():
         lib.oracle_forward.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                        ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                        ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p]
+        lib.oracle_backward_data.restype = None
+        lib.oracle_backward_data.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                             ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
+                                             ctypes.c_int32, ctypes.c_void_p]
+        lib.oracle_backward_weight.restype = None
+        lib.oracle_backward_weight.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                               ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
+                                               ctypes.c_int32, ctypes.c_void_p]
         lib.oracle_gelu.argtypes = [ctypes.c_void_p, ctypes.c_int64]
         lib.oracle_silu.argtypes = [ctypes.c_void_p, ctypes.c_int64]
         lib.oracle_round_bf16.argtypes = [ctypes.c_void_p, ctypes.c_int64]
@@ -104,6 +112,31 @@ def forward(nbr, x, w, flip: bool = False, act: str | None = None,
     if round_to_bf16:
         load().oracle_round_bf16(out.ctypes.data, out.size)
     return out
+
+
+def backward_data(nbr, dy, w, flip: bool = False) -> np.ndarray:
+    """fp64 gradient with respect to the input features (see oracle_backward_data)."""
+    nbr = np.ascontiguousarray(nbr, np.int32)
+    dy = np.ascontiguousarray(dy, np.float64)
+    w = np.ascontiguousarray(w, np.float64)
+    cout = w.shape[0]
+    cin = w.size // (27 * cout)
+    dx = np.empty((nbr.shape[0], cin), np.float64)
+    load().oracle_backward_data(nbr.ctypes.data, nbr.shape[0], dy.ctypes.data, w.ctypes.data,
+                                cin, cout, 1 if flip else 0, dx.ctypes.data)
+    return dx
+
+
+def backward_weight(nbr, x, dy, flip: bool = False) -> np.ndarray:
+    """fp64 gradient with respect to the KRSC weight, [Cout, 3, 3, 3, Cin]."""
+    nbr = np.ascontiguousarray(nbr, np.int32)
+    x = np.ascontiguousarray(x, np.float64)
+    dy = np.ascontiguousarray(dy, np.float64)
+    cin, cout = x.shape[1], dy.shape[1]
+    dw = np.empty((cout, 27, cin), np.float64)
+    load().oracle_backward_weight(nbr.ctypes.data, nbr.shape[0], x.ctypes.data, dy.ctypes.data,
+                                  cin, cout, 1 if flip else 0, dw.ctypes.data)
+    return dw.reshape(cout, 3, 3, 3, cin)
 
 
 def gelu(v) -> np.ndarray:

@@ -101,6 +101,52 @@ void oracle_forward(const int32_t* nbr, const double* x, const double* w,
   }
 }
 
+// Gradient with respect to the input features, fp64, by scattering each term of
+// the forward back to its source row:
+//   dx[j][c] += sum_o Wf[o][k][c] * dy[i][o]   for every (i, k) with nbr[i][k] = j.
+// dy is [n, cout], W is [cout, 27, cin], dx is [n, cin] (overwritten).  Serial
+// in i (the scatter targets collide); n is small in the tests that call it.
+void oracle_backward_data(const int32_t* nbr, int64_t n, const double* dy, const double* w,
+                          int32_t cin, int32_t cout, int32_t flip, double* dx) {
+  for (int64_t e = 0; e < n * cin; ++e) dx[e] = 0.0;
+  for (int64_t i = 0; i < n; ++i) {
+    for (int k = 0; k < 27; ++k) {
+      const int32_t j = nbr[i * 27 + k];
+      if (j < 0) continue;
+      const int kw = flip ? 26 - k : k;
+      for (int32_t o = 0; o < cout; ++o) {
+        const double g = dy[i * cout + o];
+        const double* wk = w + ((int64_t)o * 27 + kw) * cin;
+        for (int32_t c = 0; c < cin; ++c) dx[(int64_t)j * cin + c] += wk[c] * g;
+      }
+    }
+  }
+}
+
+// Gradient with respect to the weight, fp64:
+//   dW[o][kw][c] += dy[i][o] * x[nbr[i][k]][c]   for every (i, k), nbr[i][k] != -1,
+// kw = k (correlation) or 26 - k (flip).  dW is [cout, 27, cin] (overwritten).
+// Parallel over the output channel o (each thread owns its rows of dW).
+void oracle_backward_weight(const int32_t* nbr, int64_t n, const double* x, const double* dy,
+                            int32_t cin, int32_t cout, int32_t flip, double* dw) {
+#pragma omp parallel for schedule(static)
+  for (int32_t o = 0; o < cout; ++o) {
+    double* dwo = dw + (int64_t)o * 27 * cin;
+    for (int64_t e = 0; e < 27 * (int64_t)cin; ++e) dwo[e] = 0.0;
+    for (int64_t i = 0; i < n; ++i) {
+      const double g = dy[i * cout + o];
+      for (int k = 0; k < 27; ++k) {
+        const int32_t j = nbr[i * 27 + k];
+        if (j < 0) continue;
+        const int kw = flip ? 26 - k : k;
+        const double* xj = x + (int64_t)j * cin;
+        double* d = dwo + (int64_t)kw * cin;
+        for (int32_t c = 0; c < cin; ++c) d[c] += g * xj[c];
+      }
+    }
+  }
+}
+
 // Exact-erf GELU in place: v <- 0.5 * v * (1 + erf(v / sqrt(2))).
 void oracle_gelu(double* v, int64_t n) {
   for (int64_t i = 0; i < n; ++i) v[i] = 0.5 * v[i] * (1.0 + std::erf(v[i] / std::sqrt(2.0)));

@@ -27,7 +27,8 @@ import math
 
 import numpy as np
 
-__all__ = ["OFFSETS", "OracleError", "build_map", "forward", "gelu", "silu", "round_bf16",
+__all__ = ["OFFSETS", "OracleError", "build_map", "forward", "backward_data", "backward_weight",
+           "gelu", "silu", "round_bf16",
            "brute_force_map"]
 
 # (dz, dy, dx) for k = 0..26, kz-major: dz slowest, dx fastest.
@@ -113,6 +114,52 @@ def forward(nbr, x, w, flip: bool = False, act: str | None = None,
     if round_to_bf16:
         out = round_bf16(out)
     return out
+
+
+def backward_data(nbr, dy, w, flip: bool = False) -> np.ndarray:
+    """Gradient of the forward's output with respect to its input features, in
+    fp64, by scattering every term of the forward back to its source row:
+
+        dx[j] += Wf[:, k, :]^T @ dy[i]   for every (i, k) with nbr[i, k] = j.
+
+    dy: [N, Cout]; w: KRSC [Cout, 3, 3, 3, Cin]; returns [N, Cin].  (No
+    activation: this is the backward of the convolution itself.)
+    """
+    nbr = np.asarray(nbr)
+    dy = np.asarray(dy, np.float64)
+    w = np.asarray(w, np.float64)
+    cout = w.shape[0]
+    w27 = w.reshape(cout, 27, -1)
+    dx = np.zeros((nbr.shape[0], w27.shape[2]), np.float64)
+    for i in range(nbr.shape[0]):
+        for k in range(27):
+            j = int(nbr[i, k])
+            if j < 0:
+                continue
+            kw = 26 - k if flip else k
+            dx[j] += w27[:, kw, :].T @ dy[i]
+    return dx
+
+
+def backward_weight(nbr, x, dy, flip: bool = False) -> np.ndarray:
+    """Gradient of the forward's output with respect to the KRSC weight, in fp64:
+
+        dW[:, kw, :] += outer(dy[i], x[nbr[i, k]])   for every (i, k), nbr[i, k] != -1,
+
+    kw = k (correlation) or 26 - k (flip).  Returns [Cout, 3, 3, 3, Cin].
+    """
+    nbr = np.asarray(nbr)
+    x = np.asarray(x, np.float64)
+    dy = np.asarray(dy, np.float64)
+    dw = np.zeros((dy.shape[1], 27, x.shape[1]), np.float64)
+    for i in range(nbr.shape[0]):
+        for k in range(27):
+            j = int(nbr[i, k])
+            if j < 0:
+                continue
+            kw = 26 - k if flip else k
+            dw[:, kw, :] += np.outer(dy[i], x[j])
+    return dw.reshape(dy.shape[1], 3, 3, 3, x.shape[1])
 
 
 def gelu(v) -> np.ndarray:

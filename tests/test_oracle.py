@@ -439,3 +439,65 @@ def test_silu_closed_forms_and_torch(orc):
     # silu(v) - silu(-v) = v (sigmoid(v) + sigmoid(-v) = 1), and silu(1) = 1/(1+e^-1)
     assert np.max(np.abs(orc.silu(v) - orc.silu(-v) - v)) <= 1e-13
     assert abs(orc.silu(np.array([1.0]))[0] - 1.0 / (1.0 + math.exp(-1.0))) < 1e-15
+
+
+# ------------------------------------------------------------- the backward ---
+
+def _dense_grads(c, x, w, dy, g, batch, flip):
+    """torch autograd through the dense zero-padded conv3d on a full grid."""
+    cin = x.shape[1]
+    xd = torch.zeros(batch, cin, g, g, g, dtype=torch.float64)
+    ct = torch.from_numpy(c.astype(np.int64))
+    xd[ct[:, 0], :, ct[:, 1], ct[:, 2], ct[:, 3]] = torch.from_numpy(x)
+    xd.requires_grad_(True)
+    wk = torch.from_numpy(w).clone().requires_grad_(True)        # KRSC
+    wt = wk.permute(0, 4, 1, 2, 3)
+    if flip:
+        wt = wt.flip(2, 3, 4)
+    yd = F.conv3d(xd, wt, padding=1)
+    y = yd[ct[:, 0], :, ct[:, 1], ct[:, 2], ct[:, 3]]
+    (y * torch.from_numpy(dy)).sum().backward()
+    dx = xd.grad[ct[:, 0], :, ct[:, 1], ct[:, 2], ct[:, 3]].numpy()
+    return dx, wk.grad.numpy()
+
+
+@pytest.mark.parametrize("orc", ORACLES)
+@pytest.mark.parametrize("flip", [False, True])
+def test_backward_equals_torch_autograd_on_full_grid(orc, flip):
+    g, batch, cin, cout = 5, 2, 3, 4
+    c, x, w = _dense_case(g, batch, cin, cout, seed=21)
+    dy = np.random.default_rng(22).standard_normal((c.shape[0], cout))
+    nbr = orc.build_map(c, g, batch)
+    dx_ref, dw_ref = _dense_grads(c, x, w, dy, g, batch, flip)
+    dx = orc.backward_data(nbr, dy, w, flip=flip)
+    dw = orc.backward_weight(nbr, x, dy, flip=flip)
+    assert np.max(np.abs(dx - dx_ref)) <= 1e-12 * max(1.0, np.max(np.abs(dx_ref)))
+    assert np.max(np.abs(dw - dw_ref)) <= 1e-12 * max(1.0, np.max(np.abs(dw_ref)))
+
+
+@pytest.mark.parametrize("orc", ORACLES)
+def test_backward_adjoint_identities_on_sparse_sets(orc):
+    """<forward(x), dy> = <x, backward_data(dy)> = <W, backward_weight(x, dy)>
+    for both orientations on a random sparse set (the forward is bilinear)."""
+    rng = np.random.default_rng(23)
+    c = _rand_coords(rng, 300, 9, batch=2)
+    x = rng.standard_normal((300, 5))
+    w = rng.standard_normal((6, 3, 3, 3, 5))
+    dy = rng.standard_normal((300, 6))
+    nbr = orc.build_map(c, 9, 2)
+    for flip in (False, True):
+        lhs = float(np.sum(orc.forward(nbr, x, w, flip=flip) * dy))
+        via_x = float(np.sum(x * orc.backward_data(nbr, dy, w, flip=flip)))
+        via_w = float(np.sum(w * orc.backward_weight(nbr, x, dy, flip=flip)))
+        assert abs(lhs - via_x) <= 1e-10 * abs(lhs) and abs(lhs - via_w) <= 1e-10 * abs(lhs)
+
+
+def test_backward_python_and_cpp_agree():
+    wl = WL.make_workload("tiny")
+    nbr = C.build_map(wl.coords, wl.grid_dim)
+    x = wl.features().astype(np.float64)
+    w = wl.weights()[0].astype(np.float64)
+    dy = np.random.default_rng(24).standard_normal((wl.n, w.shape[0]))
+    for flip in (False, True):
+        assert np.max(np.abs(P.backward_data(nbr, dy, w, flip) - C.backward_data(nbr, dy, w, flip))) <= 1e-12
+        assert np.max(np.abs(P.backward_weight(nbr, x, dy, flip) - C.backward_weight(nbr, x, dy, flip))) <= 1e-10

@@ -238,6 +238,24 @@ def fused_epilogue_line(h, feats, weight, flops, flush, peak_tf, plain_ms):
             "extra_bytes": int(h.n) * cout * feats.element_size()}
 
 
+def backward_line(h, feats, weight, flops, flush, peak_tf, fp32_peak):
+    """The backward on the headline map: input gradient (a tensor-core forward
+    with the transposed weight) and weight gradient (CUDA-core FMA, fp32)."""
+    import torch
+    import sparse_voxel_conv_b200 as S
+    dy = torch.empty((h.n, weight.shape[0]), dtype=feats.dtype, device=feats.device).normal_()
+    dx = torch.empty_like(feats)
+    dw = torch.empty(weight.shape, dtype=torch.float32, device=feats.device)
+    d_ms = _time_ms(lambda: S.backward_data(h, dy, weight, out=dx), flush)
+    w_ms = _time_ms(lambda: S.backward_weight(h, feats, dy, out=dw), flush, reps=3, warm=1)
+    d_tf = flops / (d_ms / 1e3) / 1e12
+    w_tf = flops / (w_ms / 1e3) / 1e12
+    return {"data": {"ms": d_ms, "achieved": d_tf, "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": d_tf / peak_tf, "bound": "tensor"},
+            "weight": {"ms": w_ms, "achieved": w_tf, "peak": fp32_peak, "unit": "TFLOP/s",
+                       "frac": w_tf / fp32_peak, "bound": "alu"}}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -408,6 +426,8 @@ def run_ours(args):
                 float(clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965.0))
             line["fused_epilogue"] = fused_epilogue_line(h_ctx, feats, weight, flops_alg, flush,
                                                          peak_tf, fwd_avg_s * 1e3)
+            line["backward"] = backward_line(h_ctx, feats, weight, flops_alg, flush, peak_tf,
+                                             line["fp32_forward"]["peak"])
             line["context_per_offset_torch"] = per_offset_context(h_ctx, feats, weight, flush)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl, args.cpu_rows)

@@ -257,6 +257,43 @@ SUBM3D_API subm3d_status subm3d_forward_fused(const subm3d_map* map, const void*
                                               subm3d_act act, void* stream);
 
 /*
+ * Backward of one layer (the convolution itself: no bias, activation or
+ * residual) over a built map.  The pages port inference only; this is the
+ * plain gradient of the forward's definition.
+ *
+ * subm3d_backward_data: dx[j] = sum over (i, k) with nbr[i][k] = j of
+ * Wf[:, k, :]^T dy[i].  By the map's symmetry (nbr[i][k] = j <=> nbr[j][26-k]
+ * = i) that is the forward of dy with the transposed weight W^T[c][k][o] =
+ * W[o][k][c] and the opposite flip, so it writes W^T and runs the forward
+ * kernels (tensor cores for bf16: Cout and Cin multiples of 16).
+ *
+ *   dy        (device) [N, Cout] in the dtype; 16-byte aligned for bf16.
+ *   weight    (device) KRSC [Cout, 3, 3, 3, Cin], as given to the forward.
+ *   weight_t  (device) caller scratch of Cout * 27 * Cin elements, 16-byte
+ *             aligned, not overlapping weight: receives W^T [Cin, 27, Cout].
+ *   dx        (device) [N, Cin] output; must not overlap dy.
+ *   flip      the forward's orientation.
+ *
+ * subm3d_backward_weight: dW[o][kw][c] = sum_i dy[i][o] * feats[nbr[i][k]][c]
+ * over nbr[i][k] != -1, kw = k (flip = 0) or 26 - k.  dweight is fp32 KRSC
+ * [Cout, 3, 3, 3, Cin] (device, 4-byte aligned, overwritten; fp32 for both
+ * dtypes: the sum runs over all voxels).  CUDA-core FMA with fp32 atomics
+ * across voxel slices, so the summation order (and the last bits) vary from
+ * call to call.
+ *
+ * Errors: SUBM3D_E_INVALID for bad arguments or overlapping buffers; otherwise
+ * as subm3d_forward().  Both are asynchronous on `stream`.
+ */
+SUBM3D_API subm3d_status subm3d_backward_data(const subm3d_map* map, const void* dy,
+                                              const void* weight, void* weight_t, void* dx,
+                                              int32_t cin, int32_t cout, subm3d_dtype dtype,
+                                              int32_t flip, void* stream);
+SUBM3D_API subm3d_status subm3d_backward_weight(const subm3d_map* map, const void* feats,
+                                                const void* dy, float* dweight, int32_t cin,
+                                                int32_t cout, subm3d_dtype dtype, int32_t flip,
+                                                void* stream);
+
+/*
  * Device pointers into the map's x-run layout, for tests and tools: the
  * position table (int32, one entry per position: row * 4 + tag, tag 0 voxel,
  * 1 left pad of that row's voxel, 2 right pad, -1 empty), the E index table

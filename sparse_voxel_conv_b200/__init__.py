@@ -8,8 +8,9 @@ it loads the library and fails loudly if it is not built.
 """
 from . import _abi
 from ._abi import Subm3dError
-from .sparse import MapHandle, SparseTensor, SubMConv3d, SubMResBlock3d, build_map, forward, \
-    map_status, run_layout_tensors, tile_mask_tensor
+from .sparse import MapHandle, SparseTensor, SubMConv3d, SubMResBlock3d, backward_data, \
+    backward_weight, build_map, forward, map_status, run_layout_tensors, tile_mask_tensor
 
 __all__ = ["Subm3dError", "MapHandle", "SparseTensor", "SubMConv3d", "SubMResBlock3d", "build_map",
-           "forward", "map_status", "run_layout_tensors", "tile_mask_tensor"]
+           "forward", "backward_data", "backward_weight", "map_status", "run_layout_tensors",
+           "tile_mask_tensor"]

@@ -67,6 +67,10 @@ def _load() -> ctypes.CDLL:
                                                  ctypes.POINTER(vp)]),
         "subm3d_forward_fused": (ctypes.c_int, [vp, vp, vp, vp, vp, vp, i32, i32, ctypes.c_int,
                                                 i32, ctypes.c_int, vp]),
+        "subm3d_backward_data": (ctypes.c_int, [vp, vp, vp, vp, vp, i32, i32, ctypes.c_int, i32,
+                                                vp]),
+        "subm3d_backward_weight": (ctypes.c_int, [vp, vp, vp, vp, i32, i32, ctypes.c_int, i32,
+                                                  vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -196,6 +200,23 @@ def subm3d_forward_fused(handle: MapHandle, feats, weight, bias, residual, out, 
                                   _ptr(residual), _ptr(out), int(cin), int(cout), int(dtype),
                                   1 if flip else 0, int(act), _stream(stream))
     _check(st, "subm3d_forward_fused")
+
+
+def subm3d_backward_data(handle: MapHandle, dy, weight, weight_t, dx, cin: int, cout: int,
+                         dtype: int, flip: bool, stream=None) -> None:
+    """Enqueue dx = the input gradient (W^T into weight_t, then the forward)."""
+    st = lib.subm3d_backward_data(handle.ptr, _ptr(dy), _ptr(weight), _ptr(weight_t), _ptr(dx),
+                                  int(cin), int(cout), int(dtype), 1 if flip else 0,
+                                  _stream(stream))
+    _check(st, "subm3d_backward_data")
+
+
+def subm3d_backward_weight(handle: MapHandle, feats, dy, dweight, cin: int, cout: int,
+                           dtype: int, flip: bool, stream=None) -> None:
+    """Enqueue dweight (fp32 KRSC) = the weight gradient."""
+    st = lib.subm3d_backward_weight(handle.ptr, _ptr(feats), _ptr(dy), _ptr(dweight), int(cin),
+                                    int(cout), int(dtype), 1 if flip else 0, _stream(stream))
+    _check(st, "subm3d_backward_weight")
 
 
 def subm3d_map_run_layout(handle: MapHandle):

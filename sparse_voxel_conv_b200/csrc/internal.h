@@ -140,4 +140,12 @@ cudaError_t launch_forward_bf16_runs(const int32_t* pos, const int32_t* etable,
                                      int32_t flip, const Epilogue& epi, int32_t* err_word,
                                      cudaStream_t stream);
 
+// Backward (backward.cu): W [cout][27][cin] -> W^T [cin][27][cout]; and the
+// weight gradient dW [cout][27][cin] fp32 (zeroed, then accumulated).
+cudaError_t launch_transpose_weight(const void* w, void* wt, int32_t cout, int32_t cin,
+                                    bool bf16, cudaStream_t stream);
+cudaError_t launch_wgrad(const int32_t* nbr, int64_t n, const void* x, const void* dy, float* dw,
+                         int32_t cin, int32_t cout, int32_t flip, bool bf16, int num_sms,
+                         cudaStream_t stream);
+
 }  // namespace subm3d

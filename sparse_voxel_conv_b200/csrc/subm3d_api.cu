@@ -267,6 +267,50 @@ subm3d_status subm3d_forward_fused(const subm3d_map* map, const void* feats, con
                       cin, cout, dtype, flip, act, stream);
 }
 
+subm3d_status subm3d_backward_data(const subm3d_map* map, const void* dy, const void* weight,
+                                   void* weight_t, void* dx, int32_t cin, int32_t cout,
+                                   subm3d_dtype dtype, int32_t flip, void* stream) {
+  if (!map || cin < 1 || cout < 1) return SUBM3D_E_INVALID;
+  if (dtype != SUBM3D_F32 && dtype != SUBM3D_BF16) return SUBM3D_E_INVALID;
+  if (map->n == 0) return SUBM3D_OK;
+  if (!dy || !weight || !weight_t || !dx) return SUBM3D_E_INVALID;
+  const size_t esz = dtype == SUBM3D_BF16 ? 2 : 4;
+  const size_t w_bytes = static_cast<size_t>(cout) * 27 * cin * esz;
+  if (overlaps(weight, w_bytes, weight_t, w_bytes)) return SUBM3D_E_INVALID;
+  if (!aligned(weight, esz) || !aligned(weight_t, 16)) return SUBM3D_E_INVALID;
+  auto s = static_cast<cudaStream_t>(stream);
+  if (subm3d::launch_transpose_weight(weight, weight_t, cout, cin, dtype == SUBM3D_BF16, s) !=
+      cudaSuccess)
+    return SUBM3D_E_CUDA;
+  // dx = forward of dy with W^T (Cout -> Cin) and the opposite orientation
+  return forward_impl(map, map->nbr, map->tile_mask, map->n, dy, weight_t, nullptr, nullptr, dx,
+                      cout, cin, dtype, flip ? 0 : 1, SUBM3D_ACT_NONE, stream);
+}
+
+subm3d_status subm3d_backward_weight(const subm3d_map* map, const void* feats, const void* dy,
+                                     float* dweight, int32_t cin, int32_t cout,
+                                     subm3d_dtype dtype, int32_t flip, void* stream) {
+  if (!map || cin < 1 || cout < 1 || !dweight) return SUBM3D_E_INVALID;
+  if (dtype != SUBM3D_F32 && dtype != SUBM3D_BF16) return SUBM3D_E_INVALID;
+  const int64_t n = map->n;
+  if (n > 0 && (!feats || !dy)) return SUBM3D_E_INVALID;
+  const size_t esz = dtype == SUBM3D_BF16 ? 2 : 4;
+  if (!aligned(feats, esz) || !aligned(dy, esz) || !aligned(dweight, 4)) return SUBM3D_E_INVALID;
+  const size_t dw_bytes = static_cast<size_t>(cout) * 27 * cin * 4;
+  if (n > 0 && (overlaps(dweight, dw_bytes, feats, static_cast<size_t>(n) * cin * esz) ||
+                overlaps(dweight, dw_bytes, dy, static_cast<size_t>(n) * cout * esz)))
+    return SUBM3D_E_INVALID;
+  int device = 0, sms = 0;
+  if (cudaGetDevice(&device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
+    return SUBM3D_E_CUDA;
+  return subm3d::launch_wgrad(map->nbr, n, feats, dy, dweight, cin, cout, flip ? 1 : 0,
+                              dtype == SUBM3D_BF16, sms, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? SUBM3D_OK
+             : SUBM3D_E_CUDA;
+}
+
 subm3d_status subm3d_device_status(void* stream) {
   int32_t* err = device_error_word();
   if (!err) return SUBM3D_E_CUDA;

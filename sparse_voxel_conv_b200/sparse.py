@@ -16,8 +16,8 @@ import torch
 from . import _abi
 from ._abi import Subm3dError
 
-__all__ = ["MapHandle", "build_map", "forward", "SparseTensor", "SubMConv3d", "SubMResBlock3d",
-           "Subm3dError"]
+__all__ = ["MapHandle", "build_map", "forward", "backward_data", "backward_weight", "SparseTensor",
+           "SubMConv3d", "SubMResBlock3d", "Subm3dError"]
 
 MapHandle = _abi.MapHandle
 
@@ -124,6 +124,68 @@ def forward(h: MapHandle, feats: torch.Tensor, weight: torch.Tensor, flip: bool 
     return out
 
 
+def backward_data(h: MapHandle, dy: torch.Tensor, weight: torch.Tensor, flip: bool = False,
+                  out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Input gradient of the convolution: dx[j] = sum over nbr[i,k] = j of
+    Wf[:,k,:]^T dy[i] -- the forward of dy with the transposed weight and the
+    opposite orientation.  dy: [N, Cout]; returns [N, Cin] in dy's dtype."""
+    if dy.dtype not in _DTYPES:
+        raise ValueError(f"unsupported dtype {dy.dtype}")
+    dy = _cuda_contig(dy, "dy")
+    weight = _cuda_contig(weight, "weight", dy.dtype)
+    n, cout = dy.shape
+    if n != h.n or weight.shape[0] != cout:
+        raise ValueError("dy must be [N, Cout] for this map and weight")
+    cin = weight.numel() // (27 * cout)
+    weight_t = torch.empty(weight.numel(), dtype=dy.dtype, device=dy.device)
+    if out is None:
+        out = torch.empty((n, cin), dtype=dy.dtype, device=dy.device)
+    _abi.subm3d_backward_data(h, dy, weight, weight_t, out, cin, cout, _DTYPES[dy.dtype], flip,
+                              stream)
+    return out
+
+
+def backward_weight(h: MapHandle, feats: torch.Tensor, dy: torch.Tensor, flip: bool = False,
+                    out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Weight gradient: dW[o,kw,c] = sum_i dy[i,o] feats[nbr[i,k],c] (kw = k, or
+    26 - k under flip), fp32 KRSC [Cout, 3, 3, 3, Cin] for either dtype."""
+    if feats.dtype not in _DTYPES:
+        raise ValueError(f"unsupported dtype {feats.dtype}")
+    feats = _cuda_contig(feats, "feats")
+    dy = _cuda_contig(dy, "dy", feats.dtype)
+    n, cin = feats.shape
+    cout = dy.shape[1]
+    if n != h.n or dy.shape[0] != n:
+        raise ValueError("feats and dy must have the map's N rows")
+    if out is None:
+        out = torch.empty((cout, 3, 3, 3, cin), dtype=torch.float32, device=feats.device)
+    _abi.subm3d_backward_weight(h, feats, dy, out, cin, cout, _DTYPES[feats.dtype], flip, stream)
+    return out
+
+
+class _SubMConvFunction(torch.autograd.Function):
+    """out = conv(feats, weight) on a built map, differentiable in feats and
+    weight through the library's backward kernels."""
+
+    @staticmethod
+    def forward(ctx, feats, weight, h, flip):
+        ctx.save_for_backward(feats, weight)
+        ctx.h, ctx.flip = h, flip
+        return forward(h, feats, weight, flip=flip)
+
+    @staticmethod
+    def backward(ctx, grad_out):
+        feats, weight = ctx.saved_tensors
+        grad_out = grad_out.contiguous()
+        dx = dw = None
+        if ctx.needs_input_grad[0]:
+            dx = backward_data(ctx.h, grad_out, weight, flip=ctx.flip)
+        if ctx.needs_input_grad[1]:
+            dw = backward_weight(ctx.h, feats, grad_out, flip=ctx.flip).to(weight.dtype)
+            dw = dw.reshape(weight.shape)
+        return dx, dw, None, None
+
+
 def run_layout_tensors(h: MapHandle):
     """(position table, E index table [tiles, 9, 260], header) as int32 views
     of the map's workspace; call after the build has completed."""
@@ -195,6 +257,13 @@ class SubMConv3d(torch.nn.Module):
 
     def forward(self, x: SparseTensor, residual: torch.Tensor | None = None) -> SparseTensor:
         h = x.get_map(self.indice_key)
+        wants_grad = torch.is_grad_enabled() and (self.weight.requires_grad or
+                                                   x.feats.requires_grad)
+        if wants_grad:
+            if self.act is not None or self.bias is not None or residual is not None:
+                raise NotImplementedError(
+                    "gradients are implemented for the plain convolution (no act, bias, residual)")
+            return x.replace(_SubMConvFunction.apply(x.feats, self.weight, h, self.flip))
         y = forward(h, x.feats, self.weight, flip=self.flip, act=self.act, bias=self.bias,
                     residual=residual)
         return x.replace(y)

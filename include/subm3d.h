@@ -277,9 +277,12 @@ SUBM3D_API subm3d_status subm3d_forward_fused(const subm3d_map* map, const void*
  * subm3d_backward_weight: dW[o][kw][c] = sum_i dy[i][o] * feats[nbr[i][k]][c]
  * over nbr[i][k] != -1, kw = k (flip = 0) or 26 - k.  dweight is fp32 KRSC
  * [Cout, 3, 3, 3, Cin] (device, 4-byte aligned, overwritten; fp32 for both
- * dtypes: the sum runs over all voxels).  CUDA-core FMA with fp32 atomics
- * across voxel slices, so the summation order (and the last bits) vary from
- * call to call.
+ * dtypes: the sum runs over all voxels).  bf16 with Cin a multiple of 64 runs
+ * on the tensor cores over the map's x-run layout (the sum over positions as
+ * the MMA K dimension, one gathered tile per (dz, dy) pair for all three dx);
+ * other shapes and fp32 on CUDA-core FMA.  Partial sums over voxel ranges are
+ * added with fp32 atomics, so the summation order (and the last bits) vary
+ * from call to call.
  *
  * Errors: SUBM3D_E_INVALID for bad arguments or overlapping buffers; otherwise
  * as subm3d_forward().  Both are asynchronous on `stream`.

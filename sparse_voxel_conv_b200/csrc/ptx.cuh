@@ -296,6 +296,22 @@ __device__ __forceinline__ uint64_t smem_desc_sw(uint32_t saddr, uint32_t row_by
   return d;
 }
 
+// Descriptor of an MN-major operand in the 128-byte swizzle layout: rows of
+// 128 bytes (64 consecutive M or N elements) at consecutive K, 8 rows per
+// 1024-byte swizzle atom, atoms `sbo` bytes apart along K and `lbo` bytes apart
+// along M/N (the canonical ((8,n),(8,k)):((1,LBO),(8,SBO)) layout in 16-byte
+// units); layout type 2 at [61,64), version 1 at [46,48), base offset 0.
+__device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t saddr, uint32_t lbo,
+                                                       uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
 // Descriptor of a K-major operand without swizzle: 8-row x 16-byte core
 // matrices, `lbo` bytes apart along K and `sbo` bytes apart along M/N.
 __device__ __forceinline__ uint64_t smem_desc_noswizzle(uint32_t saddr, uint32_t lbo,
@@ -329,6 +345,11 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
 // [17,23), M >> 4 at [24,29).
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t m, uint32_t n) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((n >> 3) << 17) | ((m >> 4) << 24);
+}
+
+// The same with both operands MN-major (A: bit 15, B: bit 16).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_mn(uint32_t m, uint32_t n) {
+  return idesc_bf16_f32(m, n) | (1u << 15) | (1u << 16);
 }
 
 }  // namespace subm3d

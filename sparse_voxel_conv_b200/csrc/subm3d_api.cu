@@ -300,12 +300,22 @@ subm3d_status subm3d_backward_weight(const subm3d_map* map, const void* feats, c
   if (n > 0 && (overlaps(dweight, dw_bytes, feats, static_cast<size_t>(n) * cin * esz) ||
                 overlaps(dweight, dw_bytes, dy, static_cast<size_t>(n) * cout * esz)))
     return SUBM3D_E_INVALID;
+  auto s = static_cast<cudaStream_t>(stream);
+  if (n > 0 && dtype == SUBM3D_BF16 && map->pos && cin % 64 == 0 && cout % 16 == 0 &&
+      aligned(feats, 16) && aligned(dy, 16) && aligned(dweight, 16) && device_is_sm100(nullptr) == 1) {
+    int32_t* err = device_error_word();
+    if (!err) return SUBM3D_E_CUDA;
+    return subm3d::launch_wgrad_bf16_runs(map->pos, map->et, map->hdr, feats, dy, dweight, cin,
+                                          cout, flip ? 1 : 0, err, s) == cudaSuccess
+               ? SUBM3D_OK
+               : SUBM3D_E_CUDA;
+  }
   int device = 0, sms = 0;
   if (cudaGetDevice(&device) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
     return SUBM3D_E_CUDA;
   return subm3d::launch_wgrad(map->nbr, n, feats, dy, dweight, cin, cout, flip ? 1 : 0,
-                              dtype == SUBM3D_BF16, sms, static_cast<cudaStream_t>(stream)) ==
+                              dtype == SUBM3D_BF16, sms, s) ==
                  cudaSuccess
              ? SUBM3D_OK
              : SUBM3D_E_CUDA;

@@ -121,3 +121,18 @@ def test_autograd_through_subm_conv(S):
     # the weight gradient is returned in the weight's dtype (bf16): one rounding
     assert_close(conv.weight.grad.float().cpu().numpy(), C.round_bf16(dw_ref), RTOL_BF16,
                  "autograd dW")
+
+
+@pytest.mark.parametrize("cin,cout", [(128, 128), (192, 64), (64, 144)])
+@pytest.mark.parametrize("flip", [False, True])
+def test_backward_weight_tensor_core_blocks(S, shell, cin, cout, flip):
+    """The tcgen05 weight gradient over channel blocks of 128: full blocks, a
+    partial input-channel block (192 = 128 + 64), output channels below and
+    above one block (64, 144 = 128 + 16)."""
+    wl, nbr = shell
+    h, x, w, dy, xt, wt, dyt = _tensors(S, wl, "bf16", cin, cout, 61)
+    dw = S.backward_weight(h, xt, dyt, flip=flip)
+    torch.cuda.synchronize()
+    assert S._abi.subm3d_device_status() == 0
+    ref = C.backward_weight(nbr, x.astype(np.float64), dy.astype(np.float64), flip=flip)
+    assert_close(dw.cpu().numpy(), ref, RTOL_WGRAD, f"wgrad {cin}->{cout} flip={flip}")

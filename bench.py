@@ -257,6 +257,31 @@ def backward_line(h, feats, weight, flops, flush, peak_tf, fp32_peak):
                        "frac": w_tf / peak_tf, "bound": "tensor"}}
 
 
+def resample_line(coords, feats, grid, flush, hbm_gbs):
+    """Subdivide the headline set (8 children per voxel, features replicated) and
+    mean-pool the result back (the fine map built beforehand); algorithmic bytes
+    over time, against the HBM copy peak.  Pooling reads its parent count back
+    to the host, so its time includes that one synchronisation."""
+    import sparse_voxel_conv_b200 as S
+    st = S.SparseTensor(coords, feats, grid, 1)
+    n, c = feats.shape
+    esz = feats.element_size()
+    sub_ms = _time_ms(lambda: S.subdivide(st), flush)
+    fine = S.subdivide(st)
+    fine.get_map("subm0")
+    pool_ms = _time_ms(lambda: S.downsample(fine, "mean"), flush)
+    sub_bytes = n * (16 + c * esz) + 8 * n * (16 + c * esz)
+    pool_bytes = 8 * n * (16 + c * esz) + n * (16 + c * esz)
+    sub_gbs = sub_bytes / (sub_ms / 1e3) / 1e9
+    pool_gbs = pool_bytes / (pool_ms / 1e3) / 1e9
+    return {"subdivide": {"ms": sub_ms, "bytes": sub_bytes, "achieved": sub_gbs,
+                          "peak": hbm_gbs, "unit": "GB/s", "frac": sub_gbs / hbm_gbs,
+                          "bound": "hbm"},
+            "downsample_mean": {"ms": pool_ms, "bytes": pool_bytes, "achieved": pool_gbs,
+                                "peak": hbm_gbs, "unit": "GB/s", "frac": pool_gbs / hbm_gbs,
+                                "bound": "hbm", "children": 8 * n}}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -429,6 +454,8 @@ def run_ours(args):
                                                          peak_tf, fwd_avg_s * 1e3)
             line["backward"] = backward_line(h_ctx, feats, weight, flops_alg, flush, peak_tf,
                                              line["fp32_forward"]["peak"])
+            line["resample"] = resample_line(coords, feats, wl.grid_dim, flush,
+                                             float(peaks["hbm_gbs"]))
             line["context_per_offset_torch"] = per_offset_context(h_ctx, feats, weight, flush)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl, args.cpu_rows)

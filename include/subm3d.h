@@ -297,6 +297,72 @@ SUBM3D_API subm3d_status subm3d_backward_weight(const subm3d_map* map, const voi
                                                 void* stream);
 
 /*
+ * Resolution changes, factor 2 (trellis_sparse_mrp_mlx commit log; lato.2_mrp_mlx
+ * notes "Key facts").  Child slot s of a parent at (b, z, y, x) lies at
+ * (b, 2z + dz, 2y + dy, 2x + dx).
+ *
+ *   SUBM3D_EXPAND_SUBDIVIDE       every voxel emits its 8 children in C order
+ *                                 (s = 4 dz + 2 dy + dx), features replicated;
+ *                                 mask must be NULL.
+ *   SUBM3D_EXPAND_UPSAMPLE        voxel i emits child s only where mask[i*8 + s]
+ *                                 != 0; s decodes axis 0 fastest (dz = s % 2,
+ *                                 dy = s / 2 % 2, dx = s / 4 % 2); features
+ *                                 replicated; mask required.
+ *   SUBM3D_EXPAND_CHANNEL2SPATIAL as UPSAMPLE (mask optional: NULL = all 8), child
+ *                                 s takes channels [s C, (s + 1) C) of the
+ *                                 parent's 8 C (C = channels_out).
+ *
+ * subm3d_expand: coords (device) int32 [N, 4], 16-byte aligned; feats (device)
+ * [N, Cin] in dtype (Cin = channels_out, or 8 channels_out for
+ * channel2spatial); mask (device) uint8 [N, 8] or NULL.  out_coords [8N, 4]
+ * and out_feats [8N, channels_out] (device) receive the children parent-major,
+ * by ascending s; *out_count (host) = the number written.  workspace (device)
+ * >= subm3d_expand_workspace_bytes(N), 256-byte aligned.  With a mask the call
+ * reads the child count back and is blocking; without one it is asynchronous.
+ * N < 2^28.
+ */
+typedef enum {
+  SUBM3D_EXPAND_SUBDIVIDE = 0,
+  SUBM3D_EXPAND_UPSAMPLE = 1,
+  SUBM3D_EXPAND_CHANNEL2SPATIAL = 2
+} subm3d_expand_mode;
+SUBM3D_API size_t subm3d_expand_workspace_bytes(int64_t n);
+SUBM3D_API subm3d_status subm3d_expand(const int32_t* coords, const void* feats,
+                                       const uint8_t* mask, int64_t n, int32_t channels_out,
+                                       subm3d_dtype dtype, subm3d_expand_mode mode,
+                                       int32_t* out_coords, void* out_feats, void* workspace,
+                                       size_t workspace_bytes, int64_t* out_count, void* stream);
+
+/*
+ * Pooling to parents coord // 2, listed in raster order of (b, z, y, x):
+ *
+ *   SUBM3D_POOL_MAX / SUBM3D_POOL_MEAN  the element-wise max or mean over the
+ *                              children present (mean: an fp32 sum in child slot
+ *                              order, then one rounding); out_feats [P, C].
+ *   SUBM3D_POOL_SPATIAL2CHANNEL  child s's features in channels [s C, (s+1) C) of
+ *                              its parent, s = (z % 2) + 2 (y % 2) + 4 (x % 2),
+ *                              zeros where the child is absent; out_feats [P, 8 C].
+ *
+ * fine: the map built on `coords` (its table finds the children).  coords,
+ * feats [N, C] (device) are that set and its features; out_coords [N, 4] and
+ * out_feats (device) must have room for P <= N parents.  workspace >=
+ * subm3d_pool_workspace_bytes(N, grid_dim, batch) (a flag per parent cell of
+ * batch x ceil(grid_dim/2)^3; 0 = unsupported above 2^30 cells), 256-byte
+ * aligned.  Blocking: *out_count (host) = P is read back.
+ */
+typedef enum {
+  SUBM3D_POOL_MAX = 0,
+  SUBM3D_POOL_MEAN = 1,
+  SUBM3D_POOL_SPATIAL2CHANNEL = 2
+} subm3d_pool_mode;
+SUBM3D_API size_t subm3d_pool_workspace_bytes(int64_t n, int32_t grid_dim, int32_t batch);
+SUBM3D_API subm3d_status subm3d_pool(const subm3d_map* fine, const int32_t* coords,
+                                     const void* feats, int32_t channels, subm3d_dtype dtype,
+                                     subm3d_pool_mode mode, int32_t* out_coords, void* out_feats,
+                                     void* workspace, size_t workspace_bytes, int64_t* out_count,
+                                     void* stream);
+
+/*
  * Device pointers into the map's x-run layout, for tests and tools: the
  * position table (int32, one entry per position: row * 4 + tag, tag 0 voxel,
  * 1 left pad of that row's voxel, 2 right pad, -1 empty), the E index table

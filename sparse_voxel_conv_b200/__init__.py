@@ -9,8 +9,10 @@ it loads the library and fails loudly if it is not built.
 from . import _abi
 from ._abi import Subm3dError
 from .sparse import MapHandle, SparseTensor, SubMConv3d, SubMResBlock3d, backward_data, \
-    backward_weight, build_map, forward, map_status, run_layout_tensors, tile_mask_tensor
+    backward_weight, build_map, channel2spatial, downsample, forward, map_status, \
+    run_layout_tensors, spatial2channel, subdivide, tile_mask_tensor, upsample
 
 __all__ = ["Subm3dError", "MapHandle", "SparseTensor", "SubMConv3d", "SubMResBlock3d", "build_map",
            "forward", "backward_data", "backward_weight", "map_status", "run_layout_tensors",
-           "tile_mask_tensor"]
+           "tile_mask_tensor", "subdivide", "upsample", "channel2spatial", "spatial2channel",
+           "downsample"]

@@ -30,6 +30,12 @@ SUBM3D_ACT_NONE = 0
 SUBM3D_ACT_GELU = 1
 SUBM3D_ACT_SILU = 2
 SUBM3D_KVOL = 27
+SUBM3D_EXPAND_SUBDIVIDE = 0
+SUBM3D_EXPAND_UPSAMPLE = 1
+SUBM3D_EXPAND_CHANNEL2SPATIAL = 2
+SUBM3D_POOL_MAX = 0
+SUBM3D_POOL_MEAN = 1
+SUBM3D_POOL_SPATIAL2CHANNEL = 2
 SUBM3D_TILE_ROWS = 128
 
 
@@ -69,6 +75,12 @@ def _load() -> ctypes.CDLL:
                                                 i32, ctypes.c_int, vp]),
         "subm3d_backward_data": (ctypes.c_int, [vp, vp, vp, vp, vp, i32, i32, ctypes.c_int, i32,
                                                 vp]),
+        "subm3d_expand_workspace_bytes": (sz, [i64]),
+        "subm3d_expand": (ctypes.c_int, [vp, vp, vp, i64, i32, ctypes.c_int, ctypes.c_int, vp, vp,
+                                         vp, sz, ctypes.POINTER(i64), vp]),
+        "subm3d_pool_workspace_bytes": (sz, [i64, i32, i32]),
+        "subm3d_pool": (ctypes.c_int, [vp, vp, vp, i32, ctypes.c_int, ctypes.c_int, vp, vp, vp, sz,
+                                       ctypes.POINTER(i64), vp]),
         "subm3d_backward_weight": (ctypes.c_int, [vp, vp, vp, vp, i32, i32, ctypes.c_int, i32,
                                                   vp]),
     }
@@ -217,6 +229,37 @@ def subm3d_backward_weight(handle: MapHandle, feats, dy, dweight, cin: int, cout
     st = lib.subm3d_backward_weight(handle.ptr, _ptr(feats), _ptr(dy), _ptr(dweight), int(cin),
                                     int(cout), int(dtype), 1 if flip else 0, _stream(stream))
     _check(st, "subm3d_backward_weight")
+
+
+def subm3d_expand_workspace_bytes(n: int) -> int:
+    return int(lib.subm3d_expand_workspace_bytes(int(n)))
+
+
+def subm3d_expand(coords, feats, mask, n: int, channels_out: int, dtype: int, mode: int,
+                  out_coords, out_feats, workspace, workspace_bytes: int, stream=None) -> int:
+    """Enqueue an expansion; returns the number of child rows (blocking with a mask)."""
+    count = ctypes.c_int64(0)
+    st = lib.subm3d_expand(_ptr(coords), _ptr(feats), _ptr(mask), int(n), int(channels_out),
+                           int(dtype), int(mode), _ptr(out_coords), _ptr(out_feats),
+                           _ptr(workspace), int(workspace_bytes), ctypes.byref(count),
+                           _stream(stream))
+    _check(st, "subm3d_expand")
+    return int(count.value)
+
+
+def subm3d_pool_workspace_bytes(n: int, grid_dim: int, batch: int) -> int:
+    return int(lib.subm3d_pool_workspace_bytes(int(n), int(grid_dim), int(batch)))
+
+
+def subm3d_pool(handle: MapHandle, coords, feats, channels: int, dtype: int, mode: int,
+                out_coords, out_feats, workspace, workspace_bytes: int, stream=None) -> int:
+    """Pool to parents coord // 2 (blocking); returns the number of parents."""
+    count = ctypes.c_int64(0)
+    st = lib.subm3d_pool(handle.ptr, _ptr(coords), _ptr(feats), int(channels), int(dtype),
+                         int(mode), _ptr(out_coords), _ptr(out_feats), _ptr(workspace),
+                         int(workspace_bytes), ctypes.byref(count), _stream(stream))
+    _check(st, "subm3d_pool")
+    return int(count.value)
 
 
 def subm3d_map_run_layout(handle: MapHandle):

@@ -155,4 +155,36 @@ cudaError_t launch_wgrad_bf16_runs(const int32_t* pos, const int32_t* etable,
                                    float* dw, int32_t cin, int32_t cout, int32_t flip,
                                    int32_t* err_word, cudaStream_t stream);
 
+// Resolution changes (resample.cu).  Expansion: subdivide (C-order children,
+// replicated rows), upsample (masked, axis-0-fastest children, replicated) and
+// channel2spatial (masked or not, channel slices); child rows are written
+// parent-major.  Its workspace: per-1,024-voxel child counts, a total and, per
+// child row, its source (parent * 8 + slot).
+struct ExpandLayout {
+  int64_t n_blocks = 0;
+  size_t cnt_off = 0, total_off = 0, src_off = 0, bytes = 0;
+};
+ExpandLayout expand_layout(int64_t n);
+// Blocking when `mask` is given (the child count is read back); *out_count = rows.
+cudaError_t launch_expand(const int32_t* coords, const void* feats, const uint8_t* mask, int64_t n,
+                          int64_t in_row_bytes, int64_t out_row_bytes, bool slice, bool c_order,
+                          int32_t* out_coords, void* out_feats, void* workspace,
+                          int64_t* out_count, cudaStream_t stream);
+
+// Pooling to parents coord // 2 in raster order: max (0), mean (1) or
+// spatial2channel (2), through the fine set's map table.  Its workspace: a flag
+// per parent cell, per-4,096-cell counts, a total and the parents' cells.
+struct PoolLayout {
+  int32_t G = 0;
+  int64_t cells = 0, n_blocks = 0;
+  size_t flags_off = 0, cnt_off = 0, total_off = 0, cells_off = 0, bytes = 0;
+};
+PoolLayout pool_layout(int64_t n, int32_t grid_dim, int32_t batch);
+// Blocking (the parent count is read back); *out_count = parents.
+cudaError_t launch_pool(const MapLayout& map_lay, const void* map_ws, int32_t grid_dim,
+                        int32_t batch, const int32_t* coords, int64_t n, const void* feats,
+                        int32_t channels, bool bf16, int mode, int32_t* out_coords,
+                        void* out_feats, void* workspace, int64_t* out_count,
+                        cudaStream_t stream);
+
 }  // namespace subm3d

@@ -28,55 +28,10 @@
 #include <cuda_runtime.h>
 
 #include "internal.h"
+#include "map_table.cuh"
 
 namespace subm3d {
 namespace {
-
-constexpr unsigned long long kEmpty = ~0ull;
-
-__device__ __forceinline__ uint32_t mix32(uint32_t h) {
-  h ^= h >> 16;
-  h *= 0x85ebca6bu;
-  h ^= h >> 13;
-  h *= 0xc2b2ae35u;
-  h ^= h >> 16;
-  return h;
-}
-
-__device__ __forceinline__ uint32_t mix64to32(unsigned long long k) {
-  k ^= k >> 33;
-  k *= 0xff51afd7ed558ccdull;
-  k ^= k >> 33;
-  k *= 0xc4ceb9fe1a85ec53ull;
-  k ^= k >> 33;
-  return static_cast<uint32_t>(k);
-}
-
-__device__ __forceinline__ uint32_t pack32(int b, int z, int y, int x) {
-  return (static_cast<uint32_t>(b) << 30) | (static_cast<uint32_t>(z) << 20) |
-         (static_cast<uint32_t>(y) << 10) | static_cast<uint32_t>(x);
-}
-__device__ __forceinline__ unsigned long long pack64(int b, int z, int y, int x) {
-  return (static_cast<unsigned long long>(b) << 48) | (static_cast<unsigned long long>(z) << 32) |
-         (static_cast<unsigned long long>(y) << 16) | static_cast<unsigned long long>(x);
-}
-__device__ __forceinline__ uint32_t home32(uint32_t key, uint32_t capmask) {
-  return ((mix32(key >> 2) << 2) | (key & 3u)) & capmask;
-}
-__device__ __forceinline__ uint32_t home64(unsigned long long key, uint32_t capmask) {
-  return ((mix64to32(key >> 2) << 2) | static_cast<uint32_t>(key & 3u)) & capmask;
-}
-
-__device__ __forceinline__ bool in_volume(int4 c, int grid, int batch) {
-  return static_cast<unsigned>(c.x) < static_cast<unsigned>(batch) &&
-         static_cast<unsigned>(c.y) < static_cast<unsigned>(grid) &&
-         static_cast<unsigned>(c.z) < static_cast<unsigned>(grid) &&
-         static_cast<unsigned>(c.w) < static_cast<unsigned>(grid);
-}
-
-__device__ __forceinline__ int64_t cell_of(int b, int z, int y, int x, int grid) {
-  return ((static_cast<int64_t>(b) * grid + z) * grid + y) * grid + x;
-}
 
 // Fills the lookup table (`words16a` 16-byte words) with all-ones, zeroes the
 // run layout's superblock sums (`words16z` words), the status word and the
@@ -218,43 +173,6 @@ __global__ void map_insert_wide(const int4* __restrict__ coords, int64_t n, int 
     slot = (slot + 1) & capmask;
   }
   atomicOr(status, kErrTableFull);
-}
-
-enum class Kind { kDirect, kCompact, kWide };
-
-struct Tables {
-  const int32_t* cells;             // direct
-  const unsigned long long* table;  // compact slots or wide keys
-  const int32_t* rows;              // wide rows
-  uint32_t capmask;
-};
-
-template <Kind K>
-__device__ __forceinline__ int32_t lookup(const Tables& t, int b, int z, int y, int x, int grid) {
-  if constexpr (K == Kind::kDirect) {
-    return __ldg(t.cells + cell_of(b, z, y, x, grid));
-  } else if constexpr (K == Kind::kCompact) {
-    const uint32_t key = pack32(b, z, y, x);
-    uint32_t slot = home32(key, t.capmask);
-    for (uint64_t step = 0; step <= t.capmask; ++step) {
-      const unsigned long long e = __ldg(t.table + slot);
-      if (e == kEmpty) return -1;
-      if (static_cast<uint32_t>(e >> 32) == key)
-        return static_cast<int32_t>(static_cast<uint32_t>(e));
-      slot = (slot + 1) & t.capmask;
-    }
-    return -1;
-  } else {
-    const unsigned long long key = pack64(b, z, y, x);
-    uint32_t slot = home64(key, t.capmask);
-    for (uint64_t step = 0; step <= t.capmask; ++step) {
-      const unsigned long long e = __ldg(t.table + slot);
-      if (e == kEmpty) return -1;
-      if (e == key) return __ldg(t.rows + slot);
-      slot = (slot + 1) & t.capmask;
-    }
-    return -1;
-  }
 }
 
 // ----------------------------------------------------------- run layout ----

@@ -22,6 +22,8 @@ struct subm3d_map {
   const int32_t* et;      // E index table
   const int32_t* hdr;     // [runs, position tiles, positions, 0]
   int64_t ptile_max;      // position tiles reserved in the workspace
+  const void* workspace;  // the build's workspace, laid out as `layout`
+  subm3d::MapLayout layout;
   int64_t n;
   int32_t grid_dim;
   int32_t batch;
@@ -133,6 +135,8 @@ subm3d_status subm3d_build_map(const int32_t* coords, int64_t n, int32_t grid_di
   h->et = runs ? reinterpret_cast<const int32_t*>(ws + lay.et_off) : nullptr;
   h->hdr = runs ? reinterpret_cast<const int32_t*>(ws + lay.hdr_off) : nullptr;
   h->ptile_max = lay.ptile_max;
+  h->workspace = workspace;
+  h->layout = lay;
   h->n = n;
   h->grid_dim = grid_dim;
   h->batch = batch;
@@ -319,6 +323,73 @@ subm3d_status subm3d_backward_weight(const subm3d_map* map, const void* feats, c
                  cudaSuccess
              ? SUBM3D_OK
              : SUBM3D_E_CUDA;
+}
+
+size_t subm3d_expand_workspace_bytes(int64_t n) {
+  if (n < 0 || n >= (int64_t(1) << 28)) return 0;
+  return subm3d::expand_layout(n).bytes;
+}
+
+subm3d_status subm3d_expand(const int32_t* coords, const void* feats, const uint8_t* mask,
+                            int64_t n, int32_t channels_out, subm3d_dtype dtype,
+                            subm3d_expand_mode mode, int32_t* out_coords, void* out_feats,
+                            void* workspace, size_t workspace_bytes, int64_t* out_count,
+                            void* stream) {
+  if (!out_count || n < 0 || channels_out < 1) return SUBM3D_E_INVALID;
+  *out_count = 0;
+  if (dtype != SUBM3D_F32 && dtype != SUBM3D_BF16) return SUBM3D_E_INVALID;
+  if (mode != SUBM3D_EXPAND_SUBDIVIDE && mode != SUBM3D_EXPAND_UPSAMPLE &&
+      mode != SUBM3D_EXPAND_CHANNEL2SPATIAL)
+    return SUBM3D_E_INVALID;
+  if ((mode == SUBM3D_EXPAND_SUBDIVIDE && mask) || (mode == SUBM3D_EXPAND_UPSAMPLE && !mask))
+    return SUBM3D_E_INVALID;
+  if (n >= (int64_t(1) << 28)) return SUBM3D_E_UNSUPPORTED;
+  if (n == 0) return SUBM3D_OK;
+  if (!coords || !feats || !out_coords || !out_feats || !workspace) return SUBM3D_E_INVALID;
+  if (workspace_bytes < subm3d::expand_layout(n).bytes) return SUBM3D_E_INVALID;
+  const size_t esz = dtype == SUBM3D_BF16 ? 2 : 4;
+  if (!aligned(coords, 16) || !aligned(out_coords, 16) || !aligned(workspace, 256) ||
+      !aligned(feats, esz) || !aligned(out_feats, esz))
+    return SUBM3D_E_INVALID;
+  const bool slice = mode == SUBM3D_EXPAND_CHANNEL2SPATIAL;
+  const int64_t out_row = static_cast<int64_t>(channels_out) * esz;
+  const int64_t in_row = slice ? 8 * out_row : out_row;
+  const cudaError_t e = subm3d::launch_expand(
+      coords, feats, mask, n, in_row, out_row, slice, mode == SUBM3D_EXPAND_SUBDIVIDE, out_coords,
+      out_feats, workspace, out_count, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SUBM3D_OK : SUBM3D_E_CUDA;
+}
+
+size_t subm3d_pool_workspace_bytes(int64_t n, int32_t grid_dim, int32_t batch) {
+  if (n < 0 || grid_dim < 1 || grid_dim > 65535 || batch < 1 || batch > 65535) return 0;
+  const subm3d::PoolLayout l = subm3d::pool_layout(n, grid_dim, batch);
+  if (l.cells > (int64_t(1) << 30)) return 0;
+  return l.bytes;
+}
+
+subm3d_status subm3d_pool(const subm3d_map* fine, const int32_t* coords, const void* feats,
+                          int32_t channels, subm3d_dtype dtype, subm3d_pool_mode mode,
+                          int32_t* out_coords, void* out_feats, void* workspace,
+                          size_t workspace_bytes, int64_t* out_count, void* stream) {
+  if (!fine || !out_count || channels < 1) return SUBM3D_E_INVALID;
+  *out_count = 0;
+  if (dtype != SUBM3D_F32 && dtype != SUBM3D_BF16) return SUBM3D_E_INVALID;
+  if (mode != SUBM3D_POOL_MAX && mode != SUBM3D_POOL_MEAN && mode != SUBM3D_POOL_SPATIAL2CHANNEL)
+    return SUBM3D_E_INVALID;
+  const int64_t n = fine->n;
+  const size_t need = subm3d_pool_workspace_bytes(n, fine->grid_dim, fine->batch);
+  if (need == 0) return SUBM3D_E_UNSUPPORTED;
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return SUBM3D_E_INVALID;
+  if (n > 0 && (!coords || !feats || !out_coords || !out_feats)) return SUBM3D_E_INVALID;
+  const size_t esz = dtype == SUBM3D_BF16 ? 2 : 4;
+  if (!aligned(coords, 16) || !aligned(out_coords, 16) || !aligned(feats, esz) ||
+      !aligned(out_feats, esz))
+    return SUBM3D_E_INVALID;
+  const cudaError_t e = subm3d::launch_pool(
+      fine->layout, fine->workspace, fine->grid_dim, fine->batch, coords, n, feats, channels,
+      dtype == SUBM3D_BF16, static_cast<int>(mode), out_coords, out_feats, workspace, out_count,
+      static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SUBM3D_OK : SUBM3D_E_CUDA;
 }
 
 subm3d_status subm3d_device_status(void* stream) {

@@ -17,7 +17,8 @@ from . import _abi
 from ._abi import Subm3dError
 
 __all__ = ["MapHandle", "build_map", "forward", "backward_data", "backward_weight", "SparseTensor",
-           "SubMConv3d", "SubMResBlock3d", "Subm3dError"]
+           "SubMConv3d", "SubMResBlock3d", "Subm3dError", "subdivide", "upsample",
+           "channel2spatial", "spatial2channel", "downsample"]
 
 MapHandle = _abi.MapHandle
 
@@ -290,3 +291,81 @@ class SubMResBlock3d(torch.nn.Module):
 
     def forward(self, x: SparseTensor) -> SparseTensor:
         return self.conv2(self.conv1(x), residual=x.feats)
+
+
+# ------------------------------------------------------ resolution changes ----
+
+def _expand(x: "SparseTensor", mask, mode: int, channels_out: int) -> "SparseTensor":
+    coords = _cuda_contig(x.coords, "coords", torch.int32)
+    feats = _cuda_contig(x.feats, "feats")
+    if feats.dtype not in _DTYPES:
+        raise ValueError(f"unsupported dtype {feats.dtype}")
+    n = coords.shape[0]
+    if mask is not None:
+        mask = _cuda_contig(mask, "mask")
+        if mask.dtype != torch.uint8:
+            mask = (mask != 0).to(torch.uint8)
+        if tuple(mask.shape) != (n, 8):
+            raise ValueError("mask must be [N, 8]")
+    ws_bytes = max(_abi.subm3d_expand_workspace_bytes(n), 256)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=coords.device)
+    out_c = torch.empty((8 * n, 4), dtype=torch.int32, device=coords.device)
+    out_f = torch.empty((8 * n, channels_out), dtype=feats.dtype, device=coords.device)
+    m = _abi.subm3d_expand(coords, feats, mask, n, channels_out, _DTYPES[feats.dtype], mode,
+                           out_c, out_f, ws, ws_bytes)
+    return SparseTensor(out_c[:m], out_f[:m], x.grid_dim * 2, x.batch)
+
+
+def subdivide(x: "SparseTensor") -> "SparseTensor":
+    """SparseSubdivide: every voxel -> its 8 children 2*coord + (dz, dy, dx) in C
+    order (x fastest), features replicated; grid_dim doubles."""
+    return _expand(x, None, _abi.SUBM3D_EXPAND_SUBDIVIDE, x.feats.shape[1])
+
+
+def upsample(x: "SparseTensor", mask: torch.Tensor) -> "SparseTensor":
+    """Masked upsample: voxel i emits child s where mask[i, s] != 0, the child
+    index decoded axis 0 fastest (dz = s % 2, dy = s // 2 % 2, dx = s // 4 % 2);
+    features replicated."""
+    return _expand(x, mask, _abi.SUBM3D_EXPAND_UPSAMPLE, x.feats.shape[1])
+
+
+def channel2spatial(x: "SparseTensor", mask: torch.Tensor | None = None) -> "SparseTensor":
+    """Sparse depth-to-space: features [N, 8C] -> child s (axis 0 fastest) takes
+    channels [sC, (s+1)C); all 8 children or the flagged ones."""
+    c8 = x.feats.shape[1]
+    if c8 % 8:
+        raise ValueError("channel2spatial needs a multiple of 8 channels")
+    return _expand(x, mask, _abi.SUBM3D_EXPAND_CHANNEL2SPATIAL, c8 // 8)
+
+
+def _pool(x: "SparseTensor", mode: int, indice_key: str, channels_out: int) -> "SparseTensor":
+    h = x.get_map(indice_key)
+    coords = _cuda_contig(x.coords, "coords", torch.int32)
+    feats = _cuda_contig(x.feats, "feats")
+    n, c = feats.shape
+    ws_bytes = _abi.subm3d_pool_workspace_bytes(n, x.grid_dim, x.batch)
+    if ws_bytes == 0:
+        raise Subm3dError(_abi.SUBM3D_E_UNSUPPORTED, "subm3d_pool_workspace_bytes")
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=coords.device)
+    out_c = torch.empty((max(n, 1), 4), dtype=torch.int32, device=coords.device)
+    out_f = torch.empty((max(n, 1), channels_out), dtype=feats.dtype, device=coords.device)
+    p = _abi.subm3d_pool(h, coords, feats, c, _DTYPES[feats.dtype], mode, out_c, out_f, ws,
+                         ws_bytes)
+    return SparseTensor(out_c[:p], out_f[:p], (x.grid_dim + 1) // 2, x.batch)
+
+
+def downsample(x: "SparseTensor", mode: str, indice_key: str = "subm0") -> "SparseTensor":
+    """Parents coord // 2 in raster order with the max or the mean of their
+    children's features.  The pages' models differ here (LATO.2: max, Pixal3D:
+    mean by default), so the mode has no default.  Uses (or builds) the map of
+    `indice_key` on x's coordinate set."""
+    modes = {"max": _abi.SUBM3D_POOL_MAX, "mean": _abi.SUBM3D_POOL_MEAN}
+    if mode not in modes:
+        raise ValueError("mode must be 'max' or 'mean'")
+    return _pool(x, modes[mode], indice_key, x.feats.shape[1])
+
+
+def spatial2channel(x: "SparseTensor", indice_key: str = "subm0") -> "SparseTensor":
+    """Sparse space-to-depth: parents coord // 2 (raster order), child s's
+    features in channels [sC, (s+1)C), zeros for absent children."""
+    return _pool(x, _abi.SUBM3D_POOL_SPATIAL2CHANNEL, indice_key, 8 * x.feats.shape[1])

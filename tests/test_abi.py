@@ -112,3 +112,39 @@ def test_forward_argument_errors(abi):
     assert f(A, None, 10, A, W, B, 16, 24, 1, 0, 0, None) == E_UNSUP       # bf16 Cout % 16
     assert f(A, None, 10, A + 8, W, B, 16, 16, 1, 0, 0, None) == E_UNSUP   # bf16 alignment
     assert f(A, None, 10, A + 2, W, B, 3, 5, 0, 0, 0, None) == E_INVALID   # f32 alignment
+
+
+def test_resample_and_backward_argument_errors(abi):
+    """Host-side checks of the newer entry points: no CUDA call is reached."""
+    lib = abi.lib
+    cnt = ctypes.c_int64(5)
+    E_INVALID = abi.SUBM3D_E_INVALID
+    A = 1 << 20
+    assert abi.subm3d_expand_workspace_bytes(-1) == 0
+    assert abi.subm3d_expand_workspace_bytes(1000) > 8 * 1000 * 8
+    assert abi.subm3d_pool_workspace_bytes(10, 0, 1) == 0
+    assert abi.subm3d_pool_workspace_bytes(10, 64, 1) >= 32 ** 3
+    # expand: no count pointer, bad mode, subdivide with a mask, upsample without one
+    assert lib.subm3d_expand(A, A, None, 10, 8, abi.SUBM3D_F32, 0, A, A, A, 1 << 20, None,
+                             None) == E_INVALID
+    assert lib.subm3d_expand(A, A, None, 10, 8, abi.SUBM3D_F32, 7, A, A, A, 1 << 20,
+                             ctypes.byref(cnt), None) == E_INVALID and cnt.value == 0
+    assert lib.subm3d_expand(A, A, A, 10, 8, abi.SUBM3D_F32, abi.SUBM3D_EXPAND_SUBDIVIDE, A, A,
+                             A, 1 << 20, ctypes.byref(cnt), None) == E_INVALID
+    assert lib.subm3d_expand(A, A, None, 10, 8, abi.SUBM3D_F32, abi.SUBM3D_EXPAND_UPSAMPLE, A, A,
+                             A, 1 << 20, ctypes.byref(cnt), None) == E_INVALID
+    # expand: workspace too small, misaligned coordinates
+    assert lib.subm3d_expand(A, A, None, 10, 8, abi.SUBM3D_F32, 0, A, A, A, 16,
+                             ctypes.byref(cnt), None) == E_INVALID
+    assert lib.subm3d_expand(A + 4, A, None, 10, 8, abi.SUBM3D_F32, 0, A, A, A, 1 << 20,
+                             ctypes.byref(cnt), None) == E_INVALID
+    # empty expansion: nothing to do, count 0
+    assert lib.subm3d_expand(None, None, None, 0, 8, abi.SUBM3D_F32, 0, None, None, None, 0,
+                             ctypes.byref(cnt), None) == abi.SUBM3D_OK and cnt.value == 0
+    # pool / backward need a map handle
+    assert lib.subm3d_pool(None, A, A, 8, abi.SUBM3D_F32, 0, A, A, A, 1 << 20, ctypes.byref(cnt),
+                           None) == E_INVALID
+    assert lib.subm3d_backward_data(None, A, A, A, A, 8, 8, abi.SUBM3D_F32, 0, None) == E_INVALID
+    assert lib.subm3d_backward_weight(None, A, A, A, 8, 8, abi.SUBM3D_F32, 0, None) == E_INVALID
+    assert lib.subm3d_forward_fused(None, A, A, None, None, A, 8, 8, abi.SUBM3D_F32, 0, 0,
+                                    None) == E_INVALID

@@ -111,8 +111,8 @@ __global__ void __launch_bounds__(kScanThreads) expand_count(const uint8_t* __re
   if (threadIdx.x == 0) block_cnt[blockIdx.x] = sum;
 }
 
-// Child coordinates and, per child row, its source (parent * 8 + slot).  Without
-// a mask every voxel has 8 children at rows 8 i .. 8 i + 7.
+// Child coordinates and, with a mask, each child row's source (parent * 8 +
+// slot).  Without a mask every voxel has 8 children at rows 8 i .. 8 i + 7.
 __global__ void __launch_bounds__(kScanThreads)
     expand_emit(const int4* __restrict__ coords, const uint8_t* __restrict__ mask, int64_t n,
                 const int64_t* __restrict__ block_off, int c_order, int4* __restrict__ out_coords,
@@ -139,33 +139,44 @@ __global__ void __launch_bounds__(kScanThreads)
       int dz, dy, dx;
       child_offsets(s, c_order != 0, dz, dy, dx);
       out_coords[r] = make_int4(c.x, 2 * c.y + dz, 2 * c.z + dy, 2 * c.w + dx);
-      child_src[r] = i * 8 + s;
+      if (mask) child_src[r] = i * 8 + s;  // without a mask, row r's source is r itself
       ++r;
     }
   }
 }
 
-// out_feats[r] = the parent's row (replicate) or its slot's slice; one thread per
-// (child row, piece of `piece_bytes`).
-template <int PIECE>
+// out_feats[r] = the parent's row (replicate) or its slot's slice.  Each thread
+// moves kCopyPieces pieces of PIECE bytes (strided by the grid, so a warp's
+// accesses stay contiguous); without a child list (subdivide) row r's parent
+// is r / 8 and its slot r % 8.
+constexpr int kCopyPieces = 4;
+
+template <int PIECE, bool LIST>
 __global__ void __launch_bounds__(256)
     expand_copy(const uint8_t* __restrict__ feats, const int64_t* __restrict__ child_src,
                 int64_t rows, int64_t in_row_bytes, int64_t out_row_bytes, int slice,
                 uint8_t* __restrict__ out) {
   const int64_t pieces = out_row_bytes / PIECE;
-  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (t >= rows * pieces) return;
-  const int64_t r = t / pieces, p = t % pieces;
-  const int64_t src = child_src[r];
-  const int64_t parent = src >> 3, slot = src & 7;
-  const uint8_t* from = feats + parent * in_row_bytes + (slice ? slot * out_row_bytes : 0) + p * PIECE;
-  uint8_t* to = out + r * out_row_bytes + p * PIECE;
-  if constexpr (PIECE == 16)
-    *reinterpret_cast<uint4*>(to) = *reinterpret_cast<const uint4*>(from);
-  else if constexpr (PIECE == 4)
-    *reinterpret_cast<uint32_t*>(to) = *reinterpret_cast<const uint32_t*>(from);
-  else
-    *reinterpret_cast<uint16_t*>(to) = *reinterpret_cast<const uint16_t*>(from);
+  const int64_t total = rows * pieces;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+#pragma unroll
+  for (int k = 0; k < kCopyPieces; ++k) {
+    const int64_t t = t0 + k * stride;
+    if (t >= total) break;
+    const int64_t r = t / pieces, p = t % pieces;
+    const int64_t src = LIST ? child_src[r] : r;
+    const int64_t parent = src >> 3, slot = src & 7;
+    const uint8_t* from =
+        feats + parent * in_row_bytes + (slice ? slot * out_row_bytes : 0) + p * PIECE;
+    uint8_t* to = out + r * out_row_bytes + p * PIECE;
+    if constexpr (PIECE == 16)
+      *reinterpret_cast<uint4*>(to) = *reinterpret_cast<const uint4*>(from);
+    else if constexpr (PIECE == 4)
+      *reinterpret_cast<uint32_t*>(to) = *reinterpret_cast<const uint32_t*>(from);
+    else
+      *reinterpret_cast<uint16_t*>(to) = *reinterpret_cast<const uint16_t*>(from);
+  }
 }
 
 // ------------------------------------------------------------------ pool ----
@@ -245,43 +256,39 @@ enum : int { kPoolMax = 0, kPoolMean = 1, kPoolS2C = 2 };
 // One warp per parent: lanes 0-7 look up the 8 children in the fine map once
 // and broadcast their rows; the warp then streams the channels.  max / mean:
 // over the children present, in child slot order; spatial2channel: child s's
-// row (or zeros) to channel slot s.  Channels move 8 at a time (16 bytes of
-// bf16, 32 of fp32) when C is a multiple of 8, else one at a time.
+// row (or zeros) to channel slot s.  Channels move 4 at a time (8 bytes of
+// bf16, 16 of fp32: 128 channels fill the warp) when C is a multiple of 4,
+// else one at a time.
 template <typename T>
-__device__ __forceinline__ void load8(const T* p, float (&v)[8]);
+__device__ __forceinline__ void load4(const T* p, float (&v)[4]);
 template <>
-__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[8]) {
-  const uint4 r = *reinterpret_cast<const uint4*>(p);
-  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    v[2 * j] = __uint_as_float(w[j] << 16);
-    v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-  }
+__device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[4]) {
+  const uint2 r = *reinterpret_cast<const uint2*>(p);
+  v[0] = __uint_as_float(r.x << 16);
+  v[1] = __uint_as_float(r.x & 0xFFFF0000u);
+  v[2] = __uint_as_float(r.y << 16);
+  v[3] = __uint_as_float(r.y & 0xFFFF0000u);
 }
 template <>
-__device__ __forceinline__ void load8<float>(const float* p, float (&v)[8]) {
+__device__ __forceinline__ void load4<float>(const float* p, float (&v)[4]) {
   const float4 a = *reinterpret_cast<const float4*>(p);
-  const float4 b = *reinterpret_cast<const float4*>(p + 4);
-  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  v[0] = a.x;
+  v[1] = a.y;
+  v[2] = a.z;
+  v[3] = a.w;
 }
 template <typename T>
-__device__ __forceinline__ void store8(T* p, const float (&v)[8]);
+__device__ __forceinline__ void store4(T* p, const float (&v)[4]);
 template <>
-__device__ __forceinline__ void store8<__nv_bfloat16>(__nv_bfloat16* p, const float (&v)[8]) {
-  uint32_t w[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
-    w[j] = *reinterpret_cast<const uint32_t*>(&h);
-  }
-  *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+__device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* p, const float (&v)[4]) {
+  const __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
+  const __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
+  *reinterpret_cast<uint2*>(p) =
+      make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
 }
 template <>
-__device__ __forceinline__ void store8<float>(float* p, const float (&v)[8]) {
+__device__ __forceinline__ void store4<float>(float* p, const float (&v)[4]) {
   *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
-  *reinterpret_cast<float4*>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
 }
 
 template <Kind K, int MODE, typename T, bool VEC>
@@ -311,10 +318,10 @@ __global__ void __launch_bounds__(256)
     for (int s = 0; s < 8; ++s) {
       const T* src = rows[s] >= 0 ? feats + static_cast<int64_t>(rows[s]) * C : nullptr;
       if constexpr (VEC) {
-        for (int c = lane * 8; c < C; c += 256) {
-          float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-          if (src) load8<T>(src + c, v);
-          store8<T>(o + s * C + c, v);
+        for (int c = lane * 4; c < C; c += 128) {
+          float v[4] = {0.f, 0.f, 0.f, 0.f};
+          if (src) load4<T>(src + c, v);
+          store4<T>(o + s * C + c, v);
         }
       } else {
         for (int c = lane; c < C; c += 32) o[s * C + c] = src ? src[c] : from_f<T>(0.0f);
@@ -325,23 +332,23 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int s = 0; s < 8; ++s) count += rows[s] >= 0 ? 1 : 0;
     if constexpr (VEC) {
-      for (int c = lane * 8; c < C; c += 256) {
-        float acc[8];
+      for (int c = lane * 4; c < C; c += 128) {
+        float acc[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[j] = MODE == kPoolMax ? -INFINITY : 0.0f;
+        for (int j = 0; j < 4; ++j) acc[j] = MODE == kPoolMax ? -INFINITY : 0.0f;
 #pragma unroll
         for (int s = 0; s < 8; ++s) {
           if (rows[s] < 0) continue;
-          float v[8];
-          load8<T>(feats + static_cast<int64_t>(rows[s]) * C + c, v);
+          float v[4];
+          load4<T>(feats + static_cast<int64_t>(rows[s]) * C + c, v);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) acc[j] = MODE == kPoolMax ? fmaxf(acc[j], v[j]) : acc[j] + v[j];
+          for (int j = 0; j < 4; ++j) acc[j] = MODE == kPoolMax ? fmaxf(acc[j], v[j]) : acc[j] + v[j];
         }
         if (MODE == kPoolMean) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) acc[j] = count > 0 ? acc[j] / static_cast<float>(count) : 0.0f;
+          for (int j = 0; j < 4; ++j) acc[j] = count > 0 ? acc[j] / static_cast<float>(count) : 0.0f;
         }
-        store8<T>(out + p * C + c, acc);
+        store4<T>(out + p * C + c, acc);
       }
     } else {
       for (int c = lane; c < C; c += 32) {
@@ -367,8 +374,9 @@ cudaError_t launch_reduce(int mode, const int64_t* parent_cells, int64_t parents
   const unsigned blocks = static_cast<unsigned>((parents * 32 + 255) / 256);
   const auto* f = static_cast<const T*>(feats);
   auto* o = static_cast<T*>(out);
-  const bool vec = C % 8 == 0 && reinterpret_cast<uintptr_t>(feats) % 16 == 0 &&
-                   reinterpret_cast<uintptr_t>(out) % 16 == 0;
+  const size_t align = 4 * sizeof(T);  // one 4-channel piece
+  const bool vec = C % 4 == 0 && reinterpret_cast<uintptr_t>(feats) % align == 0 &&
+                   reinterpret_cast<uintptr_t>(out) % align == 0;
   auto go = [&](auto kernel) {
     kernel<<<blocks, 256, 0, stream>>>(parent_cells, parents, tab, grid, batch, G, f, C, o);
   };
@@ -432,17 +440,20 @@ cudaError_t launch_expand(const int32_t* coords, const void* feats, const uint8_
                   reinterpret_cast<uintptr_t>(feats) % 4 == 0 &&
                   reinterpret_cast<uintptr_t>(out_feats) % 4 == 0;
   const int piece = a16 ? 16 : (a4 ? 4 : 2);
-  const int64_t threads = rows * (out_row_bytes / piece);
-  const unsigned cblocks = static_cast<unsigned>((threads + 255) / 256);
+  const int64_t work = rows * (out_row_bytes / piece);
+  const unsigned cblocks =
+      static_cast<unsigned>((work + 256 * kCopyPieces - 1) / (256 * kCopyPieces));
+  auto go = [&](auto kernel) {
+    kernel<<<cblocks, 256, 0, stream>>>(f, src, rows, in_row_bytes, out_row_bytes, slice ? 1 : 0,
+                                        o);
+  };
+  const bool list = mask != nullptr;
   if (piece == 16)
-    expand_copy<16><<<cblocks, 256, 0, stream>>>(f, src, rows, in_row_bytes, out_row_bytes,
-                                                 slice ? 1 : 0, o);
+    list ? go(expand_copy<16, true>) : go(expand_copy<16, false>);
   else if (piece == 4)
-    expand_copy<4><<<cblocks, 256, 0, stream>>>(f, src, rows, in_row_bytes, out_row_bytes,
-                                                slice ? 1 : 0, o);
+    list ? go(expand_copy<4, true>) : go(expand_copy<4, false>);
   else
-    expand_copy<2><<<cblocks, 256, 0, stream>>>(f, src, rows, in_row_bytes, out_row_bytes,
-                                                slice ? 1 : 0, o);
+    list ? go(expand_copy<2, true>) : go(expand_copy<2, false>);
   return cudaGetLastError();
 }
 

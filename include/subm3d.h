@@ -16,6 +16,15 @@
  * "Unresolved").  The map is built once per coordinate set and reused by
  * every layer on that set, as spconv does with indice_key (same message).
  *
+ * Entry points, in order below: the map build (subm3d_map_workspace_bytes,
+ * subm3d_build_map, subm3d_map_status and accessors, subm3d_build_map_noalloc);
+ * the forward (subm3d_forward on nbr, subm3d_forward_map on a map,
+ * subm3d_forward_fused with a residual-block epilogue); the backward
+ * (subm3d_backward_data, subm3d_backward_weight); the resolution changes
+ * (subm3d_expand: subdivide / upsample / channel2spatial; subm3d_pool:
+ * downsample max / mean, spatial2channel); diagnostics (subm3d_map_run_layout,
+ * subm3d_device_status, subm3d_status_string, subm3d_abi_version).
+ *
  * Conventions for every entry point:
  *   - All buffers are caller-owned.  Pointers marked (device) must point to
  *     memory of the current CUDA device; (host) to host memory.  The library

@@ -13,9 +13,11 @@
 // the contraction runs over positions (MMA K), with the output channels as M
 // and the input channels as N, and both operands are the natural gathered
 // tiles -- rows of positions, channels contiguous -- i.e. MN-major operands.
-// One gathered E tile again serves all three dx: the B descriptor starts d
-// rows into it (the 128-byte swizzle is keyed on address bits, so a view
-// shifted by whole rows of an aligned slot is the same layout).
+// One gathered E tile again serves all three dx, here inside one MMA: the B
+// operand's N dimension holds three 64-channel atoms whose stride (LBO) is one
+// 128-byte row, so atom d is the tile shifted by d rows (the 128-byte swizzle
+// is keyed on address bits, so a view shifted by whole rows of an aligned slot
+// is the same layout).
 //
 // A unit is (tile range, pair, 128 output channels, 128 input channels).  Each
 // CTA takes units in turn; a unit's steps are half tiles (128 positions):
@@ -23,9 +25,11 @@
 //       -1 .. 128 of the half) x 128 channels of x, 16-byte cp.async into two
 //       64-channel 128-byte-swizzle slots each (zero-fill where absent),
 //       completing the stage's barrier with cp.async.mbarrier.arrive.noinc.
-//   warp 12 (MMA)        8 x 3 tcgen05.mma (M=128, N=128, K=16) per step into
-//       three accumulators (384 TMEM columns), one per dx.
-//   warps 0-3 (epilogue) at the end of a unit: tcgen05.ld of the three
+//   warp 12 (MMA)        8 x 2 tcgen05.mma (M=128, N=192, K=16) per step into
+//       two accumulators (384 TMEM columns), one per 64-channel chunk; the
+//       B operand's three 64-channel atoms are set 128 bytes (one row) apart,
+//       so they are the chunk's E rows shifted by dx = -1, 0, +1.
+//   warps 0-3 (epilogue) at the end of a unit: tcgen05.ld of the two
 //       accumulators and red.global.add.v4.f32 into the fp32 dW (zeroed by the
 //       launcher), the unit's partial sum over its tile range.
 // Every wait is bounded (ptx.cuh): a wait that runs out sets the library's
@@ -57,7 +61,8 @@ constexpr int GATHER_WARP0 = 4;
 constexpr int MMA_WARP = GATHER_WARP0 + NUM_GATHER_WARPS;
 constexpr int NUM_THREADS = (MMA_WARP + 1) * 32;
 constexpr int GATHER_THREADS = NUM_GATHER_WARPS * 32;
-constexpr uint32_t kTmemCols = 512;  // three 128-column accumulators
+constexpr uint32_t kAccCols = 192;   // per 64-channel chunk: dx-major, 3 x 64 columns
+constexpr uint32_t kTmemCols = 512;  // two accumulators (the two chunks of a block)
 constexpr size_t kSmemBytes = 1024 + NSTAGE * STAGE + 256;
 static_assert(kSmemBytes <= 227 * 1024, "stages exceed shared memory");
 static_assert(GATHER_THREADS == 16 * 16, "gather mapping: 16 pieces x 16 rows per pass");
@@ -212,7 +217,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) subm3d_wgrad_bf16_runs_sm100(c
   } else if (warp == MMA_WARP) {
     // -------------------------------------------------------------- MMA ----
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32_mn(OB, CB);
+      const uint32_t idesc = idesc_bf16_f32_mn(OB, kAccCols);
       WSteps st;
       st.begin(n_tiles, a.ranges, a.n_ob, a.n_cb);
       bool ok = true;
@@ -235,9 +240,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) subm3d_wgrad_bf16_runs_sm100(c
           for (int kk = 0; kk < HP / 16; ++kk) {
             const uint64_t da = smem_desc_mn_sw128(y_base + kk * 16 * ROW, Y_CHUNK, 1024);
 #pragma unroll
-            for (int d = 0; d < 3; ++d) {
-              const uint64_t db = smem_desc_mn_sw128(e_base + (kk * 16 + d) * ROW, E_CHUNK, 1024);
-              umma_bf16(tmem_base + static_cast<uint32_t>(d * CB), da, db, idesc,
+            for (int j = 0; j < 2; ++j) {
+              // N = 192: three 64-channel atoms ROW bytes apart = E rows shifted by
+              // d = 0, 1, 2, i.e. dx = -1, 0, +1 of the same chunk in one MMA
+              const uint64_t db =
+                  smem_desc_mn_sw128(e_base + j * E_CHUNK + kk * 16 * ROW, ROW, 1024);
+              umma_bf16(tmem_base + static_cast<uint32_t>(j * kAccCols), da, db, idesc,
                         (first && kk == 0) ? 0u : 1u);
             }
           }
@@ -260,23 +268,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) subm3d_wgrad_bf16_runs_sm100(c
       const int o = st.ob * OB + warp * 32 + lane;
       const int c0 = st.cb * CB;
 #pragma unroll 1
-      for (int d = 0; d < 3; ++d) {
-        const int k = 3 * st.pair + d;
-        const int kw = a.flip ? (kKvol - 1 - k) : k;
-        float* dst = a.dw + (static_cast<int64_t>(o) * kKvol + kw) * a.cin + c0;
+      for (int j = 0; j < 2; ++j) {
 #pragma unroll 1
-        for (int cc = 0; cc < CB; cc += 32) {
+        for (int cc = 0; cc < static_cast<int>(kAccCols); cc += 32) {
+          const int d = cc / 64;                  // column = d * 64 + channel in the chunk
+          const int c = c0 + j * 64 + cc % 64;    // first input channel of these 32 columns
+          const int k = 3 * st.pair + d;
+          const int kw = a.flip ? (kKvol - 1 - k) : k;
           uint32_t v[32];
           tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(warp * 32) << 16) +
-                                 static_cast<uint32_t>(d * CB + cc),
+                                 static_cast<uint32_t>(j * kAccCols + cc),
                              v);
           tmem_ld_wait();
-          if (o < a.cout) {
+          if (o < a.cout && c < a.cin) {
+            float* dst = a.dw + (static_cast<int64_t>(o) * kKvol + kw) * a.cin + c;
 #pragma unroll
-            for (int j = 0; j < 32; j += 4)
-              if (c0 + cc + j < a.cin)
-                red_add_v4(dst + cc + j, __uint_as_float(v[j]), __uint_as_float(v[j + 1]),
-                           __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+            for (int t = 0; t < 32; t += 4)
+              red_add_v4(dst + t, __uint_as_float(v[t]), __uint_as_float(v[t + 1]),
+                         __uint_as_float(v[t + 2]), __uint_as_float(v[t + 3]));
           }
         }
       }

@@ -282,6 +282,42 @@ def resample_line(coords, feats, grid, flush, hbm_gbs):
                                 "bound": "hbm", "children": 8 * n}}
 
 
+def decoder_stack_line(flush, peak_tf):
+    """The decoder stack of the batched workload (4 x 256^3 sets, 1.14 M voxels,
+    64 -> 128 -> 128 -> 128 -> 64 channels, exact GELU between layers): one map
+    build and four fused layers on it, timed as one unit."""
+    import torch
+    import sparse_voxel_conv_b200 as S
+    import workloads as WL
+    wl = WL.make_workload("batched")
+    dev = torch.device("cuda")
+    coords = torch.from_numpy(wl.coords).to(dev)
+    x0 = torch.from_numpy(WL.to_bf16_values(wl.features())).to(dev).to(torch.bfloat16)
+    ws = [torch.from_numpy(w).to(dev).to(torch.bfloat16) for w in wl.weights()]
+    n = wl.n
+    outs = [torch.empty((n, w.shape[0]), dtype=torch.bfloat16, device=dev) for w in ws]
+    nbr = torch.empty((n, 27), dtype=torch.int32, device=dev)
+    ws_bytes = S._abi.subm3d_map_workspace_bytes(n, wl.grid_dim, wl.batch)
+    work = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+
+    def run():
+        h = S.build_map(coords, wl.grid_dim, wl.batch, check=False, nbr=nbr, workspace=work)
+        x = x0
+        for li, w in enumerate(ws):
+            x = S.forward(h, x, w, act="gelu" if li < len(ws) - 1 else None, out=outs[li])
+        return x
+
+    run()
+    torch.cuda.synchronize()
+    nnz = int((nbr >= 0).sum().item())
+    ms = _time_ms(run, flush)
+    flops = sum(2.0 * nnz * w.shape[0] * w.shape[-1] for w in ws)  # KRSC: Cout ... Cin
+    tf = flops / (ms / 1e3) / 1e12
+    return {"workload": wl.name, "n_voxels": n, "ms": ms, "voxels_per_s": n / (ms / 1e3),
+            "flops": flops, "achieved": tf, "peak": peak_tf, "unit": "TFLOP/s",
+            "frac": tf / peak_tf, "what": "one map build + 4 fused bf16 layers on it"}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -481,6 +517,7 @@ def run_ours(args):
                                              line["fp32_forward"]["peak"])
             line["resample"] = resample_line(coords, feats, wl.grid_dim, flush,
                                              float(peaks["hbm_gbs"]))
+            line["decoder_stack"] = decoder_stack_line(flush, peak_tf)
             line["context_per_offset_torch"] = per_offset_context(h_ctx, feats, weight, flush)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl, args.cpu_rows)

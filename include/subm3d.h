@@ -89,7 +89,8 @@ SUBM3D_API const char* subm3d_status_string(int32_t status);
  * Workspace bytes subm3d_build_map() needs for N voxels in a batch x
  * grid_dim^3 volume: a status word, one 32-bit offset mask per 128-row tile,
  * and the lookup table -- a direct-address table of batch * grid_dim^3 int32
- * cells when that is at most 64 MB, else an open-addressing hash table of at
+ * cells when that is at most max(64 MB, 256 bytes x N) and 2^28 cells, else an
+ * open-addressing hash table of at
  * least 2N slots (8 bytes each, 12 with batch > 4 or grid_dim > 1024) -- and
  * for N < 2^29 the x-run layout of subm3d_forward_map(): run-start counts (an
  * int32 per 128-row tile and per 128 tiles), a header, a position table of 3N

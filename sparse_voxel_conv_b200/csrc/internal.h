@@ -48,8 +48,14 @@ constexpr int kKvol = 27;
 // The two lookup structures of the map build (see map_build.cu).
 enum class MapKind { kDirect, kHash };
 
-// Largest direct-address table (batch * grid_dim^3 int32 cells) the build uses.
-constexpr size_t kDirectTableMaxBytes = size_t(64) << 20;
+// The direct-address table (batch * grid_dim^3 int32 cells) is used while it
+// takes at most max(kDirectTableMinBytes, kDirectTableBytesPerVoxel * N) bytes
+// and at most kDirectTableMaxCells cells (int32 cell arithmetic in the query):
+// clearing it costs its size in HBM writes, which beats hashing N voxels until
+// the volume is a few hundred bytes per voxel.
+constexpr size_t kDirectTableMinBytes = size_t(64) << 20;
+constexpr double kDirectTableBytesPerVoxel = 256.0;
+constexpr double kDirectTableMaxCells = double(int64_t(1) << 28);
 
 // Testing knobs: force the hash table, or cap its capacity (which implies it).
 struct MapOptions {

@@ -4,8 +4,9 @@
 // (lato.2_mrp_mlx, commit 97dcdfb54a message).  Here the lookup structure is
 // one of two GPU tables over packed (b, z, y, x) keys, chosen per call:
 //
-//   direct  when batch * grid_dim^3 int32 cells fit in 64 MB (every 128^3
-//           volume): cell -> row, -1 when empty.  A collision-free perfect
+//   direct  when batch * grid_dim^3 int32 cells take at most max(64 MB,
+//           256 B x N) and 2^28 cells (every 128^3 volume; 4 x 256^3 from
+//           about a million voxels): cell -> row, -1 when empty.  A collision-free perfect
 //           hash: insert is one plain store per voxel, a lookup is one load,
 //           and voxels adjacent in raster order look up adjacent cells, so the
 //           27 lookups of a warp coalesce.  A duplicate coordinate leaves one
@@ -26,6 +27,8 @@
 // the [128, 27] block and the tile's offset mask are written with coalesced
 // stores; no atomics on the output; and the tile's share of the x-run layout).
 #include <cuda_runtime.h>
+
+#include <algorithm>
 
 #include "internal.h"
 #include "map_table.cuh"
@@ -253,7 +256,7 @@ __global__ void __launch_bounds__(kTileRows)
   if (i < n) {
     if (in_volume(c, grid, batch)) {
       if constexpr (K == Kind::kDirect) {
-        // the direct table has < 2^24 cells: int32 cell indices.  The 9 (dz, dy)
+        // the direct table has <= 2^28 cells: int32 cell indices.  The 9 (dz, dy)
         // rows are base pointers; dx = -1, 0, +1 are the cells before and after.
         const int32_t g = grid, g2 = grid * grid;
         const int32_t* centre = t.cells + (((c.x * g + c.y) * g + c.z) * g + c.w);
@@ -372,7 +375,9 @@ bool map_layout(int64_t n, int32_t grid_dim, int32_t batch, const MapOptions& op
     return false;
   MapLayout lay;
   const double cells = static_cast<double>(batch) * grid_dim * grid_dim * grid_dim;
-  const bool direct_fits = cells * 4.0 <= static_cast<double>(kDirectTableMaxBytes);
+  const double direct_budget = std::max(static_cast<double>(kDirectTableMinBytes),
+                                        kDirectTableBytesPerVoxel * static_cast<double>(n));
+  const bool direct_fits = cells * 4.0 <= direct_budget && cells <= kDirectTableMaxCells;
   lay.kind = (direct_fits && !opt.force_hash && opt.forced_capacity == 0) ? MapKind::kDirect
                                                                          : MapKind::kHash;
   lay.compact = (batch <= 4 && grid_dim <= 1024);

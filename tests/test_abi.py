@@ -65,9 +65,12 @@ def test_workspace_bytes(abi, monkeypatch):
     assert f(-1, 16, 1) == 0 and f(10, 0, 1) == 0 and f(10, 16, 0) == 0
     assert f(10, 70000, 1) == 0 and f(10, 16, 70000) == 0
     n = 329839
-    # direct table: one int32 per cell of a volume up to 64 MB
+    # direct table: one int32 per cell of a volume up to max(64 MB, 256 B x N)
     assert f(n, 128, 1) == _expected_ws(n, 4 * 128 ** 3)
     assert f(n, 256, 1) == _expected_ws(n, 4 * 256 ** 3)
+    big = 1_135_307                                  # 4 x 256^3 = 268 MB <= 256 B x N
+    assert f(big, 256, 4) == _expected_ws(big, 4 * 4 * 256 ** 3)
+    assert f(n, 256, 4) != _expected_ws(n, 4 * 4 * 256 ** 3)   # 268 MB > 84 MB: hash
     # larger volumes: hash table, 8-byte slots, capacity max(1024, pow2 >= 2N)
     assert f(n, 512, 1) == _expected_ws(n, 8 * (1 << 20))
     # wide keys (batch > 4 or grid > 1024) add a 4-byte row array

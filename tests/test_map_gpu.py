@@ -22,7 +22,7 @@ def S():
 
 @pytest.fixture(params=["auto", "hash"])
 def kind(request, monkeypatch):
-    """auto: the direct table where the volume fits in 64 MB, else the hash
+    """auto: the direct table where the volume fits max(64 MB, 256 B x N), else the hash
     table; hash: the hash table everywhere (testing knob SUBM3D_MAP_KIND)."""
     if request.param == "hash":
         monkeypatch.setenv("SUBM3D_MAP_KIND", "hash")

@@ -51,18 +51,19 @@ __device__ __forceinline__ uint4 finish_bf16x8(const float (&f)[8], bool has_res
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// Bytes of fp32 staging one bf16 epilogue warp needs: 32 positions x 32 channels.
-constexpr int kEpiWarpStageBytes = 32 * 32 * 4;
+// Bytes of fp32 staging one bf16 epilogue warp needs: 16 positions x 32 channels
+// (a 32-position chunk is staged in two halves).
+constexpr int kEpiWarpStageBytes = 16 * 32 * 4;
 
 // The epilogue of one 256-position accumulator by one warp: its 32 channels
 // (TMEM lanes; lane = channel o_warp + lane) in 8 chunks of 32 positions.  Per
-// chunk the fp32 values (bias, activation) go to the warp's staging area
-// (`stage`, kEpiWarpStageBytes; a position's 128-byte row has its 16-byte halves
-// swapped at odd positions, so the reads below are free of bank conflicts),
-// then each lane takes 8 channels of one position, adds the residual and
-// stores 16 bytes.  The output row of position j is pos[j] >> 2 when pos[j] is
-// a voxel entry (POS: the x-run layout; pads and empty positions are dropped),
-// else row0 + j below n.  Latency is hidden by prefetching: position entries
+// chunk, in two halves of 16 positions, the fp32 values (bias, activation) go to
+// the warp's staging area (`stage`, kEpiWarpStageBytes; a position's 128-byte
+// row has its 16-byte halves swapped at odd positions, so the reads below are
+// free of bank conflicts), then each lane takes 8 channels of one position,
+// adds the residual and stores 16 bytes.  The output row of position j is
+// pos[j] >> 2 when pos[j] is a voxel entry (POS: the x-run layout; pads and
+// empty positions are dropped), else row0 + j below n.  Latency is hidden by prefetching: position entries
 // two chunks ahead and each chunk's residual rows one chunk ahead, so they load
 // while the previous chunk is staged.  The chunk loop stays rolled: an
 // unrolled one inlines 256 activations and slows every warp of the kernel.
@@ -117,27 +118,30 @@ __device__ __forceinline__ void epilogue_tile_bf16(uint32_t taddr, float bias_v,
     }
     tmem_ld_wait();
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const float f = activate<ACT>(__uint_as_float(v[e]) + bias_v);
-      sts_u32(stage + e * 128 + ((lane * 4) ^ ((e & 1) << 4)), __float_as_uint(f));
-    }
-    __syncwarp();
+    for (int h = 0; h < 2; ++h) {  // positions 16h .. 16h+15 of the chunk: store slots 2h, 2h+1
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      const int j = p * 8 + lane / 4;
-      const uint32_t rb = stage + j * 128;
-      const uint32_t sw = static_cast<uint32_t>(j & 1) << 4;
-      const uint4 lo = lds_16(rb + ((q * 32) ^ sw));
-      const uint4 hi = lds_16(rb + ((q * 32 + 16) ^ sw));
-      if (rows[p] >= 0 && o_ok) {
-        const float f[8] = {__uint_as_float(lo.x), __uint_as_float(lo.y), __uint_as_float(lo.z),
-                            __uint_as_float(lo.w), __uint_as_float(hi.x), __uint_as_float(hi.y),
-                            __uint_as_float(hi.z), __uint_as_float(hi.w)};
-        *reinterpret_cast<uint4*>(out + static_cast<int64_t>(rows[p]) * cout + o) =
-            finish_bf16x8(f, residual != nullptr, res[p]);
+      for (int e = 0; e < 16; ++e) {
+        const float f = activate<ACT>(__uint_as_float(v[16 * h + e]) + bias_v);
+        sts_u32(stage + e * 128 + ((lane * 4) ^ ((e & 1) << 4)), __float_as_uint(f));
       }
+      __syncwarp();
+#pragma unroll
+      for (int p = 2 * h; p < 2 * h + 2; ++p) {
+        const int j = (p - 2 * h) * 8 + lane / 4;  // staging row (same parity as the position)
+        const uint32_t rb = stage + j * 128;
+        const uint32_t sw = static_cast<uint32_t>(j & 1) << 4;
+        const uint4 lo = lds_16(rb + ((q * 32) ^ sw));
+        const uint4 hi = lds_16(rb + ((q * 32 + 16) ^ sw));
+        if (rows[p] >= 0 && o_ok) {
+          const float f[8] = {__uint_as_float(lo.x), __uint_as_float(lo.y), __uint_as_float(lo.z),
+                              __uint_as_float(lo.w), __uint_as_float(hi.x), __uint_as_float(hi.y),
+                              __uint_as_float(hi.z), __uint_as_float(hi.w)};
+          *reinterpret_cast<uint4*>(out + static_cast<int64_t>(rows[p]) * cout + o) =
+              finish_bf16x8(f, residual != nullptr, res[p]);
+        }
+      }
+      __syncwarp();
     }
-    __syncwarp();
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
       rows[p] = rows_n[p];

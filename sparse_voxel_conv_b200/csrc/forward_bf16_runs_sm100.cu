@@ -24,13 +24,15 @@
 // Persistent kernel, one CTA per SM; a work unit is a position tile x a block
 // of 128 output channels.  Roles (14 warps):
 //
-//   warp 13 (TMA)   per E step (chunk j, pair dz-dy): bulk-copies the tile's E
-//       index list (258 rows) into the index slot of the E ring, and loads the
-//       three weight slices Wf[o0:o0+128, k, chunk j], dx = -1, 0, +1, into the
-//       W ring with 3-D TMA tiled loads (128-byte swizzle).
-//   warps 4-11      gather E: 258 rows x 128 bytes with 16-byte cp.async into
-//       the 128-byte-swizzle layout (zero-fill for absent rows), completing the
-//       E slot's barrier with cp.async.mbarrier.arrive.noinc.
+//   warp 13 (TMA)   per E step (chunk j, pair dz-dy): loads the three weight
+//       slices Wf[o0:o0+128, k, chunk j], dx = -1, 0, +1, into the W ring with
+//       3-D TMA tiled loads (128-byte swizzle).
+//   warps 4-11      gather E: once the E slot is free, 258 rows x 128 bytes with
+//       16-byte cp.async into the 128-byte-swizzle layout (zero-fill for absent
+//       rows), completing the slot's barrier with cp.async.mbarrier.arrive.noinc.
+//       Each thread reads the E index entries of its rows straight from global
+//       memory into registers one step ahead, so a freed slot waits for one
+//       memory round trip (the rows), not two (the index list, then the rows).
 //   warp 12 (MMA)   per E step, for dx = -1, 0, +1: 4 x tcgen05.mma (M=128,
 //       N=256, K=16) with the B descriptor started dx rows into the E slot.
 //       The 128-byte swizzle XORs with address bits [7,10) of each row's own
@@ -70,7 +72,6 @@ constexpr int GATHER_THREADS = NUM_GATHER_WARPS * 32;
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kERows = TP + 2;                                   // rows -1 .. 256
 constexpr uint32_t E_SLOT = ((kERows * ROW_BYTES + 1023) / 1024) * 1024;  // 33792
-constexpr uint32_t IDX_BYTES = kEtStride * 4;                  // 1040
 constexpr uint32_t A_SLOT = TO * ROW_BYTES;                      // 16384
 constexpr int kEpiStageBytes = NUM_EPI_WARPS * kEpiWarpStageBytes;
 constexpr uint32_t kTmemCols = 2 * TP;
@@ -88,19 +89,18 @@ struct RunArgs {
 };
 
 struct SmemPlan {
-  size_t e_off, idx_off, w_off, epi_off, bar_off, bytes;
+  size_t e_off, w_off, epi_off, bar_off, bytes;
 };
 
 __host__ __device__ inline SmemPlan plan_smem(int se, int sw) {
   SmemPlan p;
   p.e_off = 0;
   p.w_off = p.e_off + static_cast<size_t>(se) * E_SLOT;
-  p.idx_off = p.w_off + static_cast<size_t>(sw) * A_SLOT;
-  p.epi_off = p.idx_off + ((static_cast<size_t>(se) * IDX_BYTES + 127) / 128) * 128;
+  p.epi_off = p.w_off + static_cast<size_t>(sw) * A_SLOT;
   p.bar_off = p.epi_off + kEpiStageBytes;
-  // e_full[se], e_empty[se], idx_full[se], w_full[sw], w_empty[sw], acc_full[2],
-  // acc_empty[2], tmem slot, abort
-  p.bytes = p.bar_off + (3 * se + 2 * sw + 4) * 8 + 16 + 1024;
+  // e_full[se], e_empty[se], w_full[sw], w_empty[sw], acc_full[2], acc_empty[2],
+  // tmem slot, abort
+  p.bytes = p.bar_off + (2 * se + 2 * sw + 4) * 8 + 16 + 1024;
   return p;
 }
 
@@ -165,12 +165,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const SmemPlan plan = plan_smem(SE, SW);
   uint8_t* e_ring = base + plan.e_off;
   uint8_t* w_ring = base + plan.w_off;
-  int32_t* idx_ring = reinterpret_cast<int32_t*>(base + plan.idx_off);
   uint8_t* epi_s = base + plan.epi_off;
   uint64_t* e_full = reinterpret_cast<uint64_t*>(base + plan.bar_off);
   uint64_t* e_empty = e_full + SE;
-  uint64_t* idx_full = e_empty + SE;
-  uint64_t* w_full = idx_full + SE;
+  uint64_t* w_full = e_empty + SE;
   uint64_t* w_empty = w_full + SW;
   uint64_t* acc_full = w_empty + SW;
   uint64_t* acc_empty = acc_full + 2;
@@ -183,7 +181,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int s = 0; s < SE; ++s) {
       mbar_init(&e_full[s], GATHER_THREADS);  // every gather thread's cp.async arrive
       mbar_init(&e_empty[s], 1);              // one tcgen05.commit
-      mbar_init(&idx_full[s], 1);             // TMA thread's arrive.expect_tx
     }
     for (int s = 0; s < SW; ++s) {
       mbar_init(&w_full[s], 1);
@@ -221,24 +218,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int i = q < PPT ? rbase + q * ROWS_PER_PASS : TP + rbase;  // E index row 0..257
       dst_off[q] = i * ROW_BYTES + ((piece ^ (i & 7)) << 4);
     }
+    // the E index entries of this thread's rows for the step `t` points at
+    auto load_src = [&](const ESteps& t, int32_t (&v)[PPT + 1]) {
+      const int32_t* list = a.et + ((t.u / a.n_oblocks) * 9 + t.dzdy) * kEtStride;
+#pragma unroll
+      for (int q = 0; q <= PPT; ++q) {
+        const int i = q < PPT ? rbase + q * ROWS_PER_PASS : TP + rbase;
+        v[q] = (q < PPT || edge) ? __ldg(list + i) : -1;
+      }
+    };
     ESteps st;
     st.begin(n_units);
+    int32_t src[PPT + 1];
+    if (st.valid) load_src(st, src);
     while (st.valid) {
       const int s = st.slot;
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&idx_full[s], st.phase, abort_flag))) break;
-      const int32_t* idx = idx_ring + s * kEtStride;
+      // the E slot is free once the MMAs that read it are done
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&e_empty[s], st.phase ^ 1u, abort_flag))) break;
       const __nv_bfloat16* xcol = a.x + st.j * CHUNK + piece * 8;
       const uint32_t e_base = smem_u32(e_ring) + static_cast<uint32_t>(s) * E_SLOT;
 #pragma unroll
       for (int q = 0; q <= PPT; ++q) {
         if (q == PPT && !edge) break;
-        const int i = q < PPT ? rbase + q * ROWS_PER_PASS : TP + rbase;
-        const int32_t src = idx[i];
         cp_async_16(e_base + dst_off[q],
-                    src >= 0 ? xcol + static_cast<int64_t>(src) * a.cin : a.x, src >= 0 ? 16u : 0u);
+                    src[q] >= 0 ? xcol + static_cast<int64_t>(src[q]) * a.cin : a.x,
+                    src[q] >= 0 ? 16u : 0u);
       }
       cp_async_mbar_arrive_noinc(&e_full[s]);
       st.next(a.n_kchunks, SE);
+      if (st.valid) load_src(st, src);  // the next step's entries load while this slot fills
     }
     cp_async_wait_all();
   } else if (warp == TMA_WARP) {
@@ -248,16 +256,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     Ring w;
     bool ok = true;
     while (ok && st.valid) {
-      const int s = st.slot;
-      // the E slot (and its index slot) is free once the MMAs that read it are done
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&e_empty[s], st.phase ^ 1u, abort_flag))) break;
-      const int64_t tile = st.u / a.n_oblocks;
       const int o0 = static_cast<int>(st.u % a.n_oblocks) * TO;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&idx_full[s], IDX_BYTES);
-        bulk_load(smem_u32(idx_ring + s * kEtStride), a.et + (tile * 9 + st.dzdy) * kEtStride,
-                  IDX_BYTES, &idx_full[s]);
-      }
       for (int dx = 0; dx < 3; ++dx) {
         if (!__all_sync(0xFFFFFFFFu, mbar_wait(&w_empty[w.slot], w.phase ^ 1u, abort_flag))) {
           ok = false;
@@ -416,7 +415,7 @@ cudaError_t launch_forward_bf16_runs(const int32_t* pos, const int32_t* etable,
   int num_sms = 0;
   if ((e = device_setup(device, &num_sms)) != cudaSuccess) return e;
 
-  int se = 3, sw = 6;
+  int se = 3, sw = 7;
   while (sw > 3 && plan_smem(se, sw).bytes > static_cast<size_t>(kSmemLimit)) --sw;
   const SmemPlan plan = plan_smem(se, sw);
 

@@ -14,10 +14,28 @@
 
 namespace subm3d {
 
+// GELU in its erf form, v * Phi(v) with Phi(v) = erfc(-v / sqrt(2)) / 2, and
+// erfc by the rational-times-Gaussian approximation of Abramowitz & Stegun,
+// Handbook of Mathematical Functions, eq. 7.1.26 (after Hastings): for u >= 0,
+//   erfc(u) ~= t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-u^2),  t = 1 / (1 + p u),
+// absolute error <= 1.5e-7.  Computing erfc(|v| / sqrt 2) directly keeps the
+// negative tail free of cancellation (Phi(v) = erfc / 2 there, 1 - erfc / 2 for
+// v >= 0), and the form has no branch.
+__device__ __forceinline__ float gelu_erf(float v) {
+  constexpr float p = 0.3275911f;
+  constexpr float a1 = 0.254829592f, a2 = -0.284496736f, a3 = 1.421413741f,
+                  a4 = -1.453152027f, a5 = 1.061405429f;
+  const float u = fabsf(v) * 0.70710678118654752f;
+  const float t = __fdividef(1.0f, fmaf(p, u, 1.0f));
+  const float poly = t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, a5, a4), a3), a2), a1);
+  const float ec = poly * __expf(-u * u);  // erfc(|v| / sqrt 2)
+  return v * (v >= 0.0f ? fmaf(-0.5f, ec, 1.0f) : 0.5f * ec);
+}
+
 template <int ACT>
 __device__ __forceinline__ float activate(float v) {
   if constexpr (ACT == kActGelu) {
-    return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f));  // exact erf form
+    return gelu_erf(v);
   } else if constexpr (ACT == kActSilu) {
     // v * sigmoid(v) with the fast exponential and the fast divide (a few ulp,
     // well inside both paths' bars); for v -> -inf the divisor overflows to inf

@@ -545,18 +545,25 @@ def _oracle_step(wl, x, w, rows):
     return t1 - t0, t2 - t1
 
 
-def cpu_baseline(wl, n_rows):
+def cpu_baseline(wl, n_rows, reps=2):
     """The oracle as it stands on the host cores: map build of the full set plus
-    the forward of a sample of rows; voxels/s = 1 / (map_s / N + fwd_s / rows)."""
+    the fp64 forward of `n_rows` evenly spaced rows (all rows when n_rows <= 0),
+    `reps` times; voxels/s = 1 / mean(map_s / N + fwd_s / rows)."""
     from oracle import cpp as C
-    rows = np.linspace(0, wl.n - 1, min(n_rows, wl.n)).astype(np.int64)
+    n_rows = wl.n if n_rows <= 0 else min(n_rows, wl.n)
+    rows = np.linspace(0, wl.n - 1, n_rows).astype(np.int64)
     x, w = _oracle_inputs(wl)
-    map_s, fwd_s = _oracle_step(wl, x, w, rows)
-    per_voxel = map_s / wl.n + fwd_s / rows.size
-    return {"value": 1.0 / per_voxel, "unit": "voxels/s", "cores": C.num_threads(),
-            "kind": "oracle",
-            "sample": f"map build of all {wl.n} voxels ({map_s:.2f} s) + fp64 forward of "
-                      f"{rows.size} evenly spaced rows ({fwd_s:.2f} s)"}
+    per_voxel, map_t, fwd_t = [], [], []
+    for _ in range(reps):
+        map_s, fwd_s = _oracle_step(wl, x, w, rows)
+        map_t.append(map_s)
+        fwd_t.append(fwd_s)
+        per_voxel.append(map_s / wl.n + fwd_s / rows.size)
+    what = ("all rows" if rows.size == wl.n else f"{rows.size} evenly spaced rows")
+    return {"value": 1.0 / statistics.mean(per_voxel), "unit": "voxels/s",
+            "cores": C.num_threads(), "kind": "oracle",
+            "sample": f"{reps} x (map build of all {wl.n} voxels, {statistics.mean(map_t):.2f} s "
+                      f"+ fp64 forward of {what}, {statistics.mean(fwd_t):.2f} s)"}
 
 
 def run_reference(args):
@@ -566,7 +573,8 @@ def run_reference(args):
     from oracle import cpp as C
     wl = _workload(args.workload)
     # rows per step shrink with K so that the whole run stays within minutes
-    n_rows = max(256, min(args.cpu_rows, 2_000_000 // max(1, args.steps), wl.n))
+    cap = wl.n if args.cpu_rows <= 0 else args.cpu_rows
+    n_rows = max(256, min(cap, 2_000_000 // max(1, args.steps), wl.n))
     rows = np.linspace(0, wl.n - 1, n_rows).astype(np.int64)
     x, w = _oracle_inputs(wl)
     for _ in range(min(args.warmup, 3)):
@@ -605,7 +613,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="headline", choices=["headline", "dense", "shell_bf16"])
-    ap.add_argument("--cpu-rows", type=int, default=40000)
+    ap.add_argument("--cpu-rows", type=int, default=0,
+                    help="rows of the cpu_baseline forward (0: all rows of the workload)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-context", action="store_true",
                     help="skip the fp32-path and per-offset-loop context measurements")

@@ -128,6 +128,32 @@ def test_bf16_edge_sets(S):
     assert_close(y, C.round_bf16(centre), RTOL_BF16, "isolated")
 
 
+@pytest.mark.parametrize("flip", [False, True])
+def test_bf16_runs_edge_layouts(S, flip):
+    """The x-run kernel (Cin % 64 == 0) on the layouts whose edges matter: one
+    voxel; isolated voxels (every voxel its own run); 129 voxels of a dense
+    block; runs of 255 and 511 voxels along x (the last right pad lands on or
+    past a 256-position tile boundary, read through the next tile's edge rows);
+    random sets in 8^3."""
+    rng = np.random.default_rng(23)
+    lattice = np.array([(0, z, y, x) for z in range(0, 16, 2) for y in range(0, 16, 2)
+                        for x in range(0, 16, 2)], np.int32)
+    sets = [(np.array([[0, 7, 7, 7]], np.int32), 16), (lattice, 16),
+            (WL.dense_coords(6)[:129], 16)]
+    for length in (255, 511):
+        sets.append((np.array([[0, 3, 5, x] for x in range(length)] +
+                              [[0, 4, 5, x] for x in range(0, length, 3)], np.int32), 512))
+    for n in (2, 300):
+        cells = np.sort(rng.choice(8 ** 3, n, replace=False))
+        zyx = np.stack(np.unravel_index(cells, (8, 8, 8)), 1)
+        sets.append((np.concatenate([np.zeros((n, 1), np.int64), zyx], 1).astype(np.int32), 8))
+    for c, grid in sets:
+        x, w = _inputs(c, 64, 48, "bf16", seed=len(c))
+        _, y = _run(S, c, grid, 1, x, w, "bf16", flip=flip)
+        ref = _oracle(c, grid, 1, x, w, flip=flip, bf16_out=True)
+        assert_close(y, ref, RTOL_BF16, f"x-run n={len(c)} flip={flip}")
+
+
 def test_bf16_empty(S):
     c = np.zeros((0, 4), np.int32)
     h = S.build_map(torch.from_numpy(c).cuda(), 8, 1)

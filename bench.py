@@ -78,6 +78,12 @@ def _profiled_traffic(workload: str):
     return int(traffic.group(1))
 
 
+def _workload_config(wl, nnz_avg):
+    """The workload keys of `config`, the same in both arms."""
+    return {"workload": wl.name, "n_voxels": wl.n, "nnz_avg": nnz_avg, "cin": wl.channels[0],
+            "cout": wl.channels[1], "grid_dim": wl.grid_dim, "batch": wl.batch}
+
+
 def _workload(name):
     import workloads as WL
     return WL.make_workload(name)
@@ -478,8 +484,7 @@ def run_ours(args):
             "dtype": "bf16",
             "data": "synthetic",
             "config": {
-                "workload": wl.name, "n_voxels": n, "nnz_avg": nnz_total / n, "cin": cin,
-                "cout": cout, "grid_dim": wl.grid_dim, "batch": wl.batch,
+                **_workload_config(wl, nnz_total / n),
                 "step": f"map build ({MAP_LAUNCHES} kernels) + bf16 x-run forward (1 kernel)",
                 "l2": f"flushed before every timed step ({L2_FLUSH_BYTES >> 20} MB write)",
                 "parallelism": f"replicas x{world}, no collective on the data path",
@@ -577,6 +582,7 @@ def run_reference(args):
     n_rows = max(256, min(cap, 2_000_000 // max(1, args.steps), wl.n))
     rows = np.linspace(0, wl.n - 1, n_rows).astype(np.int64)
     x, w = _oracle_inputs(wl)
+    nnz_avg = float((C.build_map(wl.coords, wl.grid_dim, wl.batch) >= 0).sum()) / wl.n
     for _ in range(min(args.warmup, 3)):
         _oracle_step(wl, x, w, rows[:256])
     per_voxel = []
@@ -593,8 +599,9 @@ def run_reference(args):
         "warmup": args.warmup, "ms_per_step": sec_per_voxel * wl.n * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": wl.name, "n_voxels": wl.n, "cin": wl.channels[0],
-                   "cout": wl.channels[1], "parallelism": "host cores (OpenMP)"},
+        "config": {**_workload_config(wl, nnz_avg),
+                   "step": "map build + fp64 forward (C++ oracle)",
+                   "parallelism": "host cores (OpenMP)"},
         "cpu_baseline": {"value": value, "unit": "voxels/s", "cores": C.num_threads(),
                          "kind": "oracle",
                          "sample": f"per step: map build of all {wl.n} voxels + fp64 forward "

@@ -54,3 +54,49 @@ def test_single_process_is_identity():
     import bench
     assert bench.max_over_ranks(3.5, "cpu") == 3.5
     assert bench.job_rate(10, 1, 2.0) == 5.0
+
+
+def _run_bench(args, env_extra=None):
+    import json
+    import subprocess
+    import sys
+    env = dict(os.environ, **(env_extra or {}))
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], cwd=ROOT,
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [l for l in p.stdout.splitlines() if l.startswith("{")]
+    return [json.loads(l) for l in lines]
+
+
+def test_reference_arm_line():
+    """`bench.py --impl reference` (the C++ oracle on the host cores) prints one
+    JSON line with the contract's keys, the same metric and workload keys as the
+    GPU arm, a cpu_baseline describing the run and an e2e with no copies."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    lines = _run_bench(["--impl", "reference", "--workload", "shell_bf16", "--steps", "2",
+                        "--warmup", "1"])
+    assert len(lines) == 1
+    d = lines[0]
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC
+    assert d["unit"] == "voxels/s" and d["higher_is_better"] is True
+    assert d["steps"] == 2 and d["warmup"] == 1 and d["value"] > 0
+    wl = bench._workload("shell_bf16")
+    cfg = d["config"]
+    for key in ("workload", "n_voxels", "cin", "cout", "grid_dim", "batch"):
+        assert cfg[key] == bench._workload_config(wl, 0.0)[key], key
+    assert 1.0 <= cfg["nnz_avg"] <= 27.0
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_exit_without_work():
+    assert _run_bench(["--impl", "reference", "--workload", "shell_bf16", "--steps", "1",
+                       "--warmup", "1"], {"RANK": "1", "WORLD_SIZE": "2"}) == []

@@ -170,9 +170,10 @@ SUBM3D_API void subm3d_map_destroy(subm3d_map* map);
  *   dtype      SUBM3D_BF16: bf16 feats/weight/out, fp32 accumulation on the tensor
  *              cores, Cin and Cout multiples of 16 (else SUBM3D_E_UNSUPPORTED).
  *              SUBM3D_F32: fp32 throughout on CUDA-core FMA, any Cin, Cout >= 1.
- *   act        SUBM3D_ACT_NONE, SUBM3D_ACT_GELU (exact erf form) or SUBM3D_ACT_SILU
- *              (v * sigmoid(v)) on the fp32 sum; a bf16 output is rounded once,
- *              after the activation.
+ *   act        SUBM3D_ACT_NONE, SUBM3D_ACT_GELU (erf form, v * Phi(v); erfc from
+ *              Abramowitz & Stegun 7.1.26, absolute error <= 1.5e-7) or
+ *              SUBM3D_ACT_SILU (v * sigmoid(v)) on the fp32 sum; a bf16 output is
+ *              rounded once, after the activation.
  *
  * The forward never fails on data.  SUBM3D_E_UNSUPPORTED is also returned when
  * the current device is not sm_100.  A bounded device-side wait that runs out

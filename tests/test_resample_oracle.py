@@ -101,3 +101,29 @@ def test_downsample_against_numpy_unique_and_reductions():
 def test_downsample_rejects_unknown_mode():
     with pytest.raises(ValueError):
         R.downsample(np.zeros((1, 4), np.int32), np.zeros((1, 1)), "sum")
+
+
+def test_batches_never_share_a_parent():
+    # the same spatial child in two batch elements: two parents, one per element
+    c = np.array([[0, 2, 3, 4], [1, 2, 3, 4], [1, 3, 3, 5]], np.int32)
+    f = np.array([[1.0], [5.0], [7.0]])
+    pc, pmax = R.downsample(c, f, "max")
+    assert [tuple(r) for r in pc] == [(0, 1, 1, 2), (1, 1, 1, 2)]
+    assert np.array_equal(pmax, [[1.0], [7.0]])
+    _, pmean = R.downsample(c, f, "mean")
+    assert np.array_equal(pmean, [[1.0], [6.0]])
+    _, s2c = R.spatial2channel(c, f)
+    # child (2,3,4) sits in slot 0 + 2*1 + 4*0 = 2; child (3,3,5) in 1 + 2 + 4 = 7
+    assert s2c[0, 2] == 1.0 and s2c[1, 2] == 5.0 and s2c[1, 7] == 7.0
+    assert np.count_nonzero(s2c) == 3
+
+
+def test_empty_and_all_zero_mask():
+    c = np.zeros((0, 4), np.int32)
+    oc, of = R.subdivide(c, np.zeros((0, 3)))
+    assert oc.shape == (0, 4) and of.shape == (0, 3)
+    c = np.array([[0, 1, 2, 3], [0, 4, 4, 4]], np.int32)
+    oc, of = R.upsample(c, np.ones((2, 3)), np.zeros((2, 8), np.uint8))
+    assert oc.shape[0] == 0 and of.shape == (0, 3)
+    oc, of = R.channel2spatial(c, np.ones((2, 16)), np.zeros((2, 8), np.uint8))
+    assert oc.shape[0] == 0 and of.shape == (0, 2)

@@ -1,22 +1,29 @@
 """Benchmark of the SubMConv3d hot path on B200: neighbour-map build + bf16 forward.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload headline|dense|shell_bf16]
+                    [--workload headline|dense|shell_bf16|batched]
 
 One step = one pass of the whole hot path over one synthetic input: the
-neighbour-map build (hash-table init, insert, 27-probe query + tile masks) and
-the bf16 tcgen05 forward, for the headline workload (128^3 grid, 8 sphere
-shells, 329,839 voxels, 128 -> 128 channels).  Inputs are resident in HBM
-when the timed region starts; the L2 is flushed (256 MB write) before every
-timed step; each step is timed with CUDA events on the launching stream.
+neighbour-map build (table init, insert, 27-lookup query + tile masks + x-run
+layout) and the bf16 tcgen05 forward, for the headline workload (128^3 grid,
+8 sphere shells, 329,839 voxels, 128 -> 128 channels) by default; with
+--workload batched, the decoder stack (4 x 256^3 shell sets, 1,135,307
+voxels, one map build + 64 -> 128 -> 128 -> 128 -> 64 with exact GELU
+between).  Inputs are resident in HBM when the timed region starts; the L2 is
+flushed (256 MB write) before every timed step; each step is timed with CUDA
+events on the launching stream.
 
-With N > 1 (torchrun, one process per GPU) every rank runs its own replica on
-its own features (weak scaling, no collective on the data path); the job time
-is the max over ranks and `value` counts the voxels of all ranks.
+With N > 1 (torchrun, one process per GPU) there is no collective on the data
+path.  headline / dense / shell_bf16: every rank runs its own replica on its
+own features (weak scaling; `value` counts the voxels of all ranks).
+batched: rank r takes batch elements r, r + N, ... of the one batch, the
+weights replicated (strong scaling; `value` counts the batch's voxels).  The
+job time is the max over ranks.
 
---impl reference times the CPU oracle (oracle/, C++ std::map + fp64 loop) on
-the host cores, on bounded samples of the same workload, and prints the same
-line with "impl": "reference".
+--impl reference times the CPU oracle (oracle/, C++ std::map + fp64 loops) on
+the host cores, every step on the same bounded sample of the workload (a
+raster-order prefix sized to the time budget), and prints the same line with
+"impl": "reference".
 """
 from __future__ import annotations
 
@@ -81,7 +88,8 @@ def _profiled_traffic(workload: str):
 def _workload_config(wl, nnz_avg):
     """The workload keys of `config`, the same in both arms."""
     return {"workload": wl.name, "n_voxels": wl.n, "nnz_avg": nnz_avg, "cin": wl.channels[0],
-            "cout": wl.channels[1], "grid_dim": wl.grid_dim, "batch": wl.batch}
+            "cout": wl.channels[1], "channels": list(wl.channels), "grid_dim": wl.grid_dim,
+            "batch": wl.batch}
 
 
 def _workload(name):
@@ -324,6 +332,76 @@ def decoder_stack_line(flush, peak_tf):
             "frac": tf / peak_tf, "what": "one map build + 4 fused bf16 layers on it"}
 
 
+def batch_elements(rank: int, world: int, batch: int) -> list:
+    """Batch elements a rank takes when a batch is split over `world` ranks:
+    rank, rank + world, rank + 2 world, ... (none when rank >= batch)."""
+    return list(range(rank, batch, world))
+
+
+def split_batch(coords: np.ndarray, elems) -> np.ndarray:
+    """The rows of the given batch elements, in that order, their batch index
+    renumbered 0, 1, ...: batch elements never share a neighbour, so each rank
+    builds the map of its own elements alone."""
+    parts = []
+    for new_b, b in enumerate(elems):
+        c = coords[coords[:, 0] == b].copy()
+        c[:, 0] = new_b
+        parts.append(c)
+    return np.concatenate(parts) if parts else np.zeros((0, 4), np.int32)
+
+
+class Job:
+    """What one rank runs per step: its coordinate rows, features and layers.
+
+    headline / dense / shell_bf16: every rank runs a replica of the whole set on
+    its own features (weak scaling).  batched: the decoder-stack workload's
+    batch elements are split over the ranks (batch_elements), W replicated,
+    total work fixed (strong scaling); ranks past the batch size idle.  No
+    collective on the data path either way."""
+
+    def __init__(self, name: str, rank: int, world: int):
+        import workloads as WL
+        wl = WL.make_workload(name)
+        self.wl = wl
+        self.name = name
+        if name == "batched":
+            self.elems = batch_elements(rank, world, wl.batch)
+            self.coords = split_batch(wl.coords, self.elems)
+            self.batch = max(1, len(self.elems))
+            self.units_job = wl.n
+            self.scaling = "strong"
+            self.parallelism = (f"batch split x{world}: rank r takes elements r, r+{world}, ... "
+                                "(W replicated), no collective on the data path")
+        else:
+            self.elems = list(range(wl.batch))
+            self.coords = wl.coords
+            self.batch = wl.batch
+            self.units_job = wl.n * world
+            self.scaling = "weak"
+            self.parallelism = f"replicas x{world}, no collective on the data path"
+        self.n = int(self.coords.shape[0])
+        self.grid = wl.grid_dim
+        self.channels = list(wl.channels)
+        n_layers = len(self.channels) - 1
+        self.acts = ["gelu" if wl.gelu_between and li < n_layers - 1 else None
+                     for li in range(n_layers)]
+        self.weights = wl.weights()
+        self.feats = WL.to_bf16_values(WL.make_features(self.n, self.channels[0],
+                                                        feature_seed(rank)))
+
+    def flops(self, nnz: int) -> float:
+        """Algorithmic FLOPs of the layers over a map with nnz neighbour pairs."""
+        return sum(2.0 * nnz * self.channels[li] * self.channels[li + 1]
+                   for li in range(len(self.channels) - 1))
+
+    def step_text(self) -> str:
+        layers = len(self.channels) - 1
+        if layers == 1:
+            return f"map build ({MAP_LAUNCHES} kernels) + bf16 x-run forward (1 kernel)"
+        return (f"map build ({MAP_LAUNCHES} kernels) + {layers} bf16 forward layers on it "
+                f"(exact GELU between)")
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -344,34 +422,46 @@ def run_ours(args):
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
 
-    wl = _workload(args.workload)
-    import workloads as WL
-    cin, cout = wl.channels[0], wl.channels[1]
-    n = wl.n
-    coords_h = torch.from_numpy(wl.coords)
-    feats_h = torch.from_numpy(WL.to_bf16_values(WL.make_features(n, cin, feature_seed(rank))))
-    w_h = torch.from_numpy(wl.weights()[0])
+    job = Job(args.workload, rank, world)
+    wl = job.wl
+    n = job.n
+    cin, cout = job.channels[0], job.channels[-1]
+    coords_h = torch.from_numpy(job.coords)
+    feats_h = torch.from_numpy(job.feats)
+    ws_h = [torch.from_numpy(w) for w in job.weights]
     coords = coords_h.to(dev)
     feats = feats_h.to(dev).to(torch.bfloat16)
-    weight = w_h.to(dev).to(torch.bfloat16)
-    out = torch.empty((n, cout), dtype=torch.bfloat16, device=dev)
+    weights = [w.to(dev).to(torch.bfloat16) for w in ws_h]
+    outs = [torch.empty((n, w.shape[0]), dtype=torch.bfloat16, device=dev) for w in weights]
     nbr = torch.empty((n, 27), dtype=torch.int32, device=dev)
-    ws_bytes = _abi.subm3d_map_workspace_bytes(n, wl.grid_dim, wl.batch)
+    ws_bytes = max(1, _abi.subm3d_map_workspace_bytes(n, job.grid, job.batch))
     workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
-    def step(ev_fwd=None):
-        h = S.build_map(coords, wl.grid_dim, wl.batch, check=False, nbr=nbr, workspace=workspace)
+    def compute(c, x0, ws, outs_, nbr_, work, ev_fwd=None, s=None):
+        """The step's work on one buffer set: the map build, then every layer."""
+        if n == 0:
+            if ev_fwd is not None:
+                ev_fwd[0].record(stream)
+                ev_fwd[1].record(stream)
+            return None
+        h = S.build_map(c, job.grid, job.batch, check=False, nbr=nbr_, workspace=work, stream=s)
         if ev_fwd is not None:
             ev_fwd[0].record(stream)
-        S.forward(h, feats, weight, out=out)
+        x = x0
+        for li, w in enumerate(ws):
+            x = S.forward(h, x, w, act=job.acts[li], out=outs_[li], stream=s)
         if ev_fwd is not None:
             ev_fwd[1].record(stream)
         return h
 
+    def step(ev_fwd=None):
+        return compute(coords, feats, weights, outs, nbr, workspace, ev_fwd)
+
     # correctness gate before timing: the map must be valid
     h0 = step()
-    assert S.map_status(h0) == 0, "map build reported a data error"
+    if h0 is not None:
+        assert S.map_status(h0) == 0, "map build reported a data error"
     nnz_total = int((nbr >= 0).sum().item())
     assert _abi.subm3d_device_status() == 0
     for _ in range(args.warmup):
@@ -404,27 +494,28 @@ def run_ours(args):
     assert _abi.subm3d_device_status() == 0
     step_ms = [a.elapsed_time(b) for a, b in ev]
     fwd_ms = [a.elapsed_time(b) for a, b in evf]
-    map_ms = [s - f for s, f in zip(step_ms, fwd_ms)]
+    map_ms = [s_ - f for s_, f in zip(step_ms, fwd_ms)]
     total_ms = max_over_ranks(float(sum(step_ms)), dev)
 
     # e2e through the public API with host buffers: every step copies its inputs
-    # in from pinned memory, builds the map, runs the forward and copies its
+    # in from pinned memory, builds the map, runs the layers and copies the last
     # output back.  Steps are pipelined over two device buffer sets and three
     # streams (inputs in, compute, output out), ordered by events, so step k's
     # copies overlap the compute of its neighbours (PCIe is full duplex).  The
     # timed region runs from the first input copy to the last output copy.
     coords_p = coords_h.pin_memory()
     feats_p = feats_h.to(torch.bfloat16).pin_memory()
-    w_p = w_h.to(torch.bfloat16).pin_memory()
+    ws_p = [w.to(torch.bfloat16).pin_memory() for w in ws_h]
     outs_p = [torch.empty((n, cout), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    h2d = coords_p.numel() * 4 + feats_p.numel() * 2 + w_p.numel() * 2
+    h2d = coords_p.numel() * 4 + feats_p.numel() * 2 + sum(w.numel() * 2 for w in ws_p)
     d2h = outs_p[0].numel() * 2
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     bufs = [dict(coords=torch.empty_like(coords), feats=torch.empty_like(feats),
-                 weight=torch.empty_like(weight), out=torch.empty_like(out),
+                 weights=[torch.empty_like(w) for w in weights],
+                 outs=[torch.empty_like(o) for o in outs],
                  nbr=torch.empty_like(nbr), ws=torch.empty_like(workspace)) for _ in range(2)]
-    ev = lambda: torch.cuda.Event()
-    in_done, comp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    mk = lambda: torch.cuda.Event()
+    in_done, comp_done, out_done = [mk(), mk()], [mk(), mk()], [mk(), mk()]
     for e in in_done + comp_done + out_done:
         e.record(stream)
 
@@ -435,17 +526,16 @@ def run_ours(args):
             s_in.wait_event(comp_done[bset])      # the previous user of this set has read it
             B["coords"].copy_(coords_p, non_blocking=True)
             B["feats"].copy_(feats_p, non_blocking=True)
-            B["weight"].copy_(w_p, non_blocking=True)
+            for dst, src in zip(B["weights"], ws_p):
+                dst.copy_(src, non_blocking=True)
             in_done[bset].record(s_in)
         stream.wait_event(in_done[bset])
         stream.wait_event(out_done[bset])         # its output buffer has been copied out
-        h = S.build_map(B["coords"], wl.grid_dim, wl.batch, check=False, nbr=B["nbr"],
-                        workspace=B["ws"], stream=stream)
-        S.forward(h, B["feats"], B["weight"], out=B["out"], stream=stream)
+        compute(B["coords"], B["feats"], B["weights"], B["outs"], B["nbr"], B["ws"], s=stream)
         comp_done[bset].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(comp_done[bset])
-            outs_p[bset].copy_(B["out"], non_blocking=True)
+            outs_p[bset].copy_(B["outs"][-1], non_blocking=True)
             out_done[bset].record(s_out)
 
     for k in range(max(2, args.warmup)):
@@ -463,35 +553,36 @@ def run_ours(args):
 
     if rank == 0:
         peaks, peak_src = _peaks()
-        flops = 2.0 * nnz_total * cin * cout
+        flops = job.flops(nnz_total)
         fwd_avg_s = statistics.mean(fwd_ms) / 1e3
         map_avg_s = statistics.mean(map_ms) / 1e3
         achieved_tf = flops / fwd_avg_s / 1e12
         peak_tf = float(peaks["bf16_tflops"])
         map_gbs = n * MAP_BYTES_PER_VOXEL / map_avg_s / 1e9
-        voxels_total = n * world
+        n_layers = len(job.weights)
         line = {
             "metric": METRIC,
-            "value": job_rate(n, world, total_ms / 1e3 / K),
+            "value": job.units_job / (total_ms / 1e3 / K),
             "unit": "voxels/s",
             "n_gpus": world,
             "steps": K,
             "warmup": args.warmup,
             "ms_per_step": total_ms / K,
             "higher_is_better": True,
-            "scaling": "weak",
+            "scaling": job.scaling,
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic",
             "config": {
-                **_workload_config(wl, nnz_total / n),
-                "step": f"map build ({MAP_LAUNCHES} kernels) + bf16 x-run forward (1 kernel)",
+                **_workload_config(wl, nnz_total / max(n, 1)),
+                "step": job.step_text(),
                 "l2": f"flushed before every timed step ({L2_FLUSH_BYTES >> 20} MB write)",
-                "parallelism": f"replicas x{world}, no collective on the data path",
+                "parallelism": job.parallelism,
             },
-            "tflops_effective": flops * world / (total_ms / 1e3 / K) / 1e12,
+            "tflops_effective": flops / (total_ms / 1e3 / K) / 1e12,
             "roofline": {
-                "kernel": "subm3d_fwd_bf16_runs_sm100",
+                "kernel": "subm3d_fwd_bf16_runs_sm100" + (f" (x{n_layers} layers)"
+                                                         if n_layers > 1 else ""),
                 "bound": "tensor", "achieved": achieved_tf, "peak": peak_tf, "unit": "TFLOP/s",
                 "frac": achieved_tf / peak_tf, "traffic": _profiled_traffic(args.workload),
                 "traffic_unit": "bytes per launch (ncu dram read+write)",
@@ -503,72 +594,75 @@ def run_ours(args):
                 "unit": "GB/s", "frac": map_gbs / float(peaks["hbm_gbs"]),
                 "bytes_per_voxel": MAP_BYTES_PER_VOXEL, "ms_avg": map_avg_s * 1e3,
             },
-            "e2e": {"value": job_rate(n, world, e2e_ms / 1e3 / K), "unit": "voxels/s",
+            "e2e": {"value": job.units_job / (e2e_ms / 1e3 / K), "unit": "voxels/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms / K},
-            "gpu_launches": (MAP_LAUNCHES + 1) * K,
+            "gpu_launches": (MAP_LAUNCHES + n_layers) * K,
             "clocks": clocks,
         }
-        if world == 1 and not args.no_context:
+        if job.name == "batched":
+            line["config"]["batch_elements_rank0"] = job.elems
+        if world == 1 and not args.no_context and job.name == "headline":
             h_ctx = step()
             torch.cuda.synchronize()
-            flops_alg = 2.0 * nnz_total * cin * cout
+            w0 = weights[0]
             line["fp32_forward"] = fp32_forward_line(
-                h_ctx, feats.float(), weight.float(), flops_alg, flush,
+                h_ctx, feats.float(), w0.float(), flops, flush,
                 float(clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965.0))
-            line["fused_epilogue"] = fused_epilogue_line(h_ctx, feats, weight, flops_alg, flush,
+            line["fused_epilogue"] = fused_epilogue_line(h_ctx, feats, w0, flops, flush,
                                                          peak_tf, fwd_avg_s * 1e3)
-            line["backward"] = backward_line(h_ctx, feats, weight, flops_alg, flush, peak_tf,
+            line["backward"] = backward_line(h_ctx, feats, w0, flops, flush, peak_tf,
                                              line["fp32_forward"]["peak"])
             line["resample"] = resample_line(coords, feats, wl.grid_dim, flush,
                                              float(peaks["hbm_gbs"]))
             line["decoder_stack"] = decoder_stack_line(flush, peak_tf)
-            line["context_per_offset_torch"] = per_offset_context(h_ctx, feats, weight, flush)
+            line["context_per_offset_torch"] = per_offset_context(h_ctx, feats, w0, flush)
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(wl, args.cpu_rows)
+            line["cpu_baseline"] = cpu_baseline(job, args.cpu_budget_s)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
 
 
-def _oracle_inputs(wl):
-    import workloads as WL
-    x = WL.to_bf16_values(WL.make_features(wl.n, wl.channels[0], 1)).astype(np.float64)
-    w = wl.weights()[0].astype(np.float64)
-    return x, w
-
-
-def _oracle_step(wl, x, w, rows):
-    """One bounded oracle pass: the whole map (std::map) + the forward of `rows`."""
+def oracle_step(job, m: int) -> float:
+    """One pass of the whole path through the oracle (oracle/, C++ std::map and
+    fp64 loops) on a bounded sample of the job: the first m rows of its
+    coordinate set in raster order -- their map, then every layer over them
+    (GELU between where the workload has it, bf16 rounding after each layer).
+    Returns the seconds it took."""
     from oracle import cpp as C
+    c = job.coords[:m]
     t0 = time.perf_counter()
-    nbr = C.build_map(wl.coords, wl.grid_dim, wl.batch)
-    t1 = time.perf_counter()
-    C.forward(nbr, x, w, rows=rows, round_to_bf16=True)
-    t2 = time.perf_counter()
-    return t1 - t0, t2 - t1
+    nbr = C.build_map(c, job.grid, job.batch)
+    x = job.feats[:m].astype(np.float64)
+    for li, w in enumerate(job.weights):
+        x = C.forward(nbr, x, w.astype(np.float64), act=job.acts[li], round_to_bf16=True)
+    return time.perf_counter() - t0
 
 
-def cpu_baseline(wl, n_rows, reps=2):
-    """The oracle as it stands on the host cores: map build of the full set plus
-    the fp64 forward of `n_rows` evenly spaced rows (all rows when n_rows <= 0),
-    `reps` times; voxels/s = 1 / mean(map_s / N + fwd_s / rows)."""
+def oracle_sample_rows(job, seconds: float) -> int:
+    """Rows of a sample whose oracle_step takes about `seconds` (from a timed
+    pass over 4,096 rows), at most the whole set."""
+    m0 = min(job.n, 4096)
+    if m0 == 0:
+        return 0
+    per_row = oracle_step(job, m0) / m0
+    return int(max(m0, min(job.n, seconds / per_row)))
+
+
+def cpu_baseline(job, budget_s: float, reps: int = 2):
+    """The oracle as it stands on the host cores: `reps` passes of oracle_step
+    over a raster-order prefix sized to about budget_s / reps seconds (all
+    rows when they fit); voxels/s = rows / mean pass time."""
     from oracle import cpp as C
-    n_rows = wl.n if n_rows <= 0 else min(n_rows, wl.n)
-    rows = np.linspace(0, wl.n - 1, n_rows).astype(np.int64)
-    x, w = _oracle_inputs(wl)
-    per_voxel, map_t, fwd_t = [], [], []
-    for _ in range(reps):
-        map_s, fwd_s = _oracle_step(wl, x, w, rows)
-        map_t.append(map_s)
-        fwd_t.append(fwd_s)
-        per_voxel.append(map_s / wl.n + fwd_s / rows.size)
-    what = ("all rows" if rows.size == wl.n else f"{rows.size} evenly spaced rows")
-    return {"value": 1.0 / statistics.mean(per_voxel), "unit": "voxels/s",
+    m = oracle_sample_rows(job, budget_s / reps)
+    ts = [oracle_step(job, m) for _ in range(reps)]
+    what = "all rows" if m == job.n else f"the first {m} of {job.n} rows (raster order)"
+    return {"value": m / statistics.mean(ts), "unit": "voxels/s",
             "cores": C.num_threads(), "kind": "oracle",
-            "sample": f"{reps} x (map build of all {wl.n} voxels, {statistics.mean(map_t):.2f} s "
-                      f"+ fp64 forward of {what}, {statistics.mean(fwd_t):.2f} s)"}
+            "sample": f"{reps} x (map build + {len(job.weights)} fp64 layer(s)) over {what}, "
+                      f"{statistics.mean(ts):.2f} s each"}
 
 
 def run_reference(args):
@@ -576,37 +670,33 @@ def run_reference(args):
     if rank != 0:
         return
     from oracle import cpp as C
-    wl = _workload(args.workload)
-    # rows per step shrink with K so that the whole run stays within minutes
-    cap = wl.n if args.cpu_rows <= 0 else args.cpu_rows
-    n_rows = max(256, min(cap, 2_000_000 // max(1, args.steps), wl.n))
-    rows = np.linspace(0, wl.n - 1, n_rows).astype(np.int64)
-    x, w = _oracle_inputs(wl)
+    job = Job(args.workload, 0, 1)
+    wl = job.wl
+    # every step is the same bounded sample, sized so that the K timed steps
+    # take about --ref-budget-s seconds in all
+    m = oracle_sample_rows(job, args.ref_budget_s / max(1, args.steps))
     nnz_avg = float((C.build_map(wl.coords, wl.grid_dim, wl.batch) >= 0).sum()) / wl.n
-    for _ in range(min(args.warmup, 3)):
-        _oracle_step(wl, x, w, rows[:256])
-    per_voxel = []
+    for _ in range(min(args.warmup, 2)):
+        oracle_step(job, min(m, 4096))
     t_start = time.perf_counter()
-    for _ in range(args.steps):
-        map_s, fwd_s = _oracle_step(wl, x, w, rows)
-        per_voxel.append(map_s / wl.n + fwd_s / rows.size)
+    ts = [oracle_step(job, m) for _ in range(args.steps)]
     wall = time.perf_counter() - t_start
-    sec_per_voxel = statistics.mean(per_voxel)
-    value = 1.0 / sec_per_voxel
+    step_s = statistics.mean(ts)
+    value = m / step_s
+    what = "all rows" if m == job.n else f"the first {m} of {job.n} rows (raster order)"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "voxels/s",
         "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": sec_per_voxel * wl.n * 1e3,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+        "higher_is_better": True, "scaling": job.scaling, "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
         "config": {**_workload_config(wl, nnz_avg),
-                   "step": "map build + fp64 forward (C++ oracle)",
+                   "step": f"map build + {len(job.weights)} fp64 layer(s) (C++ oracle)",
                    "parallelism": "host cores (OpenMP)"},
         "cpu_baseline": {"value": value, "unit": "voxels/s", "cores": C.num_threads(),
                          "kind": "oracle",
-                         "sample": f"per step: map build of all {wl.n} voxels + fp64 forward "
-                                   f"of {rows.size} evenly spaced rows; ms_per_step extrapolates "
-                                   f"to the full set; wall {wall:.1f} s"},
+                         "sample": f"every step: map build + {len(job.weights)} fp64 layer(s) "
+                                   f"over {what}; {args.steps} steps in {wall:.1f} s"},
         "e2e": {"value": value, "unit": "voxels/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -619,9 +709,12 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="headline", choices=["headline", "dense", "shell_bf16"])
-    ap.add_argument("--cpu-rows", type=int, default=0,
-                    help="rows of the cpu_baseline forward (0: all rows of the workload)")
+    ap.add_argument("--workload", default="headline",
+                    choices=["headline", "dense", "shell_bf16", "batched"])
+    ap.add_argument("--cpu-budget-s", type=float, default=16.0,
+                    help="host seconds the cpu_baseline passes may take in all")
+    ap.add_argument("--ref-budget-s", type=float, default=60.0,
+                    help="host seconds the reference arm's timed steps may take in all")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-context", action="store_true",
                     help="skip the fp32-path and per-offset-loop context measurements")

@@ -88,14 +88,14 @@ SUBM3D_API const char* subm3d_status_string(int32_t status);
 /*
  * Workspace bytes subm3d_build_map() needs for N voxels in a batch x
  * grid_dim^3 volume: a status word, one 32-bit offset mask per 128-row tile,
- * and the lookup table -- a direct-address table of batch * grid_dim^3 int32
- * cells when that is at most max(64 MB, 256 bytes x N) and 2^28 cells, else an
- * open-addressing hash table of at
- * least 2N slots (8 bytes each, 12 with batch > 4 or grid_dim > 1024) -- and
- * for N < 2^29 the x-run layout of subm3d_forward_map(): run-start counts (an
- * int32 per 128-row tile and per 128 tiles), a header, a position table of 3N
- * int32 (rounded up) and an E index table of 9 x 260 int32 per 256 positions
- * (~110 bytes per voxel).
+ * and the lookup table -- a direct-address table of batch * (grid_dim + 2)^3
+ * int32 cells (each grid with a one-cell border) when that is at most
+ * max(64 MB, 256 bytes x N) and 2^28 cells, else an open-addressing hash table
+ * of at least 2N slots (8 bytes each, 12 with batch > 4 or grid_dim > 1024) --
+ * and for N < 2^29 the x-run layout of subm3d_forward_map(): run-start counts
+ * (an int32 per 128-row tile and per 128 tiles), a header, a position table of
+ * 3N int32 (rounded up) and an E index table of 9 lines of as many int32
+ * (~120 bytes per voxel).
  * Host-only, no CUDA
  * call.  Returns 0 for arguments subm3d_build_map() would
  * reject (N < 0, grid_dim < 1 or > 65535, batch < 1 or > 65535).
@@ -124,7 +124,7 @@ SUBM3D_API size_t subm3d_map_workspace_bytes(int64_t n, int32_t grid_dim, int32_
  * repeated are reported by subm3d_map_status(); until it returns SUBM3D_OK the
  * contents of nbr are unspecified.  Besides nbr and the tile masks the build
  * writes, for N < 2^29, the x-run position layout that subm3d_forward_map()
- * uses.  Enqueues 3 kernels; no allocation.
+ * uses.  Enqueues 3 kernels; no allocation.  N < 2^31 - 256.
  * Testing knobs, read from the environment by this function and by
  * subm3d_map_workspace_bytes() alike: SUBM3D_MAP_KIND=hash selects the hash
  * table even where the direct table fits; SUBM3D_TABLE_CAPACITY=<slots> caps
@@ -228,13 +228,17 @@ SUBM3D_API subm3d_status subm3d_build_map_noalloc(const int32_t* coords, int64_t
  * Forward of one layer over a built map -- the same op and arguments as
  * subm3d_forward(), with N, nbr and the masks taken from the map.  For bf16
  * with Cin a multiple of 64 (and a map of N < 2^29) it runs the x-run kernel,
- * which uses the map's position layout: voxels on a line of positions in row order, two pad
- * positions before every run of x-adjacent voxels, tiles of 256 positions,
- * and per tile and (dz, dy) one gathered tile of feature rows whose rows
- * p-1, p, p+1 are the dx = -1, 0, +1 neighbours of the voxel at position p;
- * the three offsets of a (dz, dy) pair share that tile through row-shifted
- * tensor-core operands, so ~3x fewer feature rows are gathered.  Other shapes
- * and fp32 run subm3d_forward().  Errors as subm3d_forward().
+ * which uses the map's position layout: voxels on a line of positions in row
+ * order, two pad positions before every run of x-adjacent voxels, tiles of
+ * 256 positions, and per tile and (dz, dy) one gathered tile of feature rows
+ * whose rows p-1, p, p+1 are the dx = -1, 0, +1 neighbours of the voxel at
+ * position p; the three offsets of a (dz, dy) pair share that tile through
+ * row-shifted tensor-core operands, so ~3x fewer feature rows are gathered.
+ * Other shapes and fp32 run subm3d_forward().  Errors as subm3d_forward().
+ * Testing knobs, read at every call: SUBM3D_FORWARD_KERNEL=gather takes the
+ * per-offset kernel of subm3d_forward() even where the x-run kernel applies;
+ * SUBM3D_WAIT_LIMIT_NS=<ns> cuts the limit of every bounded device wait of the
+ * tensor-core kernels (default 2 s) so that the timeout path can be tested.
  */
 SUBM3D_API subm3d_status subm3d_forward_map(const subm3d_map* map, const void* feats,
                                             const void* weight, void* out, int32_t cin,
@@ -377,8 +381,10 @@ SUBM3D_API subm3d_status subm3d_pool(const subm3d_map* fine, const int32_t* coor
  * Device pointers into the map's x-run layout, for tests and tools: the
  * position table (int32, one entry per position: row * 4 + tag, tag 0 voxel,
  * 1 left pad of that row's voxel, 2 right pad, -1 empty), the E index table
- * (int32 [tiles][9][260]: entry i of (tile, dz-dy) is the feature row of
- * gathered row i-1, or -1) and a 4-int header [runs, tiles, positions, 0].
+ * (int32, 9 lines, one per offset pair dz-dy = 3 (dz+1) + (dy+1), `stride`
+ * entries apart: entry q + 1 of a line is the feature row gathered as E row
+ * q, i.e. at position q, for q = -1 .. 256 tiles, or -1) and a 4-int header
+ * [runs, tiles, positions, stride].
  * Valid once the build has completed on its stream.  Host-only.
  * SUBM3D_E_UNSUPPORTED when the map has no run layout (N >= 2^29).
  */
@@ -387,8 +393,11 @@ SUBM3D_API subm3d_status subm3d_map_run_layout(const subm3d_map* map, const int3
 
 /*
  * Synchronizes `stream`, then reads and clears the library's device error word
- * of the current device: SUBM3D_E_TIMEOUT if a forward kernel gave up a
- * bounded wait since the last call, else SUBM3D_OK (or SUBM3D_E_CUDA).
+ * of the current device: SUBM3D_E_TIMEOUT if a tensor-core kernel (forward,
+ * input or weight gradient) gave up a bounded wait since the last call, else
+ * SUBM3D_OK (or SUBM3D_E_CUDA).  A kernel whose wait ran out has waited for
+ * the copies and MMAs it had issued and released its tensor memory before
+ * exiting, so later calls run normally; its own output is invalid.
  * Blocking.
  */
 SUBM3D_API subm3d_status subm3d_device_status(void* stream);

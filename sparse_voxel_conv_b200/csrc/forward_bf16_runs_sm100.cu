@@ -43,8 +43,11 @@
 //       memory, the residual, one bf16 rounding and 16-byte stores to the rows
 //       of the voxel positions (pad columns are dropped).
 //
-// Every wait is bounded (ptx.cuh); a wait that runs out sets the library's
-// device error word, the CTA lets its copies land, frees TMEM and exits.
+// Every wait is bounded (ptx.cuh).  When one runs out, every role leaves its
+// loop; after a CTA-wide barrier the TMA lane waits (bounded) for the weight
+// loads it issued and the MMA lane commits to a drain barrier and waits for
+// its MMAs, so that no copy or MMA is in flight when the CTA frees its tensor
+// memory and exits; the library's device error word is then set.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -78,14 +81,16 @@ constexpr uint32_t kTmemCols = 2 * TP;
 
 struct RunArgs {
   const int32_t* pos;     // position table
-  const int32_t* et;      // E index table
+  const int32_t* et;      // E index table: 9 lines (one per dz-dy pair), `es` entries apart
   const int32_t* hdr;     // [runs, position tiles, positions, 0]
   const __nv_bfloat16* x;
   __nv_bfloat16* out;
   const __nv_bfloat16* bias;      // [cout] or nullptr
   const __nv_bfloat16* residual;  // [N, cout] or nullptr; may be `out`
+  int64_t es;             // E line stride (entries)
   int32_t cin, cout, n_oblocks, n_kchunks, se, sw, flip;
   int32_t* err_word;
+  uint64_t wait_limit_ns;
 };
 
 struct SmemPlan {
@@ -99,8 +104,8 @@ __host__ __device__ inline SmemPlan plan_smem(int se, int sw) {
   p.epi_off = p.w_off + static_cast<size_t>(sw) * A_SLOT;
   p.bar_off = p.epi_off + kEpiStageBytes;
   // e_full[se], e_empty[se], w_full[sw], w_empty[sw], acc_full[2], acc_empty[2],
-  // tmem slot, abort
-  p.bytes = p.bar_off + (2 * se + 2 * sw + 4) * 8 + 16 + 1024;
+  // drain, WaitCtl (16 B), tmem slot
+  p.bytes = p.bar_off + (2 * se + 2 * sw + 5) * 8 + 16 + 16 + 1024;
   return p;
 }
 
@@ -172,8 +177,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* w_empty = w_full + SW;
   uint64_t* acc_full = w_empty + SW;
   uint64_t* acc_empty = acc_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint64_t* drain_bar = acc_empty + 2;
+  WaitCtl* wctl = reinterpret_cast<WaitCtl*>(drain_bar + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wctl + 1);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -190,7 +196,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], NUM_EPI_WARPS * 32);
     }
-    *abort_flag = 0;
+    mbar_init(drain_bar, 1);
+    wait_ctl_init(wctl, a.wait_limit_ns);
     fence_mbar_init();
   }
   if (warp == MMA_WARP) {
@@ -205,6 +212,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   pdl_wait();  // the setup above overlaps the map build's tail; global reads start here
   const int64_t n_tiles = __ldg(a.hdr + 1);
   const int64_t n_units = n_tiles * a.n_oblocks;
+  int64_t w_issued = 0;  // weight loads the TMA warp has issued (its abort-path drain)
 
   if (warp >= GATHER_WARP0 && warp < GATHER_WARP0 + NUM_GATHER_WARPS) {
     // ---------------------------------------------------------- gather ----
@@ -220,7 +228,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     // the E index entries of this thread's rows for the step `t` points at
     auto load_src = [&](const ESteps& t, int32_t (&v)[PPT + 1]) {
-      const int32_t* list = a.et + ((t.u / a.n_oblocks) * 9 + t.dzdy) * kEtStride;
+      // entries 256 tile .. 256 tile + 257 of the pair's line: E rows -1 .. 256
+      const int32_t* list = a.et + t.dzdy * a.es + (t.u / a.n_oblocks) * TP;
 #pragma unroll
       for (int q = 0; q <= PPT; ++q) {
         const int i = q < PPT ? rbase + q * ROWS_PER_PASS : TP + rbase;
@@ -234,7 +243,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     while (st.valid) {
       const int s = st.slot;
       // the E slot is free once the MMAs that read it are done
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&e_empty[s], st.phase ^ 1u, abort_flag))) break;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&e_empty[s], st.phase ^ 1u, wctl))) break;
       const __nv_bfloat16* xcol = a.x + st.j * CHUNK + piece * 8;
       const uint32_t e_base = smem_u32(e_ring) + static_cast<uint32_t>(s) * E_SLOT;
 #pragma unroll
@@ -258,7 +267,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     while (ok && st.valid) {
       const int o0 = static_cast<int>(st.u % a.n_oblocks) * TO;
       for (int dx = 0; dx < 3; ++dx) {
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&w_empty[w.slot], w.phase ^ 1u, abort_flag))) {
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&w_empty[w.slot], w.phase ^ 1u, wctl))) {
           ok = false;
           break;
         }
@@ -271,10 +280,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         __syncwarp();
         w.next(SW);
+        ++w_issued;
       }
       st.next(a.n_kchunks, SE);
     }
-    if (!ok) __nanosleep(20000);  // let TMA copies already issued land before exit
   } else if (warp == MMA_WARP) {
     // -------------------------------------------------------------- MMA ----
     if (lane == 0) {
@@ -286,20 +295,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       while (ok && st.valid) {
         const int local = st.local;
         const int acc = local & 1;
-        if (!mbar_wait(&acc_empty[acc], ((local >> 1) & 1) ^ 1, abort_flag)) break;
+        if (!mbar_wait(&acc_empty[acc], ((local >> 1) & 1) ^ 1, wctl)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + static_cast<uint32_t>(acc * TP);
         bool first = true;
         bool unit_done = false;
         while (!unit_done) {
           const int s = st.slot;
-          if (!mbar_wait(&e_full[s], st.phase, abort_flag)) {
+          if (!mbar_wait(&e_full[s], st.phase, wctl)) {
             ok = false;
             break;
           }
           const uint32_t e_base = smem_u32(e_ring) + static_cast<uint32_t>(s) * E_SLOT;
           for (int dx = 0; dx < 3; ++dx) {
-            if (!mbar_wait(&w_full[w.slot], w.phase, abort_flag)) {
+            if (!mbar_wait(&w_full[w.slot], w.phase, wctl)) {
               ok = false;
               break;
             }
@@ -323,7 +332,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!ok) break;
         umma_commit(&acc_full[acc]);
       }
-      if (!ok) __nanosleep(20000);  // let MMAs already issued finish before TMEM is freed
     }
   } else {
     // --------------------------------------------------------- epilogue ----
@@ -332,7 +340,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int local = 0;
     for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x, ++local) {
       const int acc = local & 1;
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&acc_full[acc], (local >> 1) & 1, abort_flag))) break;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&acc_full[acc], (local >> 1) & 1, wctl))) break;
       tc_fence_after();
       const int64_t tile = u / a.n_oblocks;
       const int o_warp = static_cast<int>(u % a.n_oblocks) * TO + warp * 32;
@@ -349,12 +357,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  __syncthreads();  // every role has left its loop; the abort word no longer changes
+  if (wait_aborted(wctl)) {
+    // copies and MMAs issued before the abort may still be in flight
+    if (warp == TMA_WARP && lane == 0) drain_ring(w_full, SW, w_issued);
+    if (warp == MMA_WARP && lane == 0) drain_mma(drain_bar);
+    tc_fence_before();
+    __syncthreads();
+  }
   if (warp == MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }
-  if (threadIdx.x == 0 && *abort_flag) atomicExch(a.err_word, 1);
+  if (threadIdx.x == 0 && wait_aborted(wctl)) atomicExch(a.err_word, 1);
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -403,9 +418,10 @@ cudaError_t device_setup(int device, int* num_sms) {
 }  // namespace
 
 cudaError_t launch_forward_bf16_runs(const int32_t* pos, const int32_t* etable,
-                                     const int32_t* header, int64_t max_tiles, const void* feats,
+                                     int64_t et_stride, const int32_t* header, int64_t max_tiles,
+                                     const void* feats,
                                      const void* weight, void* out, int32_t cin, int32_t cout,
-                                     int32_t flip, const Epilogue& epi, int32_t* err_word,
+                                     int32_t flip, const Epilogue& epi, const DeviceCtl& ctl,
                                      cudaStream_t stream) {
   EncodeTiledFn encode = encode_fn();
   if (!encode) return cudaErrorNotSupported;
@@ -433,6 +449,7 @@ cudaError_t launch_forward_bf16_runs(const int32_t* pos, const int32_t* etable,
   RunArgs a;
   a.pos = pos;
   a.et = etable;
+  a.es = et_stride;
   a.hdr = header;
   a.x = static_cast<const __nv_bfloat16*>(feats);
   a.out = static_cast<__nv_bfloat16*>(out);
@@ -445,7 +462,8 @@ cudaError_t launch_forward_bf16_runs(const int32_t* pos, const int32_t* etable,
   a.flip = flip;
   a.bias = static_cast<const __nv_bfloat16*>(epi.bias);
   a.residual = static_cast<const __nv_bfloat16*>(epi.residual);
-  a.err_word = err_word;
+  a.err_word = ctl.err_word;
+  a.wait_limit_ns = ctl.wait_limit_ns;
   // the tile count lives on the device; launch for the largest possible count
   // and let each CTA read the actual one
   const int64_t units = max_tiles * a.n_oblocks;

@@ -42,9 +42,11 @@
 //       64-byte channel runs of each voxel's row (epilogue.cuh).
 //
 // Offsets with no neighbour anywhere in the tile (bit clear in both 128-row
-// mask words) are skipped.  Every wait is bounded (ptx.cuh); a wait that runs
-// out sets the library's device error word, the CTA lets its copies land,
-// frees its tensor memory and exits.
+// mask words) are skipped.  Every wait is bounded (ptx.cuh).  When one runs
+// out, every role leaves its loop; after a CTA-wide barrier the TMA lane waits
+// (bounded) for the weight and nbr copies it issued and the MMA lane for its
+// MMAs, then the CTA frees its tensor memory, sets the library's device error
+// word and exits.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -84,6 +86,7 @@ struct FwdArgs {
   int32_t cin, cout, n_oblocks, n_kchunks, stages, flip;
   int64_t n_tiles;
   int32_t* err_word;
+  uint64_t wait_limit_ns;
 };
 
 struct SmemPlan {
@@ -99,8 +102,9 @@ __host__ __device__ inline SmemPlan plan_smem(int chunk, int stages) {
   p.nbr_off = p.b_off + stages * b_bytes;
   p.epi_off = p.nbr_off + 2 * kNbrTileBytes;
   p.bar_off = p.epi_off + kEpiStageBytes;
-  // full[S], empty[S], nbr_full[2], nbr_empty[2], acc_full[2], acc_empty[2], tmem slot, abort
-  p.bytes = p.bar_off + (2 * stages + 8) * 8 + 16 + 1024;  // + base alignment slack
+  // full[S], wfull[S], empty[S], nbr_full[2], nbr_empty[2], acc_full[2], acc_empty[2],
+  // drain, WaitCtl (16 B), tmem slot
+  p.bytes = p.bar_off + (3 * stages + 9) * 8 + 16 + 16 + 1024;  // + base alignment slack
   return p;
 }
 
@@ -188,22 +192,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* stage_b = base + plan.b_off;
   int32_t* nbr_s = reinterpret_cast<int32_t*>(base + plan.nbr_off);
   uint8_t* epi_s = base + plan.epi_off;
-  uint64_t* full = reinterpret_cast<uint64_t*>(base + plan.bar_off);
-  uint64_t* empty = full + S;
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + plan.bar_off);  // gathered B rows
+  uint64_t* wfull = full + S;                                           // TMA weight slice
+  uint64_t* empty = wfull + S;
   uint64_t* nbr_full = empty + S;
   uint64_t* nbr_empty = nbr_full + 2;
   uint64_t* acc_full = nbr_empty + 2;
   uint64_t* acc_empty = acc_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint64_t* drain_bar = acc_empty + 2;
+  WaitCtl* wctl = reinterpret_cast<WaitCtl*>(drain_bar + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wctl + 1);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], GATHER_THREADS + 1);  // every gather thread's cp.async arrive + TMA
-      mbar_init(&empty[s], 1);                    // one tcgen05.commit
+      mbar_init(&full[s], GATHER_THREADS);  // every gather thread's cp.async arrive
+      mbar_init(&wfull[s], 1);              // the TMA lane's arrive + the slice's bytes
+      mbar_init(&empty[s], 1);              // one tcgen05.commit
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&nbr_full[b], 1);
@@ -211,7 +218,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], NUM_EPI_WARPS * 32);
     }
-    *abort_flag = 0;
+    mbar_init(drain_bar, 1);
+    wait_ctl_init(wctl, a.wait_limit_ns);
     fence_mbar_init();
   }
   if (warp == MMA_WARP) {
@@ -223,6 +231,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  int64_t w_issued = 0;    // weight loads issued by the TMA warp (its abort-path drain)
+  int64_t nbr_issued = 0;  // nbr tiles staged by the TMA warp
 
   if (warp >= GATHER_WARP0 && warp < GATHER_WARP0 + NUM_GATHER_WARPS) {
     // ---------------------------------------------------------- gather ----
@@ -246,12 +256,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     while (st.valid) {
       if (st.local != ready_local) {
         if (!__all_sync(0xFFFFFFFFu,
-                        mbar_wait(&nbr_full[st.local & 1], (st.local >> 1) & 1, abort_flag)))
+                        mbar_wait(&nbr_full[st.local & 1], (st.local >> 1) & 1, wctl)))
           break;
         ready_local = st.local;
       }
       const int s = st.slot;
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[s], st.phase ^ 1u, abort_flag))) break;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[s], st.phase ^ 1u, wctl))) break;
       const int32_t* nb = nbr_s + (st.local & 1) * (TV * kKvol) + rbase * kKvol + st.k;
       const __nv_bfloat16* xcol = a.x + st.j * CHUNK + piece * 8;
       const uint32_t b_base = smem_u32(stage_b) + static_cast<uint32_t>(s) * B_STAGE;
@@ -276,7 +286,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     auto load_nbr = [&](int64_t u, int l) -> bool {
       const int buf = l & 1;
       if (!__all_sync(0xFFFFFFFFu,
-                      mbar_wait(&nbr_empty[buf], ((l >> 1) & 1) ^ 1, abort_flag)))
+                      mbar_wait(&nbr_empty[buf], ((l >> 1) & 1) ^ 1, wctl)))
         return false;
       const int64_t row0 = (u / a.n_oblocks) * TV;
       int32_t* dst = nbr_s + buf * (TV * kKvol);
@@ -293,6 +303,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&nbr_full[buf]);
       }
+      ++nbr_issued;
       return true;
     };
     bool ok = true;
@@ -310,21 +321,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       const int s = st.slot;
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[s], st.phase ^ 1u, abort_flag))) {
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[s], st.phase ^ 1u, wctl))) {
         ok = false;
         break;
       }
       if (lane == 0) {
         const int kw = a.flip ? (kKvol - 1 - st.k) : st.k;
         const int o0 = static_cast<int>(st.u % a.n_oblocks) * TO;
-        mbar_arrive_expect_tx(&full[s], A_STAGE);
-        tma_load_3d(smem_u32(stage_a) + static_cast<uint32_t>(s) * A_STAGE, &wmap, &full[s],
+        mbar_arrive_expect_tx(&wfull[s], A_STAGE);
+        tma_load_3d(smem_u32(stage_a) + static_cast<uint32_t>(s) * A_STAGE, &wmap, &wfull[s],
                     st.j * CHUNK, kw, o0);
       }
       __syncwarp();
+      ++w_issued;
       st.next(a);
     }
-    if (!ok) __nanosleep(20000);  // let TMA copies already issued land before exit
   } else if (warp == MMA_WARP) {
     // -------------------------------------------------------------- MMA ----
     if (lane == 0) {
@@ -335,14 +346,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       while (ok && st.valid) {
         const int local = st.local;
         const int acc = local & 1;
-        if (!mbar_wait(&acc_empty[acc], ((local >> 1) & 1) ^ 1, abort_flag)) break;
+        if (!mbar_wait(&acc_empty[acc], ((local >> 1) & 1) ^ 1, wctl)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + static_cast<uint32_t>(acc * TV);
         bool first = true;
         bool unit_done = false;
         while (!unit_done) {
           const int s = st.slot;
-          if (!mbar_wait(&full[s], st.phase, abort_flag)) {
+          if (!mbar_wait(&full[s], st.phase, wctl) || !mbar_wait(&wfull[s], st.phase, wctl)) {
             ok = false;
             break;
           }
@@ -362,7 +373,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!ok) break;
         umma_commit(&acc_full[acc]);
       }
-      if (!ok) __nanosleep(20000);  // let MMAs already issued finish before TMEM is freed
     }
   } else {
     // --------------------------------------------------------- epilogue ----
@@ -372,7 +382,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int local = 0;
     for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x, ++local) {
       const int acc = local & 1;
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&acc_full[acc], (local >> 1) & 1, abort_flag))) break;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&acc_full[acc], (local >> 1) & 1, wctl))) break;
       tc_fence_after();
       const int64_t row0 = (u / a.n_oblocks) * TV;
       const int o_warp = static_cast<int>(u % a.n_oblocks) * TO + warp * 32;  // this warp's channels
@@ -388,12 +398,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  __syncthreads();  // every role has left its loop; the abort word no longer changes
+  if (wait_aborted(wctl)) {
+    // copies and MMAs issued before the abort may still be in flight
+    if (warp == TMA_WARP && lane == 0) {
+      drain_ring(wfull, S, w_issued);
+      drain_ring(nbr_full, 2, nbr_issued);
+    }
+    if (warp == MMA_WARP && lane == 0) drain_mma(drain_bar);
+    tc_fence_before();
+    __syncthreads();
+  }
   if (warp == MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }
-  if (threadIdx.x == 0 && *abort_flag) atomicExch(a.err_word, 1);
+  if (threadIdx.x == 0 && wait_aborted(wctl)) atomicExch(a.err_word, 1);
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -450,7 +470,7 @@ cudaError_t device_setup(int device, int* num_sms) {
 
 cudaError_t launch_forward_bf16(const int32_t* nbr, const uint32_t* tile_mask, int64_t n,
                                 const void* feats, const void* weight, void* out, int32_t cin,
-                                int32_t cout, int32_t flip, const Epilogue& epi, int32_t* err_word,
+                                int32_t cout, int32_t flip, const Epilogue& epi, const DeviceCtl& ctl,
                                 cudaStream_t stream) {
   EncodeTiledFn encode = encode_fn();
   if (!encode) return cudaErrorNotSupported;
@@ -496,7 +516,8 @@ cudaError_t launch_forward_bf16(const int32_t* nbr, const uint32_t* tile_mask, i
   a.bias = static_cast<const __nv_bfloat16*>(epi.bias);
   a.residual = static_cast<const __nv_bfloat16*>(epi.residual);
   a.n_tiles = (n + TV - 1) / TV;
-  a.err_word = err_word;
+  a.err_word = ctl.err_word;
+  a.wait_limit_ns = ctl.wait_limit_ns;
   const int64_t units = a.n_tiles * a.n_oblocks;
   const unsigned grid = static_cast<unsigned>(units < num_sms ? units : num_sms);
   auto launch = [&](auto kernel) {

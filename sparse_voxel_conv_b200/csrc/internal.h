@@ -44,15 +44,19 @@ constexpr uint32_t kErrTableFull = 4u;
 
 constexpr int kTileRows = 128;  // rows per tile-mask word
 constexpr int kKvol = 27;
+// Largest N + 1 a map may have: row and tile arithmetic of the map kernels is
+// int32 (the last tile's end, N rounded up to 128, stays below 2^31).
+constexpr int64_t kMaxMapRows = (int64_t(1) << 31) - 256;
 
 // The two lookup structures of the map build (see map_build.cu).
 enum class MapKind { kDirect, kHash };
 
-// The direct-address table (batch * grid_dim^3 int32 cells) is used while it
-// takes at most max(kDirectTableMinBytes, kDirectTableBytesPerVoxel * N) bytes
-// and at most kDirectTableMaxCells cells (int32 cell arithmetic in the query):
-// clearing it costs its size in HBM writes, which beats hashing N voxels until
-// the volume is a few hundred bytes per voxel.
+// The direct-address table (batch * (grid_dim + 2)^3 int32 cells: each grid
+// with a one-cell border) is used while it takes at most
+// max(kDirectTableMinBytes, kDirectTableBytesPerVoxel * N) bytes and at most
+// kDirectTableMaxCells cells (int32 cell arithmetic in the query): clearing it
+// costs its size in HBM writes, which beats hashing N voxels until the volume
+// is a few hundred bytes per voxel.
 constexpr size_t kDirectTableMinBytes = size_t(64) << 20;
 constexpr double kDirectTableBytesPerVoxel = 256.0;
 constexpr double kDirectTableMaxCells = double(int64_t(1) << 28);
@@ -70,9 +74,10 @@ struct MapOptions {
 // positions: the right neighbour slot of the previous run and the left
 // neighbour slot of this one.  Positions are cut into tiles of kPosTile.
 constexpr int kPosTile = 256;
-// Row stride (int32) of the E index table: for a tile and an offset pair
-// (dz, dy), entries 0..257 are the feature rows of positions -1..256.
-constexpr int kEtStride = 260;
+// The E index table holds one line per offset pair (dz, dy), et_stride int32
+// entries apart: entry q + 1 of line dz-dy is the feature row gathered as E
+// row q (position q), for -1 <= q <= 256 * tiles, or -1.  A tile's E rows
+// -1 .. 256 are the 258 consecutive entries from 256 * tile.
 // The run layout is built for N < 2^29, so that positions (< 3N + 512) and
 // position-table entries (row * 4 + tag) fit int32; larger maps go without it.
 constexpr int64_t kRunLayoutMaxRows = int64_t(1) << 29;
@@ -93,11 +98,12 @@ struct MapLayout {
   // run layout (all kinds)
   size_t cnt_off = 0;       // int32 [n_tiles]: run starts per 128-row tile
   size_t sb_off = 0;        // int32 [ceil(n_tiles / 128)]: run starts per superblock
-  size_t hdr_off = 0;       // int32 [4]: runs, position tiles, positions, 0
+  size_t hdr_off = 0;       // int32 [4]: runs, position tiles, positions, E line stride
   size_t pos_off = 0;       // int32 [pos_max]: position table (row * 4 + tag, or -1)
   size_t pos_bytes = 0;
-  size_t et_off = 0;        // int32 [ptile_max][9][kEtStride]: E index table
-  int64_t pos_max = 0;      // positions reserved: 3N rounded up to whole tiles
+  size_t et_off = 0;        // int32 [9][et_stride]: E index table
+  int64_t et_stride = 0;    // entries per (dz, dy) line: pos_max + 4
+  int64_t pos_max = 0;      // positions reserved: 3N rounded up to whole tiles, + one tile
   int64_t ptile_max = 0;
   size_t total = 0;         // bytes
   int64_t n_tiles = 0;
@@ -108,7 +114,7 @@ bool map_layout(int64_t n, int32_t grid_dim, int32_t batch, const MapOptions& op
                 MapLayout* out);
 
 // Enqueues the three map-build kernels (init, insert, query) on `stream`.
-// Returns the launch error.
+// Returns the launch error.  Accepts N < kMaxMapRows.
 cudaError_t launch_map_build(const int32_t* coords, int64_t n, int32_t grid_dim, int32_t batch,
                              int32_t* nbr, void* workspace, const MapLayout& lay,
                              cudaStream_t stream);
@@ -131,19 +137,27 @@ cudaError_t launch_forward_f32(const int32_t* nbr, const uint32_t* tile_mask, in
                                int32_t cout, int32_t flip, const Epilogue& epi,
                                cudaStream_t stream);
 
+// What the tensor-core kernels need besides their operands: the library's
+// device error word (set to 1 by a CTA whose bounded wait ran out) and the
+// limit of each pipeline wait in ns (2 s unless a test asks for less).
+struct DeviceCtl {
+  int32_t* err_word = nullptr;
+  uint64_t wait_limit_ns = 0;
+};
+
 // bf16 forward on tcgen05 tensor cores (fp32 accumulation in TMEM).
-// err_word is the library's device error word (set when a bounded wait runs out).
 cudaError_t launch_forward_bf16(const int32_t* nbr, const uint32_t* tile_mask, int64_t n,
                                 const void* feats, const void* weight, void* out, int32_t cin,
                                 int32_t cout, int32_t flip, const Epilogue& epi,
-                                int32_t* err_word, cudaStream_t stream);
+                                const DeviceCtl& ctl, cudaStream_t stream);
 
 // bf16 forward over the x-run position layout (forward_bf16_runs_sm100.cu);
 // Cin a multiple of 64, Cout a multiple of 16.
 cudaError_t launch_forward_bf16_runs(const int32_t* pos, const int32_t* etable,
-                                     const int32_t* header, int64_t max_tiles, const void* feats,
+                                     int64_t et_stride, const int32_t* header, int64_t max_tiles,
+                                     const void* feats,
                                      const void* weight, void* out, int32_t cin, int32_t cout,
-                                     int32_t flip, const Epilogue& epi, int32_t* err_word,
+                                     int32_t flip, const Epilogue& epi, const DeviceCtl& ctl,
                                      cudaStream_t stream);
 
 // Backward (backward.cu): W [cout][27][cin] -> W^T [cin][27][cout]; and the
@@ -157,9 +171,9 @@ cudaError_t launch_wgrad(const int32_t* nbr, int64_t n, const void* x, const voi
 // bf16 weight gradient over the x-run layout on tcgen05 (wgrad_bf16_runs_sm100.cu):
 // Cin a multiple of 64, Cout a multiple of 16; zeroes dw, then accumulates.
 cudaError_t launch_wgrad_bf16_runs(const int32_t* pos, const int32_t* etable,
-                                   const int32_t* header, const void* feats, const void* dy,
+                                   int64_t et_stride, const int32_t* header, const void* feats, const void* dy,
                                    float* dw, int32_t cin, int32_t cout, int32_t flip,
-                                   int32_t* err_word, cudaStream_t stream);
+                                   const DeviceCtl& ctl, cudaStream_t stream);
 
 // Resolution changes (resample.cu).  Expansion: subdivide (C-order children,
 // replicated rows), upsample (masked, axis-0-fastest children, replicated) and

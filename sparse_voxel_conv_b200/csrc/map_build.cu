@@ -4,12 +4,14 @@
 // (lato.2_mrp_mlx, commit 97dcdfb54a message).  Here the lookup structure is
 // one of two GPU tables over packed (b, z, y, x) keys, chosen per call:
 //
-//   direct  when batch * grid_dim^3 int32 cells take at most max(64 MB,
+//   direct  when batch * (grid_dim + 2)^3 int32 cells take at most max(64 MB,
 //           256 B x N) and 2^28 cells (every 128^3 volume; 4 x 256^3 from
-//           about a million voxels): cell -> row, -1 when empty.  A collision-free perfect
-//           hash: insert is one plain store per voxel, a lookup is one load,
-//           and voxels adjacent in raster order look up adjacent cells, so the
-//           27 lookups of a warp coalesce.  A duplicate coordinate leaves one
+//           about a million voxels): cell -> row, -1 when empty; each grid has
+//           a one-cell border no voxel occupies, so a voxel's 27 neighbour
+//           cells all exist and its lookups need no bounds test.  A
+//           collision-free perfect hash: insert is one plain store per voxel,
+//           a lookup is one load, and voxels adjacent in raster order look up
+//           adjacent cells, so the 27 lookups of a warp coalesce.  A duplicate coordinate leaves one
 //           of its rows in the cell; the other row sees a foreign row at its
 //           own centre offset and raises the duplicate flag.
 //   hash    otherwise: open addressing with linear probing, capacity a power
@@ -21,11 +23,18 @@
 //           x-neighbours of a voxel usually share a 32-byte sector.  Probe
 //           loops are bounded by the capacity; a full table raises a flag.
 //
-// Kernels: map_init (table <- empty, status <- 0), map_insert (one thread per
-// voxel: 16-byte coordinate load, range check, insert), map_query (one block
-// per 128-row tile, one thread per voxel: 27 lookups into shared memory, then
-// the [128, 27] block and the tile's offset mask are written with coalesced
-// stores; no atomics on the output; and the tile's share of the x-run layout).
+// Kernels (each launched with programmatic dependent launch, so that its
+// blocks start while the previous kernel drains and do whatever touches only
+// the build's inputs before griddepcontrol.wait):
+//   map_init    table <- empty, run-count sums, status word and header <- 0;
+//   map_insert  one thread per voxel: 16-byte coordinate load, range check and
+//               the run starts of its 128-row tile (before the wait), then the
+//               insert;
+//   map_query   one block per 128-row tile, one thread per voxel: the 27
+//               lookups go to shared memory, then one bulk asynchronous copy
+//               writes the tile's [128, 27] nbr block and one store its offset
+//               mask (no atomics on the output), and the tile's share of the
+//               x-run layout.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -75,176 +84,167 @@ __device__ __forceinline__ bool x_next(int4 a, int4 b) {  // b is a's x+1 neighb
   return a.x == b.x && a.y == b.y && a.z == b.z && a.w + 1 == b.w;
 }
 
-// Called by all kInsertThreads threads of an insert block; c = coords[i] for i < n.
-__device__ __forceinline__ void count_run_starts(const int4* __restrict__ coords, int64_t n,
-                                                 int64_t i, int4 c, const RunCount& rc) {
+// The row before and the row after row i (lanes take them from their
+// neighbours; the warp's first and last lanes load them).
+__device__ __forceinline__ int4 shfl_up_int4(int4 c, int lane, const int4* coords, int i) {
+  int4 p;
+  p.x = __shfl_up_sync(0xFFFFFFFFu, c.x, 1);
+  p.y = __shfl_up_sync(0xFFFFFFFFu, c.y, 1);
+  p.z = __shfl_up_sync(0xFFFFFFFFu, c.z, 1);
+  p.w = __shfl_up_sync(0xFFFFFFFFu, c.w, 1);
+  if (lane == 0) p = i > 0 ? __ldg(coords + i - 1) : make_int4(-1, -1, -1, -1);
+  return p;
+}
+__device__ __forceinline__ int4 shfl_down_int4(int4 c, int lane, const int4* coords, int i,
+                                               int n) {
+  int4 q;
+  q.x = __shfl_down_sync(0xFFFFFFFFu, c.x, 1);
+  q.y = __shfl_down_sync(0xFFFFFFFFu, c.y, 1);
+  q.z = __shfl_down_sync(0xFFFFFFFFu, c.z, 1);
+  q.w = __shfl_down_sync(0xFFFFFFFFu, c.w, 1);
+  if (lane == 31) q = i + 1 < n ? __ldg(coords + i + 1) : make_int4(-1, -1, -1, -1);
+  return q;
+}
+
+// The coordinates of row i (i < n) or -1s, with the run-start counts of its
+// insert block written (before the kernel's wait: they depend on the
+// coordinates only).  Returns the block's run-start total in thread 0.
+__device__ __forceinline__ int32_t insert_prologue(const int4* __restrict__ coords, int n, int i,
+                                                   int4 c, const RunCount& rc) {
   __shared__ int32_t s_cnt[kInsertThreads / 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int4 prev;
-  prev.x = __shfl_up_sync(0xFFFFFFFFu, c.x, 1);
-  prev.y = __shfl_up_sync(0xFFFFFFFFu, c.y, 1);
-  prev.z = __shfl_up_sync(0xFFFFFFFFu, c.z, 1);
-  prev.w = __shfl_up_sync(0xFFFFFFFFu, c.w, 1);
-  if (lane == 0 && i > 0 && i < n) prev = __ldg(coords + i - 1);
-  const bool starts = i < n && (i == 0 || !x_next(prev, c));
+  const int4 prev = shfl_up_int4(c, lane, coords, i);
+  const bool starts = i < n && !x_next(prev, c);
   const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, starts);
   if (lane == 0) s_cnt[warp] = __popc(ballot);
   __syncthreads();
   if (threadIdx.x < 2) {
     const int h = threadIdx.x * 4;
-    const int64_t tile = static_cast<int64_t>(blockIdx.x) * 2 + threadIdx.x;
+    const int tile = blockIdx.x * 2 + threadIdx.x;
     if (tile * kTileRows < n) rc.cnt[tile] = s_cnt[h] + s_cnt[h + 1] + s_cnt[h + 2] + s_cnt[h + 3];
   }
-  if (threadIdx.x == 0) {
-    int32_t total = 0;
+  int32_t total = 0;
+  if (threadIdx.x == 0)
 #pragma unroll
     for (int w = 0; w < kInsertThreads / 32; ++w) total += s_cnt[w];
-    if (total) atomicAdd(rc.sb + (static_cast<int64_t>(blockIdx.x) * 2) / kSuperTiles, total);
-  }
+  return total;
 }
 
-__global__ void map_insert_direct(const int4* __restrict__ coords, int64_t n, int grid, int batch,
-                                  int32_t* __restrict__ cells, uint32_t* status,
-                                  RunCount rc) {
-  pdl_wait();
-  pdl_trigger();
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+template <Kind K>
+__global__ void __launch_bounds__(kInsertThreads)
+    map_insert(const int4* __restrict__ coords, int n, int grid, int batch, Tables t,
+               int32_t* __restrict__ cells, unsigned long long* __restrict__ table,
+               int32_t* __restrict__ rows, uint32_t* status, RunCount rc) {
+  const int i = blockIdx.x * kInsertThreads + threadIdx.x;
   const int4 c = i < n ? __ldg(coords + i) : make_int4(-1, -1, -1, -1);
-  if (rc.cnt) count_run_starts(coords, n, i, c, rc);
+  const int32_t total = rc.cnt ? insert_prologue(coords, n, i, c, rc) : 0;
+  pdl_wait();  // the table and the superblock sums are cleared
+  pdl_trigger();
+  if (total) atomicAdd(rc.sb + (blockIdx.x * 2) / kSuperTiles, total);
   if (i >= n) return;
   if (!in_volume(c, grid, batch)) {
     atomicOr(status, kErrRange);
     return;
   }
-  cells[cell_of(c.x, c.y, c.z, c.w, grid)] = static_cast<int32_t>(i);
-}
-
-__global__ void map_insert_compact(const int4* __restrict__ coords, int64_t n, int grid, int batch,
-                                   unsigned long long* __restrict__ table, uint32_t capmask,
-                                   uint32_t* status, RunCount rc) {
-  pdl_wait();
-  pdl_trigger();
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int4 c = i < n ? __ldg(coords + i) : make_int4(-1, -1, -1, -1);
-  if (rc.cnt) count_run_starts(coords, n, i, c, rc);
-  if (i >= n) return;
-  if (!in_volume(c, grid, batch)) {
-    atomicOr(status, kErrRange);
-    return;
-  }
-  const uint32_t key = pack32(c.x, c.y, c.z, c.w);
-  const unsigned long long entry =
-      (static_cast<unsigned long long>(key) << 32) | static_cast<uint32_t>(i);
-  uint32_t slot = home32(key, capmask);
-  for (uint64_t step = 0; step <= capmask; ++step) {
-    const unsigned long long prev = atomicCAS(table + slot, kEmpty, entry);
-    if (prev == kEmpty) return;
-    if (static_cast<uint32_t>(prev >> 32) == key) {
-      atomicOr(status, kErrDuplicate);
-      return;
+  if constexpr (K == Kind::kDirect) {
+    cells[cell_of(c.x, c.y, c.z, c.w, grid)] = i;
+  } else if constexpr (K == Kind::kCompact) {
+    const uint32_t key = pack32(c.x, c.y, c.z, c.w);
+    const unsigned long long entry =
+        (static_cast<unsigned long long>(key) << 32) | static_cast<uint32_t>(i);
+    uint32_t slot = home32(key, t.capmask);
+    for (uint64_t step = 0; step <= t.capmask; ++step) {
+      const unsigned long long prev = atomicCAS(table + slot, kEmpty, entry);
+      if (prev == kEmpty) return;
+      if (static_cast<uint32_t>(prev >> 32) == key) {
+        atomicOr(status, kErrDuplicate);
+        return;
+      }
+      slot = (slot + 1) & t.capmask;
     }
-    slot = (slot + 1) & capmask;
-  }
-  atomicOr(status, kErrTableFull);
-}
-
-__global__ void map_insert_wide(const int4* __restrict__ coords, int64_t n, int grid, int batch,
-                                unsigned long long* __restrict__ keys, int32_t* __restrict__ rows,
-                                uint32_t capmask, uint32_t* status, RunCount rc) {
-  pdl_wait();
-  pdl_trigger();
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int4 c = i < n ? __ldg(coords + i) : make_int4(-1, -1, -1, -1);
-  if (rc.cnt) count_run_starts(coords, n, i, c, rc);
-  if (i >= n) return;
-  if (!in_volume(c, grid, batch)) {
-    atomicOr(status, kErrRange);
-    return;
-  }
-  const unsigned long long key = pack64(c.x, c.y, c.z, c.w);
-  uint32_t slot = home64(key, capmask);
-  for (uint64_t step = 0; step <= capmask; ++step) {
-    const unsigned long long prev = atomicCAS(keys + slot, kEmpty, key);
-    if (prev == kEmpty) {
-      rows[slot] = static_cast<int32_t>(i);
-      return;
+    atomicOr(status, kErrTableFull);
+  } else {
+    const unsigned long long key = pack64(c.x, c.y, c.z, c.w);
+    uint32_t slot = home64(key, t.capmask);
+    for (uint64_t step = 0; step <= t.capmask; ++step) {
+      const unsigned long long prev = atomicCAS(table + slot, kEmpty, key);
+      if (prev == kEmpty) {
+        rows[slot] = i;
+        return;
+      }
+      if (prev == key) {
+        atomicOr(status, kErrDuplicate);
+        return;
+      }
+      slot = (slot + 1) & t.capmask;
     }
-    if (prev == key) {
-      atomicOr(status, kErrDuplicate);
-      return;
-    }
-    slot = (slot + 1) & capmask;
+    atomicOr(status, kErrTableFull);
   }
-  atomicOr(status, kErrTableFull);
 }
 
 // ----------------------------------------------------------- run layout ----
 // The query kernel also lays out the x-run positions: with R(v) the run starts
 // among rows 0..v, voxel v sits at position v + 2 R(v), its run's left pad (when
 // v starts the run) at the position before, the right pad (when v ends it) at
-// the one after.
+// the one after.  E row q of pair dz-dy is entry q + 1 of that pair's line.
 
-static_assert(kPosTile == 256, "et_store_row splits positions with shifts by 8");
 static_assert(kInsertThreads == 256 && kSuperTiles % 2 == 0, "insert block = two query tiles");
 
 struct RunOut {
   const int32_t* cnt;  // run starts per 128-row tile (insert kernel)
   const int32_t* sb;   // run starts per superblock of 128 tiles (insert kernel)
-  int32_t* hdr;        // [4]: runs, position tiles, positions, 0
+  int32_t* hdr;        // [4]: runs, position tiles, positions, E line stride
   int32_t* pos;        // position table
-  int32_t* et;         // E index table
+  int32_t* et;         // E index table: 9 lines of `es` entries
+  int32_t es;          // E line stride (entries)
 };
 
-// E row q of offset pair dzdy is entry (q mod 256) + 1 of tile q / 256; a tile
-// also keeps copies of its edge rows' outer neighbours (entry 0 of the next
-// tile is row 255 of this one; entry 257 of the previous tile is row 0).
-// Writes E row q for all 9 pairs, the value of pair dzdy being v[3 * dzdy].
-__device__ __forceinline__ void et_store_row(int32_t* et, int64_t q, const int32_t* v) {
-  const int64_t t = q >> 8;
-  const int i = static_cast<int>(q & 255);
-  int32_t* b = et + t * (9 * kEtStride) + i + 1;
-#pragma unroll
-  for (int dzdy = 0; dzdy < 9; ++dzdy) b[dzdy * kEtStride] = v[3 * dzdy];
-  if (i == kPosTile - 1 || (i == 0 && t > 0)) {  // one row in 128
-    int32_t* h = i == 0 ? et + (t - 1) * (9 * kEtStride) + kPosTile + 1
-                        : et + (t + 1) * (9 * kEtStride);
-#pragma unroll
-    for (int dzdy = 0; dzdy < 9; ++dzdy) h[dzdy * kEtStride] = v[3 * dzdy];
-  }
+__device__ __forceinline__ void bulk_store_smem(void* gdst, const void* ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
+               "r"(static_cast<uint32_t>(__cvta_generic_to_shared(ssrc))), "r"(bytes)
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
 // One block per 128-row tile, one thread per voxel: 27 lookups into shared
-// memory, then the [128, 27] nbr block and the tile's offset mask with
-// coalesced stores.  With RUNS, also the tile's positions and E index entries.
+// memory, then the [128, 27] nbr block (one bulk copy for a whole tile) and the
+// tile's offset mask.  With RUNS, also the tile's positions and E entries.
 template <Kind K, bool RUNS>
 __global__ void __launch_bounds__(kTileRows)
-    map_query(const int4* __restrict__ coords, int64_t n, int grid, int batch, Tables t,
+    map_query(const int4* __restrict__ coords, int n, int grid, int batch, Tables t,
               int32_t* __restrict__ nbr, uint32_t* __restrict__ tile_mask, uint32_t* status,
               RunOut ro) {
-  __shared__ __align__(16) int32_t s_nbr[kTileRows * kKvol];
+  __shared__ __align__(128) int32_t s_nbr[kTileRows * kKvol];
   __shared__ uint32_t s_bits[kTileRows / 32];
   __shared__ uint32_t s_starts[kTileRows / 32];  // run-start ballot of each warp
   __shared__ int32_t s_before[kTileRows / 32];   // partial sums of the run starts before the tile
-  __shared__ int64_t s_end;
+  __shared__ int32_t s_end;
   const int r = threadIdx.x;
   const int lane = r & 31, warp = r >> 5;
-  pdl_wait();
-  pdl_trigger();
-  const int64_t tile = blockIdx.x;
-  const int64_t row0 = tile * kTileRows;
-  const int64_t i = row0 + r;
-  int4 c = make_int4(-1, -1, -1, -1);
-  if (i < n) c = __ldg(coords + i);
+  const int tile = blockIdx.x;
+  const int row0 = tile * kTileRows;
+  const int i = row0 + r;
+  const bool live = i < n;
+  // the coordinates are the build's input: read before the wait for the table
+  const int4 c = live ? __ldg(coords + i) : make_int4(-1, -1, -1, -1);
   bool starts = false, ends = false;
   if constexpr (RUNS) {
-    if (i < n) {
-      starts = i == 0 || !x_next(__ldg(coords + i - 1), c);
-      ends = i == n - 1 || !x_next(c, __ldg(coords + i + 1));
-    }
-    const int64_t sb = tile / kSuperTiles;
+    // the same rule as the insert kernel's count, so positions match the counts
+    const int4 prev = shfl_up_int4(c, lane, coords, i);
+    const int4 next = shfl_down_int4(c, lane, coords, i, n);
+    starts = live && !x_next(prev, c);
+    ends = live && !x_next(c, next);
+  }
+  pdl_wait();  // the table, the run counts and the superblock sums are complete
+  pdl_trigger();
+  if constexpr (RUNS) {
+    const int sb = tile / kSuperTiles;
     int32_t part = 0;
-    for (int64_t j = r; j < sb; j += kTileRows) part += __ldg(ro.sb + j);
-    for (int64_t j = sb * kSuperTiles + r; j < tile; j += kTileRows) part += __ldg(ro.cnt + j);
+    for (int j = r; j < sb; j += kTileRows) part += __ldg(ro.sb + j);
+    for (int j = sb * kSuperTiles + r; j < tile; j += kTileRows) part += __ldg(ro.cnt + j);
     part = __reduce_add_sync(0xFFFFFFFFu, part);
     const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, starts);
     if (lane == 0) {
@@ -252,116 +252,129 @@ __global__ void __launch_bounds__(kTileRows)
       s_before[warp] = part;
     }
   }
-  uint32_t bits = 0u;
-  if (i < n) {
+  int32_t* nb = s_nbr + r * kKvol;
+  uint32_t absent = 0u;  // bit 26 - k set when offset k has no neighbour
+  if (live) {
     if (in_volume(c, grid, batch)) {
       if constexpr (K == Kind::kDirect) {
-        // the direct table has <= 2^28 cells: int32 cell indices.  The 9 (dz, dy)
-        // rows are base pointers; dx = -1, 0, +1 are the cells before and after.
-        const int32_t g = grid, g2 = grid * grid;
-        const int32_t* centre = t.cells + (((c.x * g + c.y) * g + c.z) * g + c.w);
-        const bool vz[3] = {c.y > 0, true, c.y < g - 1};
-        const bool vy[3] = {c.z > 0, true, c.z < g - 1};
-        const bool vx[3] = {c.w > 0, true, c.w < g - 1};
+        // the bordered table has <= 2^28 cells: int32 cell indices; every one of
+        // the 27 cells exists.  Rows (dz, dy) are base pointers, dx = -1, 0, +1
+        // the cells before and after.
+        const int32_t g = grid + 2, g2 = g * g;
+        const int32_t* centre = t.cells + (((c.x * g + c.y + 1) * g + c.z + 1) * g + c.w + 1);
 #pragma unroll
         for (int dz = 0; dz < 3; ++dz) {
 #pragma unroll
           for (int dy = 0; dy < 3; ++dy) {
-            const int32_t* row = centre + (dz - 1) * g2 + (dy - 1) * g;
+            const int32_t* row = centre + ((dz - 1) * g2 + (dy - 1) * g);
 #pragma unroll
             for (int dx = 0; dx < 3; ++dx) {
-              const int k = dz * 9 + dy * 3 + dx;
-              const int32_t found = (vz[dz] && vy[dy] && vx[dx]) ? __ldg(row + dx - 1) : -1;
-              s_nbr[r * kKvol + k] = found;
-              bits |= (found >= 0 ? 1u : 0u) << k;
+              const int32_t v = __ldg(row + dx - 1);
+              nb[dz * 9 + dy * 3 + dx] = v;
+              absent = __funnelshift_l(static_cast<uint32_t>(v), absent, 1);  // sign bit in
             }
           }
         }
-        if (s_nbr[r * kKvol + 13] != static_cast<int32_t>(i))
-          atomicOr(status, kErrDuplicate);  // another row owns this voxel's cell
+        if (nb[13] != i) atomicOr(status, kErrDuplicate);  // another row owns this cell
       } else {
 #pragma unroll
         for (int k = 0; k < kKvol; ++k) {
           const int z = c.y + k / 9 - 1;
           const int y = c.z + (k / 3) % 3 - 1;
           const int x = c.w + k % 3 - 1;
-          int32_t found = -1;
+          int32_t v = -1;
           if (static_cast<unsigned>(z) < static_cast<unsigned>(grid) &&
               static_cast<unsigned>(y) < static_cast<unsigned>(grid) &&
               static_cast<unsigned>(x) < static_cast<unsigned>(grid))
-            found = lookup<K>(t, c.x, z, y, x, grid);
-          s_nbr[r * kKvol + k] = found;
-          bits |= (found >= 0 ? 1u : 0u) << k;
+            v = lookup<K>(t, c.x, z, y, x, grid);
+          nb[k] = v;
+          absent = __funnelshift_l(static_cast<uint32_t>(v), absent, 1);
         }
       }
     } else {
 #pragma unroll
-      for (int k = 0; k < kKvol; ++k) s_nbr[r * kKvol + k] = -1;
+      for (int k = 0; k < kKvol; ++k) nb[k] = -1;
+      absent = (1u << kKvol) - 1u;
     }
-  }
-  bits = __reduce_or_sync(0xFFFFFFFFu, bits);
-  if (lane == 0) s_bits[warp] = bits;
-  __syncthreads();
-  if (r == 0) tile_mask[tile] = s_bits[0] | s_bits[1] | s_bits[2] | s_bits[3];
-  const int rows = static_cast<int>(n - row0 < kTileRows ? n - row0 : kTileRows);
-  int32_t* dst = nbr + row0 * kKvol;
-  if (rows == kTileRows) {
-    // 13824 bytes = 864 16-byte words; each tile's nbr block starts 16-byte aligned
-    const int4* src4 = reinterpret_cast<const int4*>(s_nbr);
-    int4* dst4 = reinterpret_cast<int4*>(dst);
-    for (int e = r; e < kTileRows * kKvol / 4; e += kTileRows) dst4[e] = src4[e];
   } else {
+    absent = (1u << kKvol) - 1u;
+  }
+  // bit k of the mask: offset k present somewhere in the tile
+  const uint32_t present = __brev(~absent << (32 - kKvol)) & ((1u << kKvol) - 1u);
+  const uint32_t bits = __reduce_or_sync(0xFFFFFFFFu, present);
+  if (lane == 0) s_bits[warp] = bits;
+  const int rows = n - row0 < kTileRows ? n - row0 : kTileRows;
+  if (rows == kTileRows)
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // nb -> the bulk copy
+  __syncthreads();
+  if (r == 0) {
+    tile_mask[tile] = s_bits[0] | s_bits[1] | s_bits[2] | s_bits[3];
+    // 13,824 bytes = 864 16-byte words; each tile's block starts 16-byte aligned
+    if (rows == kTileRows)
+      bulk_store_smem(nbr + static_cast<int64_t>(row0) * kKvol, s_nbr, kTileRows * kKvol * 4);
+  }
+  if (rows < kTileRows) {
+    int32_t* dst = nbr + static_cast<int64_t>(row0) * kKvol;
     for (int e = r; e < rows * kKvol; e += kTileRows) dst[e] = s_nbr[e];
   }
-  if constexpr (!RUNS) return;
-  // (the __syncthreads above also published s_starts and s_before)
-  const int64_t excl = static_cast<int64_t>(s_before[0]) + s_before[1] + s_before[2] + s_before[3];
-  const uint32_t agg = __popc(s_starts[0]) + __popc(s_starts[1]) + __popc(s_starts[2]) +
-                       __popc(s_starts[3]);
-  int64_t runs = excl;  // run starts among rows 0..i
-  for (int w = 0; w < warp; ++w) runs += __popc(s_starts[w]);
-  runs += __popc(s_starts[warp] & (0xFFFFFFFFu >> (31 - lane)));
-  if (i < n) {
-    const int64_t p = i + 2 * runs;
-    const int32_t tag = static_cast<int32_t>(i * 4);
-    ro.pos[p] = tag + kPosVoxel;
-    if (starts) ro.pos[p - 1] = tag + kPosLeftPad;
-    if (ends) ro.pos[p + 1] = tag + kPosRightPad;
-    const int32_t* nb = s_nbr + r * kKvol;  // nb[3 * dzdy + dx + 1]
-    et_store_row(ro.et, p, nb + 1);
-    if (starts) et_store_row(ro.et, p - 1, nb);
-    if (ends) et_store_row(ro.et, p + 1, nb + 2);
-    if (i == 0) {  // position 0 (the absent right pad before the first run) and row -1
-      ro.pos[0] = -1;
+  if constexpr (RUNS) {
+    // (the __syncthreads above also published s_starts and s_before)
+    const int32_t excl = s_before[0] + s_before[1] + s_before[2] + s_before[3];
+    const int32_t agg = __popc(s_starts[0]) + __popc(s_starts[1]) + __popc(s_starts[2]) +
+                        __popc(s_starts[3]);
+    int32_t runs = excl;  // run starts among rows 0..i
+    for (int w = 0; w < warp; ++w) runs += __popc(s_starts[w]);
+    runs += __popc(s_starts[warp] & (0xFFFFFFFFu >> (31 - lane)));
+    const int es = ro.es;
+    if (live) {
+      const int p = i + 2 * runs;
+      const int32_t tag = i * 4;
+      ro.pos[p] = tag + kPosVoxel;
+      if (starts) ro.pos[p - 1] = tag + kPosLeftPad;
+      if (ends) ro.pos[p + 1] = tag + kPosRightPad;
+      // E row p of pair dz-dy is the voxel's (dz, dy, 0) neighbour; its left pad
+      // (row p - 1) the (dz, dy, -1) one, its right pad (row p + 1) the (dz, dy, +1)
+      int32_t* e = ro.et + (p + 1);
 #pragma unroll
-      for (int dzdy = 0; dzdy < 9; ++dzdy) {
-        ro.et[dzdy * kEtStride] = -1;
-        ro.et[dzdy * kEtStride + 1] = -1;
+      for (int dzdy = 0; dzdy < 9; ++dzdy) e[dzdy * es] = nb[3 * dzdy + 1];
+      if (starts)
+#pragma unroll
+        for (int dzdy = 0; dzdy < 9; ++dzdy) e[dzdy * es - 1] = nb[3 * dzdy];
+      if (ends)
+#pragma unroll
+        for (int dzdy = 0; dzdy < 9; ++dzdy) e[dzdy * es + 1] = nb[3 * dzdy + 2];
+      if (i == 0) {  // position 0 (the absent right pad before the first run) and row -1
+        ro.pos[0] = -1;
+#pragma unroll
+        for (int dzdy = 0; dzdy < 9; ++dzdy) {
+          ro.et[dzdy * es] = -1;
+          ro.et[dzdy * es + 1] = -1;
+        }
+      }
+      if (i == n - 1) s_end = p + 2;  // one past the last run's right pad
+    }
+    if (row0 + kTileRows >= n) {  // the tile of row n-1: header, and the line's tail
+      __syncthreads();
+      // positions up to the last voxel: N + 2 runs - 1 (the last right pad, at
+      // position `end` - 1, is read only as E row 256 of the last tile when it
+      // falls there, and its entry is written above)
+      const int end = s_end;
+      const int positions = end - 1;
+      const int ptiles = (positions + kPosTile - 1) / kPosTile;
+      if (r == 0) {
+        ro.hdr[0] = excl + agg;
+        ro.hdr[1] = ptiles;
+        ro.hdr[2] = positions;
+        ro.hdr[3] = es;
+      }
+      for (int q = end + r; q <= ptiles * kPosTile; q += kTileRows) {
+        if (q < ptiles * kPosTile) ro.pos[q] = -1;
+#pragma unroll
+        for (int dzdy = 0; dzdy < 9; ++dzdy) ro.et[dzdy * es + q + 1] = -1;
       }
     }
-    if (i == n - 1) s_end = p + 2;  // one past the last run's right pad
   }
-  if (row0 + kTileRows >= n) {  // the tile of row n-1: header, and the line's tail
-    __syncthreads();
-    // positions up to the last voxel: N + 2 runs; the last right pad is not counted,
-    // as its only reader, row 256 of its voxel's tile, holds a copy of it
-    const int64_t end = s_end;
-    const int64_t positions = end - 1;
-    const int64_t ptiles = (positions + kPosTile - 1) / kPosTile;
-    if (r == 0) {
-      ro.hdr[0] = static_cast<int32_t>(excl + agg);
-      ro.hdr[1] = static_cast<int32_t>(ptiles);
-      ro.hdr[2] = static_cast<int32_t>(positions);
-      ro.hdr[3] = 0;
-    }
-    int32_t none[kKvol];
-#pragma unroll
-    for (int k = 0; k < kKvol; ++k) none[k] = -1;
-    for (int64_t q = end + r; q <= ptiles * kPosTile; q += kTileRows) {
-      if (q < ptiles * kPosTile) ro.pos[q] = -1;
-      et_store_row(ro.et, q, none);
-    }
-  }
+  if (r == 0 && rows == kTileRows) bulk_wait_read();  // s_nbr stays until the copy has read it
 }
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -370,11 +383,12 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 bool map_layout(int64_t n, int32_t grid_dim, int32_t batch, const MapOptions& opt,
                 MapLayout* out) {
-  if (n < 0 || n >= 0x7FFFFFFFll || grid_dim < 1 || grid_dim > 65535 || batch < 1 ||
+  if (n < 0 || n >= kMaxMapRows || grid_dim < 1 || grid_dim > 65535 || batch < 1 ||
       batch > 65535)
     return false;
   MapLayout lay;
-  const double cells = static_cast<double>(batch) * grid_dim * grid_dim * grid_dim;
+  const double gb = static_cast<double>(grid_dim) + 2.0;  // bordered grid
+  const double cells = static_cast<double>(batch) * gb * gb * gb;
   const double direct_budget = std::max(static_cast<double>(kDirectTableMinBytes),
                                         kDirectTableBytesPerVoxel * static_cast<double>(n));
   const bool direct_fits = cells * 4.0 <= direct_budget && cells <= kDirectTableMaxCells;
@@ -411,6 +425,7 @@ bool map_layout(int64_t n, int32_t grid_dim, int32_t batch, const MapOptions& op
   }
   lay.pos_max = static_cast<int64_t>(align_up(static_cast<size_t>(3 * n), kPosTile)) + kPosTile;
   lay.ptile_max = lay.pos_max / kPosTile;
+  lay.et_stride = lay.pos_max + 4;  // entries for positions -1 .. pos_max, 16-byte lines
   lay.cnt_off = end;
   lay.sb_off = align_up(lay.cnt_off + static_cast<size_t>(lay.n_tiles) * 4, 256);
   const int64_t n_super = (lay.n_tiles + kSuperTiles - 1) / kSuperTiles;
@@ -418,7 +433,7 @@ bool map_layout(int64_t n, int32_t grid_dim, int32_t batch, const MapOptions& op
   lay.pos_off = lay.hdr_off + 256;
   lay.pos_bytes = static_cast<size_t>(lay.pos_max) * 4;
   lay.et_off = align_up(lay.pos_off + lay.pos_bytes, 256);
-  lay.total = align_up(lay.et_off + static_cast<size_t>(lay.ptile_max) * 9 * kEtStride * 4, 256);
+  lay.total = align_up(lay.et_off + static_cast<size_t>(9 * lay.et_stride) * 4, 256);
   *out = lay;
   return true;
 }
@@ -426,14 +441,18 @@ bool map_layout(int64_t n, int32_t grid_dim, int32_t batch, const MapOptions& op
 namespace {
 
 template <Kind K>
-void launch_query(unsigned blocks, bool runs, const int4* c4, int64_t n, int grid, int batch,
-                  const Tables& t, int32_t* nbr, uint32_t* mask, uint32_t* status,
-                  const RunOut& ro, cudaStream_t stream) {
+void launch_build_kernels(unsigned ins_blocks, unsigned q_blocks, bool runs, const int4* c4,
+                          int n, int grid, int batch, const Tables& t, int32_t* cells,
+                          unsigned long long* table, int32_t* rows, int32_t* nbr, uint32_t* mask,
+                          uint32_t* status, const RunCount& rc, const RunOut& ro,
+                          cudaStream_t stream) {
+  launch_pdl(map_insert<K>, ins_blocks, kInsertThreads, 0, stream, c4, n, grid, batch, t, cells,
+             table, rows, status, rc);
   if (runs)
-    launch_pdl(map_query<K, true>, blocks, kTileRows, 0, stream, c4, n, grid, batch, t, nbr, mask,
-               status, ro);
+    launch_pdl(map_query<K, true>, q_blocks, kTileRows, 0, stream, c4, n, grid, batch, t, nbr,
+               mask, status, ro);
   else
-    launch_pdl(map_query<K, false>, blocks, kTileRows, 0, stream, c4, n, grid, batch, t, nbr,
+    launch_pdl(map_query<K, false>, q_blocks, kTileRows, 0, stream, c4, n, grid, batch, t, nbr,
                mask, status, ro);
 }
 
@@ -442,6 +461,7 @@ void launch_query(unsigned blocks, bool runs, const int4* c4, int64_t n, int gri
 cudaError_t launch_map_build(const int32_t* coords, int64_t n, int32_t grid_dim, int32_t batch,
                              int32_t* nbr, void* workspace, const MapLayout& lay,
                              cudaStream_t stream) {
+  if (n < 0 || n >= kMaxMapRows) return cudaErrorInvalidValue;
   auto* ws = static_cast<uint8_t*>(workspace);
   auto* status = reinterpret_cast<uint32_t*>(ws + lay.status_off);
   auto* mask = reinterpret_cast<uint32_t*>(ws + lay.mask_off);
@@ -458,6 +478,7 @@ cudaError_t launch_map_build(const int32_t* coords, int64_t n, int32_t grid_dim,
     ro.hdr = reinterpret_cast<int32_t*>(ws + lay.hdr_off);
     ro.pos = reinterpret_cast<int32_t*>(ws + lay.pos_off);
     ro.et = reinterpret_cast<int32_t*>(ws + lay.et_off);
+    ro.es = static_cast<int32_t>(lay.et_stride);
     sb_words16 = (lay.hdr_off - lay.sb_off) / 16;  // the 256-byte aligned superblock region
   }
   const size_t words16 = lay.table_bytes / 16;
@@ -472,30 +493,28 @@ cudaError_t launch_map_build(const int32_t* coords, int64_t n, int32_t grid_dim,
   }
   if (n == 0) return cudaGetLastError();
   const auto* c4 = reinterpret_cast<const int4*>(coords);
+  const int ni = static_cast<int>(n);
   const unsigned ins_blocks = static_cast<unsigned>((n + kInsertThreads - 1) / kInsertThreads);
   const unsigned q_blocks = static_cast<unsigned>(lay.n_tiles);
   Tables t{};
   t.capmask = static_cast<uint32_t>(lay.capacity - 1);
   if (lay.kind == MapKind::kDirect) {
     t.cells = reinterpret_cast<const int32_t*>(table);
-    launch_pdl(map_insert_direct, ins_blocks, kInsertThreads, 0, stream, c4, n, grid_dim, batch,
-               reinterpret_cast<int32_t*>(table), status, rc);
-    launch_query<Kind::kDirect>(q_blocks, runs, c4, n, grid_dim, batch, t, nbr, mask, status, ro,
-                                stream);
+    launch_build_kernels<Kind::kDirect>(ins_blocks, q_blocks, runs, c4, ni, grid_dim, batch, t,
+                                        reinterpret_cast<int32_t*>(table), nullptr, nullptr, nbr,
+                                        mask, status, rc, ro, stream);
   } else if (lay.compact) {
     t.table = reinterpret_cast<const unsigned long long*>(table);
-    launch_pdl(map_insert_compact, ins_blocks, kInsertThreads, 0, stream, c4, n, grid_dim, batch,
-               reinterpret_cast<unsigned long long*>(table), t.capmask, status, rc);
-    launch_query<Kind::kCompact>(q_blocks, runs, c4, n, grid_dim, batch, t, nbr, mask, status,
-                                 ro, stream);
+    launch_build_kernels<Kind::kCompact>(ins_blocks, q_blocks, runs, c4, ni, grid_dim, batch, t,
+                                         nullptr, reinterpret_cast<unsigned long long*>(table),
+                                         nullptr, nbr, mask, status, rc, ro, stream);
   } else {
     auto* rows = reinterpret_cast<int32_t*>(ws + lay.rows_off);
     t.table = reinterpret_cast<const unsigned long long*>(table);
     t.rows = rows;
-    launch_pdl(map_insert_wide, ins_blocks, kInsertThreads, 0, stream, c4, n, grid_dim, batch,
-               reinterpret_cast<unsigned long long*>(table), rows, t.capmask, status, rc);
-    launch_query<Kind::kWide>(q_blocks, runs, c4, n, grid_dim, batch, t, nbr, mask, status, ro,
-                              stream);
+    launch_build_kernels<Kind::kWide>(ins_blocks, q_blocks, runs, c4, ni, grid_dim, batch, t,
+                                      nullptr, reinterpret_cast<unsigned long long*>(table), rows,
+                                      nbr, mask, status, rc, ro, stream);
   }
   return cudaGetLastError();
 }

@@ -1,5 +1,7 @@
 // The neighbour map's lookup structures (map_build.cu builds them): a
-// direct-address table of int32 rows over batch * grid^3 cells, or an
+// direct-address table of int32 rows over batch * (grid + 2)^3 cells (each
+// batch element's grid with a one-cell border that no voxel occupies, so all
+// 27 neighbour cells of a voxel exist and lookups need no bounds test), or an
 // open-addressing hash table with linear probing -- compact 8-byte slots
 // (key32 << 32 | row) when batch <= 4 and grid_dim <= 1024, else 64-bit keys
 // with a separate int32 row array.  The home slot is 4 * h(key >> 2) + (key & 3)
@@ -55,8 +57,11 @@ __device__ __forceinline__ bool in_volume(int4 c, int grid, int batch) {
          static_cast<unsigned>(c.w) < static_cast<unsigned>(grid);
 }
 
+// Cell of (b, z, y, x) in the bordered direct table: batch element b owns a
+// block of (grid + 2)^3 cells and the voxel sits one cell in from its faces.
 __device__ __forceinline__ int64_t cell_of(int b, int z, int y, int x, int grid) {
-  return ((static_cast<int64_t>(b) * grid + z) * grid + y) * grid + x;
+  const int64_t g = grid + 2;
+  return ((static_cast<int64_t>(b) * g + (z + 1)) * g + (y + 1)) * g + (x + 1);
 }
 
 enum class Kind { kDirect, kCompact, kWide };

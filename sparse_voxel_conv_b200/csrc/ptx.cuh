@@ -1,7 +1,9 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers, cp.async, TMA tiled loads,
 // tcgen05 (TMEM allocation, UMMA issue, commit, TMEM loads) and fences.
-// Every wait in this file is bounded: it gives up after kWaitLimitNs of
-// %globaltimer time, or as soon as the CTA's abort word is set.
+// Every wait in this file is bounded.  A pipeline wait gives up after the
+// CTA's limit (WaitCtl::limit_ns of %globaltimer time, kWaitLimitNs unless the
+// caller asked for another) or as soon as the CTA's abort word is set; a drain
+// wait on the abort path has its own limit, kDrainLimitNs.
 #pragma once
 
 #include <cstdint>
@@ -9,7 +11,29 @@
 
 namespace subm3d {
 
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: default limit of a pipeline wait
+constexpr uint64_t kDrainLimitNs = 1000000000ull;  // 1 s: limit of one drain wait
+
+// Per-CTA wait control, in shared memory.  The first pipeline wait that runs
+// out of time sets `abort`; from then on every pipeline wait of the CTA
+// returns false at once, each role leaves its loop, drains what it has issued
+// (mbar_drain) and the CTA exits through its normal teardown.
+struct WaitCtl {
+  int abort;
+  int pad;
+  unsigned long long limit_ns;
+};
+
+// Called by one thread before the CTA's first __syncthreads.
+__device__ __forceinline__ void wait_ctl_init(WaitCtl* w, uint64_t limit_ns) {
+  w->abort = 0;
+  w->pad = 0;
+  w->limit_ns = limit_ns;
+}
+
+__device__ __forceinline__ bool wait_aborted(const WaitCtl* w) {
+  return *reinterpret_cast<const volatile int*>(&w->abort) != 0;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -55,28 +79,66 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// One bounded-suspension poll: the thread sleeps at most about `hint_ns`
+// (or until the phase completes) before the call returns.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity,
+                                                   uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Suspension per poll of the slow paths: a quarter of the limit, between
+// 256 ns and 100 us, so that a limit is noticed within about a quarter of itself.
+__device__ __forceinline__ uint32_t poll_hint_ns(uint64_t limit_ns) {
+  const uint64_t q = limit_ns / 4;
+  return static_cast<uint32_t>(q < 256 ? 256 : (q > 100000 ? 100000 : q));
+}
+
 // Slow path of mbar_wait, kept out of line so that the many wait sites of a
-// warp-specialised kernel share one copy of the polling loop.
-static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// warp-specialised kernel share one copy of the polling loop.  The abort word
+// and the clock are checked after every poll.
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, WaitCtl* w) {
+  volatile WaitCtl* vw = w;
+  const uint64_t limit = vw->limit_ns;
+  const uint32_t hint = poll_hint_ns(limit);
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        *abort = 1;
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_hint(bar, parity, hint)) return true;
+    if (vw->abort) return false;
+    if (globaltimer_ns() - t0 > limit) {
+      vw->abort = 1;
+      return false;
     }
   }
 }
 
 // Waits for the phase of `bar` with the given parity to complete.  Returns
-// false (and sets *abort) when the wait exceeds kWaitLimitNs, or returns false
-// at once when another role of the CTA has already set *abort.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// false (and sets the abort word) when the wait exceeds the CTA's limit, or
+// returns false at once when another role of the CTA has already set it.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, WaitCtl* w) {
   if (mbar_try_wait(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity, abort);
+  return mbar_wait_slow(bar, parity, w);
+}
+
+// Abort path: waits for the phase of `bar` with the given parity to complete,
+// whatever the abort word says, for at most kDrainLimitNs.  A role calls it
+// for each asynchronous operation it issued (a TMA or bulk copy into shared
+// memory, a tcgen05.commit after its MMAs) before the CTA frees its tensor
+// memory and exits, so that nothing still writes shared or tensor memory the
+// CTA no longer owns.  Returns false if the limit ran out.
+static __device__ __noinline__ bool mbar_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    if (mbar_try_wait_hint(bar, parity, 100000)) return true;
+    if (globaltimer_ns() - t0 > kDrainLimitNs) return false;
+  }
 }
 
 __device__ __forceinline__ void sts_u32(uint32_t addr, uint32_t v) {
@@ -244,6 +306,25 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t m, uint32_t n) {
 // The same with both operands MN-major (A: bit 15, B: bit 16).
 __host__ __device__ constexpr uint32_t idesc_bf16_f32_mn(uint32_t m, uint32_t n) {
   return idesc_bf16_f32(m, n) | (1u << 15) | (1u << 16);
+}
+
+// ------------------------------------------------------------- abort path --
+
+// A TMA producer's drain: load m of the producer went to ring slot m % slots and
+// completes the phase of parity (m / slots) & 1 of full[slot]; the last
+// min(issued, slots) loads are the only ones that can still be in flight.
+__device__ __forceinline__ void drain_ring(uint64_t* full, int slots, int64_t issued) {
+  const int64_t first = issued > slots ? issued - slots : 0;
+  for (int64_t m = first; m < issued; ++m)
+    mbar_drain(&full[m % slots], static_cast<uint32_t>((m / slots) & 1));
+}
+
+// The MMA issuer's drain: tcgen05.commit tracks every tcgen05 operation the
+// thread issued before it, so one commit to `bar` (a count-1 barrier used for
+// nothing else) and a wait for its first phase cover all of them.
+__device__ __forceinline__ void drain_mma(uint64_t* bar) {
+  umma_commit(bar);
+  mbar_drain(bar, 0);
 }
 
 }  // namespace subm3d

@@ -71,6 +71,18 @@ int device_is_sm100(int* device_out) {
   return ok;
 }
 
+// Limit of each pipeline wait inside the tensor-core kernels: 2 s, or the
+// testing knob SUBM3D_WAIT_LIMIT_NS=<ns> (read at every call), with which a
+// test makes the waits run out and checks the timeout path.
+uint64_t wait_limit_from_env() {
+  const char* v = std::getenv("SUBM3D_WAIT_LIMIT_NS");
+  if (v && *v) {
+    const unsigned long long ns = std::strtoull(v, nullptr, 10);
+    if (ns > 0) return ns;
+  }
+  return 2000000000ull;
+}
+
 int32_t* device_error_word() {
   static std::mutex mu;
   static int32_t* addr[64] = {};
@@ -178,6 +190,20 @@ bool overlaps(const void* p, size_t p_bytes, const void* q, size_t q_bytes) {
   return a < b + q_bytes && b < a + p_bytes;
 }
 
+// Kernel choice for a map with an x-run layout: the x-run kernel.  It does
+// tensor work on every position (voxels and pads) for all 27 offsets, the
+// per-offset kernel on every voxel for the offsets present in its 256-row tile
+// but with ~3x the gathered bytes; timed with the GELU epilogue on three sets
+// (x-runs of 9.3 and 4.0 voxels, 1.22 and 1.50 positions per voxel) at 64 and
+// 128 input and output channels, the x-run kernel was faster in every case, by
+// 14% (4 x 256^3 shells, 64 -> 128) to 2.1x.
+// Testing knob SUBM3D_FORWARD_KERNEL (read at every call): "gather" takes the
+// per-offset kernel even where the x-run kernel applies.
+bool prefer_gather() {
+  const char* knob = std::getenv("SUBM3D_FORWARD_KERNEL");
+  return knob && std::strcmp(knob, "gather") == 0;
+}
+
 // The forward of every entry point: map may be null (nbr-only callers), in
 // which case the x-run kernel is not available.
 subm3d_status forward_impl(const subm3d_map* map, const int32_t* nbr, const uint32_t* tile_mask,
@@ -221,15 +247,18 @@ subm3d_status forward_impl(const subm3d_map* map, const int32_t* nbr, const uint
   const int sm100 = device_is_sm100(nullptr);
   if (sm100 < 0) return SUBM3D_E_CUDA;
   if (sm100 == 0) return SUBM3D_E_UNSUPPORTED;
-  int32_t* err = device_error_word();
-  if (!err) return SUBM3D_E_CUDA;
+  subm3d::DeviceCtl ctl;
+  ctl.err_word = device_error_word();
+  if (!ctl.err_word) return SUBM3D_E_CUDA;
+  ctl.wait_limit_ns = wait_limit_from_env();
   cudaError_t e;
-  if (map && map->pos && cin % 64 == 0)
-    e = subm3d::launch_forward_bf16_runs(map->pos, map->et, map->hdr, map->ptile_max, feats,
-                                         weight, out, cin, cout, flip01, epi, err, s);
+  if (map && map->pos && cin % 64 == 0 && !prefer_gather())
+    e = subm3d::launch_forward_bf16_runs(map->pos, map->et, map->layout.et_stride, map->hdr,
+                                         map->ptile_max, feats,
+                                         weight, out, cin, cout, flip01, epi, ctl, s);
   else
     e = subm3d::launch_forward_bf16(nbr, tile_mask, n, feats, weight, out, cin, cout, flip01, epi,
-                                    err, s);
+                                    ctl, s);
   if (e == cudaErrorNotSupported) return SUBM3D_E_UNSUPPORTED;
   return e == cudaSuccess ? SUBM3D_OK : SUBM3D_E_CUDA;
 }
@@ -307,10 +336,13 @@ subm3d_status subm3d_backward_weight(const subm3d_map* map, const void* feats, c
   auto s = static_cast<cudaStream_t>(stream);
   if (n > 0 && dtype == SUBM3D_BF16 && map->pos && cin % 64 == 0 && cout % 16 == 0 &&
       aligned(feats, 16) && aligned(dy, 16) && aligned(dweight, 16) && device_is_sm100(nullptr) == 1) {
-    int32_t* err = device_error_word();
-    if (!err) return SUBM3D_E_CUDA;
-    return subm3d::launch_wgrad_bf16_runs(map->pos, map->et, map->hdr, feats, dy, dweight, cin,
-                                          cout, flip ? 1 : 0, err, s) == cudaSuccess
+    subm3d::DeviceCtl ctl;
+    ctl.err_word = device_error_word();
+    if (!ctl.err_word) return SUBM3D_E_CUDA;
+    ctl.wait_limit_ns = wait_limit_from_env();
+    return subm3d::launch_wgrad_bf16_runs(map->pos, map->et, map->layout.et_stride, map->hdr,
+                                          feats, dy, dweight, cin,
+                                          cout, flip ? 1 : 0, ctl, s) == cudaSuccess
                ? SUBM3D_OK
                : SUBM3D_E_CUDA;
   }

@@ -69,13 +69,15 @@ static_assert(GATHER_THREADS == 16 * 16, "gather mapping: 16 pieces x 16 rows pe
 
 struct WgradArgs {
   const int32_t* pos;  // position table
-  const int32_t* et;   // E index table
+  const int32_t* et;   // E index table: 9 lines (one per dz-dy pair), `es` entries apart
+  int64_t es;          // E line stride (entries)
   const int32_t* hdr;  // [runs, position tiles, positions, 0]
   const __nv_bfloat16* x;
   const __nv_bfloat16* dy;
   float* dw;           // [cout][27][cin], zeroed
   int32_t cin, cout, n_ob, n_cb, ranges, flip;
   int32_t* err_word;
+  uint64_t wait_limit_ns;
 };
 
 // The step sequence of a CTA, walked identically by every role: units
@@ -148,8 +150,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) subm3d_wgrad_bf16_runs_sm100(c
   uint64_t* empty = full + NSTAGE;
   uint64_t* acc_full = empty + NSTAGE;
   uint64_t* acc_empty = acc_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint64_t* drain_bar = acc_empty + 1;
+  WaitCtl* wctl = reinterpret_cast<WaitCtl*>(drain_bar + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wctl + 1);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -160,7 +163,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) subm3d_wgrad_bf16_runs_sm100(c
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, NUM_EPI_WARPS * 32);
-    *abort_flag = 0;
+    mbar_init(drain_bar, 1);
+    wait_ctl_init(wctl, a.wait_limit_ns);
     fence_mbar_init();
   }
   if (warp == MMA_WARP) {
@@ -185,13 +189,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) subm3d_wgrad_bf16_runs_sm100(c
     st.begin(n_tiles, a.ranges, a.n_ob, a.n_cb);
     while (st.valid) {
       const int s = st.slot;
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[s], st.phase ^ 1u, abort_flag))) break;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[s], st.phase ^ 1u, wctl))) break;
       const uint32_t y_base = smem_u32(ring) + static_cast<uint32_t>(s) * STAGE;
       const uint32_t e_base = y_base + 2 * Y_CHUNK;
       const int o = st.ob * OB + chunk * 64 + col * 8;   // dy channel of this piece
       const int c = st.cb * CB + chunk * 64 + col * 8;   // x channel of this piece
       const int32_t* posp = a.pos + st.tile * kPosTile + st.half * HP;
-      const int32_t* etp = a.et + (st.tile * 9 + st.pair) * kEtStride + st.half * HP;
+      const int32_t* etp = a.et + st.pair * a.es + st.tile * kPosTile + st.half * HP;
 #pragma unroll
       for (int q = 0; q < YROWS / 16; ++q) {
         const int r = rbase + 16 * q;
@@ -223,13 +227,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) subm3d_wgrad_bf16_runs_sm100(c
       bool ok = true;
       while (ok && st.valid) {
         // the accumulators are free once the previous unit's epilogue has read them
-        if (!mbar_wait(acc_empty, (st.local & 1) ^ 1, abort_flag)) break;
+        if (!mbar_wait(acc_empty, (st.local & 1) ^ 1, wctl)) break;
         tc_fence_after();
         bool first = true;
         bool unit_done = false;
         while (!unit_done) {
           const int s = st.slot;
-          if (!mbar_wait(&full[s], st.phase, abort_flag)) {
+          if (!mbar_wait(&full[s], st.phase, wctl)) {
             ok = false;
             break;
           }
@@ -256,14 +260,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) subm3d_wgrad_bf16_runs_sm100(c
         if (!ok) break;
         umma_commit(acc_full);
       }
-      if (!ok) __nanosleep(20000);  // let MMAs already issued finish before TMEM is freed
     }
   } else {
     // --------------------------------------------------------- epilogue ----
     WSteps st;
     st.begin(n_tiles, a.ranges, a.n_ob, a.n_cb);
     while (st.valid) {
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(acc_full, st.local & 1, abort_flag))) break;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(acc_full, st.local & 1, wctl))) break;
       tc_fence_after();
       const int o = st.ob * OB + warp * 32 + lane;
       const int c0 = st.cb * CB;
@@ -298,20 +301,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) subm3d_wgrad_bf16_runs_sm100(c
   }
 
   tc_fence_before();
-  __syncthreads();
+  __syncthreads();  // every role has left its loop; the abort word no longer changes
+  if (wait_aborted(wctl)) {
+    // MMAs issued before the abort may still be running (the gather threads have
+    // already waited for their own copies)
+    if (warp == MMA_WARP && lane == 0) drain_mma(drain_bar);
+    tc_fence_before();
+    __syncthreads();
+  }
   if (warp == MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }
-  if (threadIdx.x == 0 && *abort_flag) atomicExch(a.err_word, 1);
+  if (threadIdx.x == 0 && wait_aborted(wctl)) atomicExch(a.err_word, 1);
 }
 
 }  // namespace
 
 cudaError_t launch_wgrad_bf16_runs(const int32_t* pos, const int32_t* etable,
-                                   const int32_t* header, const void* feats, const void* dy,
+                                   int64_t et_stride, const int32_t* header, const void* feats, const void* dy,
                                    float* dw, int32_t cin, int32_t cout, int32_t flip,
-                                   int32_t* err_word, cudaStream_t stream) {
+                                   const DeviceCtl& ctl, cudaStream_t stream) {
   static std::mutex mu;
   static int sms[64] = {0};
   int device = 0;
@@ -337,6 +347,7 @@ cudaError_t launch_wgrad_bf16_runs(const int32_t* pos, const int32_t* etable,
   WgradArgs a;
   a.pos = pos;
   a.et = etable;
+  a.es = et_stride;
   a.hdr = header;
   a.x = static_cast<const __nv_bfloat16*>(feats);
   a.dy = static_cast<const __nv_bfloat16*>(dy);
@@ -349,7 +360,8 @@ cudaError_t launch_wgrad_bf16_runs(const int32_t* pos, const int32_t* etable,
   const int combos = 9 * a.n_ob * a.n_cb;
   a.ranges = num_sms / combos > 0 ? num_sms / combos : 1;
   a.flip = flip;
-  a.err_word = err_word;
+  a.err_word = ctl.err_word;
+  a.wait_limit_ns = ctl.wait_limit_ns;
   const int64_t units = static_cast<int64_t>(a.ranges) * combos;
   const unsigned grid = static_cast<unsigned>(units < num_sms ? units : num_sms);
   return launch_pdl(subm3d_wgrad_bf16_runs_sm100, grid, NUM_THREADS, kSmemBytes, stream, a);

@@ -188,16 +188,18 @@ class _SubMConvFunction(torch.autograd.Function):
 
 
 def run_layout_tensors(h: MapHandle):
-    """(position table, E index table [tiles, 9, 260], header) as int32 views
-    of the map's workspace; call after the build has completed."""
+    """(position table [256 tiles], E index table [9, 256 tiles + 2], header) as
+    int32 views of the map's workspace; call after the build has completed.
+    Row dz-dy of the E table holds, at column q + 1, the feature row gathered
+    as E row q (position q) for the offset pair (dz, dy), q = -1 .. 256 tiles."""
     pos_p, et_p, hdr_p = _abi.subm3d_map_run_layout(h)
     base = h.workspace.data_ptr()
     ws = h.workspace
     hdr = ws[hdr_p - base:hdr_p - base + 16].view(torch.int32)
-    tiles = int(hdr[1].item())
+    tiles, stride = int(hdr[1].item()), int(hdr[3].item())
     pos = ws[pos_p - base:pos_p - base + 4 * 256 * tiles].view(torch.int32)
-    et = ws[et_p - base:et_p - base + 4 * tiles * 9 * 260].view(torch.int32).view(tiles, 9, 260)
-    return pos, et, hdr
+    lines = ws[et_p - base:et_p - base + 4 * 9 * stride].view(torch.int32).view(9, stride)
+    return pos, lines[:, :256 * tiles + 2], hdr
 
 
 class SparseTensor:

@@ -46,8 +46,8 @@ def test_version_and_strings(abi):
 def _expected_ws(n, table_bytes):
     """Workspace layout: 256-B status block, tile masks, lookup table, run-start
     counts (one int32 per 128-row tile, one per 128 tiles), 256-B header,
-    position table (3N rounded to 256, + 256), E index table (one [9, 260]
-    int32 block per 256 positions); 256-B aligned parts."""
+    position table (3N rounded to 256, + 256), E index table (9 lines of
+    pos_max + 4 int32); 256-B aligned parts."""
     up = lambda v: (v + 255) // 256 * 256
     head = up(256 + 4 * ((n + 127) // 128))
     tiles = (n + 127) // 128
@@ -55,7 +55,7 @@ def _expected_ws(n, table_bytes):
     after_table = up(head + table_bytes)
     pos_off = up(up(after_table + 4 * tiles) + 4 * ((tiles + 127) // 128)) + 256
     et_off = up(pos_off + 4 * pos_max)
-    return up(et_off + (pos_max // 256) * 9 * 260 * 4)
+    return up(et_off + 9 * (pos_max + 4) * 4)
 
 
 def test_workspace_bytes(abi, monkeypatch):
@@ -65,12 +65,16 @@ def test_workspace_bytes(abi, monkeypatch):
     assert f(-1, 16, 1) == 0 and f(10, 0, 1) == 0 and f(10, 16, 0) == 0
     assert f(10, 70000, 1) == 0 and f(10, 16, 70000) == 0
     n = 329839
-    # direct table: one int32 per cell of a volume up to max(64 MB, 256 B x N)
-    assert f(n, 128, 1) == _expected_ws(n, 4 * 128 ** 3)
-    assert f(n, 256, 1) == _expected_ws(n, 4 * 256 ** 3)
-    big = 1_135_307                                  # 4 x 256^3 = 268 MB <= 256 B x N
-    assert f(big, 256, 4) == _expected_ws(big, 4 * 4 * 256 ** 3)
-    assert f(n, 256, 4) != _expected_ws(n, 4 * 4 * 256 ** 3)   # 268 MB > 84 MB: hash
+    # direct table: one int32 per cell of each bordered grid, (grid + 2)^3 cells,
+    # while that takes at most max(64 MB, 256 B x N)
+    up = lambda v: (v + 255) // 256 * 256
+    assert f(n, 128, 1) == _expected_ws(n, up(4 * 130 ** 3))
+    small = 1000                                     # budget 64 MB
+    assert f(small, 254, 1) == _expected_ws(small, up(4 * 256 ** 3))   # exactly 64 MB
+    assert f(small, 255, 1) == _expected_ws(small, 8 * 2048)           # just over: hash
+    big = 1_135_307                                  # 4 x 258^3 = 275 MB <= 256 B x N
+    assert f(big, 256, 4) == _expected_ws(big, up(4 * 4 * 258 ** 3))
+    assert f(n, 256, 4) == _expected_ws(n, 8 * (1 << 20))      # 275 MB > 84 MB: hash
     # larger volumes: hash table, 8-byte slots, capacity max(1024, pow2 >= 2N)
     assert f(n, 512, 1) == _expected_ws(n, 8 * (1 << 20))
     # wide keys (batch > 4 or grid > 1024) add a 4-byte row array

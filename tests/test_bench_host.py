@@ -1,6 +1,8 @@
 """Host logic of the multi-GPU benchmark, run as two gloo ranks on CPU: every
-rank gets its own input seed, the job time is the max over ranks, and the
-weak-scaling rate counts the voxels of all ranks."""
+rank gets its own input seed, the job time is the max over ranks, the
+weak-scaling rate counts the voxels of all ranks, and the batched workload's
+elements are split over the ranks (each element on exactly one rank, batch
+indices renumbered per rank) with a strong-scaling rate."""
 import os
 import socket
 
@@ -100,3 +102,77 @@ def test_reference_arm_line():
 def test_reference_arm_other_ranks_exit_without_work():
     assert _run_bench(["--impl", "reference", "--workload", "shell_bf16", "--steps", "1",
                        "--warmup", "1"], {"RANK": "1", "WORLD_SIZE": "2"}) == []
+
+
+def _four_elements():
+    """Four batch elements of different sizes (the batched workload's structure:
+    independent sets that share no neighbour), raster order."""
+    import numpy as np
+    parts = []
+    for b, n in enumerate((5, 9, 3, 7)):
+        rng = np.random.default_rng(b)
+        cells = np.sort(rng.choice(6 ** 3, n, replace=False))
+        zyx = np.stack(np.unravel_index(cells, (6, 6, 6)), 1)
+        parts.append(np.concatenate([np.full((n, 1), b), zyx], 1).astype(np.int32))
+    return np.concatenate(parts)
+
+
+def _split_rank_main(rank, world, port, out):
+    import datetime
+    import sys
+    sys.path.insert(0, ROOT)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import torch.distributed as dist
+    import bench
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        coords = _four_elements()
+        elems = bench.batch_elements(rank, world, 4)
+        sub = bench.split_batch(coords, elems)
+        local_ms = 4.0 * sub.shape[0]          # time grows with the rank's rows
+        job_ms = bench.max_over_ranks(local_ms, "cpu")
+        out[rank] = (elems, sub.tolist(), job_ms)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_batch_split():
+    import numpy as np
+    import sys
+    sys.path.insert(0, ROOT)
+    world = 2
+    port = _free_port()
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_split_rank_main, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    coords = _four_elements()
+    assert res[0][0] == [0, 2] and res[1][0] == [1, 3]     # rank r: elements r, r + world
+    seen = []
+    for r in range(world):
+        sub = np.array(res[r][1], np.int32)
+        for new_b, b in enumerate(res[r][0]):
+            mine = sub[sub[:, 0] == new_b]
+            orig = coords[coords[:, 0] == b]
+            assert np.array_equal(mine[:, 1:], orig[:, 1:])  # same rows, same order
+            seen.append(b)
+        assert set(sub[:, 0].tolist()) == set(range(len(res[r][0])))  # renumbered 0..m-1
+    assert sorted(seen) == [0, 1, 2, 3]                      # every element exactly once
+    rows = [len(res[r][1]) for r in range(world)]
+    assert sum(rows) == coords.shape[0]
+    job_ms = res[0][2]
+    assert job_ms == res[1][2] == 4.0 * max(rows)            # the slowest rank's time
+    # strong scaling: the job's rate counts the batch's voxels once
+    assert coords.shape[0] == 24
+    assert coords.shape[0] / (job_ms / 1e3) == pytest.approx(24 / (4.0 * max(rows) / 1e3))
+
+
+def test_batch_split_more_ranks_than_elements():
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    assert [bench.batch_elements(r, 8, 4) for r in range(8)] == [[0], [1], [2], [3], [], [], [], []]
+    assert bench.batch_elements(0, 1, 4) == [0, 1, 2, 3]
+    assert bench.split_batch(_four_elements(), []).shape == (0, 4)

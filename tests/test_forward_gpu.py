@@ -256,3 +256,33 @@ def test_bf16_both_kernels_agree_with_oracle(S, name, flip):
         y = S.forward(h, xt, wt, flip=flip, kernel=kernel).float().cpu().numpy()
         assert S._abi.subm3d_device_status() == 0
         assert_close(y[rows], ref, RTOL_BF16, f"{name} {kernel} flip={flip}")
+
+
+def test_kernel_choice_and_knob(S, monkeypatch):
+    """subm3d_forward_map runs the x-run kernel wherever its layout applies, on
+    short runs too (the 64^3 shell: runs of ~4 voxels, 1.50 N positions), at 64
+    and 128 input channels; SUBM3D_FORWARD_KERNEL=gather switches it to the
+    per-offset kernel of subm3d_forward.  Each kernel is deterministic, so the
+    results match bit for bit the kernel that ran."""
+    wl = WL.make_workload("shell_bf16")
+    c = torch.from_numpy(wl.coords).cuda()
+    h = S.build_map(c, wl.grid_dim, wl.batch)
+    hdr = S.run_layout_tensors(h)[2].cpu().numpy()
+    assert hdr[2] > 1.45 * wl.n
+    for cin in (64, 128):
+        xt = torch.from_numpy(WL.to_bf16_values(WL.make_features(wl.n, cin, 41))).cuda().to(
+            torch.bfloat16)
+        wt = torch.from_numpy(WL.to_bf16_values(WL.make_weight(64, cin, 42))).cuda().to(
+            torch.bfloat16)
+        auto = S.forward(h, xt, wt)
+        gather = S.forward(h, xt, wt, kernel="gather")       # subm3d_forward on nbr
+        monkeypatch.setenv("SUBM3D_FORWARD_KERNEL", "gather")
+        knob = S.forward(h, xt, wt)
+        monkeypatch.delenv("SUBM3D_FORWARD_KERNEL")
+        torch.cuda.synchronize()
+        assert S._abi.subm3d_device_status() == 0
+        assert torch.equal(knob, gather), cin
+        ref = _oracle(wl.coords, wl.grid_dim, 1, xt.float().cpu().numpy(),
+                      wt.float().cpu().numpy(), bf16_out=True)
+        for what, y in (("auto", auto), ("gather", gather)):
+            assert_close(y.float().cpu().numpy(), ref, RTOL_BF16, f"{what} cin={cin}")

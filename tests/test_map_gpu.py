@@ -32,8 +32,11 @@ def kind(request, monkeypatch):
 
 
 def _gpu_map(S, coords, grid, batch):
+    """The GPU map, and its tile masks as whole unsigned 32-bit words: compared
+    with the oracle's 27-bit masks, the five high bits must be zero too."""
     h = S.build_map(torch.from_numpy(np.ascontiguousarray(coords)).cuda(), grid, batch)
-    return h, h.nbr.cpu().numpy(), S.tile_mask_tensor(h).cpu().numpy().astype(np.int64) & 0x7FFFFFF
+    words = S.tile_mask_tensor(h).cpu().numpy().view(np.uint32).astype(np.int64)
+    return h, h.nbr.cpu().numpy(), words
 
 
 @pytest.mark.parametrize("name", ["tiny", "shell", "headline", "dense", "batched"])
@@ -146,7 +149,7 @@ def _check_run_layout(S, coords, grid, batch):
     runs = int(starts.sum())
     positions = n + 2 * runs
     assert hdr[0] == runs and hdr[2] == positions and hdr[1] == (positions + 255) // 256
-    assert pos.shape[0] == 256 * hdr[1] and et.shape == (hdr[1], 9, 260)
+    assert pos.shape[0] == 256 * hdr[1] and et.shape == (9, 256 * hdr[1] + 2)
     voxel_pos = np.nonzero((pos >= 0) & ((pos & 3) == 0))[0]
     assert np.array_equal(pos[voxel_pos] >> 2, np.arange(n))      # every row once, in order
     assert np.array_equal(voxel_pos, np.arange(n) + 2 * np.cumsum(starts))
@@ -158,12 +161,14 @@ def _check_run_layout(S, coords, grid, batch):
     assert np.array_equal(right, (voxel_pos[ends] + 1)[inside])
     assert pos[0] == -1 and (pos[positions + 1:] == -1).all()
     assert ((pos >= 0) | (pos == -1)).all()
-    assert (et[:, :, :258] >= -1).all() and (et[:, :, :258] < n).all()
-    tile, local = voxel_pos // 256, voxel_pos % 256
+    assert (et >= -1).all() and (et < n).all()   # every entry a tile reads is written
     for k in range(27):
         dzdy, dx = k // 3, k % 3 - 1
-        got = et[tile, dzdy, local + dx + 1]
+        got = et[dzdy, voxel_pos + dx + 1]
         assert np.array_equal(got, ref[:, k]), f"offset {k}"
+    # E rows that are not a voxel's neighbour row: positions -1 and 0, and the
+    # tail after the last right pad, are empty
+    assert (et[:, :2] == -1).all() and (et[:, positions + 2:] == -1).all()
 
 
 @pytest.mark.parametrize("name", ["tiny", "shell", "headline", "batched"])

@@ -54,6 +54,31 @@ def test_noalloc_matches_workspace_build_on_consecutive_calls():
     assert torch.equal(y, y_ref)
 
 
+def test_noalloc_wide_keys_match_oracle():
+    """batch > 4 or grid_dim > 1024 takes the 64-bit key form, whose hash table
+    keeps its rows in a separate region of the fixed scratch array.  Its maps
+    are checked against the oracle directly, on two calls in a row."""
+    from oracle import cpp as C
+    from sparse_voxel_conv_b200 import _abi as A
+    from tests.helpers import masks_from_nbr
+
+    parts = []
+    for b in range(5):                                    # batch 5: wide keys
+        c = WL.tiny_coords(seed=30 + b)
+        c[:, 0] = b
+        parts.append(c)
+    five = np.concatenate(parts)[WL.permute_rows(sum(len(p) for p in parts), 31)]
+    far = WL.tiny_coords(seed=32)
+    far[:, 1:] += 1500                                    # grid 2048: wide keys
+    for coords, grid, batch in ((five, 16, 5), (far, 2048, 1)):
+        st, c, nbr, mask = _noalloc(A, coords, grid, batch)
+        assert st == A.SUBM3D_OK, A.subm3d_status_string(st)
+        ref = C.build_map(coords, grid, batch)
+        assert np.array_equal(nbr.cpu().numpy(), ref)
+        words = mask.cpu().numpy().view(np.uint32).astype(np.int64)
+        assert np.array_equal(words, masks_from_nbr(ref))
+
+
 def test_noalloc_reports_data_errors_and_rejects_oversize():
     from sparse_voxel_conv_b200 import _abi as A
 

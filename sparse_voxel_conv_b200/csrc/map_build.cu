@@ -189,6 +189,8 @@ __global__ void __launch_bounds__(kInsertThreads)
 // the one after.  E row q of pair dz-dy is entry q + 1 of that pair's line.
 
 static_assert(kInsertThreads == 256 && kSuperTiles % 2 == 0, "insert block = two query tiles");
+// Positions one warp's 32 rows can occupy: each row its own run, with both pads.
+constexpr int kWarpSpan = 3 * 32;
 
 struct RunOut {
   const int32_t* cnt;  // run starts per 128-row tile (insert kernel)
@@ -222,6 +224,7 @@ __global__ void __launch_bounds__(kTileRows)
   __shared__ uint32_t s_starts[kTileRows / 32];  // run-start ballot of each warp
   __shared__ int32_t s_before[kTileRows / 32];   // partial sums of the run starts before the tile
   __shared__ int32_t s_end;
+  __shared__ uint8_t s_src[RUNS ? 4 * kWarpSpan : 4];  // position -> row and kind, per warp
   const int r = threadIdx.x;
   const int lane = r & 31, warp = r >> 5;
   const int tile = blockIdx.x;
@@ -326,23 +329,39 @@ __global__ void __launch_bounds__(kTileRows)
     for (int w = 0; w < warp; ++w) runs += __popc(s_starts[w]);
     runs += __popc(s_starts[warp] & (0xFFFFFFFFu >> (31 - lane)));
     const int es = ro.es;
+    const int p = i + 2 * runs;  // this row's position (when live)
+    // Position-major stores: the warp's positions form one range [w0, w1] (its
+    // first row's left pad, if that row starts a run, to its last row's right
+    // pad, if that row ends one; at most 96), every position the voxel, left pad
+    // or right pad of one of its rows.  Each lane records which row and which of
+    // the three occupies its positions, then the lanes write the range's
+    // position entries and E entries in order, 32 consecutive positions per
+    // store, instead of scattered single stores for the pads.
+    const uint32_t live_lanes = __ballot_sync(0xFFFFFFFFu, live);
+    int w0 = 0, w1 = -1;
+    if (live_lanes) {
+      w0 = __shfl_sync(0xFFFFFFFFu, starts ? p - 1 : p, __ffs(live_lanes) - 1);
+      w1 = __shfl_sync(0xFFFFFFFFu, ends ? p + 1 : p, 31 - __clz(live_lanes));
+    }
+    uint8_t* src_of = s_src + warp * kWarpSpan;  // position - w0 -> lane * 4 + kind
     if (live) {
-      const int p = i + 2 * runs;
-      const int32_t tag = i * 4;
-      ro.pos[p] = tag + kPosVoxel;
-      if (starts) ro.pos[p - 1] = tag + kPosLeftPad;
-      if (ends) ro.pos[p + 1] = tag + kPosRightPad;
-      // E row p of pair dz-dy is the voxel's (dz, dy, 0) neighbour; its left pad
-      // (row p - 1) the (dz, dy, -1) one, its right pad (row p + 1) the (dz, dy, +1)
-      int32_t* e = ro.et + (p + 1);
+      src_of[p - w0] = static_cast<uint8_t>(lane * 4 + 1);                 // the voxel
+      if (starts) src_of[p - 1 - w0] = static_cast<uint8_t>(lane * 4 + 0);  // its left pad
+      if (ends) src_of[p + 1 - w0] = static_cast<uint8_t>(lane * 4 + 2);    // its right pad
+    }
+    __syncwarp();
+    for (int q = w0 + lane; q <= w1; q += 32) {
+      const int code = src_of[q - w0];
+      const int r_src = warp * 32 + (code >> 2), kind = code & 3;  // kind = dx + 1
+      ro.pos[q] = (row0 + r_src) * 4 +
+                  (kind == 1 ? kPosVoxel : (kind == 0 ? kPosLeftPad : kPosRightPad));
+      // E row q of pair dz-dy: the (dz, dy, dx) neighbour of the row's voxel
+      const int32_t* nbs = s_nbr + r_src * kKvol + kind;
+      int32_t* e = ro.et + (q + 1);
 #pragma unroll
-      for (int dzdy = 0; dzdy < 9; ++dzdy) e[dzdy * es] = nb[3 * dzdy + 1];
-      if (starts)
-#pragma unroll
-        for (int dzdy = 0; dzdy < 9; ++dzdy) e[dzdy * es - 1] = nb[3 * dzdy];
-      if (ends)
-#pragma unroll
-        for (int dzdy = 0; dzdy < 9; ++dzdy) e[dzdy * es + 1] = nb[3 * dzdy + 2];
+      for (int dzdy = 0; dzdy < 9; ++dzdy) e[dzdy * es] = nbs[3 * dzdy];
+    }
+    if (live) {
       if (i == 0) {  // position 0 (the absent right pad before the first run) and row -1
         ro.pos[0] = -1;
 #pragma unroll

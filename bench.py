@@ -114,6 +114,19 @@ def max_over_ranks(value: float, device) -> float:
     return float(t.item())
 
 
+def sum_over_ranks(value: float, device) -> float:
+    """The job's total of a per-rank quantity (all-reduce SUM of a float; the
+    value itself without an initialised process group).  Bookkeeping only,
+    outside the timed region."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
 def job_rate(units_per_rank: int, world: int, job_seconds: float) -> float:
     """Weak-scaling throughput: the units every rank processed / the job time."""
     return units_per_rank * world / job_seconds
@@ -550,6 +563,7 @@ def run_ours(args):
     e1.record(s_out)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    job_flops = sum_over_ranks(job.flops(nnz_total), dev)  # every rank's layers
 
     if rank == 0:
         peaks, peak_src = _peaks()
@@ -579,7 +593,7 @@ def run_ours(args):
                 "l2": f"flushed before every timed step ({L2_FLUSH_BYTES >> 20} MB write)",
                 "parallelism": job.parallelism,
             },
-            "tflops_effective": flops / (total_ms / 1e3 / K) / 1e12,
+            "tflops_effective": job_flops / (total_ms / 1e3 / K) / 1e12,
             "roofline": {
                 "kernel": "subm3d_fwd_bf16_runs_sm100" + (f" (x{n_layers} layers)"
                                                          if n_layers > 1 else ""),

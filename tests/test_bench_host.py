@@ -32,7 +32,8 @@ def _rank_main(rank, world, port, out):
         local_ms = 10.0 + 5.0 * rank  # rank 1 is the slowest
         job_ms = bench.max_over_ranks(local_ms, "cpu")
         out[rank] = (bench.feature_seed(rank), job_ms,
-                     bench.job_rate(1000, world, job_ms / 1e3))
+                     bench.job_rate(1000, world, job_ms / 1e3),
+                     bench.sum_over_ranks(1.5 + rank, "cpu"))
     finally:
         dist.destroy_process_group()
 
@@ -48,6 +49,7 @@ def test_two_rank_reduction_and_rate():
     assert len(seeds) == world                        # each replica has its own input
     assert res[0][1] == res[1][1] == pytest.approx(15.0)   # max over ranks on every rank
     assert res[0][2] == pytest.approx(2 * 1000 / 0.015)    # all ranks' voxels / job time
+    assert res[0][3] == res[1][3] == pytest.approx(4.0)    # a per-rank quantity summed
 
 
 def test_single_process_is_identity():
@@ -55,6 +57,7 @@ def test_single_process_is_identity():
     sys.path.insert(0, ROOT)
     import bench
     assert bench.max_over_ranks(3.5, "cpu") == 3.5
+    assert bench.sum_over_ranks(3.5, "cpu") == 3.5
     assert bench.job_rate(10, 1, 2.0) == 5.0
 
 

@@ -193,11 +193,11 @@ cudaError_t launch_expand(const int32_t* coords, const void* feats, const uint8_
 
 // Pooling to parents coord // 2 in raster order: max (0), mean (1) or
 // spatial2channel (2), through the fine set's map table.  Its workspace: a flag
-// per parent cell, per-4,096-cell counts, a total and the parents' cells.
+// per parent cell, per-4,096-cell counts and the total.
 struct PoolLayout {
   int32_t G = 0;
   int64_t cells = 0, n_blocks = 0;
-  size_t flags_off = 0, cnt_off = 0, total_off = 0, cells_off = 0, bytes = 0;
+  size_t flags_off = 0, cnt_off = 0, total_off = 0, bytes = 0;
 };
 PoolLayout pool_layout(int64_t n, int32_t grid_dim, int32_t batch);
 // Blocking (the parent count is read back); *out_count = parents.

@@ -2,12 +2,19 @@
 //
 // out[i] = act( sum_k Wf[:, k, :] . x[nbr[i][k]] + bias ) + residual[i],
 // Wf[:, k] = W[:, k] or W[:, 26-k] with flip (correlation / mirrored kernel,
-// lato.2_mrp_mlx commit 97dcdfb54a message); bias and residual optional.  Implicit gather-GEMM: a 64-row x 64-column output tile
-// per block, 256 threads with a 4x4 register tile each.  For every offset the
-// tile needs, 16-channel slices of the 64 gathered input rows (zero where
-// nbr = -1) and of the weight slice are staged in shared memory and
-// contracted; the accumulators stay in registers across all 27 offsets, so
-// there is no scatter and no atomics.  Any Cin, Cout >= 1.
+// lato.2_mrp_mlx commit 97dcdfb54a message); bias and residual optional.
+//
+// Implicit gather-GEMM, one 128-row x 128-column output tile per block (the
+// rows are one tile-mask tile): 256 threads with an 8 x 8 register tile each
+// (rows 4 ty .. 4 ty + 3 and 64 + 4 ty ..; columns likewise with tx).  The K
+// loop runs over the offsets present in the tile (its mask word) and, for each,
+// 16-channel slices of Cin.  A step stages the 128 gathered input rows' slice
+// (zeros where nbr = -1) and the weight slice in shared memory, k-major with a
+// 4-float pad so that the transposing stores are conflict-free; the next step's
+// slices load into registers, 8 channels at a time, while this step's 64 FMAs
+// per thread and channel run, with two shared buffers and one barrier per step.  The accumulators stay
+// in registers across all 27 offsets: no scatter, no atomics.  Any Cin, Cout
+// >= 1; 16-byte loads and stores where Cin and Cout are multiples of 4.
 //
 // fp32 FMA rather than TF32 tensor cores: TF32's 10-bit mantissa cannot meet a
 // 1e-5 relative tolerance over 27*Cin terms.
@@ -19,89 +26,178 @@
 namespace subm3d {
 namespace {
 
-constexpr int BM = 64, BN = 64, BK = 16, NT = 256;
+constexpr int BM = 128, BN = 128, BK = 16, HK = BK / 2, NT = 256, PAD = 4;
+static_assert(BM == kTileRows, "one tile-mask word per block");
+
+// The four channels c .. c + 3 of row `src` (zeros past cin or for src < 0).
+template <bool VEC>
+__device__ __forceinline__ float4 load4(const float* __restrict__ base, int64_t src, int c,
+                                        int cin) {
+  if (src < 0 || c >= cin) return make_float4(0.f, 0.f, 0.f, 0.f);
+  const float* p = base + src * cin + c;
+  if constexpr (VEC) return __ldg(reinterpret_cast<const float4*>(p));
+  float v[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) v[j] = c + j < cin ? __ldg(p + j) : 0.f;
+  return make_float4(v[0], v[1], v[2], v[3]);
+}
 
 // out may alias residual (an in-place residual add): neither is __restrict__.
-template <int ACT>
-__global__ void __launch_bounds__(NT)
+template <int ACT, bool VEC>
+__global__ void __launch_bounds__(NT, 2)
     fwd_f32_kernel(const int32_t* __restrict__ nbr, const uint32_t* __restrict__ tile_mask,
                    int64_t n, const float* __restrict__ x, const float* __restrict__ w,
                    float* out, int cin, int cout, int flip, const float* bias,
                    const float* residual) {
   __shared__ int32_t s_nbr[BM * kKvol];
-  __shared__ __align__(16) float s_a[BK][BM];
-  __shared__ __align__(16) float s_b[BK][BN];
+  __shared__ int32_t s_off[kKvol + 1];
+  __shared__ __align__(16) float s_a[2][BK][BM + PAD];
+  __shared__ __align__(16) float s_b[2][BK][BN + PAD];
 
   const int t = threadIdx.x;
   const int64_t row0 = static_cast<int64_t>(blockIdx.x) * BM;
   const int col0 = blockIdx.y * BN;
   for (int e = t; e < BM * kKvol; e += NT) {
     const int64_t r = row0 + e / kKvol;
-    s_nbr[e] = (r < n) ? nbr[row0 * kKvol + e] : -1;
+    s_nbr[e] = (r < n) ? __ldg(nbr + row0 * kKvol + e) : -1;
   }
-  const uint32_t mask = tile_mask ? tile_mask[row0 / kTileRows] : 0x7FFFFFFu;
+  if (t == 0) {
+    const uint32_t mask = tile_mask ? __ldg(tile_mask + blockIdx.x) : 0x7FFFFFFu;
+    int cnt = 0;
+    for (int k = 0; k < kKvol; ++k)
+      if ((mask >> k) & 1u) s_off[cnt++] = k;
+    s_off[kKvol] = cnt;
+  }
   __syncthreads();
 
-  const int ty = t / 16, tx = t % 16;
-  float acc[4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+  // staging role: row / output column t / 2, channels 4 (t % 2) .. + 3 of the slice
+  const int sr = t >> 1, sh = (t & 1) * 4;
+  const int so = col0 + sr;
+  // compute role
+  const int ty = t >> 4, tx = t & 15;
+  const int steps = s_off[kKvol] * ((cin + BK - 1) / BK);
 
-  uint32_t m = mask;
-  while (m) {
-    const int k = __ffs(m) - 1;
-    m &= m - 1;
+  float4 ra, rb;  // the next half-step's slices
+  int f_ki = 0, f_c = 0;  // the step fetch() loads next: offset index, slice start
+  // one half (8 channels) of the step at (f_ki, f_c); the second half advances
+  auto fetch = [&](int half) {
+    const int k = s_off[f_ki];
     const int kw = flip ? (kKvol - 1 - k) : k;
-    for (int c0 = 0; c0 < cin; c0 += BK) {
-#pragma unroll
-      for (int e = 0; e < (BM * BK) / NT; ++e) {
-        const int idx = t + e * NT;
-        const int r = idx / BK, kk = idx % BK;
-        const int src = s_nbr[r * kKvol + k];
-        const int c = c0 + kk;
-        s_a[kk][r] = (src >= 0 && c < cin) ? __ldg(x + static_cast<int64_t>(src) * cin + c) : 0.f;
+    const int c = f_c + half * HK + sh;
+    ra = load4<VEC>(x, s_nbr[sr * kKvol + k], c, cin);
+    rb = load4<VEC>(w, so < cout ? static_cast<int64_t>(so) * kKvol + kw : -1, c, cin);
+    if (half) {
+      f_c += BK;
+      if (f_c >= cin) {
+        f_c = 0;
+        ++f_ki;
       }
-#pragma unroll
-      for (int e = 0; e < (BN * BK) / NT; ++e) {
-        const int idx = t + e * NT;
-        const int col = idx / BK, kk = idx % BK;
-        const int o = col0 + col, c = c0 + kk;
-        s_b[kk][col] = (o < cout && c < cin)
-                           ? __ldg(w + (static_cast<int64_t>(o) * kKvol + kw) * cin + c)
-                           : 0.f;
-      }
-      __syncthreads();
-#pragma unroll
-      for (int kk = 0; kk < BK; ++kk) {
-        const float4 a4 = *reinterpret_cast<const float4*>(&s_a[kk][ty * 4]);
-        const float4 b4 = *reinterpret_cast<const float4*>(&s_b[kk][tx * 4]);
-        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-        const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-      }
-      __syncthreads();
     }
+  };
+  auto stage = [&](int buf, int half) {
+    const int kk = half * HK + sh;
+    s_a[buf][kk + 0][sr] = ra.x;
+    s_a[buf][kk + 1][sr] = ra.y;
+    s_a[buf][kk + 2][sr] = ra.z;
+    s_a[buf][kk + 3][sr] = ra.w;
+    s_b[buf][kk + 0][sr] = rb.x;
+    s_b[buf][kk + 1][sr] = rb.y;
+    s_b[buf][kk + 2][sr] = rb.z;
+    s_b[buf][kk + 3][sr] = rb.w;
+  };
+
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+  auto compute = [&](int buf, int half) {
+#pragma unroll
+    for (int q = 0; q < HK; ++q) {
+      const int kk = half * HK + q;
+      const float4 a0 = *reinterpret_cast<const float4*>(&s_a[buf][kk][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&s_a[buf][kk][64 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&s_b[buf][kk][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&s_b[buf][kk][64 + tx * 4]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+  };
+
+  if (steps > 0) {
+    fetch(0);
+    stage(0, 0);
+    fetch(1);
+    stage(0, 1);
+    __syncthreads();
+  }
+  // buffer s & 1 holds step s; step s + 1 is fetched into registers half by
+  // half and staged in the other buffer (free since the last barrier)
+  for (int s = 0; s < steps; ++s) {
+    const int buf = s & 1;
+    const bool more = s + 1 < steps;
+    if (more) fetch(0);
+    compute(buf, 0);
+    if (more) {
+      stage(buf ^ 1, 0);
+      fetch(1);
+    }
+    compute(buf, 1);
+    if (more) stage(buf ^ 1, 1);
+    __syncthreads();
   }
 
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int64_t r = row0 + ty * 4 + i;
+  for (int i = 0; i < 8; ++i) {
+    const int64_t r = row0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4);
     if (r >= n) continue;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int o = col0 + tx * 4 + j;
-      if (o >= cout) continue;
-      float v = activate<ACT>(acc[i][j] + (bias ? bias[o] : 0.0f));
-      if (residual) v += residual[r * cout + o];
-      out[r * cout + o] = v;
+    for (int h = 0; h < 2; ++h) {
+      const int o0 = col0 + h * 64 + tx * 4;
+      float v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int o = o0 + j;
+        v[j] = o < cout ? activate<ACT>(acc[i][4 * h + j] + (bias ? bias[o] : 0.0f)) : 0.0f;
+      }
+      float* dst = out + r * cout + o0;
+      if (VEC && o0 + 3 < cout) {
+        if (residual) {
+          const float4 q = *reinterpret_cast<const float4*>(residual + r * cout + o0);
+          v[0] += q.x;
+          v[1] += q.y;
+          v[2] += q.z;
+          v[3] += q.w;
+        }
+        *reinterpret_cast<float4*>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (o0 + j >= cout) break;
+          dst[j] = v[j] + (residual ? residual[r * cout + o0 + j] : 0.0f);
+        }
+      }
     }
   }
 }
+
+template <int ACT>
+void launch_act(dim3 grid, bool vec, cudaStream_t stream, const int32_t* nbr,
+                const uint32_t* tile_mask, int64_t n, const float* x, const float* w, float* out,
+                int cin, int cout, int flip, const float* bias, const float* res) {
+  if (vec)
+    fwd_f32_kernel<ACT, true><<<grid, NT, 0, stream>>>(nbr, tile_mask, n, x, w, out, cin, cout,
+                                                       flip, bias, res);
+  else
+    fwd_f32_kernel<ACT, false><<<grid, NT, 0, stream>>>(nbr, tile_mask, n, x, w, out, cin, cout,
+                                                        flip, bias, res);
+}
+
+bool aligned16(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; }
 
 }  // namespace
 
@@ -113,15 +209,18 @@ cudaError_t launch_forward_f32(const int32_t* nbr, const uint32_t* tile_mask, in
                   static_cast<unsigned>((cout + BN - 1) / BN));
   const auto* bias = static_cast<const float*>(epi.bias);
   const auto* res = static_cast<const float*>(epi.residual);
+  // 16-byte rows: feats, weight, out and residual rows start on 16 bytes
+  const bool vec = cin % 4 == 0 && cout % 4 == 0 && aligned16(feats) && aligned16(weight) &&
+                   aligned16(out) && (!res || aligned16(res));
   if (epi.act == kActGelu)
-    fwd_f32_kernel<kActGelu><<<grid, NT, 0, stream>>>(nbr, tile_mask, n, feats, weight, out, cin,
-                                                      cout, flip, bias, res);
+    launch_act<kActGelu>(grid, vec, stream, nbr, tile_mask, n, feats, weight, out, cin, cout, flip,
+                         bias, res);
   else if (epi.act == kActSilu)
-    fwd_f32_kernel<kActSilu><<<grid, NT, 0, stream>>>(nbr, tile_mask, n, feats, weight, out, cin,
-                                                      cout, flip, bias, res);
+    launch_act<kActSilu>(grid, vec, stream, nbr, tile_mask, n, feats, weight, out, cin, cout, flip,
+                         bias, res);
   else
-    fwd_f32_kernel<kActNone><<<grid, NT, 0, stream>>>(nbr, tile_mask, n, feats, weight, out, cin,
-                                                      cout, flip, bias, res);
+    launch_act<kActNone>(grid, vec, stream, nbr, tile_mask, n, feats, weight, out, cin, cout, flip,
+                         bias, res);
   return cudaGetLastError();
 }
 

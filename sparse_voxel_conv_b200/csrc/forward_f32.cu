@@ -8,7 +8,7 @@
 // rows are one tile-mask tile): 256 threads with an 8 x 8 register tile each
 // (rows 4 ty .. 4 ty + 3 and 64 + 4 ty ..; columns likewise with tx).  The K
 // loop runs over the offsets present in the tile (its mask word) and, for each,
-// 16-channel slices of Cin.  A step stages the 128 gathered input rows' slice
+// 32-channel slices of Cin.  A step stages the 128 gathered input rows' slice
 // (zeros where nbr = -1) and the weight slice in shared memory, k-major with a
 // 4-float pad so that the transposing stores are conflict-free; the next step's
 // slices load into registers, 8 channels at a time, while this step's 64 FMAs
@@ -26,7 +26,10 @@
 namespace subm3d {
 namespace {
 
-constexpr int BM = 128, BN = 128, BK = 16, HK = BK / 2, NT = 256, PAD = 4;
+constexpr int BM = 128, BN = 128, BK = 32, HK = 8, NP = BK / HK, NT = 256, PAD = 4;
+// dynamic shared memory: two k-major buffers of each operand, then the tile's nbr rows
+constexpr int kOperandFloats = BK * (BM + PAD);  // BN == BM
+constexpr size_t kSmemBytes = (4 * kOperandFloats + BM * kKvol + kKvol + 1) * 4;
 static_assert(BM == kTileRows, "one tile-mask word per block");
 
 // The four channels c .. c + 3 of row `src` (zeros past cin or for src < 0).
@@ -49,10 +52,12 @@ __global__ void __launch_bounds__(NT, 2)
                    int64_t n, const float* __restrict__ x, const float* __restrict__ w,
                    float* out, int cin, int cout, int flip, const float* bias,
                    const float* residual) {
-  __shared__ int32_t s_nbr[BM * kKvol];
-  __shared__ int32_t s_off[kKvol + 1];
-  __shared__ __align__(16) float s_a[2][BK][BM + PAD];
-  __shared__ __align__(16) float s_b[2][BK][BN + PAD];
+  extern __shared__ float4 smem_f4[];
+  auto s_a = reinterpret_cast<float (*)[BK][BM + PAD]>(smem_f4);                       // [2]
+  auto s_b = reinterpret_cast<float (*)[BK][BN + PAD]>(reinterpret_cast<float*>(smem_f4) +
+                                                       2 * kOperandFloats);           // [2]
+  int32_t* s_nbr = reinterpret_cast<int32_t*>(smem_f4) + 4 * kOperandFloats;
+  int32_t* s_off = s_nbr + BM * kKvol;
 
   const int t = threadIdx.x;
   const int64_t row0 = static_cast<int64_t>(blockIdx.x) * BM;
@@ -79,14 +84,14 @@ __global__ void __launch_bounds__(NT, 2)
 
   float4 ra, rb;  // the next half-step's slices
   int f_ki = 0, f_c = 0;  // the step fetch() loads next: offset index, slice start
-  // one half (8 channels) of the step at (f_ki, f_c); the second half advances
-  auto fetch = [&](int half) {
+  // part `part` (8 channels) of the step at (f_ki, f_c); the last part advances
+  auto fetch = [&](int part) {
     const int k = s_off[f_ki];
     const int kw = flip ? (kKvol - 1 - k) : k;
-    const int c = f_c + half * HK + sh;
+    const int c = f_c + part * HK + sh;
     ra = load4<VEC>(x, s_nbr[sr * kKvol + k], c, cin);
     rb = load4<VEC>(w, so < cout ? static_cast<int64_t>(so) * kKvol + kw : -1, c, cin);
-    if (half) {
+    if (part == NP - 1) {
       f_c += BK;
       if (f_c >= cin) {
         f_c = 0;
@@ -94,8 +99,8 @@ __global__ void __launch_bounds__(NT, 2)
       }
     }
   };
-  auto stage = [&](int buf, int half) {
-    const int kk = half * HK + sh;
+  auto stage = [&](int buf, int part) {
+    const int kk = part * HK + sh;
     s_a[buf][kk + 0][sr] = ra.x;
     s_a[buf][kk + 1][sr] = ra.y;
     s_a[buf][kk + 2][sr] = ra.z;
@@ -111,10 +116,10 @@ __global__ void __launch_bounds__(NT, 2)
   for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-  auto compute = [&](int buf, int half) {
+  auto compute = [&](int buf, int part) {
 #pragma unroll
     for (int q = 0; q < HK; ++q) {
-      const int kk = half * HK + q;
+      const int kk = part * HK + q;
       const float4 a0 = *reinterpret_cast<const float4*>(&s_a[buf][kk][ty * 4]);
       const float4 a1 = *reinterpret_cast<const float4*>(&s_a[buf][kk][64 + ty * 4]);
       const float4 b0 = *reinterpret_cast<const float4*>(&s_b[buf][kk][tx * 4]);
@@ -129,25 +134,24 @@ __global__ void __launch_bounds__(NT, 2)
   };
 
   if (steps > 0) {
-    fetch(0);
-    stage(0, 0);
-    fetch(1);
-    stage(0, 1);
+#pragma unroll 1
+    for (int part = 0; part < NP; ++part) {
+      fetch(part);
+      stage(0, part);
+    }
     __syncthreads();
   }
-  // buffer s & 1 holds step s; step s + 1 is fetched into registers half by
-  // half and staged in the other buffer (free since the last barrier)
+  // buffer s & 1 holds step s; step s + 1 is fetched into registers 8 channels
+  // at a time and staged in the other buffer (free since the last barrier)
   for (int s = 0; s < steps; ++s) {
     const int buf = s & 1;
     const bool more = s + 1 < steps;
-    if (more) fetch(0);
-    compute(buf, 0);
-    if (more) {
-      stage(buf ^ 1, 0);
-      fetch(1);
+#pragma unroll
+    for (int part = 0; part < NP; ++part) {
+      if (more) fetch(part);
+      compute(buf, part);
+      if (more) stage(buf ^ 1, part);
     }
-    compute(buf, 1);
-    if (more) stage(buf ^ 1, 1);
     __syncthreads();
   }
 
@@ -185,16 +189,35 @@ __global__ void __launch_bounds__(NT, 2)
   }
 }
 
+template <int ACT, bool VEC>
+cudaError_t launch_one(dim3 grid, cudaStream_t stream, const int32_t* nbr,
+                       const uint32_t* tile_mask, int64_t n, const float* x, const float* w,
+                       float* out, int cin, int cout, int flip, const float* bias,
+                       const float* res) {
+  static bool attr_set[64] = {};  // per device and instantiation; a repeat set is harmless
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    e = cudaFuncSetAttribute(fwd_f32_kernel<ACT, VEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes));
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  fwd_f32_kernel<ACT, VEC><<<grid, NT, kSmemBytes, stream>>>(nbr, tile_mask, n, x, w, out, cin,
+                                                             cout, flip, bias, res);
+  return cudaGetLastError();
+}
+
 template <int ACT>
-void launch_act(dim3 grid, bool vec, cudaStream_t stream, const int32_t* nbr,
-                const uint32_t* tile_mask, int64_t n, const float* x, const float* w, float* out,
-                int cin, int cout, int flip, const float* bias, const float* res) {
-  if (vec)
-    fwd_f32_kernel<ACT, true><<<grid, NT, 0, stream>>>(nbr, tile_mask, n, x, w, out, cin, cout,
-                                                       flip, bias, res);
-  else
-    fwd_f32_kernel<ACT, false><<<grid, NT, 0, stream>>>(nbr, tile_mask, n, x, w, out, cin, cout,
-                                                        flip, bias, res);
+cudaError_t launch_act(dim3 grid, bool vec, cudaStream_t stream, const int32_t* nbr,
+                       const uint32_t* tile_mask, int64_t n, const float* x, const float* w,
+                       float* out, int cin, int cout, int flip, const float* bias,
+                       const float* res) {
+  return vec ? launch_one<ACT, true>(grid, stream, nbr, tile_mask, n, x, w, out, cin, cout, flip,
+                                     bias, res)
+             : launch_one<ACT, false>(grid, stream, nbr, tile_mask, n, x, w, out, cin, cout, flip,
+                                      bias, res);
 }
 
 bool aligned16(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; }
@@ -213,15 +236,13 @@ cudaError_t launch_forward_f32(const int32_t* nbr, const uint32_t* tile_mask, in
   const bool vec = cin % 4 == 0 && cout % 4 == 0 && aligned16(feats) && aligned16(weight) &&
                    aligned16(out) && (!res || aligned16(res));
   if (epi.act == kActGelu)
-    launch_act<kActGelu>(grid, vec, stream, nbr, tile_mask, n, feats, weight, out, cin, cout, flip,
-                         bias, res);
-  else if (epi.act == kActSilu)
-    launch_act<kActSilu>(grid, vec, stream, nbr, tile_mask, n, feats, weight, out, cin, cout, flip,
-                         bias, res);
-  else
-    launch_act<kActNone>(grid, vec, stream, nbr, tile_mask, n, feats, weight, out, cin, cout, flip,
-                         bias, res);
-  return cudaGetLastError();
+    return launch_act<kActGelu>(grid, vec, stream, nbr, tile_mask, n, feats, weight, out, cin,
+                                cout, flip, bias, res);
+  if (epi.act == kActSilu)
+    return launch_act<kActSilu>(grid, vec, stream, nbr, tile_mask, n, feats, weight, out, cin,
+                                cout, flip, bias, res);
+  return launch_act<kActNone>(grid, vec, stream, nbr, tile_mask, n, feats, weight, out, cin, cout,
+                              flip, bias, res);
 }
 
 }  // namespace subm3d

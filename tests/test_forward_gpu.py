@@ -82,6 +82,24 @@ def test_f32_without_tile_mask(S):
     assert_close(y, _oracle(c, 16, 1, x, w), RTOL_F32, "f32 no mask")
 
 
+def test_f32_headline_full(S):
+    # the size bench.py times: 2,577 tiles of 128 rows (the last one 111 rows),
+    # 128 -> 128, every output against the oracle
+    wl = WL.make_workload("headline")
+    x, w = wl.features(), wl.weights()[0]
+    _, y = _run(S, wl.coords, 128, 1, x, w, "f32")
+    assert_close(y, _oracle(wl.coords, 128, 1, x, w), RTOL_F32, "headline f32")
+
+
+def test_f32_headline_flip_gelu_sampled(S):
+    wl = WL.make_workload("headline")
+    x, w = wl.features(), wl.weights()[0]
+    _, y = _run(S, wl.coords, 128, 1, x, w, "f32", flip=True, act="gelu")
+    rows = sample_rows(wl.n, 4000, seed=3)  # includes the first and the ragged last tiles
+    ref = _oracle(wl.coords, 128, 1, x, w, flip=True, act="gelu", rows=rows)
+    assert_close(y[rows], ref, RTOL_F32, "headline f32 flip gelu")
+
+
 # ------------------------------------------------------------------ bf16 ----
 
 @pytest.mark.parametrize("flip", [False, True])

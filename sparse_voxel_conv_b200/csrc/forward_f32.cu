@@ -38,11 +38,14 @@ __device__ __forceinline__ float4 load4(const float* __restrict__ base, int64_t 
                                         int cin) {
   if (src < 0 || c >= cin) return make_float4(0.f, 0.f, 0.f, 0.f);
   const float* p = base + src * cin + c;
-  if constexpr (VEC) return __ldg(reinterpret_cast<const float4*>(p));
-  float v[4];
+  if constexpr (VEC) {
+    return __ldg(reinterpret_cast<const float4*>(p));
+  } else {
+    float v[4];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) v[j] = c + j < cin ? __ldg(p + j) : 0.f;
-  return make_float4(v[0], v[1], v[2], v[3]);
+    for (int j = 0; j < 4; ++j) v[j] = c + j < cin ? __ldg(p + j) : 0.f;
+    return make_float4(v[0], v[1], v[2], v[3]);
+  }
 }
 
 // out may alias residual (an in-place residual add): neither is __restrict__.

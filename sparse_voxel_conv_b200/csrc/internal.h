@@ -48,22 +48,34 @@ constexpr int kKvol = 27;
 // int32 (the last tile's end, N rounded up to 128, stays below 2^31).
 constexpr int64_t kMaxMapRows = (int64_t(1) << 31) - 256;
 
-// The two lookup structures of the map build (see map_build.cu).
-enum class MapKind { kDirect, kHash };
+// The three lookup structures of the map build (see map_build.cu).
+enum class MapKind { kDirect, kHash, kBrick };
 
 // The direct-address table (batch * (grid_dim + 2)^3 int32 cells: each grid
-// with a one-cell border) is used while it takes at most
+// with a one-cell border) may be used while it takes at most
 // max(kDirectTableMinBytes, kDirectTableBytesPerVoxel * N) bytes and at most
-// kDirectTableMaxCells cells (int32 cell arithmetic in the query): clearing it
-// costs its size in HBM writes, which beats hashing N voxels until the volume
-// is a few hundred bytes per voxel.
+// kDirectTableMaxCells cells (int32 cell arithmetic in the query).  Clearing it
+// costs its size in HBM writes, so it is chosen while it is small (at most
+// kDirectTableMinBytes) or dense (at most kDirectCellsPerVoxel cells per
+// voxel); sparser volumes take the brick table when its directory fits the
+// same budget, and the hash table otherwise.
 constexpr size_t kDirectTableMinBytes = size_t(64) << 20;
 constexpr double kDirectTableBytesPerVoxel = 256.0;
 constexpr double kDirectTableMaxCells = double(int64_t(1) << 28);
+constexpr double kDirectCellsPerVoxel = 16.0;
 
-// Testing knobs: force the hash table, or cap its capacity (which implies it).
+// The brick table cuts each bordered grid into bricks of 8 (x) x 4 (y) x 2 (z)
+// cells: a directory of int32 (one per brick: -1, or the brick's slot) and a
+// pool of 64-cell int32 blocks, one per occupied brick (at most min(N, bricks)
+// of them, so at most 256 bytes per voxel).
+constexpr int kBrickCells = 64;
+
+// Testing knobs: force one table kind (where it fits), or cap the hash
+// table's capacity (which implies the hash table).
 struct MapOptions {
   bool force_hash = false;
+  bool force_brick = false;
+  bool force_direct = false;
   uint64_t forced_capacity = 0;  // a power of two, or 0
   bool run_layout = true;        // also build the x-run layout (subm3d_forward_map)
 };
@@ -89,12 +101,16 @@ struct MapLayout {
   MapKind kind = MapKind::kDirect;
   bool compact = true;      // hash: 32-bit keys in 8-byte (key, row) slots; else 64-bit keys + rows
   uint64_t capacity = 0;    // hash slots, a power of two >= 4
-  uint64_t cells = 0;       // direct: batch * grid_dim^3
-  size_t status_off = 0;    // uint32 status word
+  uint64_t cells = 0;       // direct: batch * (grid_dim + 2)^3
+  int32_t bgx = 0, bgy = 0, bgz = 0;  // brick: bricks along x, y, z of one bordered grid
+  uint64_t bricks_max = 0;  // brick: pool blocks reserved, min(N, directory entries)
+  size_t status_off = 0;    // uint32 status word (+ the brick counter, uint32, after it)
   size_t mask_off = 0;      // uint32 [n_tiles]
-  size_t table_off = 0;     // direct: int32 [cells]; hash: uint64 [capacity] (slots or keys)
+  size_t table_off = 0;     // direct: int32 [cells]; hash: uint64 [capacity] (slots or keys);
+                            // brick: int32 directory [batch * bgz * bgy * bgx]
   size_t table_bytes = 0;   // bytes of the table (a multiple of 16)
-  size_t rows_off = 0;      // hash, wide keys only: int32 rows [capacity]
+  size_t rows_off = 0;      // hash, wide keys only: int32 rows [capacity];
+                            // brick: int32 pool [bricks_max * kBrickCells]
   // run layout (all kinds)
   size_t cnt_off = 0;       // int32 [n_tiles]: run starts per 128-row tile
   size_t sb_off = 0;        // int32 [ceil(n_tiles / 128)]: run starts per superblock
@@ -113,7 +129,7 @@ struct MapLayout {
 bool map_layout(int64_t n, int32_t grid_dim, int32_t batch, const MapOptions& opt,
                 MapLayout* out);
 
-// Enqueues the three map-build kernels (init, insert, query) on `stream`.
+// Enqueues the map-build kernels (init, [brick allocation,] insert, query) on `stream`.
 // Returns the launch error.  Accepts N < kMaxMapRows.
 cudaError_t launch_map_build(const int32_t* coords, int64_t n, int32_t grid_dim, int32_t batch,
                              int32_t* nbr, void* workspace, const MapLayout& lay,

@@ -2,18 +2,24 @@
 //
 // The pages build a "sorted-key indice map (27 lookups/voxel vectorised)"
 // (lato.2_mrp_mlx, commit 97dcdfb54a message).  Here the lookup structure is
-// one of two GPU tables over packed (b, z, y, x) keys, chosen per call:
+// one of three GPU tables over packed (b, z, y, x) keys, chosen per call:
 //
 //   direct  when batch * (grid_dim + 2)^3 int32 cells take at most max(64 MB,
-//           256 B x N) and 2^28 cells (every 128^3 volume; 4 x 256^3 from
-//           about a million voxels): cell -> row, -1 when empty; each grid has
-//           a one-cell border no voxel occupies, so a voxel's 27 neighbour
-//           cells all exist and its lookups need no bounds test.  A
+//           256 B x N) and 2^28 cells, and the table is small (<= 64 MB) or
+//           dense (<= 16 cells per voxel): cell -> row, -1 when empty; each
+//           grid has a one-cell border no voxel occupies, so a voxel's 27
+//           neighbour cells all exist and its lookups need no bounds test.  A
 //           collision-free perfect hash: insert is one plain store per voxel,
 //           a lookup is one load, and voxels adjacent in raster order look up
-//           adjacent cells, so the 27 lookups of a warp coalesce.  A duplicate coordinate leaves one
-//           of its rows in the cell; the other row sees a foreign row at its
-//           own centre offset and raises the duplicate flag.
+//           adjacent cells, so the 27 lookups of a warp coalesce.  A duplicate
+//           coordinate leaves one of its rows in the cell; the other row sees
+//           a foreign row at its own centre offset and raises the duplicate
+//           flag (likewise in the brick table).
+//   brick   for sparser volumes whose brick directory fits the same budget: the
+//           bordered cells in bricks of 8 (x) x 4 (y) x 2 (z); the directory
+//           (one int32 per brick) is cleared, the occupied bricks get 64-cell
+//           blocks from a counter, and lookups go directory -> block.  Only the
+//           directory and the blocks in use are written, not the whole volume.
 //   hash    otherwise: open addressing with linear probing, capacity a power
 //           of two >= 2N.  With batch <= 4 and grid_dim <= 1024 a key is
 //           b:2|z:10|y:10|x:10 and a slot the 8-byte word (key << 32 | row),
@@ -26,7 +32,9 @@
 // Kernels (each launched with programmatic dependent launch, so that its
 // blocks start while the previous kernel drains and do whatever touches only
 // the build's inputs before griddepcontrol.wait):
-//   map_init    table <- empty, run-count sums, status word and header <- 0;
+//   map_init    table (brick: directory) <- empty, run-count sums, status
+//               word, brick counter and header <- 0;
+//   map_brick_alloc (brick table only) a pool block for every occupied brick;
 //   map_insert  one thread per voxel: 16-byte coordinate load, range check and
 //               the run starts of its 128-row tile (before the wait), then the
 //               insert;
@@ -58,7 +66,8 @@ __global__ void map_init(uint4* a, size_t words16a, uint4* z, size_t words16z, u
   for (size_t t = t0; t < words16a; t += stride) a[t] = ones;
   for (size_t t = t0; t < words16z; t += stride) z[t] = make_uint4(0u, 0u, 0u, 0u);
   if (t0 == 0) {
-    *status = 0u;
+    status[0] = 0u;  // error bits
+    status[1] = 0u;  // brick table: pool blocks handed out
     if (hdr)
       for (int k = 0; k < 4; ++k) hdr[k] = 0;
   }
@@ -130,6 +139,30 @@ __device__ __forceinline__ int32_t insert_prologue(const int4* __restrict__ coor
   return total;
 }
 
+// Brick table: each occupied brick gets a pool block.  The first voxel to
+// claim its directory entry (-1 -> -2) takes the next block from the counter
+// after the status word, fills it with -1 and publishes the block's index; the
+// insert kernel, launched after this grid completes, writes rows into it.
+// Voxels outside the volume are left to the insert kernel's range check.
+__global__ void __launch_bounds__(256)
+    map_brick_alloc(const int4* __restrict__ coords, int n, int grid, int batch, Tables t,
+                    int32_t* __restrict__ dir, int32_t* __restrict__ pool, uint32_t* status) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  const int4 c = i < n ? __ldg(coords + i) : make_int4(-1, -1, -1, -1);
+  pdl_wait();  // the directory and the counter are cleared
+  pdl_trigger();
+  if (i >= n || !in_volume(c, grid, batch)) return;
+  int32_t* d = dir + brick_of(t, c.x, c.y + 1, c.z + 1, c.w + 1);
+  if (*reinterpret_cast<volatile int32_t*>(d) != -1) return;  // claimed already
+  if (atomicCAS(d, -1, -2) != -1) return;
+  const uint32_t slot = atomicAdd(status + 1, 1u);  // < min(N, bricks): one per occupied brick
+  uint4* blk = reinterpret_cast<uint4*>(pool + static_cast<int64_t>(slot) * kBrickCells);
+  const uint4 ones = make_uint4(~0u, ~0u, ~0u, ~0u);
+#pragma unroll
+  for (int k = 0; k < kBrickCells / 4; ++k) blk[k] = ones;
+  *d = static_cast<int32_t>(slot);
+}
+
 template <Kind K>
 __global__ void __launch_bounds__(kInsertThreads)
     map_insert(const int4* __restrict__ coords, int n, int grid, int batch, Tables t,
@@ -148,6 +181,9 @@ __global__ void __launch_bounds__(kInsertThreads)
   }
   if constexpr (K == Kind::kDirect) {
     cells[cell_of(c.x, c.y, c.z, c.w, grid)] = i;
+  } else if constexpr (K == Kind::kBrick) {  // `cells` is the pool, t.rows the directory
+    const int32_t slot = __ldg(t.rows + brick_of(t, c.x, c.y + 1, c.z + 1, c.w + 1));
+    cells[static_cast<int64_t>(slot) * kBrickCells + brick_cell(c.y + 1, c.z + 1, c.w + 1)] = i;
   } else if constexpr (K == Kind::kCompact) {
     const uint32_t key = pack32(c.x, c.y, c.z, c.w);
     const unsigned long long entry =
@@ -277,6 +313,25 @@ __global__ void __launch_bounds__(kTileRows)
               absent = __funnelshift_l(static_cast<uint32_t>(v), absent, 1);  // sign bit in
             }
           }
+        }
+        if (nb[13] != i) atomicOr(status, kErrDuplicate);  // another row owns this cell
+      } else if constexpr (K == Kind::kBrick) {
+        // bordered cells: the 27 directory loads first (mostly one brick), then
+        // the cells of the bricks that exist
+        const int Z = c.y + 1, Y = c.z + 1, X = c.w + 1;
+        int32_t slot[kKvol];
+#pragma unroll
+        for (int k = 0; k < kKvol; ++k)
+          slot[k] = __ldg(t.rows + brick_of(t, c.x, Z + k / 9 - 1, Y + (k / 3) % 3 - 1,
+                                            X + k % 3 - 1));
+#pragma unroll
+        for (int k = 0; k < kKvol; ++k) {
+          const int32_t v =
+              slot[k] < 0 ? -1
+                          : __ldg(t.cells + static_cast<int64_t>(slot[k]) * kBrickCells +
+                                  brick_cell(Z + k / 9 - 1, Y + (k / 3) % 3 - 1, X + k % 3 - 1));
+          nb[k] = v;
+          absent = __funnelshift_l(static_cast<uint32_t>(v), absent, 1);
         }
         if (nb[13] != i) atomicOr(status, kErrDuplicate);  // another row owns this cell
       } else {
@@ -411,8 +466,26 @@ bool map_layout(int64_t n, int32_t grid_dim, int32_t batch, const MapOptions& op
   const double direct_budget = std::max(static_cast<double>(kDirectTableMinBytes),
                                         kDirectTableBytesPerVoxel * static_cast<double>(n));
   const bool direct_fits = cells * 4.0 <= direct_budget && cells <= kDirectTableMaxCells;
-  lay.kind = (direct_fits && !opt.force_hash && opt.forced_capacity == 0) ? MapKind::kDirect
-                                                                         : MapKind::kHash;
+  // brick directory over the bordered grids: bricks of 8 (x) x 4 (y) x 2 (z) cells
+  const int64_t g2 = static_cast<int64_t>(grid_dim) + 2;
+  lay.bgx = static_cast<int32_t>((g2 + 7) / 8);
+  lay.bgy = static_cast<int32_t>((g2 + 3) / 4);
+  lay.bgz = static_cast<int32_t>((g2 + 1) / 2);
+  const double dir_cells = static_cast<double>(batch) * lay.bgz * lay.bgy * lay.bgx;
+  const bool brick_fits = dir_cells * 4.0 <= direct_budget;
+  if (opt.force_hash || opt.forced_capacity != 0)
+    lay.kind = MapKind::kHash;
+  else if (opt.force_brick && brick_fits)
+    lay.kind = MapKind::kBrick;
+  else if (opt.force_direct && direct_fits)
+    lay.kind = MapKind::kDirect;
+  else if (direct_fits && (cells * 4.0 <= static_cast<double>(kDirectTableMinBytes) ||
+                           cells <= kDirectCellsPerVoxel * static_cast<double>(n)))
+    lay.kind = MapKind::kDirect;  // small or dense: clearing the table is cheap
+  else if (brick_fits)
+    lay.kind = MapKind::kBrick;
+  else
+    lay.kind = direct_fits ? MapKind::kDirect : MapKind::kHash;
   lay.compact = (batch <= 4 && grid_dim <= 1024);
   uint64_t cap = 1024;
   while (cap < 2ull * static_cast<uint64_t>(n)) cap <<= 1;
@@ -421,7 +494,7 @@ bool map_layout(int64_t n, int32_t grid_dim, int32_t batch, const MapOptions& op
     while (cap < opt.forced_capacity) cap <<= 1;
   }
   lay.capacity = cap;
-  lay.cells = direct_fits ? static_cast<uint64_t>(cells) : 0;
+  lay.cells = lay.kind == MapKind::kDirect ? static_cast<uint64_t>(cells) : 0;
   lay.n_tiles = (n + kTileRows - 1) / kTileRows;
   lay.status_off = 0;
   lay.mask_off = 256;
@@ -431,6 +504,12 @@ bool map_layout(int64_t n, int32_t grid_dim, int32_t batch, const MapOptions& op
     lay.table_bytes = align_up(lay.cells * 4, 256);
     lay.rows_off = lay.table_off + lay.table_bytes;
     end = lay.rows_off;
+  } else if (lay.kind == MapKind::kBrick) {
+    const uint64_t dir_n = static_cast<uint64_t>(dir_cells);
+    lay.bricks_max = std::max<uint64_t>(1, std::min<uint64_t>(static_cast<uint64_t>(n), dir_n));
+    lay.table_bytes = align_up(dir_n * 4, 256);
+    lay.rows_off = lay.table_off + lay.table_bytes;
+    end = align_up(lay.rows_off + lay.bricks_max * kBrickCells * 4, 256);
   } else {
     lay.table_bytes = cap * 8;
     lay.rows_off = align_up(lay.table_off + lay.table_bytes, 256);
@@ -522,6 +601,18 @@ cudaError_t launch_map_build(const int32_t* coords, int64_t n, int32_t grid_dim,
     launch_build_kernels<Kind::kDirect>(ins_blocks, q_blocks, runs, c4, ni, grid_dim, batch, t,
                                         reinterpret_cast<int32_t*>(table), nullptr, nullptr, nbr,
                                         mask, status, rc, ro, stream);
+  } else if (lay.kind == MapKind::kBrick) {
+    auto* dir = reinterpret_cast<int32_t*>(table);
+    auto* pool = reinterpret_cast<int32_t*>(ws + lay.rows_off);
+    t.cells = pool;
+    t.rows = dir;
+    t.bgx = lay.bgx;
+    t.bgy = lay.bgy;
+    t.bgz = lay.bgz;
+    launch_pdl(map_brick_alloc, static_cast<unsigned>((n + 255) / 256), 256, 0, stream, c4, ni,
+               grid_dim, batch, t, dir, pool, status);
+    launch_build_kernels<Kind::kBrick>(ins_blocks, q_blocks, runs, c4, ni, grid_dim, batch, t,
+                                       pool, nullptr, nullptr, nbr, mask, status, rc, ro, stream);
   } else if (lay.compact) {
     t.table = reinterpret_cast<const unsigned long long*>(table);
     launch_build_kernels<Kind::kCompact>(ins_blocks, q_blocks, runs, c4, ni, grid_dim, batch, t,

@@ -1,8 +1,11 @@
 // The neighbour map's lookup structures (map_build.cu builds them): a
 // direct-address table of int32 rows over batch * (grid + 2)^3 cells (each
 // batch element's grid with a one-cell border that no voxel occupies, so all
-// 27 neighbour cells of a voxel exist and lookups need no bounds test), or an
-// open-addressing hash table with linear probing -- compact 8-byte slots
+// 27 neighbour cells of a voxel exist and lookups need no bounds test); a
+// brick table over the same bordered cells (a directory of 8 x 4 x 2-cell
+// bricks, x fastest, pointing at 64-cell row blocks for the occupied bricks
+// only, -1 elsewhere: two dependent loads per lookup, no bounds test either);
+// or an open-addressing hash table with linear probing -- compact 8-byte slots
 // (key32 << 32 | row) when batch <= 4 and grid_dim <= 1024, else 64-bit keys
 // with a separate int32 row array.  The home slot is 4 * h(key >> 2) + (key & 3)
 // with a 32-bit avalanche mix h, so the x-neighbours of a voxel usually share a
@@ -64,19 +67,34 @@ __device__ __forceinline__ int64_t cell_of(int b, int z, int y, int x, int grid)
   return ((static_cast<int64_t>(b) * g + (z + 1)) * g + (y + 1)) * g + (x + 1);
 }
 
-enum class Kind { kDirect, kCompact, kWide };
+enum class Kind { kDirect, kCompact, kWide, kBrick };
 
 struct Tables {
-  const int32_t* cells;             // direct
+  const int32_t* cells;             // direct cells; brick: the pool of 64-cell blocks
   const unsigned long long* table;  // compact slots or wide keys
-  const int32_t* rows;              // wide rows
+  const int32_t* rows;              // wide rows; brick: the directory
   uint32_t capmask;
+  int32_t bgx, bgy, bgz;            // brick: bricks per bordered grid along x, y, z
 };
+
+// Brick of bordered cell (b, Z, Y, X) (Z = z + 1 ...) in the directory, and the
+// cell's index inside its 64-cell block.
+__device__ __forceinline__ int64_t brick_of(const Tables& t, int b, int Z, int Y, int X) {
+  return ((static_cast<int64_t>(b) * t.bgz + (Z >> 1)) * t.bgy + (Y >> 2)) * t.bgx + (X >> 3);
+}
+__device__ __forceinline__ int brick_cell(int Z, int Y, int X) {
+  return ((Z & 1) * 4 + (Y & 3)) * 8 + (X & 7);
+}
 
 template <Kind K>
 __device__ __forceinline__ int32_t lookup(const Tables& t, int b, int z, int y, int x, int grid) {
   if constexpr (K == Kind::kDirect) {
     return __ldg(t.cells + cell_of(b, z, y, x, grid));
+  } else if constexpr (K == Kind::kBrick) {
+    (void)grid;  // -1 <= z, y, x <= grid: every bordered cell has a directory entry
+    const int32_t s = __ldg(t.rows + brick_of(t, b, z + 1, y + 1, x + 1));
+    return s < 0 ? -1
+                 : __ldg(t.cells + static_cast<int64_t>(s) * 64 + brick_cell(z + 1, y + 1, x + 1));
   } else if constexpr (K == Kind::kCompact) {
     const uint32_t key = pack32(b, z, y, x);
     uint32_t slot = home32(key, t.capmask);

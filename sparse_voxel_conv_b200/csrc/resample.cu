@@ -574,6 +574,16 @@ cudaError_t launch_pool(const MapLayout& map_lay, const void* map_ws, int32_t gr
                                                            feats, channels, out_feats, stream)
              : launch_reduce<Kind::kDirect, float>(mode, pc, total, n, t, grid_dim, batch, feats,
                                                    channels, out_feats, stream);
+  } else if (map_lay.kind == MapKind::kBrick) {
+    t.rows = reinterpret_cast<const int32_t*>(mws + map_lay.table_off);   // directory
+    t.cells = reinterpret_cast<const int32_t*>(mws + map_lay.rows_off);   // blocks
+    t.bgx = map_lay.bgx;
+    t.bgy = map_lay.bgy;
+    t.bgz = map_lay.bgz;
+    e = bf16 ? launch_reduce<Kind::kBrick, __nv_bfloat16>(mode, pc, total, n, t, grid_dim, batch,
+                                                          feats, channels, out_feats, stream)
+             : launch_reduce<Kind::kBrick, float>(mode, pc, total, n, t, grid_dim, batch, feats,
+                                                  channels, out_feats, stream);
   } else if (map_lay.compact) {
     t.table = reinterpret_cast<const unsigned long long*>(mws + map_lay.table_off);
     e = bf16 ? launch_reduce<Kind::kCompact, __nv_bfloat16>(mode, pc, total, n, t, grid_dim,

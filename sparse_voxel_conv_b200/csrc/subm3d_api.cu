@@ -38,13 +38,17 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 //   SUBM3D_TABLE_CAPACITY=<slots>  caps the hash table (and selects it), so that
 //                                  a full table can be exercised;
 //   SUBM3D_MAP_KIND=hash           uses the hash table even where the direct
-//                                  table would fit.
+//                                  or brick table would fit;
+//   SUBM3D_MAP_KIND=brick|direct   uses that table wherever it fits (within
+//                                  the direct table's size budget).
 subm3d::MapOptions options_from_env() {
   subm3d::MapOptions o;
   const char* cap = std::getenv("SUBM3D_TABLE_CAPACITY");
   if (cap && *cap) o.forced_capacity = std::strtoull(cap, nullptr, 10);
   const char* kind = std::getenv("SUBM3D_MAP_KIND");
   if (kind && std::strcmp(kind, "hash") == 0) o.force_hash = true;
+  if (kind && std::strcmp(kind, "brick") == 0) o.force_brick = true;
+  if (kind && std::strcmp(kind, "direct") == 0) o.force_direct = true;
   return o;
 }
 

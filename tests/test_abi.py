@@ -58,6 +58,15 @@ def _expected_ws(n, table_bytes):
     return up(et_off + 9 * (pos_max + 4) * 4)
 
 
+def _brick_bytes(n, grid, batch):
+    """Brick table: an int32 directory over the bordered grids in bricks of
+    8 (x) x 4 (y) x 2 (z) cells, then min(N, bricks) blocks of 64 int32 cells."""
+    up = lambda v: (v + 255) // 256 * 256
+    g2 = grid + 2
+    dirn = batch * ((g2 + 1) // 2) * ((g2 + 3) // 4) * ((g2 + 7) // 8)
+    return up(4 * dirn) + 256 * max(1, min(n, dirn))
+
+
 def test_workspace_bytes(abi, monkeypatch):
     monkeypatch.delenv("SUBM3D_MAP_KIND", raising=False)
     monkeypatch.delenv("SUBM3D_TABLE_CAPACITY", raising=False)
@@ -66,19 +75,28 @@ def test_workspace_bytes(abi, monkeypatch):
     assert f(10, 70000, 1) == 0 and f(10, 16, 70000) == 0
     n = 329839
     # direct table: one int32 per cell of each bordered grid, (grid + 2)^3 cells,
-    # while that takes at most max(64 MB, 256 B x N)
+    # while that fits max(64 MB, 256 B x N) and is at most 64 MB or 16 cells per voxel
     up = lambda v: (v + 255) // 256 * 256
     assert f(n, 128, 1) == _expected_ws(n, up(4 * 130 ** 3))
     small = 1000                                     # budget 64 MB
     assert f(small, 254, 1) == _expected_ws(small, up(4 * 256 ** 3))   # exactly 64 MB
-    assert f(small, 255, 1) == _expected_ws(small, 8 * 2048)           # just over: hash
-    big = 1_135_307                                  # 4 x 258^3 = 275 MB <= 256 B x N
-    assert f(big, 256, 4) == _expected_ws(big, up(4 * 4 * 258 ** 3))
-    assert f(n, 256, 4) == _expected_ws(n, 8 * (1 << 20))      # 275 MB > 84 MB: hash
-    # larger volumes: hash table, 8-byte slots, capacity max(1024, pow2 >= 2N)
-    assert f(n, 512, 1) == _expected_ws(n, 8 * (1 << 20))
-    # wide keys (batch > 4 or grid > 1024) add a 4-byte row array
+    assert f(small, 255, 1) == _expected_ws(small, _brick_bytes(small, 255, 1))  # just over
+    dense = 2_097_152                                # 130^3 cells, 1.05 per voxel
+    assert f(dense, 128, 1) == _expected_ws(dense, up(4 * 130 ** 3))
+    # sparser volumes: the brick table while its directory fits the budget
+    big = 1_135_307                                  # 4 x 258^3 cells = 60 per voxel
+    assert f(big, 256, 4) == _expected_ws(big, _brick_bytes(big, 256, 4))
+    assert f(n, 256, 4) == _expected_ws(n, _brick_bytes(n, 256, 4))
+    assert f(n, 512, 1) == _expected_ws(n, _brick_bytes(n, 512, 1))
+    # beyond: hash table, 8-byte slots, capacity max(1024, pow2 >= 2N); wide keys
+    # (batch > 4 or grid > 1024) add a 4-byte row array
     assert f(n, 2048, 1) == _expected_ws(n, 12 * (1 << 20))
+    assert f(1000, 4000, 1) == _expected_ws(1000, 12 * 2048)
+    monkeypatch.setenv("SUBM3D_MAP_KIND", "direct")  # where it fits
+    assert f(big, 256, 4) == _expected_ws(big, up(4 * 4 * 258 ** 3))
+    assert f(n, 512, 1) == _expected_ws(n, _brick_bytes(n, 512, 1))
+    monkeypatch.setenv("SUBM3D_MAP_KIND", "brick")
+    assert f(n, 128, 1) == _expected_ws(n, _brick_bytes(n, 128, 1))
     monkeypatch.setenv("SUBM3D_MAP_KIND", "hash")
     assert f(n, 128, 1) == _expected_ws(n, 8 * (1 << 20))
     assert f(n, 128, 5) == _expected_ws(n, 12 * (1 << 20))

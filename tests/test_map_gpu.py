@@ -20,14 +20,15 @@ def S():
     return S
 
 
-@pytest.fixture(params=["auto", "hash"])
+@pytest.fixture(params=["auto", "direct", "brick", "hash"])
 def kind(request, monkeypatch):
-    """auto: the direct table where the volume fits max(64 MB, 256 B x N), else the hash
-    table; hash: the hash table everywhere (testing knob SUBM3D_MAP_KIND)."""
-    if request.param == "hash":
-        monkeypatch.setenv("SUBM3D_MAP_KIND", "hash")
-    else:
+    """auto: the library's choice (the direct table for small or dense volumes,
+    the brick table for sparser ones, the hash table beyond both); direct /
+    brick / hash: that table wherever it fits (testing knob SUBM3D_MAP_KIND)."""
+    if request.param == "auto":
         monkeypatch.delenv("SUBM3D_MAP_KIND", raising=False)
+    else:
+        monkeypatch.setenv("SUBM3D_MAP_KIND", request.param)
     return request.param
 
 

@@ -23,12 +23,12 @@ def S():
     return S
 
 
-@pytest.fixture(params=["auto", "hash"])
+@pytest.fixture(params=["auto", "brick", "hash"])
 def kind(request, monkeypatch):
-    if request.param == "hash":
-        monkeypatch.setenv("SUBM3D_MAP_KIND", "hash")
-    else:
+    if request.param == "auto":
         monkeypatch.delenv("SUBM3D_MAP_KIND", raising=False)
+    else:
+        monkeypatch.setenv("SUBM3D_MAP_KIND", request.param)
     return request.param
 
 

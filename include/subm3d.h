@@ -88,10 +88,16 @@ SUBM3D_API const char* subm3d_status_string(int32_t status);
 /*
  * Workspace bytes subm3d_build_map() needs for N voxels in a batch x
  * grid_dim^3 volume: a status word, one 32-bit offset mask per 128-row tile,
- * and the lookup table -- a direct-address table of batch * (grid_dim + 2)^3
- * int32 cells (each grid with a one-cell border) when that is at most
- * max(64 MB, 256 bytes x N) and 2^28 cells, else an open-addressing hash table
- * of at least 2N slots (8 bytes each, 12 with batch > 4 or grid_dim > 1024) --
+ * and the lookup table -- with budget = max(64 MB, 256 bytes x N):
+ *   a direct-address table of batch * (grid_dim + 2)^3 int32 cells (each grid
+ *   with a one-cell border) when that fits the budget and 2^28 cells and is at
+ *   most 64 MB or 16 cells per voxel;
+ *   else a brick table when its directory fits the budget: one int32 per brick
+ *   of 8 (x) x 4 (y) x 2 (z) bordered cells, then min(N, bricks) blocks of 64
+ *   int32 cells (at most 256 bytes per voxel; only occupied bricks' blocks are
+ *   written);
+ *   else an open-addressing hash table of at least 2N slots (8 bytes each, 12
+ *   with batch > 4 or grid_dim > 1024) --
  * and for N < 2^29 the x-run layout of subm3d_forward_map(): run-start counts
  * (an int32 per 128-row tile and per 128 tiles), a header, a position table of
  * 3N int32 (rounded up) and an E index table of 9 lines of as many int32
@@ -104,7 +110,8 @@ SUBM3D_API size_t subm3d_map_workspace_bytes(int64_t n, int32_t grid_dim, int32_
 
 /*
  * Build the neighbour map of a coordinate set ("sorted-key indice map, 27
- * lookups/voxel", lato.2_mrp_mlx commit 97dcdfb54a; here a GPU hash table).
+ * lookups/voxel", lato.2_mrp_mlx commit 97dcdfb54a; here a direct-address,
+ * brick or hash table on the GPU, see subm3d_map_workspace_bytes()).
  *
  *   coords     (device) int32 [N, 4] rows (b, z, y, x), 16-byte aligned, any row order.
  *   n          N >= 0; N < 2^31 - 1.
@@ -120,14 +127,16 @@ SUBM3D_API size_t subm3d_map_workspace_bytes(int64_t n, int32_t grid_dim, int32_
  *   out_map    (host) receives a new handle; release it with subm3d_map_destroy().
  *
  * The map is bit-identical to the plain definition for every valid input and
- * does not depend on the hash layout.  Coordinates outside the volume or
+ * does not depend on the table kind or its layout.  Coordinates outside the volume or
  * repeated are reported by subm3d_map_status(); until it returns SUBM3D_OK the
  * contents of nbr are unspecified.  Besides nbr and the tile masks the build
  * writes, for N < 2^29, the x-run position layout that subm3d_forward_map()
- * uses.  Enqueues 3 kernels; no allocation.  N < 2^31 - 256.
+ * uses.  Enqueues 3 kernels (4 with the brick table); no allocation.
+ * N < 2^31 - 256.
  * Testing knobs, read from the environment by this function and by
- * subm3d_map_workspace_bytes() alike: SUBM3D_MAP_KIND=hash selects the hash
- * table even where the direct table fits; SUBM3D_TABLE_CAPACITY=<slots> caps
+ * subm3d_map_workspace_bytes() alike: SUBM3D_MAP_KIND=direct|brick|hash
+ * selects that table wherever it fits the budget (the hash table always
+ * does); SUBM3D_TABLE_CAPACITY=<slots> caps
  * the hash table (and selects it) so that SUBM3D_E_TABLE_FULL can be
  * exercised -- probe loops stop after `capacity` steps instead of spinning.
  */

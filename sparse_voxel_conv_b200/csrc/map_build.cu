@@ -139,28 +139,54 @@ __device__ __forceinline__ int32_t insert_prologue(const int4* __restrict__ coor
   return total;
 }
 
-// Brick table: each occupied brick gets a pool block.  The first voxel to
-// claim its directory entry (-1 -> -2) takes the next block from the counter
-// after the status word, fills it with -1 and publishes the block's index; the
-// insert kernel, launched after this grid completes, writes rows into it.
-// Voxels outside the volume are left to the insert kernel's range check.
-__global__ void __launch_bounds__(256)
+// Brick table: each occupied brick gets a pool block.  Among a warp's lanes
+// that share a brick the lowest one claims its directory entry (-1 -> -2, after
+// a plain read that turns most claims away); the block's winners then take
+// consecutive blocks from the counter after the status word with one atomic
+// add, fill them with -1 and publish their indices.  The insert kernel,
+// launched after this grid completes, writes rows into them.  Voxels outside
+// the volume are left to the insert kernel's range check.
+constexpr int kAllocThreads = 256;
+
+__global__ void __launch_bounds__(kAllocThreads)
     map_brick_alloc(const int4* __restrict__ coords, int n, int grid, int batch, Tables t,
                     int32_t* __restrict__ dir, int32_t* __restrict__ pool, uint32_t* status) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  __shared__ uint32_t s_won[kAllocThreads / 32];
+  __shared__ uint32_t s_base;
+  const int i = blockIdx.x * kAllocThreads + threadIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int4 c = i < n ? __ldg(coords + i) : make_int4(-1, -1, -1, -1);
+  const bool valid = i < n && in_volume(c, grid, batch);
+  const long long brick = valid ? brick_of(t, c.x, c.y + 1, c.z + 1, c.w + 1) : -1ll;
+  const unsigned peers = __match_any_sync(0xFFFFFFFFu, brick);
   pdl_wait();  // the directory and the counter are cleared
   pdl_trigger();
-  if (i >= n || !in_volume(c, grid, batch)) return;
-  int32_t* d = dir + brick_of(t, c.x, c.y + 1, c.z + 1, c.w + 1);
-  if (*reinterpret_cast<volatile int32_t*>(d) != -1) return;  // claimed already
-  if (atomicCAS(d, -1, -2) != -1) return;
-  const uint32_t slot = atomicAdd(status + 1, 1u);  // < min(N, bricks): one per occupied brick
-  uint4* blk = reinterpret_cast<uint4*>(pool + static_cast<int64_t>(slot) * kBrickCells);
-  const uint4 ones = make_uint4(~0u, ~0u, ~0u, ~0u);
+  bool won = false;
+  if (valid && __ffs(peers) - 1 == lane) {
+    int32_t* d = dir + brick;
+    won = *reinterpret_cast<volatile int32_t*>(d) == -1 && atomicCAS(d, -1, -2) == -1;
+  }
+  const unsigned wins = __ballot_sync(0xFFFFFFFFu, won);
+  if (lane == 0) s_won[warp] = __popc(wins);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t total = 0;
+    for (int w = 0; w < kAllocThreads / 32; ++w) {
+      const uint32_t k = s_won[w];
+      s_won[w] = total;  // exclusive prefix over the warps
+      total += k;
+    }
+    s_base = total ? atomicAdd(status + 1, total) : 0u;  // < min(N, bricks) blocks in all
+  }
+  __syncthreads();
+  if (won) {
+    const uint32_t slot = s_base + s_won[warp] + __popc(wins & ((1u << lane) - 1u));
+    uint4* blk = reinterpret_cast<uint4*>(pool + static_cast<int64_t>(slot) * kBrickCells);
+    const uint4 ones = make_uint4(~0u, ~0u, ~0u, ~0u);
 #pragma unroll
-  for (int k = 0; k < kBrickCells / 4; ++k) blk[k] = ones;
-  *d = static_cast<int32_t>(slot);
+    for (int k = 0; k < kBrickCells / 4; ++k) blk[k] = ones;
+    dir[brick] = static_cast<int32_t>(slot);
+  }
 }
 
 template <Kind K>
@@ -609,8 +635,8 @@ cudaError_t launch_map_build(const int32_t* coords, int64_t n, int32_t grid_dim,
     t.bgx = lay.bgx;
     t.bgy = lay.bgy;
     t.bgz = lay.bgz;
-    launch_pdl(map_brick_alloc, static_cast<unsigned>((n + 255) / 256), 256, 0, stream, c4, ni,
-               grid_dim, batch, t, dir, pool, status);
+    launch_pdl(map_brick_alloc, static_cast<unsigned>((n + kAllocThreads - 1) / kAllocThreads),
+               kAllocThreads, 0, stream, c4, ni, grid_dim, batch, t, dir, pool, status);
     launch_build_kernels<Kind::kBrick>(ins_blocks, q_blocks, runs, c4, ni, grid_dim, batch, t,
                                        pool, nullptr, nullptr, nbr, mask, status, rc, ro, stream);
   } else if (lay.compact) {

@@ -78,6 +78,22 @@ def test_map_wide_keys(S, kind, grid, batch, shift):
     assert np.array_equal(masks, masks_from_nbr(ref))
 
 
+@pytest.fixture(scope="module")
+def large_sparse():
+    """Two 512^3 grids of large shells: 615,658 voxels, 441 cells per voxel, so
+    the direct table (1.09 GB) exceeds the budget and the library's choice is the
+    brick table (a 17 MB directory)."""
+    c = WL.batched_coords(batch=2, grid=512, min_voxels=120_000, seed0=7, r_lo=40.0, r_hi=120.0)
+    return c, C.build_map(c, 512, 2)
+
+
+def test_map_large_sparse_volume(S, kind, large_sparse):
+    c, ref = large_sparse
+    _, nbr, masks = _gpu_map(S, c, 512, 2)
+    assert np.array_equal(nbr, ref)
+    assert np.array_equal(masks, masks_from_nbr(ref))
+
+
 def test_map_edge_sizes(S, kind):
     for c in (np.zeros((0, 4), np.int32), np.array([[0, 3, 3, 3]], np.int32),
               WL.dense_coords(5)[:129], WL.dense_coords(2)):

@@ -236,7 +236,8 @@ SUBM3D_API subm3d_status subm3d_build_map_noalloc(const int32_t* coords, int64_t
 /*
  * Forward of one layer over a built map -- the same op and arguments as
  * subm3d_forward(), with N, nbr and the masks taken from the map.  For bf16
- * with Cin a multiple of 64 (and a map of N < 2^29) it runs the x-run kernel,
+ * with Cin >= 48 (and a map of N < 2^29) it runs the x-run kernel (Cin in
+ * 64-channel chunks, the last one zero-padded when Cin is not a multiple of 64),
  * which uses the map's position layout: voxels on a line of positions in row
  * order, two pad positions before every run of x-adjacent voxels, tiles of
  * 256 positions, and per tile and (dz, dy) one gathered tile of feature rows

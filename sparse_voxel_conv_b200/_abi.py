@@ -196,7 +196,7 @@ def subm3d_forward(nbr, tile_mask, n: int, feats, weight, out, cin: int, cout: i
 def subm3d_forward_map(handle: MapHandle, feats, weight, out, cin: int, cout: int, dtype: int,
                        flip: bool, act: int, stream=None) -> None:
     """Enqueue one layer's forward over a built map (x-run kernel for bf16 with
-    Cin % 64 == 0); raises Subm3dError on an argument error."""
+    Cin >= 48); raises Subm3dError on an argument error."""
     st = lib.subm3d_forward_map(handle.ptr, _ptr(feats), _ptr(weight), _ptr(out), int(cin),
                                 int(cout), int(dtype), 1 if flip else 0, int(act),
                                 _stream(stream))

@@ -246,12 +246,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&e_empty[s], st.phase ^ 1u, wctl))) break;
       const __nv_bfloat16* xcol = a.x + st.j * CHUNK + piece * 8;
       const uint32_t e_base = smem_u32(e_ring) + static_cast<uint32_t>(s) * E_SLOT;
+      if (st.j * CHUNK + piece * 8 < a.cin) {
 #pragma unroll
-      for (int q = 0; q <= PPT; ++q) {
-        if (q == PPT && !edge) break;
-        cp_async_16(e_base + dst_off[q],
-                    src[q] >= 0 ? xcol + static_cast<int64_t>(src[q]) * a.cin : a.x,
-                    src[q] >= 0 ? 16u : 0u);
+        for (int q = 0; q <= PPT; ++q) {
+          if (q == PPT && !edge) break;
+          cp_async_16(e_base + dst_off[q],
+                      src[q] >= 0 ? xcol + static_cast<int64_t>(src[q]) * a.cin : a.x,
+                      src[q] >= 0 ? 16u : 0u);
+        }
+      } else {
+        // a piece past cin (the last chunk of a cin that is not a multiple of
+        // 64): zeros, so that the chunk's four K steps add nothing there (the
+        // weight slice's columns past cin are zero-filled by the TMA load)
+#pragma unroll
+        for (int q = 0; q <= PPT; ++q) {
+          if (q == PPT && !edge) break;
+          cp_async_16(e_base + dst_off[q], a.x, 0u);
+        }
       }
       cp_async_mbar_arrive_noinc(&e_full[s]);
       st.next(a.n_kchunks, SE);
@@ -456,7 +467,7 @@ cudaError_t launch_forward_bf16_runs(const int32_t* pos, const int32_t* etable,
   a.cin = cin;
   a.cout = cout;
   a.n_oblocks = (cout + TO - 1) / TO;
-  a.n_kchunks = cin / CHUNK;
+  a.n_kchunks = (cin + CHUNK - 1) / CHUNK;
   a.se = se;
   a.sw = sw;
   a.flip = flip;

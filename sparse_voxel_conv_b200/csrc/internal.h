@@ -168,7 +168,7 @@ cudaError_t launch_forward_bf16(const int32_t* nbr, const uint32_t* tile_mask, i
                                 const DeviceCtl& ctl, cudaStream_t stream);
 
 // bf16 forward over the x-run position layout (forward_bf16_runs_sm100.cu);
-// Cin a multiple of 64, Cout a multiple of 16.
+// Cin and Cout multiples of 16 (Cin in 64-channel chunks, the last zero-padded).
 cudaError_t launch_forward_bf16_runs(const int32_t* pos, const int32_t* etable,
                                      int64_t et_stride, const int32_t* header, int64_t max_tiles,
                                      const void* feats,

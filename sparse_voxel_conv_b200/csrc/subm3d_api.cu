@@ -194,13 +194,16 @@ bool overlaps(const void* p, size_t p_bytes, const void* q, size_t q_bytes) {
   return a < b + q_bytes && b < a + p_bytes;
 }
 
-// Kernel choice for a map with an x-run layout: the x-run kernel.  It does
-// tensor work on every position (voxels and pads) for all 27 offsets, the
-// per-offset kernel on every voxel for the offsets present in its 256-row tile
-// but with ~3x the gathered bytes; timed with the GELU epilogue on three sets
-// (x-runs of 9.3 and 4.0 voxels, 1.22 and 1.50 positions per voxel) at 64 and
-// 128 input and output channels, the x-run kernel was faster in every case, by
-// 14% (4 x 256^3 shells, 64 -> 128) to 2.1x.
+// Kernel choice for a map with an x-run layout: the x-run kernel when Cin >= 48.
+// It does tensor work on every position (voxels and pads) for all 27 offsets,
+// the per-offset kernel on every voxel for the offsets present in its 256-row
+// tile but with ~3x the gathered bytes; timed with the GELU epilogue on three
+// sets (x-runs of 9.3 and 4.0 voxels, 1.22 and 1.50 positions per voxel) at 64
+// and 128 input and output channels, the x-run kernel was faster in every case,
+// by 14% (4 x 256^3 shells, 64 -> 128) to 2.1x; with a partial last chunk it is
+// 2.0-2.3x faster at 48 and 80 input channels on the headline set and 1.4x at
+// 96 -> 64 on the decoder-stack set, but at 32 channels (half of its only
+// chunk zeros) it is no faster than the per-offset kernel, which keeps Cin < 48.
 // Testing knob SUBM3D_FORWARD_KERNEL (read at every call): "gather" takes the
 // per-offset kernel even where the x-run kernel applies.
 bool prefer_gather() {
@@ -256,7 +259,7 @@ subm3d_status forward_impl(const subm3d_map* map, const int32_t* nbr, const uint
   if (!ctl.err_word) return SUBM3D_E_CUDA;
   ctl.wait_limit_ns = wait_limit_from_env();
   cudaError_t e;
-  if (map && map->pos && cin % 64 == 0 && !prefer_gather())
+  if (map && map->pos && cin >= 48 && !prefer_gather())  // cin % 16 == 0 (checked above)
     e = subm3d::launch_forward_bf16_runs(map->pos, map->et, map->layout.et_stride, map->hdr,
                                          map->ptile_max, feats,
                                          weight, out, cin, cout, flip01, epi, ctl, s);

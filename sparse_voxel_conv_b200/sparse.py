@@ -88,7 +88,7 @@ def forward(h: MapHandle, feats: torch.Tensor, weight: torch.Tensor, flip: bool 
     act: None, "gelu" (exact erf form) or "silu".  bias: optional [Cout];
     residual: optional [N, Cout] (may be `out`), both of the feature dtype.
     kernel: "auto" runs subm3d_forward_fused (the x-run kernel for bf16 with
-    Cin % 64 == 0); "gather" runs subm3d_forward on nbr and the tile masks
+    Cin >= 48); "gather" runs subm3d_forward on nbr and the tile masks
     (use_tile_mask=False: no masks; no bias or residual there).
     """
     if feats.dtype not in _DTYPES:

@@ -196,6 +196,17 @@ def test_bf16_headline_flip_sampled(S):
     assert_close(y[rows], ref, RTOL_BF16, "headline flip")
 
 
+@pytest.mark.parametrize("cin,cout", [(80, 128), (48, 48)])
+def test_bf16_headline_partial_chunk_sampled(S, cin, cout):
+    # the x-run kernel with a partial last 64-channel chunk, over all 1,567 tiles
+    wl = WL.make_workload("headline")
+    x, w = _inputs(wl.coords, cin, cout, "bf16", seed=cin)
+    _, y = _run(S, wl.coords, 128, 1, x, w, "bf16", act="gelu")
+    rows = sample_rows(wl.n, 4000, seed=cin)
+    ref = _oracle(wl.coords, 128, 1, x, w, act="gelu", bf16_out=True, rows=rows)
+    assert_close(y[rows], ref, RTOL_BF16, f"headline {cin}->{cout}")
+
+
 def test_bf16_dense_sampled_and_vs_conv3d(S):
     wl = WL.make_workload("dense")
     x, w = wl.features(), wl.weights()[0]
@@ -277,17 +288,18 @@ def test_bf16_both_kernels_agree_with_oracle(S, name, flip):
 
 
 def test_kernel_choice_and_knob(S, monkeypatch):
-    """subm3d_forward_map runs the x-run kernel wherever its layout applies, on
-    short runs too (the 64^3 shell: runs of ~4 voxels, 1.50 N positions), at 64
-    and 128 input channels; SUBM3D_FORWARD_KERNEL=gather switches it to the
-    per-offset kernel of subm3d_forward.  Each kernel is deterministic, so the
-    results match bit for bit the kernel that ran."""
+    """subm3d_forward_map runs the x-run kernel wherever its layout applies and
+    Cin >= 48, on short runs too (the 64^3 shell: runs of ~4 voxels, 1.50 N
+    positions); at 48 and 80 input channels its last 64-channel chunk is partial
+    (zero-filled past Cin).  Below 48 channels it takes the per-offset kernel of
+    subm3d_forward, and SUBM3D_FORWARD_KERNEL=gather does so everywhere.  Each
+    kernel is deterministic, so results match bit for bit the kernel that ran."""
     wl = WL.make_workload("shell_bf16")
     c = torch.from_numpy(wl.coords).cuda()
     h = S.build_map(c, wl.grid_dim, wl.batch)
     hdr = S.run_layout_tensors(h)[2].cpu().numpy()
     assert hdr[2] > 1.45 * wl.n
-    for cin in (64, 128):
+    for cin in (32, 48, 64, 80, 128):
         xt = torch.from_numpy(WL.to_bf16_values(WL.make_features(wl.n, cin, 41))).cuda().to(
             torch.bfloat16)
         wt = torch.from_numpy(WL.to_bf16_values(WL.make_weight(64, cin, 42))).cuda().to(
@@ -300,6 +312,8 @@ def test_kernel_choice_and_knob(S, monkeypatch):
         torch.cuda.synchronize()
         assert S._abi.subm3d_device_status() == 0
         assert torch.equal(knob, gather), cin
+        if cin < 48:
+            assert torch.equal(auto, gather), cin
         ref = _oracle(wl.coords, wl.grid_dim, 1, xt.float().cpu().numpy(),
                       wt.float().cpu().numpy(), bf16_out=True)
         for what, y in (("auto", auto), ("gather", gather)):

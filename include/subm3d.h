@@ -302,10 +302,10 @@ SUBM3D_API subm3d_status subm3d_forward_fused(const subm3d_map* map, const void*
  * subm3d_backward_weight: dW[o][kw][c] = sum_i dy[i][o] * feats[nbr[i][k]][c]
  * over nbr[i][k] != -1, kw = k (flip = 0) or 26 - k.  dweight is fp32 KRSC
  * [Cout, 3, 3, 3, Cin] (device, 4-byte aligned, overwritten; fp32 for both
- * dtypes: the sum runs over all voxels).  bf16 with Cin a multiple of 64 runs
- * on the tensor cores over the map's x-run layout (the sum over positions as
+ * dtypes: the sum runs over all voxels).  bf16 (with the map's x-run layout)
+ * runs on the tensor cores over that layout (the sum over positions as
  * the MMA K dimension, one gathered tile per (dz, dy) pair for all three dx);
- * other shapes and fp32 on CUDA-core FMA.  Partial sums over voxel ranges are
+ * fp32, and maps without that layout, on CUDA-core FMA.  Partial sums over voxel ranges are
  * added with fp32 atomics, so the summation order (and the last bits) vary
  * from call to call.
  *

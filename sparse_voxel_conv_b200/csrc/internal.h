@@ -185,7 +185,7 @@ cudaError_t launch_wgrad(const int32_t* nbr, int64_t n, const void* x, const voi
                          cudaStream_t stream);
 
 // bf16 weight gradient over the x-run layout on tcgen05 (wgrad_bf16_runs_sm100.cu):
-// Cin a multiple of 64, Cout a multiple of 16; zeroes dw, then accumulates.
+// Cin and Cout multiples of 16; zeroes dw, then accumulates.
 cudaError_t launch_wgrad_bf16_runs(const int32_t* pos, const int32_t* etable,
                                    int64_t et_stride, const int32_t* header, const void* feats, const void* dy,
                                    float* dw, int32_t cin, int32_t cout, int32_t flip,

@@ -341,7 +341,7 @@ subm3d_status subm3d_backward_weight(const subm3d_map* map, const void* feats, c
                 overlaps(dweight, dw_bytes, dy, static_cast<size_t>(n) * cout * esz)))
     return SUBM3D_E_INVALID;
   auto s = static_cast<cudaStream_t>(stream);
-  if (n > 0 && dtype == SUBM3D_BF16 && map->pos && cin % 64 == 0 && cout % 16 == 0 &&
+  if (n > 0 && dtype == SUBM3D_BF16 && map->pos && cin % 16 == 0 && cout % 16 == 0 &&
       aligned(feats, 16) && aligned(dy, 16) && aligned(dweight, 16) && device_is_sm100(nullptr) == 1) {
     subm3d::DeviceCtl ctl;
     ctl.err_word = device_error_word();

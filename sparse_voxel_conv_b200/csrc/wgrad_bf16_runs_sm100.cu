@@ -285,10 +285,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) subm3d_wgrad_bf16_runs_sm100(c
           tmem_ld_wait();
           if (o < a.cout && c < a.cin) {
             float* dst = a.dw + (static_cast<int64_t>(o) * kKvol + kw) * a.cin + c;
+            // cin is a multiple of 16: each 4-channel group is inside or past it
 #pragma unroll
             for (int t = 0; t < 32; t += 4)
-              red_add_v4(dst + t, __uint_as_float(v[t]), __uint_as_float(v[t + 1]),
-                         __uint_as_float(v[t + 2]), __uint_as_float(v[t + 3]));
+              if (c + t < a.cin)
+                red_add_v4(dst + t, __uint_as_float(v[t]), __uint_as_float(v[t + 1]),
+                           __uint_as_float(v[t + 2]), __uint_as_float(v[t + 3]));
           }
         }
       }

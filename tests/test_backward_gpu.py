@@ -19,7 +19,7 @@ pytestmark = pytest.mark.gpu
 RTOL_WGRAD = 1e-4
 
 # (name, dtype, cin, cout).  The input gradient is a forward Cout -> Cin, so
-# xrun runs the x-run kernel there (Cout % 64 == 0), gather the per-offset one.
+# xrun runs the x-run kernel there (Cout >= 48), gather the per-offset one.
 PATHS = [("xrun", "bf16", 64, 128), ("gather", "bf16", 48, 32), ("f32", "f32", 24, 40)]
 
 
@@ -123,12 +123,13 @@ def test_autograd_through_subm_conv(S):
                  "autograd dW")
 
 
-@pytest.mark.parametrize("cin,cout", [(128, 128), (192, 64), (64, 144)])
+@pytest.mark.parametrize("cin,cout", [(128, 128), (192, 64), (64, 144), (80, 64), (48, 48)])
 @pytest.mark.parametrize("flip", [False, True])
 def test_backward_weight_tensor_core_blocks(S, shell, cin, cout, flip):
     """The tcgen05 weight gradient over channel blocks of 128: full blocks, a
     partial input-channel block (192 = 128 + 64), output channels below and
-    above one block (64, 144 = 128 + 16)."""
+    above one block (64, 144 = 128 + 16), and input channels that end inside a
+    64-channel chunk (80 = 64 + 16, 48)."""
     wl, nbr = shell
     h, x, w, dy, xt, wt, dyt = _tensors(S, wl, "bf16", cin, cout, 61)
     dw = S.backward_weight(h, xt, dyt, flip=flip)

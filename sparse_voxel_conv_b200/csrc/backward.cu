@@ -10,12 +10,12 @@
 //
 // Weight gradient.  dW[o][kw][c] = sum_i dy[i][o] * x[nbr[i][k]][c], kw = k or
 // 26-k under flip: for each offset a [Cout x N] . [N x Cin] product whose
-// reduction runs over the voxels.  wgrad_kernel: a block takes a 64 x 64 (o, c)
-// tile of one offset and a slice of the voxels, stages 16-voxel slices of dy and
-// of the gathered x rows (zero where nbr = -1) in shared memory, accumulates a
-// 4 x 4 fp32 register tile per thread and adds the block's partial tile into
-// the fp32 dW with atomics (dW is zeroed first).  CUDA-core FMA; bf16 inputs are
-// widened to fp32.
+// reduction runs over the voxels.  wgrad_kernel: a block takes a 128 x 128
+// (o, c) tile of one offset and a slice of the voxels, stages 32-voxel slices of
+// dy and of the gathered x rows (zero where nbr = -1) in shared memory,
+// accumulates an 8 x 8 fp32 register tile per thread and adds the block's
+// partial tile into the fp32 dW with atomics (dW is zeroed first).  CUDA-core
+// FMA; bf16 inputs are widened to fp32.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -55,64 +55,145 @@ __global__ void __launch_bounds__(256) transpose_weight_kernel(const T* __restri
   }
 }
 
-constexpr int WB = 64, WK = 16, WT = 256;  // tile 64 x 64, 16 voxels per slice, 256 threads
+// Weight-gradient tile: 128 output x 128 input channels of one offset per block,
+// 256 threads with an 8 x 8 register tile each (o = 4 ty .. 4 ty + 3 and
+// 64 + 4 ty ..; c likewise with tx), K = the voxels of the block's slice in
+// steps of 32.  Both operands are voxel-major rows -- dy[i][o0 ..] and the
+// gathered x[nbr[i][k]][c0 ..] (zero where nbr = -1) -- so a step stages them
+// with 16-byte stores as they come, in two shared buffers; the next step loads
+// into registers in four 8-voxel parts while this step's FMAs run.
+constexpr int WB = 128, WK = 32, WT = 256, WP = 8;
+constexpr int kWgradFloats = WK * WB;                       // one operand, one buffer
+constexpr size_t kWgradSmemBytes = 4 * kWgradFloats * 4;    // two operands x two buffers
 
-template <typename T>
-__global__ void __launch_bounds__(WT)
+// Four consecutive values at p (converted to fp32), zeros where past `limit`.
+template <typename T, bool VEC>
+__device__ __forceinline__ float4 load4_row(const T* __restrict__ p, int first, int limit) {
+  if (first >= limit) return make_float4(0.f, 0.f, 0.f, 0.f);
+  if constexpr (VEC) {
+    if constexpr (sizeof(T) == 4) {
+      return __ldg(reinterpret_cast<const float4*>(p));
+    } else {
+      const uint2 r = __ldg(reinterpret_cast<const uint2*>(p));
+      return make_float4(__uint_as_float(r.x << 16), __uint_as_float(r.x & 0xFFFF0000u),
+                         __uint_as_float(r.y << 16), __uint_as_float(r.y & 0xFFFF0000u));
+    }
+  } else {
+    float v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] = first + j < limit ? to_f32(p[j]) : 0.f;
+    return make_float4(v[0], v[1], v[2], v[3]);
+  }
+}
+
+template <typename T, bool VEC>
+__global__ void __launch_bounds__(WT, 2)
     wgrad_kernel(const int32_t* __restrict__ nbr, int64_t n, const T* __restrict__ x,
                  const T* __restrict__ dy, float* __restrict__ dw, int cin, int cout, int flip,
                  int64_t rows_per_split) {
-  __shared__ __align__(16) float s_a[WK][WB];  // dy slice: [voxel][o]
-  __shared__ __align__(16) float s_b[WK][WB];  // gathered x slice: [voxel][c]
+  extern __shared__ float4 smem_w4[];
+  auto s_a = reinterpret_cast<float (*)[WK][WB]>(smem_w4);                       // [2] dy
+  auto s_b = reinterpret_cast<float (*)[WK][WB]>(reinterpret_cast<float*>(smem_w4) +
+                                                 2 * kWgradFloats);             // [2] x
   const int k = blockIdx.y;
   const int n_ct = (cin + WB - 1) / WB;
   const int o0 = (blockIdx.x / n_ct) * WB, c0 = (blockIdx.x % n_ct) * WB;
   const int64_t i_begin = static_cast<int64_t>(blockIdx.z) * rows_per_split;
   const int64_t i_end = i_begin + rows_per_split < n ? i_begin + rows_per_split : n;
-  const int t = threadIdx.x, tx = t % 16, ty = t / 16;
-  float acc[4][4] = {};
-  for (int64_t i0 = i_begin; i0 < i_end; i0 += WK) {
-    // 16 voxels x 64 channels of each operand: 1024 elements, 4 per thread
+  const int steps = static_cast<int>((i_end - i_begin + WK - 1) / WK);
+  const int t = threadIdx.x;
+  // staging role: voxel t / 32 of the part, channels 4 (t % 32) .. + 3
+  const int sv = t >> 5, sg = (t & 31) * 4;
+  // compute role
+  const int ty = t >> 4, tx = t & 15;
+
+  float4 ra, rb;
+  auto fetch = [&](int step, int part) {
+    const int v = part * WP + sv;
+    const int64_t i = i_begin + static_cast<int64_t>(step) * WK + v;
+    if (i < i_end) {
+      ra = load4_row<T, VEC>(dy + i * cout + o0 + sg, o0 + sg, cout);
+      const int32_t j = __ldg(nbr + i * kKvol + k);
+      rb = j >= 0 ? load4_row<T, VEC>(x + static_cast<int64_t>(j) * cin + c0 + sg, c0 + sg, cin)
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
+    } else {
+      ra = rb = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  auto stage = [&](int buf, int part) {
+    const int v = part * WP + sv;
+    *reinterpret_cast<float4*>(&s_a[buf][v][sg]) = ra;
+    *reinterpret_cast<float4*>(&s_b[buf][v][sg]) = rb;
+  };
+  float acc[8][8];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int idx = t + e * WT;
-      const int v = idx / WB, col = idx % WB;
-      const int64_t i = i0 + v;
-      float a = 0.0f, b = 0.0f;
-      if (i < i_end) {
-        if (o0 + col < cout) a = to_f32(dy[i * cout + o0 + col]);
-        const int32_t j = nbr[i * kKvol + k];
-        if (j >= 0 && c0 + col < cin) b = to_f32(x[static_cast<int64_t>(j) * cin + c0 + col]);
-      }
-      s_a[v][col] = a;
-      s_b[v][col] = b;
+  for (int m = 0; m < 8; ++m)
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[m][q] = 0.f;
+
+  if (steps > 0) {
+#pragma unroll 1
+    for (int part = 0; part < WK / WP; ++part) {
+      fetch(0, part);
+      stage(0, part);
     }
     __syncthreads();
+  }
+  for (int s = 0; s < steps; ++s) {
+    const int buf = s & 1;
+    const bool more = s + 1 < steps;
 #pragma unroll
-    for (int kk = 0; kk < WK; ++kk) {
-      float av[4], bv[4];
+    for (int part = 0; part < WK / WP; ++part) {
+      if (more) fetch(s + 1, part);
 #pragma unroll
-      for (int m = 0; m < 4; ++m) av[m] = s_a[kk][ty * 4 + m];
+      for (int q = 0; q < WP; ++q) {
+        const int kk = part * WP + q;
+        const float4 a0 = *reinterpret_cast<const float4*>(&s_a[buf][kk][ty * 4]);
+        const float4 a1 = *reinterpret_cast<const float4*>(&s_a[buf][kk][64 + ty * 4]);
+        const float4 b0 = *reinterpret_cast<const float4*>(&s_b[buf][kk][tx * 4]);
+        const float4 b1 = *reinterpret_cast<const float4*>(&s_b[buf][kk][64 + tx * 4]);
+        const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-      for (int m = 0; m < 4; ++m) bv[m] = s_b[kk][tx * 4 + m];
+        for (int m = 0; m < 8; ++m)
 #pragma unroll
-      for (int m = 0; m < 4; ++m)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[m][q] = fmaf(av[m], bv[q], acc[m][q]);
+          for (int r = 0; r < 8; ++r) acc[m][r] = fmaf(av[m], bv[r], acc[m][r]);
+      }
+      if (more) stage(buf ^ 1, part);
     }
     __syncthreads();
   }
   const int kw = flip ? 26 - k : k;
 #pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    const int o = o0 + ty * 4 + m;
+  for (int m = 0; m < 8; ++m) {
+    const int o = o0 + (m < 4 ? ty * 4 + m : 64 + ty * 4 + m - 4);
     if (o >= cout) continue;
+    float* row = dw + (static_cast<int64_t>(o) * kKvol + kw) * cin;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int c = c0 + tx * 4 + q;
-      if (c < cin) atomicAdd(dw + (static_cast<int64_t>(o) * kKvol + kw) * cin + c, acc[m][q]);
+    for (int r = 0; r < 8; ++r) {
+      const int c = c0 + (r < 4 ? tx * 4 + r : 64 + tx * 4 + r - 4);
+      if (c < cin) atomicAdd(row + c, acc[m][r]);
     }
   }
+}
+
+template <typename T, bool VEC>
+cudaError_t launch_wgrad_kernel(dim3 grid, cudaStream_t stream, const int32_t* nbr, int64_t n,
+                                const void* x, const void* dy, float* dw, int cin, int cout,
+                                int flip, int64_t rows) {
+  static bool attr_set[64] = {};  // per device and instantiation; a repeat set is harmless
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    e = cudaFuncSetAttribute(wgrad_kernel<T, VEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kWgradSmemBytes));
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  wgrad_kernel<T, VEC><<<grid, WT, kWgradSmemBytes, stream>>>(
+      nbr, n, static_cast<const T*>(x), static_cast<const T*>(dy), dw, cin, cout, flip, rows);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -136,22 +217,27 @@ cudaError_t launch_wgrad(const int32_t* nbr, int64_t n, const void* x, const voi
       cudaMemsetAsync(dw, 0, static_cast<size_t>(cout) * kKvol * cin * sizeof(float), stream);
   if (e != cudaSuccess || n == 0) return e;
   const int tiles = ((cout + WB - 1) / WB) * ((cin + WB - 1) / WB);
-  // split the voxels so that the grid covers the SMs about 8 times over
+  // split the voxels so that the grid covers the SMs (two blocks each) about 4 times
   int64_t splits = (static_cast<int64_t>(num_sms) * 8 + tiles * kKvol - 1) / (tiles * kKvol);
   if (splits < 1) splits = 1;
   int64_t rows = (n + splits - 1) / splits;
   rows = (rows + WK - 1) / WK * WK;
   splits = (n + rows - 1) / rows;
   const dim3 grid(static_cast<unsigned>(tiles), kKvol, static_cast<unsigned>(splits));
+  // 16-byte (fp32) or 8-byte (bf16) row pieces where the rows allow
+  const size_t esz = bf16 ? 2 : 4;
+  const bool vec = cin % 4 == 0 && cout % 4 == 0 &&
+                   reinterpret_cast<uintptr_t>(x) % (4 * esz) == 0 &&
+                   reinterpret_cast<uintptr_t>(dy) % (4 * esz) == 0;
   if (bf16)
-    wgrad_kernel<__nv_bfloat16><<<grid, WT, 0, stream>>>(
-        nbr, n, static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(dy), dw,
-        cin, cout, flip, rows);
-  else
-    wgrad_kernel<float><<<grid, WT, 0, stream>>>(nbr, n, static_cast<const float*>(x),
-                                                 static_cast<const float*>(dy), dw, cin, cout,
-                                                 flip, rows);
-  return cudaGetLastError();
+    return vec ? launch_wgrad_kernel<__nv_bfloat16, true>(grid, stream, nbr, n, x, dy, dw, cin,
+                                                         cout, flip, rows)
+               : launch_wgrad_kernel<__nv_bfloat16, false>(grid, stream, nbr, n, x, dy, dw, cin,
+                                                          cout, flip, rows);
+  return vec ? launch_wgrad_kernel<float, true>(grid, stream, nbr, n, x, dy, dw, cin, cout, flip,
+                                                rows)
+             : launch_wgrad_kernel<float, false>(grid, stream, nbr, n, x, dy, dw, cin, cout, flip,
+                                                 rows);
 }
 
 }  // namespace subm3d

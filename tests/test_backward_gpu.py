@@ -99,6 +99,33 @@ def test_backward_weight_ragged_and_empty(S):
     assert torch.count_nonzero(dw0).item() == 0     # the gradient of an empty sum is zero
 
 
+@pytest.mark.parametrize("cin,cout", [(3, 5), (70, 130), (128, 128)])
+def test_backward_weight_f32_shapes(S, shell, cin, cout):
+    """The CUDA-core weight gradient (fp32): element-wise row pieces where Cin or
+    Cout is not a multiple of 4, two output-channel blocks (130), whole tiles."""
+    wl, nbr = shell
+    h, x, w, dy, xt, wt, dyt = _tensors(S, wl, "f32", cin, cout, 71)
+    dw = S.backward_weight(h, xt, dyt)
+    torch.cuda.synchronize()
+    ref = C.backward_weight(nbr, x.astype(np.float64), dy.astype(np.float64))
+    assert_close(dw.cpu().numpy(), ref, RTOL_WGRAD, f"f32 wgrad {cin}->{cout}")
+
+
+def test_backward_weight_f32_headline_slices(S):
+    """fp32 128 -> 128 on the headline set (329,839 voxels, many voxel slices):
+    dW[o][k][c] depends on dy[:, o] and x[:, c] only, so rows and columns of the
+    full gradient are checked against the oracle on those columns."""
+    wl = WL.make_workload("headline")
+    x = WL.make_features(wl.n, 128, 81)
+    dy = WL.make_features(wl.n, 128, 82)
+    h = S.build_map(torch.from_numpy(wl.coords).cuda(), wl.grid_dim, 1)
+    dw = S.backward_weight(h, torch.from_numpy(x).cuda(), torch.from_numpy(dy).cuda()).cpu().numpy()
+    osel, csel = np.r_[0:8, 60:68, 120:128], np.r_[0:8, 64:72, 124:128]
+    nbr = C.build_map(wl.coords, wl.grid_dim, 1)
+    ref = C.backward_weight(nbr, x[:, csel].astype(np.float64), dy[:, osel].astype(np.float64))
+    assert_close(dw[osel][:, :, :, :, csel], ref, RTOL_WGRAD, "f32 wgrad headline")
+
+
 def test_autograd_through_subm_conv(S):
     """SubMConv3d with a trainable weight: loss = sum(y * g); torch autograd
     calls the library's backward kernels."""

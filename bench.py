@@ -45,7 +45,8 @@ METRIC = "SubMConv3d fwd voxels/s and TFLOP/s at 128^3/128ch bf16; % of B200 roo
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # Kernels one map build launches: table init, insert, and the query, which
-# also lays out the x-run positions and the E index table.
+# also lays out the x-run positions and the E index table; the brick table
+# adds its block allocation.
 MAP_LAUNCHES = 3
 
 # Algorithmic bytes of the map build per voxel: int32 (b,z,y,x) in + int32 [27] out.
@@ -209,18 +210,23 @@ def _time_ms(fn, flush, reps=5, warm=2):
 
 
 def fp32_forward_line(h, feats_f32, w_f32, flops, flush, sm_mhz):
-    """The fp32 path (CUDA-core FMA) on the same map, against the FP32 peak
-    SMs x 128 lanes x 2 flop x SM clock."""
+    """The fp32 path (CUDA-core FMA) on the same map, forward and weight
+    gradient, against the FP32 peak SMs x 128 lanes x 2 flop x SM clock."""
     import torch
     import sparse_voxel_conv_b200 as S
     out = torch.empty((h.n, w_f32.shape[0]), dtype=torch.float32, device=feats_f32.device)
     ms = _time_ms(lambda: S.forward(h, feats_f32, w_f32, out=out), flush)
+    dy = torch.empty_like(out).normal_()
+    dw = torch.empty(w_f32.shape, dtype=torch.float32, device=feats_f32.device)
+    w_ms = _time_ms(lambda: S.backward_weight(h, feats_f32, dy, out=dw), flush, reps=3, warm=1)
     sms = torch.cuda.get_device_properties(feats_f32.device).multi_processor_count
     peak = sms * 128 * 2 * sm_mhz * 1e6 / 1e12
     achieved = flops / (ms / 1e3) / 1e12
+    w_achieved = flops / (w_ms / 1e3) / 1e12
     return {"bound": "alu", "ms": ms, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
             "frac": achieved / peak,
-            "peak_source": f"{sms} SMs x 128 FP32 lanes x 2 x {sm_mhz:.0f} MHz"}
+            "peak_source": f"{sms} SMs x 128 FP32 lanes x 2 x {sm_mhz:.0f} MHz",
+            "weight_gradient": {"ms": w_ms, "achieved": w_achieved, "frac": w_achieved / peak}}
 
 
 def per_offset_context(h, feats, weight, flush):
@@ -407,12 +413,12 @@ class Job:
         return sum(2.0 * nnz * self.channels[li] * self.channels[li + 1]
                    for li in range(len(self.channels) - 1))
 
-    def step_text(self) -> str:
+    def step_text(self, map_launches: int = MAP_LAUNCHES, table: str = "direct") -> str:
         layers = len(self.channels) - 1
+        build = f"map build ({table} table, {map_launches} kernels)"
         if layers == 1:
-            return f"map build ({MAP_LAUNCHES} kernels) + bf16 x-run forward (1 kernel)"
-        return (f"map build ({MAP_LAUNCHES} kernels) + {layers} bf16 forward layers on it "
-                f"(exact GELU between)")
+            return f"{build} + bf16 x-run forward (1 kernel)"
+        return f"{build} + {layers} bf16 forward layers on it (exact GELU between)"
 
 
 def run_ours(args):
@@ -473,8 +479,13 @@ def run_ours(args):
 
     # correctness gate before timing: the map must be valid
     h0 = step()
+    map_launches, table = MAP_LAUNCHES, "direct"
     if h0 is not None:
         assert S.map_status(h0) == 0, "map build reported a data error"
+        kind = _abi.subm3d_map_table(h0)
+        table = {_abi.SUBM3D_TABLE_DIRECT: "direct", _abi.SUBM3D_TABLE_HASH: "hash",
+                 _abi.SUBM3D_TABLE_BRICK: "brick"}[kind]
+        map_launches = MAP_LAUNCHES + (1 if kind == _abi.SUBM3D_TABLE_BRICK else 0)
     nnz_total = int((nbr >= 0).sum().item())
     assert _abi.subm3d_device_status() == 0
     for _ in range(args.warmup):
@@ -589,7 +600,7 @@ def run_ours(args):
             "data": "synthetic",
             "config": {
                 **_workload_config(wl, nnz_total / max(n, 1)),
-                "step": job.step_text(),
+                "step": job.step_text(map_launches, table),
                 "l2": f"flushed before every timed step ({L2_FLUSH_BYTES >> 20} MB write)",
                 "parallelism": job.parallelism,
             },
@@ -611,7 +622,7 @@ def run_ours(args):
             "e2e": {"value": job.units_job / (e2e_ms / 1e3 / K), "unit": "voxels/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms / K},
-            "gpu_launches": (MAP_LAUNCHES + n_layers) * K,
+            "gpu_launches": (map_launches + n_layers) * K,
             "clocks": clocks,
         }
         if job.name == "batched":

@@ -156,6 +156,11 @@ SUBM3D_API const int32_t* subm3d_map_nbr(const subm3d_map* map);        /* (devi
 SUBM3D_API const uint32_t* subm3d_map_tile_mask(const subm3d_map* map); /* (device) [ceil(N/128)]    */
 SUBM3D_API int64_t subm3d_map_size(const subm3d_map* map);              /* N                         */
 
+/* The lookup table the build chose (see subm3d_map_workspace_bytes()); the
+ * build enqueues 4 kernels with the brick table, 3 otherwise.  -1 for NULL. */
+typedef enum { SUBM3D_TABLE_DIRECT = 0, SUBM3D_TABLE_HASH = 1, SUBM3D_TABLE_BRICK = 2 } subm3d_table;
+SUBM3D_API int32_t subm3d_map_table(const subm3d_map* map);
+
 /* Frees the host handle only; the caller's nbr and workspace are untouched. */
 SUBM3D_API void subm3d_map_destroy(subm3d_map* map);
 

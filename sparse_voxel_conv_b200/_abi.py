@@ -62,6 +62,7 @@ def _load() -> ctypes.CDLL:
         "subm3d_map_nbr": (vp, [vp]),
         "subm3d_map_tile_mask": (vp, [vp]),
         "subm3d_map_size": (i64, [vp]),
+        "subm3d_map_table": (ctypes.c_int32, [vp]),
         "subm3d_map_destroy": (None, [vp]),
         "subm3d_forward": (ctypes.c_int, [vp, vp, i64, vp, vp, vp, i32, i32, ctypes.c_int, i32,
                                           ctypes.c_int, vp]),
@@ -182,6 +183,14 @@ def subm3d_map_tile_mask(handle: MapHandle) -> int:
 
 def subm3d_map_size(handle: MapHandle) -> int:
     return int(lib.subm3d_map_size(handle.ptr))
+
+
+SUBM3D_TABLE_DIRECT, SUBM3D_TABLE_HASH, SUBM3D_TABLE_BRICK = 0, 1, 2
+
+
+def subm3d_map_table(handle: MapHandle) -> int:
+    """The lookup table the build chose: SUBM3D_TABLE_DIRECT, _HASH or _BRICK."""
+    return int(lib.subm3d_map_table(handle.ptr))
 
 
 def subm3d_forward(nbr, tile_mask, n: int, feats, weight, out, cin: int, cout: int,

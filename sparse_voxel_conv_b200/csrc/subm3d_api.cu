@@ -184,6 +184,14 @@ const uint32_t* subm3d_map_tile_mask(const subm3d_map* map) {
   return map ? map->tile_mask : nullptr;
 }
 int64_t subm3d_map_size(const subm3d_map* map) { return map ? map->n : -1; }
+int32_t subm3d_map_table(const subm3d_map* map) {
+  if (!map) return -1;
+  switch (map->layout.kind) {
+    case subm3d::MapKind::kDirect: return SUBM3D_TABLE_DIRECT;
+    case subm3d::MapKind::kBrick: return SUBM3D_TABLE_BRICK;
+    default: return SUBM3D_TABLE_HASH;
+  }
+}
 void subm3d_map_destroy(subm3d_map* map) { delete map; }
 
 namespace {

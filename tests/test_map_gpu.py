@@ -78,6 +78,24 @@ def test_map_wide_keys(S, kind, grid, batch, shift):
     assert np.array_equal(masks, masks_from_nbr(ref))
 
 
+def test_map_table_choice(S, monkeypatch):
+    """The table each set gets (subm3d_map_table): direct for the headline and
+    the dense sets (small or dense volumes), brick for the decoder-stack set (60
+    cells per voxel); the testing knob forces the hash table."""
+    A = S._abi
+    monkeypatch.delenv("SUBM3D_MAP_KIND", raising=False)
+    want = {"headline": A.SUBM3D_TABLE_DIRECT, "dense": A.SUBM3D_TABLE_DIRECT,
+            "batched": A.SUBM3D_TABLE_BRICK}
+    for name, table in want.items():
+        wl = WL.make_workload(name)
+        h = S.build_map(torch.from_numpy(wl.coords).cuda(), wl.grid_dim, wl.batch)
+        assert A.subm3d_map_table(h) == table, name
+    monkeypatch.setenv("SUBM3D_MAP_KIND", "hash")
+    wl = WL.make_workload("shell")
+    h = S.build_map(torch.from_numpy(wl.coords).cuda(), wl.grid_dim, wl.batch)
+    assert A.subm3d_map_table(h) == A.SUBM3D_TABLE_HASH
+
+
 @pytest.fixture(scope="module")
 def large_sparse():
     """Two 512^3 grids of large shells: 615,658 voxels, 441 cells per voxel, so

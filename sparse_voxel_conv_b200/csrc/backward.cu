@@ -86,6 +86,18 @@ __device__ __forceinline__ float4 load4_row(const T* __restrict__ p, int first, 
   }
 }
 
+// Two fp32 FMAs in one instruction (each lane of the pair rounded as fmaf):
+// d = a * b + c on (lo, hi) pairs held in 64-bit registers.
+__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
+                                                  unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long pack2(float lo, float hi) {
+  return (static_cast<unsigned long long>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+}
+
 template <typename T, bool VEC>
 __global__ void __launch_bounds__(WT, 2)
     wgrad_kernel(const int32_t* __restrict__ nbr, int64_t n, const T* __restrict__ x,
@@ -125,11 +137,12 @@ __global__ void __launch_bounds__(WT, 2)
     *reinterpret_cast<float4*>(&s_a[buf][v][sg]) = ra;
     *reinterpret_cast<float4*>(&s_b[buf][v][sg]) = rb;
   };
-  float acc[8][8];
+  // accumulator pairs: acc2[m][p] holds columns 2p, 2p + 1 of row m
+  unsigned long long acc2[8][4];
 #pragma unroll
   for (int m = 0; m < 8; ++m)
 #pragma unroll
-    for (int q = 0; q < 8; ++q) acc[m][q] = 0.f;
+    for (int p = 0; p < 4; ++p) acc2[m][p] = 0ull;
 
   if (steps > 0) {
 #pragma unroll 1
@@ -150,14 +163,16 @@ __global__ void __launch_bounds__(WT, 2)
         const int kk = part * WP + q;
         const float4 a0 = *reinterpret_cast<const float4*>(&s_a[buf][kk][ty * 4]);
         const float4 a1 = *reinterpret_cast<const float4*>(&s_a[buf][kk][64 + ty * 4]);
-        const float4 b0 = *reinterpret_cast<const float4*>(&s_b[buf][kk][tx * 4]);
-        const float4 b1 = *reinterpret_cast<const float4*>(&s_b[buf][kk][64 + tx * 4]);
+        const ulonglong2 b0 = *reinterpret_cast<const ulonglong2*>(&s_b[buf][kk][tx * 4]);
+        const ulonglong2 b1 = *reinterpret_cast<const ulonglong2*>(&s_b[buf][kk][64 + tx * 4]);
         const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-        const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        const unsigned long long bp[4] = {b0.x, b0.y, b1.x, b1.y};
 #pragma unroll
-        for (int m = 0; m < 8; ++m)
+        for (int m = 0; m < 8; ++m) {
+          const unsigned long long am = pack2(av[m], av[m]);
 #pragma unroll
-          for (int r = 0; r < 8; ++r) acc[m][r] = fmaf(av[m], bv[r], acc[m][r]);
+          for (int p = 0; p < 4; ++p) acc2[m][p] = fma2(am, bp[p], acc2[m][p]);
+        }
       }
       if (more) stage(buf ^ 1, part);
     }
@@ -172,7 +187,9 @@ __global__ void __launch_bounds__(WT, 2)
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int c = c0 + (r < 4 ? tx * 4 + r : 64 + tx * 4 + r - 4);
-      if (c < cin) atomicAdd(row + c, acc[m][r]);
+      const unsigned long long pr = acc2[m][r >> 1];
+      if (c < cin)
+        atomicAdd(row + c, __uint_as_float(static_cast<uint32_t>((r & 1) ? (pr >> 32) : pr)));
     }
   }
 }

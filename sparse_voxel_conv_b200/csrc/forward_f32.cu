@@ -48,6 +48,18 @@ __device__ __forceinline__ float4 load4(const float* __restrict__ base, int64_t 
   }
 }
 
+// Two fp32 FMAs in one instruction (each lane of the pair rounded as fmaf):
+// d = a * b + c on (lo, hi) pairs held in 64-bit registers.
+__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
+                                                  unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long pack2(float lo, float hi) {
+  return (static_cast<unsigned long long>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+}
+
 // out may alias residual (an in-place residual add): neither is __restrict__.
 template <int ACT, bool VEC>
 __global__ void __launch_bounds__(NT, 2)
@@ -114,25 +126,28 @@ __global__ void __launch_bounds__(NT, 2)
     s_b[buf][kk + 3][sr] = rb.w;
   };
 
-  float acc[8][8];
+  // accumulator pairs: acc2[i][p] holds columns 2p, 2p + 1 of row i
+  unsigned long long acc2[8][4];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    for (int p = 0; p < 4; ++p) acc2[i][p] = 0ull;
   auto compute = [&](int buf, int part) {
 #pragma unroll
     for (int q = 0; q < HK; ++q) {
       const int kk = part * HK + q;
       const float4 a0 = *reinterpret_cast<const float4*>(&s_a[buf][kk][ty * 4]);
       const float4 a1 = *reinterpret_cast<const float4*>(&s_a[buf][kk][64 + ty * 4]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&s_b[buf][kk][tx * 4]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&s_b[buf][kk][64 + tx * 4]);
+      const ulonglong2 b0 = *reinterpret_cast<const ulonglong2*>(&s_b[buf][kk][tx * 4]);
+      const ulonglong2 b1 = *reinterpret_cast<const ulonglong2*>(&s_b[buf][kk][64 + tx * 4]);
       const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      const unsigned long long bp[4] = {b0.x, b0.y, b1.x, b1.y};
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
+      for (int i = 0; i < 8; ++i) {
+        const unsigned long long ai = pack2(av[i], av[i]);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        for (int p = 0; p < 4; ++p) acc2[i][p] = fma2(ai, bp[p], acc2[i][p]);
+      }
     }
   };
 
@@ -169,7 +184,10 @@ __global__ void __launch_bounds__(NT, 2)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int o = o0 + j;
-        v[j] = o < cout ? activate<ACT>(acc[i][4 * h + j] + (bias ? bias[o] : 0.0f)) : 0.0f;
+        const int col = 4 * h + j;
+        const unsigned long long pr = acc2[i][col >> 1];
+        const float av = __uint_as_float(static_cast<uint32_t>((col & 1) ? (pr >> 32) : pr));
+        v[j] = o < cout ? activate<ACT>(av + (bias ? bias[o] : 0.0f)) : 0.0f;
       }
       float* dst = out + r * cout + o0;
       if (VEC && o0 + 3 < cout) {

@@ -16,10 +16,11 @@ from tests.helpers import RTOL_BF16, RTOL_F32, assert_close
 
 pytestmark = pytest.mark.gpu
 
-# (name, dtype, cin, cout): the x-run kernel takes bf16 with Cin % 64 == 0, the
-# gather kernel other bf16 widths, fp32 the CUDA-core kernel
+# (name, dtype, cin, cout): the x-run kernel takes bf16 with Cin >= 48 (48: a
+# partial 64-channel chunk), the gather kernel narrower bf16, fp32 the
+# CUDA-core kernel
 PATHS = [("xrun64", "bf16", 64, 64), ("xrun128", "bf16", 128, 128),
-         ("gather48", "bf16", 48, 32), ("f32", "f32", 24, 40)]
+         ("xrun48", "bf16", 48, 32), ("gather32", "bf16", 32, 48), ("f32", "f32", 24, 40)]
 
 
 @pytest.fixture(scope="module")

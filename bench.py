@@ -346,9 +346,22 @@ def decoder_stack_line(flush, peak_tf):
     ms = _time_ms(run, flush)
     flops = sum(2.0 * nnz * w.shape[0] * w.shape[-1] for w in ws)  # KRSC: Cout ... Cin
     tf = flops / (ms / 1e3) / 1e12
+    # where the time goes: the map build and each layer alone (L2 flushed before each)
+    h = S.build_map(coords, wl.grid_dim, wl.batch, check=False, nbr=nbr, workspace=work)
+    parts = {"map_build": _time_ms(lambda: S.build_map(coords, wl.grid_dim, wl.batch,
+                                                         check=False, nbr=nbr, workspace=work),
+                                   flush)}
+    ins = [x0] + outs[:-1]
+    for li, w in enumerate(ws):
+        act = "gelu" if li < len(ws) - 1 else None
+        parts[f"layer{li} {w.shape[-1]}->{w.shape[0]}"] = _time_ms(
+            lambda li=li, w=w, act=act: S.forward(h, ins[li], w, act=act, out=outs[li]), flush)
+    table = {S._abi.SUBM3D_TABLE_DIRECT: "direct", S._abi.SUBM3D_TABLE_HASH: "hash",
+             S._abi.SUBM3D_TABLE_BRICK: "brick"}[S._abi.subm3d_map_table(h)]
     return {"workload": wl.name, "n_voxels": n, "ms": ms, "voxels_per_s": n / (ms / 1e3),
             "flops": flops, "achieved": tf, "peak": peak_tf, "unit": "TFLOP/s",
-            "frac": tf / peak_tf, "what": "one map build + 4 fused bf16 layers on it"}
+            "frac": tf / peak_tf, "what": "one map build + 4 fused bf16 layers on it",
+            "map_table": table, "parts_ms": parts}
 
 
 def batch_elements(rank: int, world: int, batch: int) -> list:

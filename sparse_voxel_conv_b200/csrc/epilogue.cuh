@@ -118,10 +118,10 @@ __device__ __forceinline__ void epilogue_tile_bf16(uint32_t taddr, float bias_v,
                  : make_uint4(0u, 0u, 0u, 0u);
   };
   // chunk 0's rows and residual now, chunk 1's pos entry in flight
-  int32_t pe_next = POS ? __ldg(pos + 32 + lane) : 0;
+  int32_t pe_next = POS ? ld_dep(pos + 32 + lane) : 0;
   int32_t rows[4];
   uint4 res[4];
-  rows_of(0, POS ? __ldg(pos + lane) : 0, rows);
+  rows_of(0, POS ? ld_dep(pos + lane) : 0, rows);
   load_res(rows, res);
 #pragma unroll 1
   for (int ci = 0; ci < kChunks; ++ci) {
@@ -132,7 +132,7 @@ __device__ __forceinline__ void epilogue_tile_bf16(uint32_t taddr, float bias_v,
     if (ci + 1 < kChunks) {  // next chunk's rows and residual (and the pos entry after it)
       rows_of(ci + 1, pe_next, rows_n);
       load_res(rows_n, res_n);
-      if (POS && ci + 2 < kChunks) pe_next = __ldg(pos + (ci + 2) * 32 + lane);
+      if (POS && ci + 2 < kChunks) pe_next = ld_dep(pos + (ci + 2) * 32 + lane);
     }
     tmem_ld_wait();
 #pragma unroll

@@ -210,7 +210,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait();  // the setup above overlaps the map build's tail; global reads start here
-  const int64_t n_tiles = __ldg(a.hdr + 1);
+  const int64_t n_tiles = ld_dep(a.hdr + 1);
   const int64_t n_units = n_tiles * a.n_oblocks;
   int64_t w_issued = 0;  // weight loads the TMA warp has issued (its abort-path drain)
 
@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
       for (int q = 0; q <= PPT; ++q) {
         const int i = q < PPT ? rbase + q * ROWS_PER_PASS : TP + rbase;
-        v[q] = (q < PPT || edge) ? __ldg(list + i) : -1;
+        v[q] = (q < PPT || edge) ? ld_dep(list + i) : -1;
       }
     };
     ESteps st;

@@ -21,6 +21,26 @@ __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Loads, after pdl_wait(), of data that an earlier kernel of the chain writes.
+// A kernel launched with the attribute can be running while that kernel still
+// writes, so such data must not go through the non-coherent read-only path
+// (ld.global.nc, __ldg): that path takes the data to be unchanged for the
+// reading kernel's whole lifetime, and the compiler may schedule those loads
+// above griddepcontrol.wait.  (A forward that read the map's header through it,
+// queued right behind the build, at times saw the value from before the build
+// and skipped whole tiles.)  These are ordinary coherent loads (ld.global.ca),
+// written as volatile asm so that they stay after the wait.
+__device__ __forceinline__ int32_t ld_dep(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.global.ca.b32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ unsigned long long ld_dep(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.global.ca.b64 %0, [%1];" : "=l"(v) : "l"(p));
+  return v;
+}
+
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                        cudaStream_t stream, Args&&... args) {

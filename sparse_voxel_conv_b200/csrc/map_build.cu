@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(kInsertThreads)
   if constexpr (K == Kind::kDirect) {
     cells[cell_of(c.x, c.y, c.z, c.w, grid)] = i;
   } else if constexpr (K == Kind::kBrick) {  // `cells` is the pool, t.rows the directory
-    const int32_t slot = __ldg(t.rows + brick_of(t, c.x, c.y + 1, c.z + 1, c.w + 1));
+    const int32_t slot = ld_dep(t.rows + brick_of(t, c.x, c.y + 1, c.z + 1, c.w + 1));
     cells[static_cast<int64_t>(slot) * kBrickCells + brick_cell(c.y + 1, c.z + 1, c.w + 1)] = i;
   } else if constexpr (K == Kind::kCompact) {
     const uint32_t key = pack32(c.x, c.y, c.z, c.w);
@@ -308,8 +308,8 @@ __global__ void __launch_bounds__(kTileRows)
   if constexpr (RUNS) {
     const int sb = tile / kSuperTiles;
     int32_t part = 0;
-    for (int j = r; j < sb; j += kTileRows) part += __ldg(ro.sb + j);
-    for (int j = sb * kSuperTiles + r; j < tile; j += kTileRows) part += __ldg(ro.cnt + j);
+    for (int j = r; j < sb; j += kTileRows) part += ld_dep(ro.sb + j);
+    for (int j = sb * kSuperTiles + r; j < tile; j += kTileRows) part += ld_dep(ro.cnt + j);
     part = __reduce_add_sync(0xFFFFFFFFu, part);
     const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, starts);
     if (lane == 0) {
@@ -334,7 +334,7 @@ __global__ void __launch_bounds__(kTileRows)
             const int32_t* row = centre + ((dz - 1) * g2 + (dy - 1) * g);
 #pragma unroll
             for (int dx = 0; dx < 3; ++dx) {
-              const int32_t v = __ldg(row + dx - 1);
+              const int32_t v = ld_dep(row + dx - 1);
               nb[dz * 9 + dy * 3 + dx] = v;
               absent = __funnelshift_l(static_cast<uint32_t>(v), absent, 1);  // sign bit in
             }
@@ -348,13 +348,13 @@ __global__ void __launch_bounds__(kTileRows)
         int32_t slot[kKvol];
 #pragma unroll
         for (int k = 0; k < kKvol; ++k)
-          slot[k] = __ldg(t.rows + brick_of(t, c.x, Z + k / 9 - 1, Y + (k / 3) % 3 - 1,
+          slot[k] = ld_dep(t.rows + brick_of(t, c.x, Z + k / 9 - 1, Y + (k / 3) % 3 - 1,
                                             X + k % 3 - 1));
 #pragma unroll
         for (int k = 0; k < kKvol; ++k) {
           const int32_t v =
               slot[k] < 0 ? -1
-                          : __ldg(t.cells + static_cast<int64_t>(slot[k]) * kBrickCells +
+                          : ld_dep(t.cells + static_cast<int64_t>(slot[k]) * kBrickCells +
                                   brick_cell(Z + k / 9 - 1, Y + (k / 3) % 3 - 1, X + k % 3 - 1));
           nb[k] = v;
           absent = __funnelshift_l(static_cast<uint32_t>(v), absent, 1);

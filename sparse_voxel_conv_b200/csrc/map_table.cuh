@@ -9,11 +9,15 @@
 // (key32 << 32 | row) when batch <= 4 and grid_dim <= 1024, else 64-bit keys
 // with a separate int32 row array.  The home slot is 4 * h(key >> 2) + (key & 3)
 // with a 32-bit avalanche mix h, so the x-neighbours of a voxel usually share a
-// 32-byte sector.  Probe loops are bounded by the capacity.
+// 32-byte sector.  Probe loops are bounded by the capacity.  Lookups read the
+// tables with ld_dep(): the query kernel may start while the insert kernel
+// still writes them.
 #pragma once
 
 #include <cstdint>
 #include <cuda_runtime.h>
+
+#include "internal.h"
 
 namespace subm3d {
 namespace {
@@ -89,17 +93,17 @@ __device__ __forceinline__ int brick_cell(int Z, int Y, int X) {
 template <Kind K>
 __device__ __forceinline__ int32_t lookup(const Tables& t, int b, int z, int y, int x, int grid) {
   if constexpr (K == Kind::kDirect) {
-    return __ldg(t.cells + cell_of(b, z, y, x, grid));
+    return ld_dep(t.cells + cell_of(b, z, y, x, grid));
   } else if constexpr (K == Kind::kBrick) {
     (void)grid;  // -1 <= z, y, x <= grid: every bordered cell has a directory entry
-    const int32_t s = __ldg(t.rows + brick_of(t, b, z + 1, y + 1, x + 1));
+    const int32_t s = ld_dep(t.rows + brick_of(t, b, z + 1, y + 1, x + 1));
     return s < 0 ? -1
-                 : __ldg(t.cells + static_cast<int64_t>(s) * 64 + brick_cell(z + 1, y + 1, x + 1));
+                 : ld_dep(t.cells + static_cast<int64_t>(s) * 64 + brick_cell(z + 1, y + 1, x + 1));
   } else if constexpr (K == Kind::kCompact) {
     const uint32_t key = pack32(b, z, y, x);
     uint32_t slot = home32(key, t.capmask);
     for (uint64_t step = 0; step <= t.capmask; ++step) {
-      const unsigned long long e = __ldg(t.table + slot);
+      const unsigned long long e = ld_dep(t.table + slot);
       if (e == kEmpty) return -1;
       if (static_cast<uint32_t>(e >> 32) == key)
         return static_cast<int32_t>(static_cast<uint32_t>(e));
@@ -110,9 +114,9 @@ __device__ __forceinline__ int32_t lookup(const Tables& t, int b, int z, int y, 
     const unsigned long long key = pack64(b, z, y, x);
     uint32_t slot = home64(key, t.capmask);
     for (uint64_t step = 0; step <= t.capmask; ++step) {
-      const unsigned long long e = __ldg(t.table + slot);
+      const unsigned long long e = ld_dep(t.table + slot);
       if (e == kEmpty) return -1;
-      if (e == key) return __ldg(t.rows + slot);
+      if (e == key) return ld_dep(t.rows + slot);
       slot = (slot + 1) & t.capmask;
     }
     return -1;

@@ -176,7 +176,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) subm3d_wgrad_bf16_runs_sm100(c
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait();
-  const int64_t n_tiles = __ldg(a.hdr + 1);
+  const int64_t n_tiles = ld_dep(a.hdr + 1);
 
   if (warp >= GATHER_WARP0 && warp < MMA_WARP) {
     // ---------------------------------------------------------- gather ----
@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) subm3d_wgrad_bf16_runs_sm100(c
 #pragma unroll
       for (int q = 0; q < YROWS / 16; ++q) {
         const int r = rbase + 16 * q;
-        const int32_t e = __ldg(posp + r);
+        const int32_t e = ld_dep(posp + r);
         const bool ok = e >= 0 && (e & 3) == kPosVoxel && o < a.cout;
         const uint32_t dst = y_base + chunk * Y_CHUNK + r * ROW + ((col ^ (r & 7)) << 4);
         cp_async_16(dst, ok ? a.dy + static_cast<int64_t>(e >> 2) * a.cout + o : a.dy,
@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) subm3d_wgrad_bf16_runs_sm100(c
       for (int q = 0; q <= HP / 16; ++q) {
         const int r = rbase + 16 * q;  // E slot row r = E row r - 1 of the half
         if (q == HP / 16 && r >= EROWS) break;
-        const int32_t e = __ldg(etp + r);
+        const int32_t e = ld_dep(etp + r);
         const bool ok = e >= 0 && c < a.cin;
         const uint32_t dst = e_base + chunk * E_CHUNK + r * ROW + ((col ^ (r & 7)) << 4);
         cp_async_16(dst, ok ? a.x + static_cast<int64_t>(e) * a.cin + c : a.x, ok ? 16u : 0u);

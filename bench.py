@@ -75,7 +75,7 @@ def _profiled_traffic(workload: str):
     try:
         text = open(prof).read()
         h = hashlib.sha256()
-        for f in ("forward_bf16_runs_sm100.cu", "ptx.cuh", "epilogue.cuh"):
+        for f in ("forward_bf16_runs_sm100.cu", "ptx.cuh", "epilogue.cuh", "internal.h"):
             h.update(open(os.path.join(csrc, f), "rb").read())
     except OSError:
         return None

@@ -37,6 +37,12 @@
  *     on the device and reported by subm3d_map_status().
  *   - Every function is safe to call from several host threads on different
  *     streams; calls that share a workspace must be ordered by the caller.
+ *   - Stream order is enough: a call on a map may be enqueued right behind its
+ *     build, and a build may reuse the nbr buffer and workspace of maps whose
+ *     calls are enqueued before it on the same stream (those calls see their
+ *     own map).  The kernels use programmatic dependent launch, read what an
+ *     earlier kernel wrote only after griddepcontrol.wait, and never through
+ *     the non-coherent load path.
  */
 #ifndef SUBM3D_H_
 #define SUBM3D_H_

@@ -25,11 +25,63 @@ __device__ __forceinline__ float gelu_erf(float v) {
   constexpr float p = 0.3275911f;
   constexpr float a1 = 0.254829592f, a2 = -0.284496736f, a3 = 1.421413741f,
                   a4 = -1.453152027f, a5 = 1.061405429f;
-  const float u = fabsf(v) * 0.70710678118654752f;
-  const float t = __fdividef(1.0f, fmaf(p, u, 1.0f));
-  const float poly = t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, a5, a4), a3), a2), a1);
-  const float ec = poly * __expf(-u * u);  // erfc(|v| / sqrt 2)
-  return v * (v >= 0.0f ? fmaf(-0.5f, ec, 1.0f) : 0.5f * ec);
+  const float u = __fmul_rn(fabsf(v), 0.70710678118654752f);
+  const float t = __fdividef(1.0f, __fmaf_rn(p, u, 1.0f));
+  const float poly =
+      __fmul_rn(t, __fmaf_rn(t, __fmaf_rn(t, __fmaf_rn(t, __fmaf_rn(t, a5, a4), a3), a2), a1));
+  const float ec = __fmul_rn(poly, __expf(-__fmul_rn(u, u)));  // erfc(|v| / sqrt 2)
+  return __fmul_rn(v, v >= 0.0f ? __fmaf_rn(-0.5f, ec, 1.0f) : __fmul_rn(0.5f, ec));
+}
+
+// Two lanes of fp32 in one 64-bit register: the packed add / multiply / fma of
+// sm_100 (add / mul / fma .rn.f32x2: two independent IEEE operations each).
+__device__ __forceinline__ unsigned long long f2_pack(float lo, float hi) {
+  unsigned long long d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ void f2_unpack(unsigned long long d, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(d));
+}
+__device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long f2_mul(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b,
+                                                     unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// gelu_erf on two values at once: the same operations in the same order (so
+// the same bits), the multiplies and fmas as f32x2 pairs; the reciprocal and
+// the exponential stay per value.
+__device__ __forceinline__ void gelu_erf2(float& v0, float& v1) {
+  const auto k = [](float c) { return f2_pack(c, c); };
+  const unsigned long long u = f2_mul(f2_pack(fabsf(v0), fabsf(v1)), k(0.70710678118654752f));
+  float d0, d1;
+  f2_unpack(f2_fma(k(0.3275911f), u, k(1.0f)), d0, d1);
+  const unsigned long long t = f2_pack(__fdividef(1.0f, d0), __fdividef(1.0f, d1));
+  unsigned long long q = f2_fma(t, k(1.061405429f), k(-1.453152027f));
+  q = f2_fma(t, q, k(1.421413741f));
+  q = f2_fma(t, q, k(-0.284496736f));
+  q = f2_fma(t, q, k(0.254829592f));
+  const unsigned long long poly = f2_mul(t, q);
+  float w0, w1;
+  f2_unpack(f2_mul(u, u), w0, w1);
+  const unsigned long long ec = f2_mul(poly, f2_pack(__expf(-w0), __expf(-w1)));
+  float hi0, hi1, lo0, lo1;  // Phi for v >= 0 and for v < 0
+  f2_unpack(f2_fma(k(-0.5f), ec, k(1.0f)), hi0, hi1);
+  f2_unpack(f2_mul(k(0.5f), ec), lo0, lo1);
+  f2_unpack(f2_mul(f2_pack(v0, v1), f2_pack(v0 >= 0.0f ? hi0 : lo0, v1 >= 0.0f ? hi1 : lo1)),
+            v0, v1);
 }
 
 template <int ACT>
@@ -138,9 +190,19 @@ __device__ __forceinline__ void epilogue_tile_bf16(uint32_t taddr, float bias_v,
 #pragma unroll
     for (int h = 0; h < 2; ++h) {  // positions 16h .. 16h+15 of the chunk: store slots 2h, 2h+1
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const float f = activate<ACT>(__uint_as_float(v[16 * h + e]) + bias_v);
-        sts_u32(stage + e * 128 + ((lane * 4) ^ ((e & 1) << 4)), __float_as_uint(f));
+      for (int e = 0; e < 16; e += 2) {  // bias and activation on pairs of positions
+        float f0, f1;
+        f2_unpack(f2_add(f2_pack(__uint_as_float(v[16 * h + e]), __uint_as_float(v[16 * h + e + 1])),
+                         f2_pack(bias_v, bias_v)),
+                  f0, f1);
+        if constexpr (ACT == kActGelu) {
+          gelu_erf2(f0, f1);
+        } else {
+          f0 = activate<ACT>(f0);
+          f1 = activate<ACT>(f1);
+        }
+        sts_u32(stage + e * 128 + (lane * 4), __float_as_uint(f0));
+        sts_u32(stage + (e + 1) * 128 + ((lane * 4) ^ 16), __float_as_uint(f1));
       }
       __syncwarp();
 #pragma unroll

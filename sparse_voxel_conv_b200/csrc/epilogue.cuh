@@ -127,11 +127,13 @@ constexpr int kEpiWarpStageBytes = 16 * 32 * 4;
 
 // The epilogue of one 256-position accumulator by one warp: its 32 channels
 // (TMEM lanes; lane = channel o_warp + lane) in 8 chunks of 32 positions.  Per
-// chunk, in two halves of 16 positions, the fp32 values (bias, activation) go to
-// the warp's staging area (`stage`, kEpiWarpStageBytes; a position's 128-byte
-// row has its 16-byte halves swapped at odd positions, so the reads below are
-// free of bank conflicts), then each lane takes 8 channels of one position,
-// adds the residual and stores 16 bytes.  The output row of position j is
+// chunk, in two halves of 16 positions, the values after bias and activation go
+// to the warp's staging area (`stage`, kEpiWarpStageBytes), then each lane takes
+// 8 channels of one position and stores 16 bytes.  With a residual they are
+// staged in fp32 (a position's 128-byte row has its 16-byte halves swapped at
+// odd positions, so the reads are free of bank conflicts) and the lane adds the
+// residual before the one bf16 rounding; without one they are rounded first and
+// staged as 64-byte bf16 rows.  The output row of position j is
 // pos[j] >> 2 when pos[j] is a voxel entry (POS: the x-run layout; pads and
 // empty positions are dropped), else row0 + j below n.  Latency is hidden by prefetching: position entries
 // two chunks ahead and each chunk's residual rows one chunk ahead, so they load
@@ -174,7 +176,56 @@ __device__ __forceinline__ void epilogue_tile_bf16(uint32_t taddr, float bias_v,
   int32_t rows[4];
   uint4 res[4];
   rows_of(0, POS ? ld_dep(pos + lane) : 0, rows);
-  load_res(rows, res);
+  if (residual != nullptr) load_res(rows, res);
+  if (residual == nullptr) {
+    // No residual: round to bf16 before staging (the same single rounding), so
+    // the staging holds 64-byte rows of 32 bf16 channels and each lane reads its
+    // 8 channels with one 16-byte load -- half the shared-memory traffic.
+#pragma unroll 1
+    for (int ci = 0; ci < kChunks; ++ci) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(taddr + ci * 32, v);
+      int32_t rows_n[4];
+      if (ci + 1 < kChunks) {
+        rows_of(ci + 1, pe_next, rows_n);
+        if (POS && ci + 2 < kChunks) pe_next = ld_dep(pos + (ci + 2) * 32 + lane);
+      }
+      tmem_ld_wait();
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {  // positions e, e+1 of the half
+          float f0, f1;
+          f2_unpack(f2_add(f2_pack(__uint_as_float(v[16 * h + e]),
+                                   __uint_as_float(v[16 * h + e + 1])),
+                           f2_pack(bias_v, bias_v)),
+                    f0, f1);
+          if constexpr (ACT == kActGelu) {
+            gelu_erf2(f0, f1);
+          } else {
+            f0 = activate<ACT>(f0);
+            f1 = activate<ACT>(f1);
+          }
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(f0, f1);
+          const uint32_t w = *reinterpret_cast<const uint32_t*>(&b2);
+          sts_u16(stage + e * 64 + lane * 2, static_cast<uint16_t>(w & 0xFFFFu));
+          sts_u16(stage + (e + 1) * 64 + lane * 2, static_cast<uint16_t>(w >> 16));
+        }
+        __syncwarp();
+#pragma unroll
+        for (int p = 2 * h; p < 2 * h + 2; ++p) {
+          const int j = (p - 2 * h) * 8 + lane / 4;  // staging row
+          const uint4 val = lds_16(stage + j * 64 + q * 16);
+          if (rows[p] >= 0 && o_ok)
+            *reinterpret_cast<uint4*>(out + static_cast<int64_t>(rows[p]) * cout + o) = val;
+        }
+        __syncwarp();
+      }
+#pragma unroll
+      for (int p = 0; p < 4; ++p) rows[p] = rows_n[p];
+    }
+    return;
+  }
 #pragma unroll 1
   for (int ci = 0; ci < kChunks; ++ci) {
     uint32_t v[32];

@@ -360,8 +360,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(acc * TP);
       // voxel positions store to their row; pads and empty positions are dropped
-      epilogue_tile_bf16<ACT, true>(taddr, bias_v, stage, lane, o_warp, a.cout, a.pos + tile * TP,
-                                    0, 0, a.out, a.residual);
+      if (o_warp < a.cout)  // a warp whose 32 channels all lie past Cout has nothing to store
+        epilogue_tile_bf16<ACT, true>(taddr, bias_v, stage, lane, o_warp, a.cout,
+                                      a.pos + tile * TP, 0, 0, a.out, a.residual);
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
     }

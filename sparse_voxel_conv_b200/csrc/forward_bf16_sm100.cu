@@ -390,8 +390,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           (a.bias && o_warp + lane < a.cout) ? __bfloat162float(a.bias[o_warp + lane]) : 0.0f;
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(acc * TV);
-      epilogue_tile_bf16<ACT, false>(taddr, bias_v, stage, lane, o_warp, a.cout, nullptr, row0,
-                                     a.n, a.out, a.residual);
+      if (o_warp < a.cout)  // a warp whose 32 channels all lie past Cout has nothing to store
+        epilogue_tile_bf16<ACT, false>(taddr, bias_v, stage, lane, o_warp, a.cout, nullptr,
+                                       row0, a.n, a.out, a.residual);
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
     }

@@ -35,6 +35,33 @@ def _cuda_contig(t: torch.Tensor, name: str, dtype=None) -> torch.Tensor:
     return t.contiguous()
 
 
+def _new(t, orig):
+    """t when this binding made it (an allocation or a contiguous copy), else None."""
+    return None if t is orig else t
+
+
+def _on_side_stream(stream, *made) -> None:
+    """Before a call enqueued on `stream` when that is not torch's current stream.
+
+    This binding allocates outputs and scratch, and makes contiguous copies, on
+    the current stream; the caching allocator hands out memory that is free in
+    that stream's order only.  So the side stream first waits for the work
+    already queued on the current stream, and the tensors made here are
+    recorded as in use by the side stream (their memory is not handed out again
+    before its work has run).  `made`: only tensors created here (None skipped);
+    the caller's own tensors are the caller's to manage."""
+    if stream is None:
+        return
+    side = stream if isinstance(stream, torch.cuda.Stream) else torch.cuda.ExternalStream(int(stream))
+    current = torch.cuda.current_stream()
+    if side.cuda_stream == current.cuda_stream:
+        return
+    side.wait_stream(current)
+    for t in made:
+        if t is not None:
+            t.record_stream(side)
+
+
 def build_map(coords: torch.Tensor, grid_dim: int, batch: int = 1, stream=None,
               check: bool = True, nbr: torch.Tensor | None = None,
               workspace: torch.Tensor | None = None) -> MapHandle:
@@ -45,6 +72,7 @@ def build_map(coords: torch.Tensor, grid_dim: int, batch: int = 1, stream=None,
     coordinates; with check=False it stays asynchronous (call .status later).
     nbr / workspace may be passed in to reuse memory.
     """
+    coords_in, nbr_in, workspace_in = coords, nbr, workspace
     coords = _cuda_contig(coords, "coords", torch.int32)
     if coords.dim() != 2 or coords.shape[1] != 4:
         raise ValueError("coords must have shape [N, 4]")
@@ -57,6 +85,8 @@ def build_map(coords: torch.Tensor, grid_dim: int, batch: int = 1, stream=None,
         nbr = torch.empty((n, 27), dtype=torch.int32, device=dev)
     if workspace is None or workspace.numel() * workspace.element_size() < ws_bytes:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    _on_side_stream(stream, _new(coords, coords_in), _new(nbr, nbr_in),
+                    _new(workspace, workspace_in))
     h = _abi.subm3d_build_map(coords, n, grid_dim, batch, nbr, workspace, ws_bytes, stream)
     h.coords = coords
     if check:
@@ -93,6 +123,7 @@ def forward(h: MapHandle, feats: torch.Tensor, weight: torch.Tensor, flip: bool 
     """
     if feats.dtype not in _DTYPES:
         raise ValueError(f"unsupported feature dtype {feats.dtype}")
+    given = (feats, weight, bias, residual, out)
     feats = _cuda_contig(feats, "feats")
     weight = _cuda_contig(weight, "weight", feats.dtype)
     n, cin = feats.shape
@@ -111,6 +142,8 @@ def forward(h: MapHandle, feats: torch.Tensor, weight: torch.Tensor, flip: bool 
             raise ValueError("residual must have shape [N, Cout]")
     if out is None:
         out = torch.empty((n, cout), dtype=feats.dtype, device=feats.device)
+    _on_side_stream(stream, *(_new(t, g) for t, g in zip((feats, weight, bias, residual, out),
+                                                          given)))
     if kernel == "auto" and use_tile_mask:
         _abi.subm3d_forward_fused(h, feats, weight, bias, residual, out, cin, cout,
                                   _DTYPES[feats.dtype], flip, _ACTS[act], stream)
@@ -132,6 +165,7 @@ def backward_data(h: MapHandle, dy: torch.Tensor, weight: torch.Tensor, flip: bo
     opposite orientation.  dy: [N, Cout]; returns [N, Cin] in dy's dtype."""
     if dy.dtype not in _DTYPES:
         raise ValueError(f"unsupported dtype {dy.dtype}")
+    given = (dy, weight, out)
     dy = _cuda_contig(dy, "dy")
     weight = _cuda_contig(weight, "weight", dy.dtype)
     n, cout = dy.shape
@@ -141,6 +175,7 @@ def backward_data(h: MapHandle, dy: torch.Tensor, weight: torch.Tensor, flip: bo
     weight_t = torch.empty(weight.numel(), dtype=dy.dtype, device=dy.device)
     if out is None:
         out = torch.empty((n, cin), dtype=dy.dtype, device=dy.device)
+    _on_side_stream(stream, weight_t, *(_new(t, g) for t, g in zip((dy, weight, out), given)))
     _abi.subm3d_backward_data(h, dy, weight, weight_t, out, cin, cout, _DTYPES[dy.dtype], flip,
                               stream)
     return out
@@ -152,6 +187,7 @@ def backward_weight(h: MapHandle, feats: torch.Tensor, dy: torch.Tensor, flip: b
     26 - k under flip), fp32 KRSC [Cout, 3, 3, 3, Cin] for either dtype."""
     if feats.dtype not in _DTYPES:
         raise ValueError(f"unsupported dtype {feats.dtype}")
+    given = (feats, dy, out)
     feats = _cuda_contig(feats, "feats")
     dy = _cuda_contig(dy, "dy", feats.dtype)
     n, cin = feats.shape
@@ -160,6 +196,7 @@ def backward_weight(h: MapHandle, feats: torch.Tensor, dy: torch.Tensor, flip: b
         raise ValueError("feats and dy must have the map's N rows")
     if out is None:
         out = torch.empty((cout, 3, 3, 3, cin), dtype=torch.float32, device=feats.device)
+    _on_side_stream(stream, *(_new(t, g) for t, g in zip((feats, dy, out), given)))
     _abi.subm3d_backward_weight(h, feats, dy, out, cin, cout, _DTYPES[feats.dtype], flip, stream)
     return out
 

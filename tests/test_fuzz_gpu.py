@@ -1,0 +1,74 @@
+"""A seeded random sweep through the map build and the forward kernels.
+
+Small random coordinate sets -- several grid sizes (odd ones included), batch
+sizes, densities and row orders (raster, permuted, reversed) -- with channel
+pairs that reach every forward kernel: the x-run bf16 kernel (Cin >= 48, whole
+and partial 64-channel chunks, Cout below, at and above 128), the per-offset
+bf16 kernel (Cin < 48) and the fp32 kernel (any size).  nbr must equal the
+oracle's bit for bit and every output row must meet the path's bar against the
+oracle (bf16 2e-2, fp32 1e-5 of |ref| + rms ref).
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads as WL
+from oracle import cpp as C
+from tests.helpers import RTOL_BF16, RTOL_F32, assert_close
+
+pytestmark = pytest.mark.gpu
+
+_CHANNELS = [(16, 16, "bf16"), (32, 48, "bf16"), (48, 32, "bf16"), (64, 64, "bf16"),
+             (80, 144, "bf16"), (128, 128, "bf16"), (96, 16, "bf16"), (8, 24, "f32"),
+             (20, 12, "f32")]
+
+
+def _cases(count=45, seed=2024):
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(count):
+        grid = int(rng.choice([5, 9, 17, 24, 33]))
+        batch = int(rng.integers(1, 4))
+        p = float(rng.choice([0.03, 0.15, 0.4]))
+        order = ["raster", "permuted", "reversed"][i % 3]
+        cin, cout, dtype = _CHANNELS[i % len(_CHANNELS)]
+        act = [None, "gelu", "silu"][int(rng.integers(0, 3))]
+        flip = bool(rng.integers(0, 2))
+        out.append((1000 + i, grid, batch, p, order, cin, cout, dtype, act, flip))
+    return out
+
+
+@pytest.fixture(scope="module")
+def S():
+    import sparse_voxel_conv_b200 as S
+    return S
+
+
+@pytest.mark.parametrize("case", _cases(), ids=lambda c: f"s{c[0]}-g{c[1]}b{c[2]}-{c[4]}-{c[5]}x{c[6]}{c[7]}")
+def test_random_sets_against_oracle(S, case):
+    seed, grid, batch, p, order, cin, cout, dtype, act, flip = case
+    coords = WL.random_coords(seed, grid, batch, p)
+    n = coords.shape[0]
+    if order == "permuted":
+        coords = coords[WL.permute_rows(n, seed)]
+    elif order == "reversed":
+        coords = coords[::-1]
+    coords = np.ascontiguousarray(coords)
+    x = WL.make_features(n, cin, seed + 1)
+    w = WL.make_weight(cout, cin, seed + 2)
+    if dtype == "bf16":
+        x, w = WL.to_bf16_values(x), WL.to_bf16_values(w)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+
+    h = S.build_map(torch.from_numpy(coords).cuda(), grid, batch)
+    want_nbr = C.build_map(coords, grid, batch)
+    assert np.array_equal(h.nbr.cpu().numpy(), want_nbr), case
+
+    y = S.forward(h, torch.from_numpy(x).cuda().to(tdt), torch.from_numpy(w).cuda().to(tdt),
+                  flip=flip, act=act)
+    torch.cuda.synchronize()
+    assert S._abi.subm3d_device_status() == 0
+    ref = C.forward(want_nbr, np.asarray(x, np.float64), np.asarray(w, np.float64), flip=flip,
+                    act=act, round_to_bf16=(dtype == "bf16"))
+    assert_close(y.float().cpu().numpy(), ref, RTOL_BF16 if dtype == "bf16" else RTOL_F32,
+                 f"random set {case}")

@@ -21,7 +21,7 @@ from dataclasses import dataclass, field
 import numpy as np
 
 __all__ = [
-    "Workload", "WORKLOADS", "make_workload", "tiny_coords", "shell_coords",
+    "Workload", "WORKLOADS", "make_workload", "tiny_coords", "random_coords", "shell_coords",
     "headline_coords", "dense_coords", "batched_coords", "make_features",
     "make_weight", "permute_rows", "to_bf16_values",
 ]
@@ -55,6 +55,14 @@ def tiny_coords(seed: int = 0, grid: int = 16, p: float = 0.3) -> np.ndarray:
     """Batch 1, 16^3 grid, each cell occupied i.i.d. with probability p (1,223 voxels at seed 0)."""
     occ = np.random.default_rng(seed).random((grid, grid, grid)) < p
     return _raster(occ)
+
+
+def random_coords(seed: int, grid: int, batch: int, p: float) -> np.ndarray:
+    """`batch` grids of grid^3 cells, each cell occupied i.i.d. with probability
+    p; rows in raster order (b, z, y, x)."""
+    rng = np.random.default_rng(seed)
+    parts = [_raster(rng.random((grid, grid, grid)) < p, b) for b in range(batch)]
+    return np.concatenate(parts) if parts else np.empty((0, 4), np.int32)
 
 
 def shell_coords(grid: int = 64, radius: float = 24.0, half: float = 1.0) -> np.ndarray:

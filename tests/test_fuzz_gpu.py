@@ -1,4 +1,5 @@
-"""A seeded random sweep through the map build and the forward kernels.
+"""A seeded random sweep through the map build, the forward kernels, the
+gradients and the resolution changes.
 
 Small random coordinate sets -- several grid sizes (odd ones included), batch
 sizes, densities and row orders (raster, permuted, reversed) -- with channel
@@ -47,13 +48,7 @@ def S():
 @pytest.mark.parametrize("case", _cases(), ids=lambda c: f"s{c[0]}-g{c[1]}b{c[2]}-{c[4]}-{c[5]}x{c[6]}{c[7]}")
 def test_random_sets_against_oracle(S, case):
     seed, grid, batch, p, order, cin, cout, dtype, act, flip = case
-    coords = WL.random_coords(seed, grid, batch, p)
-    n = coords.shape[0]
-    if order == "permuted":
-        coords = coords[WL.permute_rows(n, seed)]
-    elif order == "reversed":
-        coords = coords[::-1]
-    coords = np.ascontiguousarray(coords)
+    coords, n = _case_inputs(case)
     x = WL.make_features(n, cin, seed + 1)
     w = WL.make_weight(cout, cin, seed + 2)
     if dtype == "bf16":
@@ -72,3 +67,83 @@ def test_random_sets_against_oracle(S, case):
                     act=act, round_to_bf16=(dtype == "bf16"))
     assert_close(y.float().cpu().numpy(), ref, RTOL_BF16 if dtype == "bf16" else RTOL_F32,
                  f"random set {case}")
+
+
+RTOL_WGRAD = 1e-4  # fp32 weight gradient: fp32 atomics over up to N terms per entry
+
+
+def _case_inputs(case):
+    seed, grid, batch, p, order, cin, cout, dtype, act, flip = case
+    coords = WL.random_coords(seed, grid, batch, p)
+    n = coords.shape[0]
+    if order == "permuted":
+        coords = coords[WL.permute_rows(n, seed)]
+    elif order == "reversed":
+        coords = coords[::-1]
+    return np.ascontiguousarray(coords), n
+
+
+@pytest.mark.parametrize("case", _cases(count=18, seed=77),
+                         ids=lambda c: f"s{c[0]}-g{c[1]}b{c[2]}-{c[4]}-{c[5]}x{c[6]}{c[7]}")
+def test_random_sets_gradients_against_oracle(S, case):
+    """Input and weight gradients on random sets (the input gradient is a forward
+    Cout -> Cin, so the channel pairs reach the x-run and per-offset kernels in
+    that direction too)."""
+    seed, grid, batch, p, order, cin, cout, dtype, act, flip = case
+    coords, n = _case_inputs(case)
+    x = WL.make_features(n, cin, seed + 3)
+    w = WL.make_weight(cout, cin, seed + 4)
+    dy = WL.make_features(n, cout, seed + 5)
+    if dtype == "bf16":
+        x, w, dy = WL.to_bf16_values(x), WL.to_bf16_values(w), WL.to_bf16_values(dy)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda().to(tdt)
+    h = S.build_map(torch.from_numpy(coords).cuda(), grid, batch)
+    dx = S.backward_data(h, t(dy), t(w), flip=flip)
+    dw = S.backward_weight(h, t(x), t(dy), flip=flip)
+    torch.cuda.synchronize()
+    assert S._abi.subm3d_device_status() == 0
+    nbr = C.build_map(coords, grid, batch)
+    ref_dx = C.backward_data(nbr, np.asarray(dy, np.float64), np.asarray(w, np.float64), flip=flip)
+    if dtype == "bf16":
+        ref_dx = C.round_bf16(ref_dx)
+    assert_close(dx.float().cpu().numpy(), ref_dx, RTOL_BF16 if dtype == "bf16" else RTOL_F32,
+                 f"input gradient {case}")
+    ref_dw = C.backward_weight(nbr, np.asarray(x, np.float64), np.asarray(dy, np.float64), flip=flip)
+    assert_close(dw.cpu().numpy(), ref_dw, RTOL_WGRAD, f"weight gradient {case}")
+
+
+@pytest.mark.parametrize("case", _cases(count=12, seed=99),
+                         ids=lambda c: f"s{c[0]}-g{c[1]}b{c[2]}-{c[4]}-{c[7]}")
+def test_random_sets_resampling_against_oracle(S, case):
+    """Subdivide, max / mean downsample and spatial2channel on random sets, every
+    row against the resampling oracle."""
+    from oracle import resample_oracle as R
+    seed, grid, batch, p, order, cin, cout, dtype, act, flip = case
+    coords, n = _case_inputs(case)
+    # the pooling oracle and kernels take raster-ordered parents from any child order
+    f = WL.make_features(n, cin, seed + 6)
+    if dtype == "bf16":
+        f = WL.to_bf16_values(f)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    st = S.SparseTensor(torch.from_numpy(coords).cuda(), torch.from_numpy(f).cuda().to(tdt),
+                        grid_dim=grid, batch=batch)
+    npf = lambda t: t.float().cpu().numpy() if t.is_floating_point() else t.cpu().numpy()
+    fine = S.subdivide(st)
+    rc, rf = R.subdivide(coords, f)
+    assert np.array_equal(npf(fine.coords), rc) and np.array_equal(npf(fine.feats), rf), case
+    for mode in ("max", "mean"):
+        out = S.downsample(st, mode)
+        rc, rf = R.downsample(coords, f, mode)
+        assert np.array_equal(npf(out.coords), rc), (case, mode)
+        if mode == "max":
+            assert np.array_equal(npf(out.feats), rf.astype(np.float32)), (case, mode)
+        else:
+            ref = WL.to_bf16_values(rf.astype(np.float32)) if dtype == "bf16" else rf
+            assert_close(npf(out.feats), ref, RTOL_BF16 if dtype == "bf16" else RTOL_F32,
+                         f"mean pooling {case}")
+    out = S.spatial2channel(st)
+    rc, rf = R.spatial2channel(coords, f)
+    assert np.array_equal(npf(out.coords), rc) and np.array_equal(npf(out.feats), rf), case
+    torch.cuda.synchronize()
+    assert S._abi.subm3d_device_status() == 0

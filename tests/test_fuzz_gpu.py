@@ -147,3 +147,33 @@ def test_random_sets_resampling_against_oracle(S, case):
     assert np.array_equal(npf(out.coords), rc) and np.array_equal(npf(out.feats), rf), case
     torch.cuda.synchronize()
     assert S._abi.subm3d_device_status() == 0
+
+
+@pytest.mark.parametrize("kind", ["brick", "hash"])
+@pytest.mark.parametrize("case", _cases(count=15, seed=123),
+                         ids=lambda c: f"s{c[0]}-g{c[1]}b{c[2]}-{c[4]}-{c[5]}x{c[6]}{c[7]}")
+def test_random_sets_table_kinds(S, case, kind, monkeypatch):
+    """The brick and hash tables (forced with the testing knob SUBM3D_MAP_KIND)
+    give the oracle's nbr, and the forward on their maps equals, bit for bit,
+    the forward on the direct table's map: the map, and the x-run layout built
+    from it, do not depend on the table."""
+    seed, grid, batch, p, order, cin, cout, dtype, act, flip = case
+    coords, n = _case_inputs(case)
+    x = WL.make_features(n, cin, seed + 7)
+    w = WL.make_weight(cout, cin, seed + 8)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    xt = torch.from_numpy(x).cuda().to(tdt)
+    wt = torch.from_numpy(w).cuda().to(tdt)
+    ct = torch.from_numpy(coords).cuda()
+    monkeypatch.delenv("SUBM3D_MAP_KIND", raising=False)
+    h_direct = S.build_map(ct, grid, batch)
+    y_direct = S.forward(h_direct, xt, wt, flip=flip, act=act)
+    monkeypatch.setenv("SUBM3D_MAP_KIND", kind)
+    h = S.build_map(ct, grid, batch)
+    y = S.forward(h, xt, wt, flip=flip, act=act)
+    torch.cuda.synchronize()
+    assert S._abi.subm3d_device_status() == 0
+    want = {"brick": S._abi.SUBM3D_TABLE_BRICK, "hash": S._abi.SUBM3D_TABLE_HASH}[kind]
+    assert S._abi.subm3d_map_table(h) == want
+    assert np.array_equal(h.nbr.cpu().numpy(), C.build_map(coords, grid, batch)), case
+    assert torch.equal(y, y_direct), case

@@ -5,7 +5,8 @@ Small random coordinate sets -- several grid sizes (odd ones included), batch
 sizes, densities and row orders (raster, permuted, reversed) -- with channel
 pairs that reach every forward kernel: the x-run bf16 kernel (Cin >= 48, whole
 and partial 64-channel chunks, Cout below, at and above 128), the per-offset
-bf16 kernel (Cin < 48) and the fp32 kernel (any size).  nbr must equal the
+bf16 kernel (Cin < 48) and the fp32 kernel (any size), some with a bias and a
+residual in the fused epilogue.  nbr must equal the
 oracle's bit for bit and every output row must meet the path's bar against the
 oracle (bf16 2e-2, fp32 1e-5 of |ref| + rms ref).
 """
@@ -54,17 +55,26 @@ def test_random_sets_against_oracle(S, case):
     if dtype == "bf16":
         x, w = WL.to_bf16_values(x), WL.to_bf16_values(w)
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    # the fused epilogue's inputs on some of the sets: a bias on odd seeds, a
+    # residual on every third (fp32 staging in the bf16 kernels then)
+    bias = WL.make_features(1, cout, seed + 9)[0] if seed % 2 else None
+    res = WL.make_features(n, cout, seed + 10) if seed % 3 == 0 else None
+    if dtype == "bf16":
+        bias = None if bias is None else WL.to_bf16_values(bias)
+        res = None if res is None else WL.to_bf16_values(res)
+    t = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).cuda().to(tdt)
 
     h = S.build_map(torch.from_numpy(coords).cuda(), grid, batch)
     want_nbr = C.build_map(coords, grid, batch)
     assert np.array_equal(h.nbr.cpu().numpy(), want_nbr), case
 
-    y = S.forward(h, torch.from_numpy(x).cuda().to(tdt), torch.from_numpy(w).cuda().to(tdt),
-                  flip=flip, act=act)
+    y = S.forward(h, t(x), t(w), flip=flip, act=act, bias=t(bias), residual=t(res))
     torch.cuda.synchronize()
     assert S._abi.subm3d_device_status() == 0
     ref = C.forward(want_nbr, np.asarray(x, np.float64), np.asarray(w, np.float64), flip=flip,
-                    act=act, round_to_bf16=(dtype == "bf16"))
+                    act=act, round_to_bf16=(dtype == "bf16"),
+                    bias=None if bias is None else np.asarray(bias, np.float64),
+                    residual=None if res is None else np.asarray(res, np.float64))
     assert_close(y.float().cpu().numpy(), ref, RTOL_BF16 if dtype == "bf16" else RTOL_F32,
                  f"random set {case}")
 

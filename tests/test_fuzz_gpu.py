@@ -187,3 +187,30 @@ def test_random_sets_table_kinds(S, case, kind, monkeypatch):
     assert S._abi.subm3d_map_table(h) == want
     assert np.array_equal(h.nbr.cpu().numpy(), C.build_map(coords, grid, batch)), case
     assert torch.equal(y, y_direct), case
+
+
+@pytest.mark.parametrize("kind", ["auto", "brick", "hash"])
+@pytest.mark.parametrize("seed,grid,batch,p", [(2001, 7, 5, 0.3), (2002, 12, 6, 0.1),
+                                              (2003, 20, 7, 0.05)])
+def test_random_sets_wide_keys(S, seed, grid, batch, p, kind, monkeypatch):
+    """Batches above 4 take the wide (64-bit) keys in the hash table and more
+    grids in the direct and brick tables: nbr against the oracle, in permuted
+    row order, and the x-run forward against the oracle."""
+    if kind == "auto":
+        monkeypatch.delenv("SUBM3D_MAP_KIND", raising=False)
+    else:
+        monkeypatch.setenv("SUBM3D_MAP_KIND", kind)
+    coords = WL.random_coords(seed, grid, batch, p)
+    n = coords.shape[0]
+    coords = np.ascontiguousarray(coords[WL.permute_rows(n, seed)])
+    h = S.build_map(torch.from_numpy(coords).cuda(), grid, batch)
+    nbr = C.build_map(coords, grid, batch)
+    assert np.array_equal(h.nbr.cpu().numpy(), nbr)
+    x = WL.to_bf16_values(WL.make_features(n, 64, seed + 1))
+    w = WL.to_bf16_values(WL.make_weight(64, 64, seed + 2))
+    y = S.forward(h, torch.from_numpy(x).cuda().to(torch.bfloat16),
+                  torch.from_numpy(w).cuda().to(torch.bfloat16))
+    torch.cuda.synchronize()
+    assert S._abi.subm3d_device_status() == 0
+    ref = C.forward(nbr, np.asarray(x, np.float64), np.asarray(w, np.float64), round_to_bf16=True)
+    assert_close(y.float().cpu().numpy(), ref, RTOL_BF16, f"wide keys {kind} b={batch}")

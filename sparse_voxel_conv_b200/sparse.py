@@ -52,7 +52,8 @@ def _on_side_stream(stream, *made) -> None:
     the caller's own tensors are the caller's to manage."""
     if stream is None:
         return
-    side = stream if isinstance(stream, torch.cuda.Stream) else torch.cuda.ExternalStream(int(stream))
+    side = (stream if isinstance(stream, torch.cuda.Stream)
+            else torch.cuda.ExternalStream(int(stream)))
     current = torch.cuda.current_stream()
     if side.cuda_stream == current.cuda_stream:
         return

@@ -46,7 +46,11 @@ def S():
     return S
 
 
-@pytest.mark.parametrize("case", _cases(), ids=lambda c: f"s{c[0]}-g{c[1]}b{c[2]}-{c[4]}-{c[5]}x{c[6]}{c[7]}")
+def _case_id(c):
+    return f"s{c[0]}-g{c[1]}b{c[2]}-{c[4]}-{c[5]}x{c[6]}{c[7]}"
+
+
+@pytest.mark.parametrize("case", _cases(), ids=_case_id)
 def test_random_sets_against_oracle(S, case):
     seed, grid, batch, p, order, cin, cout, dtype, act, flip = case
     coords, n = _case_inputs(case)
@@ -93,8 +97,7 @@ def _case_inputs(case):
     return np.ascontiguousarray(coords), n
 
 
-@pytest.mark.parametrize("case", _cases(count=18, seed=77),
-                         ids=lambda c: f"s{c[0]}-g{c[1]}b{c[2]}-{c[4]}-{c[5]}x{c[6]}{c[7]}")
+@pytest.mark.parametrize("case", _cases(count=18, seed=77), ids=_case_id)
 def test_random_sets_gradients_against_oracle(S, case):
     """Input and weight gradients on random sets (the input gradient is a forward
     Cout -> Cin, so the channel pairs reach the x-run and per-offset kernels in
@@ -119,7 +122,8 @@ def test_random_sets_gradients_against_oracle(S, case):
         ref_dx = C.round_bf16(ref_dx)
     assert_close(dx.float().cpu().numpy(), ref_dx, RTOL_BF16 if dtype == "bf16" else RTOL_F32,
                  f"input gradient {case}")
-    ref_dw = C.backward_weight(nbr, np.asarray(x, np.float64), np.asarray(dy, np.float64), flip=flip)
+    ref_dw = C.backward_weight(nbr, np.asarray(x, np.float64), np.asarray(dy, np.float64),
+                               flip=flip)
     assert_close(dw.cpu().numpy(), ref_dw, RTOL_WGRAD, f"weight gradient {case}")
 
 
@@ -160,8 +164,7 @@ def test_random_sets_resampling_against_oracle(S, case):
 
 
 @pytest.mark.parametrize("kind", ["brick", "hash"])
-@pytest.mark.parametrize("case", _cases(count=15, seed=123),
-                         ids=lambda c: f"s{c[0]}-g{c[1]}b{c[2]}-{c[4]}-{c[5]}x{c[6]}{c[7]}")
+@pytest.mark.parametrize("case", _cases(count=15, seed=123), ids=_case_id)
 def test_random_sets_table_kinds(S, case, kind, monkeypatch):
     """The brick and hash tables (forced with the testing knob SUBM3D_MAP_KIND)
     give the oracle's nbr, and the forward on their maps equals, bit for bit,
